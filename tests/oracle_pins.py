@@ -1,0 +1,271 @@
+"""Pins for the CPU oracle: checks against facts fixed by the pages and by
+mathematics, never against the oracle itself.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError
+when the oracle disagrees.  ``tests/test_oracle.py`` runs them on the real
+oracle; ``tests/test_oracle_mutants.py`` runs them on deliberately broken
+copies to show that each plausible mistake is caught by at least one pin.
+"""
+from __future__ import annotations
+
+import itertools
+import os
+
+import numpy as np
+
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "worked_example.txt")
+
+# bf16 bit patterns of the small alphabet {0, -0, +-1, +-2, +-3, +-4}.
+_ALPHABET = np.array([0x0000, 0x8000, 0x3F80, 0xBF80, 0x4000, 0xC000,
+                      0x4040, 0xC040, 0x4080, 0xC080], dtype=np.uint16)
+
+
+def _bf16(x) -> np.ndarray:
+    return synth.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+def _f64(bits) -> np.ndarray:
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def brute_force_pair(group_abs) -> tuple[int, int]:
+    """Frobenius-optimal 2:4 choice by enumeration of all six index pairs.
+
+    A pair is optimal when every kept magnitude is >= every dropped one (the
+    hard-thresholding optimum of HASSLE-free section 4.1.1); among optimal
+    pairs take the lexicographically smallest (the lower-index tie rule).
+    """
+    best = None
+    for a, b in itertools.combinations(range(4), 2):
+        dropped = [group_abs[p] for p in range(4) if p not in (a, b)]
+        if min(group_abs[a], group_abs[b]) >= max(dropped):
+            if best is None or (a, b) < best:
+                best = (a, b)
+    return best
+
+
+def decode_meta(meta_row: np.ndarray, groups: int):
+    out = []
+    for g in range(groups):
+        nib = (int(meta_row[g // 2]) >> (4 * (g % 2))) & 0xF
+        out.append((nib & 3, nib >> 2))
+    return out
+
+
+def read_golden(path: str = GOLDEN):
+    rows = {}
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            rows.setdefault(key, []).append(vals)
+    hexrows = lambda k: np.array([[int(v, 16) for v in r] for r in rows[k]], dtype=np.uint16)
+    return {
+        "W": hexrows("W"), "VALS": hexrows("VALS"),
+        "META": np.array([[int(v, 16) for v in r] for r in rows["META"]], dtype=np.uint8),
+        "X": hexrows("X"), "U": hexrows("U"), "V": hexrows("V"),
+        "Y": np.array([[float(v) for v in r] for r in rows["Y"]]),
+        "B": np.array([[float(v) for v in r] for r in rows["B"]]),
+    }
+
+
+# --------------------------------------------------------------------------- pack pins
+
+def pin_pack_golden(o):
+    g = read_golden()
+    vals, meta = o.pack_2to4(g["W"])
+    np.testing.assert_array_equal(vals, g["VALS"])
+    np.testing.assert_array_equal(meta, g["META"])
+
+
+def pin_pack_exhaustive_alphabet(o):
+    """Every group of four over the 10-letter alphabet (10^4 groups)."""
+    groups = np.array(list(itertools.product(range(len(_ALPHABET)), repeat=4)))
+    W = _ALPHABET[groups].reshape(-1, 4)        # one group per row, d_in = 4
+    vals, meta = o.pack_2to4(W)
+    absf = np.abs(_f64(W))
+    for i in range(W.shape[0]):
+        a, b = brute_force_pair(absf[i])
+        nib = int(meta[i, 0]) & 0xF
+        assert (nib & 3, nib >> 2) == (a, b), (i, W[i], (nib & 3, nib >> 2), (a, b))
+        assert vals[i, 0] == W[i, a] and vals[i, 1] == W[i, b], (i, W[i], vals[i])
+        assert int(meta[i, 0]) >> 4 == 0
+
+
+def pin_pack_random_bruteforce(o, seed: int = 7):
+    """Random bf16 groups with a narrow exponent range (many exact ties)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    sign = rng.integers(0, 2, size=(300, 24)).astype(np.uint16) << 15
+    expo = rng.integers(125, 129, size=(300, 24)).astype(np.uint16) << 7
+    mant = rng.integers(0, 4, size=(300, 24)).astype(np.uint16) << 5
+    W = (sign | expo | mant).astype(np.uint16)
+    vals, meta = o.pack_2to4(W)
+    absf = np.abs(_f64(W))
+    for i in range(W.shape[0]):
+        pairs = decode_meta(meta[i], 6)
+        for g in range(6):
+            a, b = brute_force_pair(absf[i, 4 * g:4 * g + 4])
+            assert pairs[g] == (a, b), (i, g)
+            assert vals[i, 2 * g] == W[i, 4 * g + a] and vals[i, 2 * g + 1] == W[i, 4 * g + b]
+
+
+def pin_pack_invariants(o):
+    layer = synth.CONFIGS[1].layers[0]
+    W = layer.weight()
+    vals, meta = o.pack_2to4(W)
+    d_out, d_in = W.shape
+    S = o.unpack_2to4(vals, meta, d_in)
+    Wf = np.abs(_f64(W))
+    for i in range(0, d_out, 7):
+        pairs = decode_meta(meta[i], d_in // 4)
+        for g, (a, b) in enumerate(pairs):
+            assert 0 <= a < b <= 3
+            grp = Wf[i, 4 * g:4 * g + 4]
+            dropped = [grp[p] for p in range(4) if p not in (a, b)]
+            assert min(grp[a], grp[b]) >= max(dropped)
+            assert np.count_nonzero(S[i, 4 * g:4 * g + 4] & 0x7FFF) <= 2
+            for p in range(4):
+                if p not in (a, b):
+                    assert S[i, 4 * g + p] == 0
+                else:
+                    assert S[i, 4 * g + p] == W[i, 4 * g + p]
+
+
+def pin_pack_roundtrip(o):
+    W = synth.gaussian_bf16((64, 96), 0.02, 11)
+    vals, meta = o.pack_2to4(W)
+    S = o.unpack_2to4(vals, meta, 96)
+    vals2, meta2 = o.pack_2to4(S)          # idempotent on an already-projected matrix
+    np.testing.assert_array_equal(vals2, vals)
+    np.testing.assert_array_equal(meta2, meta)
+    # A matrix that is 2:4 by construction packs losslessly.
+    rng = np.random.Generator(np.random.PCG64(12))
+    dense = np.zeros((32, 64), dtype=np.uint16)
+    for i in range(32):
+        for g in range(16):
+            a, b = sorted(rng.choice(4, size=2, replace=False))
+            dense[i, 4 * g + a] = _bf16([rng.uniform(0.5, 2.0) * rng.choice([-1, 1])])[0]
+            dense[i, 4 * g + b] = _bf16([rng.uniform(0.5, 2.0) * rng.choice([-1, 1])])[0]
+    v3, m3 = o.pack_2to4(dense)
+    np.testing.assert_array_equal(o.unpack_2to4(v3, m3, 64), dense)
+
+
+def pin_pack_specials(o):
+    """NaN/Inf/-0 follow the integer magnitude key (a stated reading)."""
+    W = np.array([[0x3F80, 0x7FC0, 0x7F80, 0xFF80,      # 1, NaN, +Inf, -Inf -> keep NaN, +Inf
+                   0x8000, 0x0000, 0x8000, 0x0000]],     # -0, +0, -0, +0     -> keep idx 0, 1
+                 dtype=np.uint16)
+    vals, meta = o.pack_2to4(W)
+    np.testing.assert_array_equal(vals, [[0x7FC0, 0x7F80, 0x8000, 0x0000]])
+    assert int(meta[0, 0]) == ((1 | 2 << 2) | ((0 | 1 << 2) << 4))
+
+
+def pin_pack_odd_groups(o):
+    """d_in = 12: three groups, the last meta byte holds one nibble."""
+    W = _bf16([[1, 2, 3, 4, 4, 3, 2, 1, 0, 5, 0, 5]])
+    vals, meta = o.pack_2to4(W)
+    assert meta.shape == (1, 2)
+    np.testing.assert_array_equal(vals, _bf16([[3, 4, 4, 3, 5, 5]]))
+    assert int(meta[0, 0]) == ((2 | 3 << 2) | ((0 | 1 << 2) << 4))
+    assert int(meta[0, 1]) == (1 | 3 << 2)
+
+
+# --------------------------------------------------------------------------- forward pins
+
+def pin_forward_golden(o):
+    g = read_golden()
+    Y, B = o.forward(g["X"], g["VALS"], g["META"], g["U"], g["V"])
+    np.testing.assert_array_equal(Y, g["Y"])
+    np.testing.assert_array_equal(B, g["B"])
+
+
+def _small_int_problem(seed, M, d_out, d_in, r):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    X = _bf16(rng.integers(-3, 4, size=(M, d_in)))
+    W = _bf16(rng.integers(-4, 5, size=(d_out, d_in)))
+    U = _bf16(rng.integers(-2, 3, size=(d_out, r)))
+    V = _bf16(rng.integers(-2, 3, size=(r, d_in)))
+    return X, W, U, V
+
+
+def pin_forward_identity_exact(o):
+    """X (S + U V)^T == X S^T + (X V^T) U^T, exactly, with small integers
+    (every partial sum is an integer well inside fp64's exact range)."""
+    for seed, (M, d_out, d_in, r) in enumerate([(5, 12, 16, 3), (3, 8, 24, 1), (7, 20, 8, 6)]):
+        X, W, U, V = _small_int_problem(100 + seed, M, d_out, d_in, r)
+        vals, meta = o.pack_2to4(W)
+        S = _f64(o.unpack_2to4(vals, meta, d_in))
+        Xf, Uf, Vf = _f64(X), _f64(U), _f64(V)
+        rhs = Xf @ S.T + (Xf @ Vf.T) @ Uf.T
+        Y, B = o.forward(X, vals, meta, U, V)
+        np.testing.assert_array_equal(Y, rhs)
+        np.testing.assert_array_equal(B, np.abs(Xf) @ np.abs(S + Uf @ Vf).T)
+
+
+def pin_forward_numpy(o):
+    """fp64 library GEMM cross-check on non-square shapes (catches transposes)."""
+    for (M, d_out, d_in, r, seed) in [(8, 256, 256, 8, 1), (6, 40, 72, 5, 2), (9, 24, 64, 16, 3)]:
+        X = synth.gaussian_bf16((M, d_in), 1.0, seed * 10 + 1)
+        W = synth.gaussian_bf16((d_out, d_in), 0.02, seed * 10 + 2)
+        U = synth.gaussian_bf16((d_out, r), 0.3, seed * 10 + 3)
+        V = synth.gaussian_bf16((r, d_in), 0.3, seed * 10 + 4)
+        vals, meta = o.pack_2to4(W)
+        S = _f64(o.unpack_2to4(vals, meta, d_in))
+        Wp = S + _f64(U) @ _f64(V)
+        ref = _f64(X) @ Wp.T
+        Y, B = o.forward(X, vals, meta, U, V)
+        scale = np.abs(_f64(X)) @ np.abs(Wp).T
+        assert np.all(np.abs(Y - ref) <= 1e-12 * scale + 1e-300)
+        assert np.all(np.abs(B - scale) <= 1e-12 * scale + 1e-300)
+        assert np.all(np.abs(Y) <= B * (1 + 1e-12))
+
+
+def pin_forward_one_hot(o):
+    """X = e_j picks column j of W' = S + U V."""
+    d_out, d_in, r = 16, 32, 4
+    _, W, U, V = _small_int_problem(5, 1, d_out, d_in, r)
+    vals, meta = o.pack_2to4(W)
+    S = _f64(o.unpack_2to4(vals, meta, d_in))
+    Wp = S + _f64(U) @ _f64(V)
+    X = np.zeros((d_in, d_in), dtype=np.uint16)
+    X[np.arange(d_in), np.arange(d_in)] = 0x3F80
+    Y, _ = o.forward(X, vals, meta, U, V)
+    np.testing.assert_array_equal(Y, Wp.T)
+
+
+def pin_forward_sparse_only(o):
+    """r = 0 (and U = 0) leaves X S^T."""
+    X, W, U, V = _small_int_problem(6, 4, 12, 16, 3)
+    vals, meta = o.pack_2to4(W)
+    S = _f64(o.unpack_2to4(vals, meta, 16))
+    Y0, _ = o.forward(X, vals, meta, None, None)
+    np.testing.assert_array_equal(Y0, _f64(X) @ S.T)
+    Yz, _ = o.forward(X, vals, meta, np.zeros_like(U), V)
+    np.testing.assert_array_equal(Yz, _f64(X) @ S.T)
+
+
+def pin_forward_row_subset(o):
+    X, W, U, V = _small_int_problem(8, 10, 12, 16, 2)
+    vals, meta = o.pack_2to4(W)
+    Yall, Ball = o.forward(X, vals, meta, U, V)
+    rows = [7, 0, 3, 3]
+    Ys, Bs = o.forward(X, vals, meta, U, V, rows=rows)
+    np.testing.assert_array_equal(Ys, Yall[rows])
+    np.testing.assert_array_equal(Bs, Ball[rows])
+
+
+def pin_lowrank_project(o):
+    X, _, _, V = _small_int_problem(9, 6, 4, 24, 5)
+    np.testing.assert_array_equal(o.lowrank_project(X, V), _f64(X) @ _f64(V).T)
+
+
+ALL_PINS = [
+    pin_pack_golden, pin_pack_exhaustive_alphabet, pin_pack_random_bruteforce,
+    pin_pack_invariants, pin_pack_roundtrip, pin_pack_specials, pin_pack_odd_groups,
+    pin_forward_golden, pin_forward_identity_exact, pin_forward_numpy, pin_forward_one_hot,
+    pin_forward_sparse_only, pin_forward_row_subset, pin_lowrank_project,
+]

@@ -1,0 +1,62 @@
+"""Plant plausible mistakes in a copy of the oracle (on the CPU) and check
+that at least one pin catches each of them.  This is evidence that the pins in
+tests/oracle_pins.py constrain every step of the oracle, not just some."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+TESTS = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(TESTS)
+
+# Runs every pin against one compiled library in a child process (a mutant may
+# crash) and prints the names of the pins that failed.
+_CHILD = """
+import sys
+sys.path[:0] = [{root!r}, {tests!r}]
+import oracle
+from oracle_pins import ALL_PINS
+o = oracle.Oracle({lib!r})
+for pin in ALL_PINS:
+    try:
+        pin(o)
+    except (AssertionError, ValueError, IndexError):
+        print("CAUGHT", pin.__name__)
+"""
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "slr_oracle.c")
+
+# (name, text to replace, replacement, expected number of occurrences)
+MUTANTS = [
+    ("tie_to_higher_index", "(kq == kp && q < p)", "(kq == kp && q > p)", 1),
+    ("signed_key", " & 0x7FFFu;", ";", 2),
+    ("smallest_magnitude", "if (rank < 2) kept[n++] = p;", "if (rank >= 2) kept[n++] = p;", 1),
+    ("kept_order_swapped", "*idx0 = kept[0];\n    *idx1 = kept[1];", "*idx0 = kept[1];\n    *idx1 = kept[0];", 1),
+    ("nibble_fields_swapped", "(unsigned)a | ((unsigned)b << 2)", "(unsigned)b | ((unsigned)a << 2)", 1),
+    ("nibble_position_swapped", "nib << (4 * (g % 2))", "nib << (4 * ((g + 1) % 2))", 1),
+    ("lowrank_sign", "row[j] += lr;", "row[j] -= lr;", 1),
+    ("lowrank_dropped", "row[j] += lr;", "(void)lr;", 1),
+    ("V_transposed", "V[k * d_in + j]", "V[j * r + k]", 2),
+    ("U_wrong_row", "U[i * r + k]", "U[k]", 1),
+    ("X_wrong_row", "xr[j] = bf16_bits_to_double(X[m * d_in + j]);", "xr[j] = bf16_bits_to_double(X[j]);", 1),
+    ("bound_signed", "fabs(xr[j]) * fabs(row[j])", "xr[j] * row[j]", 1),
+    ("sparse_vals_swapped", "row[4 * g + a] = bf16_bits_to_double(vals[i * (d_in / 2) + 2 * g + 0]);",
+     "row[4 * g + a] = bf16_bits_to_double(vals[i * (d_in / 2) + 2 * g + 1]);", 1),
+]
+
+
+@pytest.mark.parametrize("name,old,new,count", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(name, old, new, count, tmp_path):
+    text = open(SRC).read()
+    assert text.count(old) == count, f"mutation site for {name} not found"
+    src = tmp_path / f"{name}.c"
+    src.write_text(text.replace(old, new))
+    lib = oracle.compile_source(str(src), str(tmp_path / f"lib{name}.so"))
+    proc = subprocess.run([sys.executable, "-c", _CHILD.format(root=ROOT, tests=TESTS, lib=lib)],
+                          capture_output=True, text=True, timeout=300)
+    caught = [l.split()[1] for l in proc.stdout.splitlines() if l.startswith("CAUGHT")]
+    # A crash of the mutant also counts as detection, but say so.
+    assert caught or proc.returncode != 0, f"no pin caught mutant {name}: {proc.stderr[-500:]}"
