@@ -1,0 +1,471 @@
+#!/usr/bin/env python
+"""Benchmark of the 2:4-sparse + low-rank linear forward on B200.
+
+Metric: S+LR linear forward TFLOP/s at M = 2048 (Llama-3-8B gate/up shape,
+14336 x 4096, r = 64; dense-equivalent FLOPs 2*M*d_out*d_in per step) and GB/s
+at M = 1 (Llama-3-8B q_proj shape, 4096 x 4096, r = 64), each with its
+fraction of the roofline.  One JSON line on stdout (rank 0).
+
+A step is one forward pass (rank projection T = X V^T, then the fused 2:4 +
+rank-r tensor-core kernel) over one batch of synthetic tokens, inputs
+resident in HBM.  The 2:4 pack is the one-time weight preparation; it is timed
+in the same run and reported under "pack".  Buffers rotate over enough copies
+that the working set of consecutive steps exceeds the 126 MB L2.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+runs its own batch (weak scaling, no collective on the data path) and the
+reported time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+PREFILL = dict(cfg=3, name="gate_up", M=2048)
+DECODE = dict(cfg=2, name="q_proj", M=1)
+
+# Fallback peaks (the profiling recipe's earlier measurement on this machine),
+# used only when MEASURED_PEAKS.json is absent.
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPARSE_RATIO = 2.0   # nominal 2:4 sparse / dense tensor throughput ratio
+
+# DRAM bytes per launch of the dominant kernel from the committed ncu capture
+# (profiles/); valid only for the kernel source it was taken on.
+NCU_TRAFFIC = {}
+
+
+def layer_of(cfg, name):
+    return next(l for l in synth.CONFIGS[cfg].layers if l.name == name)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_bytes(M, d_out, d_in, r):
+    """X + vals + meta + U + V + Y (T's round trip excluded)."""
+    return 2 * M * d_in + d_out * d_in + d_out * d_in // 8 + 2 * r * (d_out + d_in) + 2 * M * d_out
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    with open(os.path.join(ROOT, "sparse_rank_linear_02_b200", "csrc", "tc_forward.cu"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    QUERY = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus_id = bus_id
+        self.proc = None
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.bus_id:
+            cmd.insert(1, f"--id={self.bus_id}")
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.samples = []
+        if self.proc is None:
+            return False
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for row in csv.reader(io.StringIO(out)):
+            if len(row) >= 10:
+                self.samples.append([c.strip() for c in row])
+        return False
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        mx = [float(s[3]) for s in self.samples if s[3].replace(".", "").isdigit()]
+        load = [v for v in sm if v > 0.5 * max(sm)] if sm else []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, dist):
+    import torch
+    import sparse_rank_linear_02_b200 as slr
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ------------------------------------------------ prefill workload (the metric)
+    L = layer_of(PREFILL["cfg"], PREFILL["name"])
+    M, d_out, d_in, r = PREFILL["M"], L.d_out, L.d_in, L.r
+    W = to_dev(L.weight())
+    Uh, Vh = L.factors()
+    Xh = L.activations(M)
+    path = slr.select_path(M, d_out, d_in, r)
+    ws_bytes = slr.workspace_size(M, d_out, d_in, r)
+    vals0, meta0 = slr.pack_2to4(W)
+    set_bytes = algorithmic_bytes(M, d_out, d_in, r) + ws_bytes
+    n_copies = max(2, math.ceil(2.0 * L2_BYTES / set_bytes))
+    sets = []
+    for _ in range(n_copies):
+        sets.append(dict(X=to_dev(Xh), vals=vals0.clone(), meta=meta0.clone(), U=to_dev(Uh), V=to_dev(Vh),
+                         Y=torch.empty((M, d_out), dtype=torch.bfloat16, device=dev),
+                         ws=torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)))
+
+    def step(s, ev_mid=None):
+        slr.forward_project(s["X"], s["V"], d_out, s["ws"], path=path)
+        if ev_mid is not None:
+            ev_mid.record()
+        slr.forward_combine(s["X"], s["vals"], s["meta"], s["U"], s["Y"], s["ws"], path=path)
+
+    for i in range(args.warmup):
+        step(sets[i % n_copies])
+    slr.check_kernel_error()
+    K = args.steps
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    evm = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    bus = getattr(torch.cuda.get_device_properties(dev), "pci_bus_id", None)
+    barrier()
+    with ClockSampler(bus if rank == 0 else None) as clk:
+        for k in range(K):
+            ev0[k].record()
+            step(sets[k % n_copies], evm[k])
+            ev1[k].record()
+        torch.cuda.synchronize()
+    barrier()
+    slr.check_kernel_error()
+    total_ms = max_over_ranks(ev0[0].elapsed_time(ev1[K - 1]))
+    combine_ms = statistics.mean(evm[k].elapsed_time(ev1[k]) for k in range(K))
+    project_ms = statistics.mean(ev0[k].elapsed_time(evm[k]) for k in range(K))
+    ms_per_step = total_ms / K
+    flops_dense = 2.0 * M * d_out * d_in                 # dense-equivalent work per step
+    flops_lr = 2.0 * M * r * (d_in + d_out)
+    flops_exec = M * d_out * d_in + flops_lr              # MACs on kept weights x2 / 2 + rank-r GEMMs
+    value = world * flops_dense / (total_ms / K * 1e-3) / 1e12
+
+    p_dense = peaks["bf16_tflops"]
+    p_sparse = SPARSE_RATIO * p_dense
+    # dominant kernel (the fused 2:4 + rank-r tensor-core combine): sparse
+    # product at the 2:4 peak plus the rank-r expansion T U^T at the dense peak.
+    k_flops_sp = flops_dense
+    k_flops_lr = 2.0 * M * r * d_out
+    t_roof_k = k_flops_sp / (p_sparse * 1e12) + k_flops_lr / (p_dense * 1e12)
+    achieved_k = (k_flops_sp + k_flops_lr) / (combine_ms * 1e-3) / 1e12
+    peak_k = (k_flops_sp + k_flops_lr) / t_roof_k / 1e12
+    sha = kernel_source_sha()
+    traffic = NCU_TRAFFIC.get("tc_forward", {})
+    traffic_bytes = traffic.get("bytes_per_launch") if traffic.get("source_sha") == sha else None
+    roofline = {"bound": "tensor", "kernel": "tc_forward_kernel (2:4 tcgen05.mma.sp + rank-r tcgen05.mma)",
+                "achieved": round(achieved_k, 1), "peak": round(peak_k, 1), "unit": "TFLOP/s",
+                "frac": round(achieved_k / peak_k, 4), "traffic": traffic_bytes,
+                "algorithmic_flops_per_launch": k_flops_sp + k_flops_lr,
+                "kernel_ms": round(combine_ms, 4),
+                "peak_source": f"{peak_src}: 2:4 peak = {SPARSE_RATIO:g} x bf16_tflops {p_dense:g} (burst) for "
+                               f"2*M*d_out*d_in, bf16_tflops for 2*M*r*d_out"}
+    # whole-step roofline (all kernels, the SURVEY's model)
+    step_bytes = algorithmic_bytes(M, d_out, d_in, r)
+    t_roof_step = max(step_bytes / (peaks["hbm_gbs"] * 1e9),
+                      flops_dense / (p_sparse * 1e12) + flops_lr / (p_dense * 1e12))
+    prefill = {"tflops_dense_equiv": round(value / world, 1), "tflops_executed": round(flops_exec / (ms_per_step * 1e-3) / 1e12, 1),
+               "gbs": round(step_bytes / (ms_per_step * 1e-3) / 1e9, 1),
+               "frac_of_roofline": round(t_roof_step / (ms_per_step * 1e-3), 4),
+               "project_ms": round(project_ms, 4), "combine_ms": round(combine_ms, 4)}
+    clocks = clk.summary()
+
+    # ------------------------------------------------ e2e through host buffers
+    X_pin = torch.from_numpy(Xh.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Y_pin = torch.empty((M, d_out), dtype=torch.bfloat16).pin_memory()
+    s0 = sets[0]
+    for _ in range(2):
+        s0["X"].copy_(X_pin, non_blocking=True)
+        slr.forward(s0["X"], s0["vals"], s0["meta"], s0["U"], s0["V"], out=s0["Y"], workspace=s0["ws"])
+        Y_pin.copy_(s0["Y"], non_blocking=True)
+    Ke = max(3, K // 2)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for k in range(Ke):
+        s = sets[k % n_copies]
+        s["X"].copy_(X_pin, non_blocking=True)
+        slr.forward(s["X"], s["vals"], s["meta"], s["U"], s["V"], out=s["Y"], workspace=s["ws"])
+        Y_pin.copy_(s["Y"], non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / Ke
+    e2e = {"value": round(world * flops_dense / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(X_pin.numel() * 2), "d2h_bytes_per_step": int(Y_pin.numel() * 2),
+           "ms_per_step": round(e2e_ms, 4)}
+    del sets, s0
+
+    # ------------------------------------------------ decode leg (M = 1)
+    decode = run_decode_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier)
+
+    # ------------------------------------------------ pack leg
+    pack = run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier)
+    del W
+
+    # ------------------------------------------------ CPU baseline (oracle), rank 0 at N = 1
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_prefill(L, rows=args.cpu_rows)
+
+    line = {
+        "metric": "S+LR linear fwd TFLOP/s (M=2048) & GB/s (M=1), % of roofline",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, Llama-3-8B gate/up shape)",
+        "config": {"workload": "Llama-3-8B gate/up prefill: d_out=14336, d_in=4096, r=64, M=2048 tokens/GPU, "
+                               "2:4 S + rank-64 U,V, bf16 in, fp32 accumulate",
+                   "tokens_per_gpu": M, "d_out": d_out, "d_in": d_in, "rank": r, "path": path,
+                   "l2": f"rotating {n_copies} buffer sets of {set_bytes / 1e6:.1f} MB (> L2 126 MB)",
+                   "parallelism": f"dp{world} (independent token batches, no collective)"},
+        "prefill": prefill,
+        "decode_m1": decode,
+        "pack": pack,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+        "peaks": {"source": peak_src, **peaks},
+        "kernel_source_sha": sha,
+    }
+    return line
+
+
+def run_decode_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier):
+    L = layer_of(DECODE["cfg"], DECODE["name"])
+    M, d_out, d_in, r = DECODE["M"], L.d_out, L.d_in, L.r
+    W = to_dev(L.weight())
+    vals0, meta0 = slr.pack_2to4(W)
+    del W
+    Uh, Vh = L.factors()
+    Xh = L.activations(M)
+    path = slr.select_path(M, d_out, d_in, r)
+    ws_bytes = slr.workspace_size(M, d_out, d_in, r)
+    nbytes = algorithmic_bytes(M, d_out, d_in, r)
+    n_copies = max(2, math.ceil(3.0 * L2_BYTES / nbytes))
+    sets = [dict(X=to_dev(Xh), vals=vals0.clone(), meta=meta0.clone(), U=to_dev(Uh), V=to_dev(Vh),
+                 Y=torch.empty((M, d_out), dtype=torch.bfloat16, device=dev),
+                 ws=torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)) for _ in range(n_copies)]
+    K = max(50, 10 * args.steps)
+
+    def step(s, ev_mid=None):
+        slr.forward_project(s["X"], s["V"], d_out, s["ws"], path=path)
+        if ev_mid is not None:
+            ev_mid.record()
+        slr.forward_combine(s["X"], s["vals"], s["meta"], s["U"], s["Y"], s["ws"], path=path)
+
+    for i in range(max(args.warmup, 10)):
+        step(sets[i % n_copies])
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    evm = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    barrier()
+    for k in range(K):
+        ev0[k].record()
+        step(sets[k % n_copies], evm[k])
+        ev1[k].record()
+    torch.cuda.synchronize()
+    barrier()
+    total_ms = max_over_ranks(ev0[0].elapsed_time(ev1[K - 1]))
+    combine_ms = statistics.mean(evm[k].elapsed_time(ev1[k]) for k in range(K))
+    ms = total_ms / K
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    # the streaming kernel alone moves vals + meta + X + U + Y (V is read by the projection)
+    k_bytes = nbytes - 2 * r * d_in
+    k_gbs = k_bytes / (combine_ms * 1e-3) / 1e9
+    del sets
+    return {"workload": "Llama-3-8B q_proj decode: 4096x4096, r=64, M=1", "path": path,
+            "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 5), "steps": K,
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "algorithmic_bytes": nbytes,
+            "kernel": {"name": "decode_forward_kernel", "ms": round(combine_ms, 5), "bytes": k_bytes,
+                       "gbs": round(k_gbs, 1), "frac": round(k_gbs / peaks["hbm_gbs"], 4)},
+            "l2": f"rotating {n_copies} buffer sets of {nbytes / 1e6:.1f} MB"}
+
+
+def run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier):
+    d_out, d_in = W.shape
+    nbytes = d_out * d_in * 2 + d_out * d_in + d_out * d_in // 8   # read W, write vals + meta
+    n_copies = max(2, math.ceil(2.0 * L2_BYTES / nbytes))
+    Ws = [W if i == 0 else W.clone() for i in range(n_copies)]
+    outs = [(torch.empty((d_out, d_in // 2), dtype=torch.bfloat16, device=dev),
+             torch.empty((d_out, d_in // 8), dtype=torch.uint8, device=dev)) for _ in range(n_copies)]
+    lib = slr.lib()
+
+    def pack(i):
+        v, m = outs[i % n_copies]
+        w = Ws[i % n_copies]
+        st = lib.slr_pack_2to4(slr._ptr(w), d_out, d_in, d_in, slr._ptr(v), slr._ptr(m), slr._stream())
+        assert st == 0, st
+
+    for i in range(3):
+        pack(i)
+    K = max(10, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record()
+    for k in range(K):
+        pack(k)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1)) / K
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": f"2:4 pack of the {d_out}x{d_in} gate/up weight", "value": round(gbs, 1),
+            "unit": "GB/s", "ms_per_launch": round(ms, 5), "bytes_per_launch": nbytes,
+            "frac": round(gbs / peaks["hbm_gbs"], 4)}
+
+
+def cpu_baseline_prefill(L, rows: int):
+    import oracle
+    W = L.weight()
+    U, V = L.factors()
+    X = L.activations(PREFILL["M"])
+    vals, meta = oracle.pack_2to4(W)
+    sel = np.sort(np.random.Generator(np.random.PCG64(77)).choice(PREFILL["M"], size=rows, replace=False))
+    threads = oracle.max_threads()
+    t0 = time.perf_counter()
+    oracle.forward(X, vals, meta, U, V, rows=sel, with_bound=False, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return {"value": round(2.0 * rows * L.d_out * L.d_in / dt / 1e12, 6), "unit": "TFLOP/s",
+            "cores": threads, "kind": "oracle",
+            "sample": f"{rows} of {PREFILL['M']} token rows of the gate/up workload (all {L.d_out} outputs), "
+                      f"fp64 oracle incl. forming W' = S + U V once, {dt:.2f} s wall"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The oracle as the reference arm: a bounded row sample per step."""
+    import oracle
+    L = layer_of(PREFILL["cfg"], PREFILL["name"])
+    W = L.weight()
+    U, V = L.factors()
+    X = L.activations(PREFILL["M"])
+    vals, meta = oracle.pack_2to4(W)
+    rows = args.ref_rows
+    threads = oracle.max_threads()
+    rng = np.random.Generator(np.random.PCG64(5))
+    for _ in range(args.warmup):
+        oracle.forward(X, vals, meta, U, V, rows=rng.choice(PREFILL["M"], rows, replace=False),
+                       with_bound=False, nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward(X, vals, meta, U, V, rows=rng.choice(PREFILL["M"], rows, replace=False),
+                       with_bound=False, nthreads=threads)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = 2.0 * rows * L.d_out * L.d_in / dt / 1e12
+    sample = (f"{rows} random token rows of the M=2048 gate/up workload per step, all {L.d_out} outputs, "
+              f"fp64 oracle (forms W' = S + U V each step)")
+    return {"impl": "reference", "metric": "S+LR linear fwd TFLOP/s (M=2048) & GB/s (M=1), % of roofline",
+            "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "Llama-3-8B gate/up prefill: d_out=14336, d_in=4096, r=64, M=2048 tokens"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=64, help="token rows in the oracle CPU baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=8, help="token rows per step of the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        line = run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,178 @@
+/*
+ * slr.h -- C ABI of the 2:4-sparse + low-rank linear layer library (libslr.so).
+ *
+ * The layer (LoSparse, arXiv 2306.11222, sections 3 and 3.2; HASSLE-free,
+ * arXiv 2502.00899, section 1 and the abstract's 2:4 + rank-64 scheme) stores a
+ * weight W (d_out x d_in) as a 2:4 semi-structured sparse matrix S plus a
+ * rank-r product U*V, and evaluates the two terms side by side:
+ *
+ *        Y = X * S^T + (X * V^T) * U^T            (bf16 in, fp32 accumulate, bf16 out)
+ *
+ * All matrices are row-major with dense rows unless a leading dimension is
+ * passed.  Every pointer argument of a compute call is a DEVICE pointer on the
+ * current CUDA device; the caller owns all memory (the library allocates
+ * nothing and frees nothing).  All work is queued on `stream` and runs
+ * asynchronously; no call synchronises.
+ *
+ * Error behaviour: argument checks (null pointers, shapes, alignment,
+ * workspace size, device capability) run on the host before anything is
+ * queued, in that order, and return the first failing status with nothing
+ * launched.  A launch failure returns SLR_ERR_CUDA.  Faults inside a kernel
+ * surface, as usual for CUDA, at the caller's next synchronisation.
+ *
+ * Threading: calls are safe from several host threads; calls on one stream
+ * execute in order.  Outputs must not alias inputs.
+ */
+#ifndef SLR_H
+#define SLR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SLR_API __attribute__((visibility("default")))
+#else
+#define SLR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st *slr_stream_t;
+
+typedef enum slr_status {
+    SLR_OK = 0,
+    SLR_ERR_NULL = 1,      /* a required pointer is NULL                         */
+    SLR_ERR_SHAPE = 2,     /* a size is negative or violates a divisibility rule */
+    SLR_ERR_ALIGN = 3,     /* a pointer is not 16-byte aligned                   */
+    SLR_ERR_WORKSPACE = 4, /* workspace smaller than slr_forward_workspace_size  */
+    SLR_ERR_DEVICE = 5,    /* no CUDA device, or the current device is not sm_100 */
+    SLR_ERR_CUDA = 6,      /* a CUDA runtime/driver call or kernel launch failed */
+    SLR_ERR_TIMEOUT = 7,   /* a kernel gave up a bounded wait (see the forward)  */
+    SLR_ERR_ARG = 8        /* an enum argument is out of range                   */
+} slr_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+SLR_API const char *slr_status_string(slr_status s);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+SLR_API int slr_version(void);
+
+/* --------------------------------------------------------------------------
+ * 2:4 projection and packing.
+ *
+ * Hard-thresholding onto 2:4 (HASSLE-free, section 4.1.1: with an identity
+ * Hessian the optimal sparse update keeps the largest-magnitude entries; the
+ * 2:4 pattern, "two nonzeros in every four weights", as on the 3BASiL page).
+ * For every row i and every aligned group g of four columns 4g..4g+3, the two
+ * positions with the largest magnitude are kept (magnitude = the bf16 bits
+ * with the sign cleared, compared as integers; equal magnitudes keep the
+ * lower index; NaN ranks above Inf).  Exactly two positions are kept per
+ * group, even when they hold zeros.
+ *
+ *   W     device, bf16 [d_out, ldw] (ldw >= d_in), read only.
+ *   vals  device, bf16 [d_out, d_in/2], dense rows: the two kept values of
+ *         group g at columns 2g, 2g+1, in ascending index order (bit copies).
+ *   meta  device, uint8 [d_out, slr_meta_row_bytes(d_in)], dense rows: byte j
+ *         of a row holds group 2j in its low nibble and group 2j+1 in its high
+ *         nibble; nibble = idx0 | idx1 << 2 with 0 <= idx0 < idx1 <= 3.  When
+ *         d_in/4 is odd the last high nibble is 0.
+ *
+ * Requirements: d_out >= 0, d_in >= 0, d_in % 4 == 0, ldw >= d_in; W, vals and
+ * meta non-NULL unless d_out * d_in == 0.  Any alignment is accepted; 16-byte
+ * aligned W with d_in and ldw multiples of 8 takes the vectorised path.
+ * The result is bit-exact and deterministic.
+ * ------------------------------------------------------------------------ */
+SLR_API slr_status slr_pack_2to4(const void *W, int64_t d_out, int64_t d_in, int64_t ldw,
+                         void *vals, void *meta, slr_stream_t stream);
+
+/* Bytes per metadata row: ceil(d_in / 8). */
+SLR_API int64_t slr_meta_row_bytes(int64_t d_in);
+
+/* --------------------------------------------------------------------------
+ * Forward pass  Y = X * S^T + (X * V^T) * U^T.
+ *
+ * LoSparse, section 3.2: the compressed layer computes the low-rank and sparse
+ * terms in parallel instead of X * W.  Here W' = S + U*V with U d_out x r and
+ * V r x d_in; (X V^T) is the rank-r projection T (M x r).
+ *
+ *   X     device, bf16 [M, d_in]          activations, one token per row.
+ *   vals  device, bf16 [d_out, d_in/2]    from slr_pack_2to4.
+ *   meta  device, uint8 [d_out, d_in/8]   from slr_pack_2to4.
+ *   U     device, bf16 [d_out, r]         (ignored, may be NULL, when r == 0).
+ *   V     device, bf16 [r, d_in]          (ignored, may be NULL, when r == 0).
+ *   Y     device, bf16 [M, d_out]         output, written once, RNE rounded.
+ *   workspace / workspace_bytes: device scratch of at least
+ *         slr_forward_workspace_size(M, d_out, d_in, r) bytes, 256-byte
+ *         aligned; its contents on entry do not matter and are clobbered.
+ *
+ * Arithmetic: products of bf16 inputs are accumulated in fp32.  T is kept in
+ * fp32 on the small-M path and rounded to bf16 before the second product on
+ * the tensor-core path.  Accuracy contract (tested): relative Frobenius error
+ * <= 5e-3 and |err_ij| <= 1e-2 * (|X| |W'|^T)_ij + 1e-3 against the exact
+ * result on the same bf16 inputs.
+ *
+ * Requirements: M >= 0 (M == 0 returns SLR_OK before any pointer is looked
+ * at), d_out >= 1, d_in >= 128 with d_in % 128 == 0, r >= 0 with r % 8 == 0,
+ * M, d_out, d_in < 2^31, all pointers 16-byte aligned.  The tensor-core path
+ * additionally needs d_out % 8 == 0 (SLR_PATH_AUTO avoids it otherwise).
+ * ------------------------------------------------------------------------ */
+SLR_API slr_status slr_forward(const void *X, int64_t M, const void *vals, const void *meta,
+                       int64_t d_out, int64_t d_in, const void *U, const void *V, int64_t r,
+                       void *Y, void *workspace, size_t workspace_bytes, slr_stream_t stream);
+
+/* Scratch bytes slr_forward needs for this problem (0 when none). */
+SLR_API size_t slr_forward_workspace_size(int64_t M, int64_t d_out, int64_t d_in, int64_t r);
+
+/* Execution paths of the forward pass. */
+typedef enum slr_path {
+    SLR_PATH_AUTO = 0,   /* choose by M (slr_forward_select_path)                  */
+    SLR_PATH_DECODE = 1, /* small-M path: CUDA-core streaming kernel over S rows    */
+    SLR_PATH_TENSOR = 2  /* 2:4 tcgen05 tensor-core GEMM with the rank-r term fused */
+} slr_path;
+
+/* The path SLR_PATH_AUTO takes for this problem. */
+SLR_API slr_path slr_forward_select_path(int64_t M, int64_t d_out, int64_t d_in, int64_t r);
+
+/* slr_forward with an explicit path (for tests and measurement); same
+ * arguments, requirements and result contract as slr_forward. */
+SLR_API slr_status slr_forward_with_path(const void *X, int64_t M, const void *vals, const void *meta,
+                                 int64_t d_out, int64_t d_in, const void *U, const void *V,
+                                 int64_t r, void *Y, void *workspace, size_t workspace_bytes,
+                                 slr_path path, slr_stream_t stream);
+
+/* The two stages of slr_forward, for callers that schedule or time them
+ * separately.  slr_forward(...) == slr_forward_project(...) followed on the same
+ * stream by slr_forward_combine(...) with the same path and workspace.
+ *
+ * slr_forward_project: T = X * V^T (the rank-r projection, LoSparse section
+ * 3.2) into `workspace`, in the layout the resolved path reads (fp32 [M, r]
+ * for SLR_PATH_DECODE, bf16 [M, r] for SLR_PATH_TENSOR).  d_out only selects
+ * the path.  vals/meta/U/Y are not read.
+ *
+ * slr_forward_combine: Y = X * S^T + T * U^T with T taken from `workspace`
+ * as written by slr_forward_project for the same (M, d_out, r, path).  V is
+ * not read.  Requirements and errors are those of slr_forward restricted to
+ * the arguments each stage takes. */
+SLR_API slr_status slr_forward_project(const void *X, int64_t M, const void *V, int64_t d_out, int64_t d_in,
+                                       int64_t r, void *workspace, size_t workspace_bytes, slr_path path,
+                                       slr_stream_t stream);
+SLR_API slr_status slr_forward_combine(const void *X, int64_t M, const void *vals, const void *meta,
+                                       int64_t d_out, int64_t d_in, const void *U, int64_t r, void *Y,
+                                       const void *workspace, size_t workspace_bytes, slr_path path,
+                                       slr_stream_t stream);
+
+/* Synchronises the current device, then reports (and clears) the error word
+ * that the tensor-core kernel sets when one of its bounded waits expires:
+ * SLR_ERR_TIMEOUT if any launch since the last check gave up, SLR_OK
+ * otherwise.  Kernels that time out leave their output incomplete but free
+ * their resources and return, so the CUDA context stays usable. */
+SLR_API slr_status slr_check_kernel_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLR_H */

@@ -75,7 +75,7 @@ class Oracle:
         lib.oracle_unpack_2to4.restype = ctypes.c_int
         lib.oracle_unpack_2to4.argtypes = [p, p, i64, i64, p]
         lib.oracle_forward.restype = ctypes.c_int
-        lib.oracle_forward.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, i64, p, p, ctypes.c_int]
+        lib.oracle_forward.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, i64, p, i64, p, p, ctypes.c_int]
         lib.oracle_lowrank_project.restype = ctypes.c_int
         lib.oracle_lowrank_project.argtypes = [p, i64, p, i64, i64, p]
         lib.oracle_max_threads.restype = ctypes.c_int
@@ -114,12 +114,14 @@ class Oracle:
             raise ValueError("oracle_unpack_2to4 rejected its arguments")
         return S
 
-    def forward(self, X, vals, meta, U, V, rows=None, with_bound: bool = True, nthreads: int = 0):
+    def forward(self, X, vals, meta, U, V, rows=None, outs=None, with_bound: bool = True,
+                nthreads: int = 0):
         """fp64 ``Y = X @ (S + U @ V).T`` and the bound ``|X| @ |S + U @ V|.T``.
 
-        ``rows`` selects token rows of X (default: all).  ``U``/``V`` may be
-        None (no low-rank term).  Returns ``(Y, B)`` as float64
-        [n_rows, d_out]; ``B`` is None when ``with_bound`` is False.
+        ``rows`` selects token rows of X and ``outs`` output features (default:
+        all of each).  ``U``/``V`` may be None (no low-rank term).  Returns
+        ``(Y, B)`` as float64 [n_rows, n_outs]; ``B`` is None when
+        ``with_bound`` is False.
         """
         X = _u16(X)
         vals = _u16(vals)
@@ -139,12 +141,18 @@ class Oracle:
         else:
             rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
             n = rows_arr.shape[0]
-        Y = np.zeros((n, d_out), dtype=np.float64)
-        B = np.zeros((n, d_out), dtype=np.float64) if with_bound else None
+        if outs is None:
+            no, outs_arr = d_out, None
+        else:
+            outs_arr = np.ascontiguousarray(outs, dtype=np.int64)
+            no = outs_arr.shape[0]
+        Y = np.zeros((n, no), dtype=np.float64)
+        B = np.zeros((n, no), dtype=np.float64) if with_bound else None
         rc = self._lib.oracle_forward(
             _ptr(X), M, _ptr(vals), _ptr(meta), d_out, d_in,
             _ptr(U) if r else None, _ptr(V) if r else None, r,
             _ptr(rows_arr) if rows_arr is not None else None, n,
+            _ptr(outs_arr) if outs_arr is not None else None, no,
             _ptr(Y), _ptr(B) if B is not None else None, int(nthreads))
         if rc != 0:
             raise ValueError(f"oracle_forward failed (rc={rc})")
@@ -188,8 +196,9 @@ def unpack_2to4(vals, meta, d_in: int):
     return default().unpack_2to4(vals, meta, d_in)
 
 
-def forward(X, vals, meta, U, V, rows=None, with_bound: bool = True, nthreads: int = 0):
-    return default().forward(X, vals, meta, U, V, rows=rows, with_bound=with_bound, nthreads=nthreads)
+def forward(X, vals, meta, U, V, rows=None, outs=None, with_bound: bool = True, nthreads: int = 0):
+    return default().forward(X, vals, meta, U, V, rows=rows, outs=outs, with_bound=with_bound,
+                             nthreads=nthreads)
 
 
 def lowrank_project(X, V):

@@ -166,18 +166,25 @@ static void dense_row(const uint16_t *vals, const uint8_t *meta, const uint16_t 
 /* Forward pass in fp64:  Y[m, i] = sum_j X[m, j] * W'[i, j],
  *                        B[m, i] = sum_j |X[m, j]| * |W'[i, j]|.
  * rows      : the n_rows indices of X (tokens) to evaluate, or NULL for all M.
- * Y, Bound  : n_rows x d_out doubles (row t is token rows[t]); Bound may be NULL.
+ * outs      : the n_outs output indices i to evaluate, or NULL for all d_out.
+ * Y, Bound  : n_rows x n_outs doubles (entry [t, o] is token rows[t], output
+ *             outs[o]); Bound may be NULL.
  * r may be 0 (no low-rank term; U and V are then ignored). */
 int oracle_forward(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                    int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *V,
-                   int64_t r, const int64_t *rows, int64_t n_rows, double *Y,
-                   double *Bound, int nthreads)
+                   int64_t r, const int64_t *rows, int64_t n_rows, const int64_t *outs,
+                   int64_t n_outs, double *Y, double *Bound, int nthreads)
 {
     if (d_in % 4 != 0 || d_out < 0 || M < 0 || r < 0) return -1;
     if (rows == NULL) n_rows = M;
+    if (outs == NULL) n_outs = d_out;
     for (int64_t t = 0; t < n_rows; ++t) {
         int64_t m = rows ? rows[t] : t;
         if (m < 0 || m >= M) return -1;
+    }
+    for (int64_t o = 0; o < n_outs; ++o) {
+        int64_t i = outs ? outs[o] : o;
+        if (i < 0 || i >= d_out) return -1;
     }
     set_threads(nthreads);
     int failed = 0;
@@ -190,7 +197,8 @@ int oracle_forward(const uint16_t *X, int64_t M, const uint16_t *vals, const uin
             failed = 1;
         } else {
 #pragma omp for schedule(dynamic, 4)
-            for (int64_t i = 0; i < d_out; ++i) {
+            for (int64_t o = 0; o < n_outs; ++o) {
+                int64_t i = outs ? outs[o] : o;
                 dense_row(vals, meta, U, V, d_in, r, i, row);
                 for (int64_t t = 0; t < n_rows; ++t) {
                     int64_t m = rows ? rows[t] : t;
@@ -200,8 +208,8 @@ int oracle_forward(const uint16_t *X, int64_t M, const uint16_t *vals, const uin
                         acc += xr[j] * row[j];
                         bound += fabs(xr[j]) * fabs(row[j]);
                     }
-                    Y[t * d_out + i] = acc;
-                    if (Bound) Bound[t * d_out + i] = bound;
+                    Y[t * n_outs + o] = acc;
+                    if (Bound) Bound[t * n_outs + o] = bound;
                 }
             }
         }

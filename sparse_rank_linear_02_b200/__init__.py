@@ -1,0 +1,162 @@
+"""Python binding of libslr: the 2:4-sparse + low-rank linear layer on B200.
+
+Argument marshalling only.  Every step of the computation runs in the CUDA
+kernels of ``libslr.so`` (built in-tree by ``python -m
+sparse_rank_linear_02_b200.build``); there is no fallback of any kind, and the
+import fails if the library is missing.
+
+Functions mirror the C ABI in ``include/slr.h``:
+
+* ``pack_2to4(W) -> (vals, meta)``  -- ``slr_pack_2to4``
+* ``forward(X, vals, meta, U, V) -> Y``  -- ``slr_forward`` /
+  ``slr_forward_with_path``
+* ``workspace_size``, ``select_path``, ``check_kernel_error``
+
+Tensors are torch CUDA tensors (torch only provides memory and the current
+stream): bf16 for W, X, U, V, vals and Y, uint8 for meta.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libslr.so")
+
+SLR_OK = 0
+STATUS_NAMES = {0: "SLR_OK", 1: "SLR_ERR_NULL", 2: "SLR_ERR_SHAPE", 3: "SLR_ERR_ALIGN",
+                4: "SLR_ERR_WORKSPACE", 5: "SLR_ERR_DEVICE", 6: "SLR_ERR_CUDA",
+                7: "SLR_ERR_TIMEOUT", 8: "SLR_ERR_ARG"}
+PATHS = {"auto": 0, "decode": 1, "tensor": 2}
+PATH_NAMES = {v: k for k, v in PATHS.items()}
+
+
+class SlrError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} "
+                         f"({_lib.slr_status_string(status).decode()})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with "
+                          f"`python -m sparse_rank_linear_02_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    i64, p, sz, st = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    lib.slr_status_string.restype = ctypes.c_char_p
+    lib.slr_status_string.argtypes = [st]
+    lib.slr_version.restype = ctypes.c_int
+    lib.slr_pack_2to4.restype = st
+    lib.slr_pack_2to4.argtypes = [p, i64, i64, i64, p, p, p]
+    lib.slr_meta_row_bytes.restype = i64
+    lib.slr_meta_row_bytes.argtypes = [i64]
+    lib.slr_forward.restype = st
+    lib.slr_forward.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, p, sz, p]
+    lib.slr_forward_with_path.restype = st
+    lib.slr_forward_with_path.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, p, sz, st, p]
+    lib.slr_forward_workspace_size.restype = sz
+    lib.slr_forward_workspace_size.argtypes = [i64, i64, i64, i64]
+    lib.slr_forward_select_path.restype = st
+    lib.slr_forward_select_path.argtypes = [i64, i64, i64, i64]
+    lib.slr_check_kernel_error.restype = st
+    lib.slr_check_kernel_error.argtypes = []
+    lib.slr_forward_project.restype = st
+    lib.slr_forward_project.argtypes = [p, i64, p, i64, i64, i64, p, sz, st, p]
+    lib.slr_forward_combine.restype = st
+    lib.slr_forward_combine.argtypes = [p, i64, p, p, i64, i64, p, i64, p, p, sz, st, p]
+    return lib
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ``libslr.so`` (for direct C-ABI calls)."""
+    return _lib
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(status: int, what: str):
+    if status != SLR_OK:
+        raise SlrError(status, what)
+
+
+def meta_row_bytes(d_in: int) -> int:
+    return int(_lib.slr_meta_row_bytes(d_in))
+
+
+def pack_2to4(W: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+    """2:4 projection by magnitude and packing of bf16 ``W`` [d_out, d_in]."""
+    if W.dtype != torch.bfloat16 or W.dim() != 2 or not W.is_cuda or W.stride(1) != 1:
+        raise ValueError("W must be a 2-D CUDA bf16 tensor with unit column stride")
+    d_out, d_in = W.shape
+    vals = torch.empty((d_out, d_in // 2), dtype=torch.bfloat16, device=W.device)
+    meta = torch.empty((d_out, meta_row_bytes(d_in)), dtype=torch.uint8, device=W.device)
+    _check(_lib.slr_pack_2to4(_ptr(W), d_out, d_in, W.stride(0), _ptr(vals), _ptr(meta), _stream()),
+           "slr_pack_2to4")
+    return vals, meta
+
+
+def workspace_size(M: int, d_out: int, d_in: int, r: int) -> int:
+    return int(_lib.slr_forward_workspace_size(M, d_out, d_in, r))
+
+
+def select_path(M: int, d_out: int, d_in: int, r: int) -> str:
+    return PATH_NAMES[int(_lib.slr_forward_select_path(M, d_out, d_in, r))]
+
+
+def forward(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, U: torch.Tensor | None,
+            V: torch.Tensor | None, *, path: str = "auto", out: torch.Tensor | None = None,
+            workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """``Y = X @ S.T + (X @ V.T) @ U.T`` with S given packed by ``pack_2to4``."""
+    M, d_in = X.shape
+    d_out = vals.shape[0]
+    r = 0 if U is None else U.shape[1]
+    if out is None:
+        out = torch.empty((M, d_out), dtype=torch.bfloat16, device=X.device)
+    need = workspace_size(M, d_out, d_in, r)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.slr_forward_with_path(_ptr(X), M, _ptr(vals), _ptr(meta), d_out, d_in, _ptr(U), _ptr(V), r,
+                                      _ptr(out), _ptr(workspace), ws_bytes, PATHS[path], _stream()),
+           "slr_forward")
+    return out
+
+
+def forward_project(X: torch.Tensor, V: torch.Tensor | None, d_out: int, workspace: torch.Tensor, *,
+                    path: str = "auto") -> None:
+    """Stage 1 of ``forward``: T = X V^T into ``workspace`` (``slr_forward_project``)."""
+    M, d_in = X.shape
+    r = 0 if V is None else V.shape[0]
+    _check(_lib.slr_forward_project(_ptr(X), M, _ptr(V), d_out, d_in, r, _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), PATHS[path], _stream()),
+           "slr_forward_project")
+
+
+def forward_combine(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, U: torch.Tensor | None,
+                    out: torch.Tensor, workspace: torch.Tensor | None, *, path: str = "auto") -> torch.Tensor:
+    """Stage 2 of ``forward``: Y = X S^T + T U^T with T from ``workspace``."""
+    M, d_in = X.shape
+    d_out = vals.shape[0]
+    r = 0 if U is None else U.shape[1]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.slr_forward_combine(_ptr(X), M, _ptr(vals), _ptr(meta), d_out, d_in, _ptr(U), r, _ptr(out),
+                                    _ptr(workspace), ws_bytes, PATHS[path], _stream()),
+           "slr_forward_combine")
+    return out
+
+
+def check_kernel_error() -> None:
+    """Synchronise and raise if a tensor-core kernel reported a bounded-wait timeout."""
+    _check(_lib.slr_check_kernel_error(), "slr_check_kernel_error")

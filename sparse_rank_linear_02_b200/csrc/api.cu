@@ -1,0 +1,223 @@
+// api.cu -- the exported C ABI (include/slr.h): argument checks, workspace
+// layout and path dispatch.  No arithmetic of the layer happens here.
+#include <mutex>
+
+#include "common.cuh"
+#include "tc_forward.cuh"
+
+namespace slr {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// sm_100 check, cached per device ordinal.
+slr_status check_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+        cudaGetLastError();
+        return SLR_ERR_DEVICE;
+    }
+    static std::mutex mu;
+    static int verdict[64] = {0};  // 0 unknown, 1 ok, 2 bad
+    if (dev >= 64) return SLR_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(mu);
+    if (verdict[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return SLR_ERR_DEVICE;
+        }
+        verdict[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    }
+    return verdict[dev] == 1 ? SLR_OK : SLR_ERR_DEVICE;
+}
+
+// Token count up to which the CUDA-core streaming path is used.
+constexpr int64_t kDecodeMaxM = 16;
+
+size_t workspace_bytes_for(int64_t M, int64_t r, slr_path path) {
+    if (M <= 0 || r <= 0) return 0;
+    if (path == SLR_PATH_DECODE) return round_up((size_t)M * r * sizeof(float), kAlign);
+    return round_up((size_t)M * r * sizeof(uint16_t), kAlign);
+}
+
+// The tensor-core path stores Y with TMA, whose row pitch must be a multiple
+// of 16 bytes (d_out % 8 == 0); other shapes stay on the streaming path.
+bool tensor_ok(int64_t d_out) { return d_out % 8 == 0; }
+
+slr_path resolve(slr_path path, int64_t M, int64_t d_out) {
+    if (path != SLR_PATH_AUTO) return path;
+    return (M <= kDecodeMaxM || !tensor_ok(d_out)) ? SLR_PATH_DECODE : SLR_PATH_TENSOR;
+}
+
+// Host-side validation shared by the forward entry points.  `need_factors`
+// selects which low-rank operands the stage reads.
+slr_status validate(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out, int64_t d_in,
+                    const void *U, const void *V, int64_t r, const void *Y, const void *workspace,
+                    size_t workspace_bytes, slr_path path, bool need_sparse, bool need_U, bool need_V,
+                    slr_path *resolved) {
+    if (path != SLR_PATH_AUTO && path != SLR_PATH_DECODE && path != SLR_PATH_TENSOR) return SLR_ERR_ARG;
+    if (M < 0 || d_out < 0 || d_in < 0 || r < 0) return SLR_ERR_SHAPE;
+    const slr_path p = resolve(path, M, d_out);
+    *resolved = p;
+    if (M == 0) return SLR_OK;
+    const size_t need = workspace_bytes_for(M, r, p);
+    if (X == nullptr) return SLR_ERR_NULL;
+    if (need_sparse && (vals == nullptr || meta == nullptr || Y == nullptr)) return SLR_ERR_NULL;
+    if (r > 0 && ((need_U && U == nullptr) || (need_V && V == nullptr))) return SLR_ERR_NULL;
+    if (need > 0 && workspace == nullptr) return SLR_ERR_NULL;
+    if (d_out < 1 || d_in < 128 || d_in % 128 != 0 || r % 8 != 0) return SLR_ERR_SHAPE;
+    if (p == SLR_PATH_TENSOR && !tensor_ok(d_out)) return SLR_ERR_SHAPE;
+    if (M > INT32_MAX || d_out > INT32_MAX || d_in > INT32_MAX) return SLR_ERR_SHAPE;
+    if (!aligned16(X)) return SLR_ERR_ALIGN;
+    if (need_sparse && (!aligned16(vals) || !aligned16(meta) || !aligned16(Y))) return SLR_ERR_ALIGN;
+    if (r > 0 && ((need_U && !aligned16(U)) || (need_V && !aligned16(V)))) return SLR_ERR_ALIGN;
+    if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0) return SLR_ERR_ALIGN;
+    if (workspace_bytes < need) return SLR_ERR_WORKSPACE;
+    return check_device();
+}
+
+// Stage 1: T = X V^T into the workspace, fp32 for the streaming path and bf16
+// for the tensor-core path.
+cudaError_t run_project(const void *X, int64_t M, const void *V, int64_t d_in, int64_t r, void *workspace,
+                        slr_path p, cudaStream_t stream) {
+    if (r == 0) return cudaSuccess;
+    const uint16_t *x = static_cast<const uint16_t *>(X);
+    const uint16_t *vv = static_cast<const uint16_t *>(V);
+    if (p == SLR_PATH_DECODE) return launch_lowrank_project(x, M, vv, d_in, r, static_cast<float *>(workspace), nullptr, stream);
+    return launch_lowrank_project(x, M, vv, d_in, r, nullptr, static_cast<uint16_t *>(workspace), stream);
+}
+
+// Stage 2: Y = X S^T + T U^T with T read from the workspace.
+cudaError_t run_combine(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out, int64_t d_in,
+                        const void *U, int64_t r, void *Y, const void *workspace, slr_path p,
+                        cudaStream_t stream) {
+    const uint16_t *x = static_cast<const uint16_t *>(X);
+    const uint16_t *v = static_cast<const uint16_t *>(vals);
+    const uint8_t *m = static_cast<const uint8_t *>(meta);
+    const uint16_t *u = static_cast<const uint16_t *>(U);
+    uint16_t *y = static_cast<uint16_t *>(Y);
+    if (p == SLR_PATH_DECODE)
+        return launch_decode_forward(x, M, v, m, d_out, d_in, u, r > 0 ? static_cast<const float *>(workspace) : nullptr,
+                                     r, y, stream);
+    return launch_tc_forward(x, M, v, m, d_out, d_in, u, r > 0 ? static_cast<const uint16_t *>(workspace) : nullptr,
+                             r, y, stream);
+}
+
+slr_status forward_impl(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out,
+                        int64_t d_in, const void *U, const void *V, int64_t r, void *Y, void *workspace,
+                        size_t workspace_bytes, slr_path path, cudaStream_t stream) {
+    slr_path p;
+    const slr_status st = validate(X, M, vals, meta, d_out, d_in, U, V, r, Y, workspace, workspace_bytes, path,
+                                   true, true, true, &p);
+    if (st != SLR_OK || M == 0) return st;
+    cudaError_t err = run_project(X, M, V, d_in, r, workspace, p, stream);
+    if (err == cudaSuccess) err = run_combine(X, M, vals, meta, d_out, d_in, U, r, Y, workspace, p, stream);
+    return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace slr
+
+extern "C" {
+
+const char *slr_status_string(slr_status s) {
+    switch (s) {
+        case SLR_OK: return "SLR_OK";
+        case SLR_ERR_NULL: return "SLR_ERR_NULL: a required pointer is NULL";
+        case SLR_ERR_SHAPE: return "SLR_ERR_SHAPE: a size is negative or violates a divisibility rule";
+        case SLR_ERR_ALIGN: return "SLR_ERR_ALIGN: a pointer is not 16-byte aligned";
+        case SLR_ERR_WORKSPACE: return "SLR_ERR_WORKSPACE: workspace too small";
+        case SLR_ERR_DEVICE: return "SLR_ERR_DEVICE: no sm_100 CUDA device is current";
+        case SLR_ERR_CUDA: return "SLR_ERR_CUDA: a CUDA call or kernel launch failed";
+        case SLR_ERR_TIMEOUT: return "SLR_ERR_TIMEOUT: a kernel gave up a bounded wait";
+        case SLR_ERR_ARG: return "SLR_ERR_ARG: an enum argument is out of range";
+    }
+    return "SLR_ERR_UNKNOWN";
+}
+
+int slr_version(void) { return 100; }
+
+int64_t slr_meta_row_bytes(int64_t d_in) { return d_in < 0 ? 0 : (d_in / 4 + 1) / 2; }
+
+slr_status slr_pack_2to4(const void *W, int64_t d_out, int64_t d_in, int64_t ldw, void *vals, void *meta,
+                         slr_stream_t stream) {
+    if (d_out < 0 || d_in < 0 || d_in % 4 != 0 || ldw < d_in) return SLR_ERR_SHAPE;
+    if (d_out == 0 || d_in == 0) return SLR_OK;
+    if (W == nullptr || vals == nullptr || meta == nullptr) return SLR_ERR_NULL;
+    const slr_status dev = slr::check_device();
+    if (dev != SLR_OK) return dev;
+    const cudaError_t err = slr::launch_pack_2to4(static_cast<const uint16_t *>(W), d_out, d_in, ldw,
+                                                  static_cast<uint16_t *>(vals), static_cast<uint8_t *>(meta),
+                                                  reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
+}
+
+size_t slr_forward_workspace_size(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
+    (void)d_out;
+    (void)d_in;
+    const size_t a = slr::workspace_bytes_for(M, r, SLR_PATH_DECODE);
+    const size_t b = slr::workspace_bytes_for(M, r, SLR_PATH_TENSOR);
+    return a > b ? a : b;
+}
+
+slr_path slr_forward_select_path(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
+    (void)d_out;
+    (void)d_in;
+    (void)r;
+    return slr::resolve(SLR_PATH_AUTO, M, d_out);
+}
+
+slr_status slr_check_kernel_error(void) {
+    if (slr::check_device() != SLR_OK) return SLR_ERR_DEVICE;
+    if (cudaDeviceSynchronize() != cudaSuccess) return SLR_ERR_CUDA;
+    unsigned code = 0;
+    if (slr::read_and_clear_kernel_error(&code) != cudaSuccess) return SLR_ERR_CUDA;
+    return code ? SLR_ERR_TIMEOUT : SLR_OK;
+}
+
+slr_status slr_forward(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out, int64_t d_in,
+                       const void *U, const void *V, int64_t r, void *Y, void *workspace, size_t workspace_bytes,
+                       slr_stream_t stream) {
+    return slr::forward_impl(X, M, vals, meta, d_out, d_in, U, V, r, Y, workspace, workspace_bytes, SLR_PATH_AUTO,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+slr_status slr_forward_project(const void *X, int64_t M, const void *V, int64_t d_out, int64_t d_in, int64_t r,
+                               void *workspace, size_t workspace_bytes, slr_path path, slr_stream_t stream) {
+    slr_path p;
+    const void *dummy = X;
+    const slr_status st = slr::validate(X, M, dummy, dummy, d_out, d_in, nullptr, V, r, dummy, workspace,
+                                        workspace_bytes, path, false, false, true, &p);
+    if (st != SLR_OK || M == 0) return st;
+    return slr::run_project(X, M, V, d_in, r, workspace, p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SLR_OK
+               : SLR_ERR_CUDA;
+}
+
+slr_status slr_forward_combine(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out,
+                               int64_t d_in, const void *U, int64_t r, void *Y, const void *workspace,
+                               size_t workspace_bytes, slr_path path, slr_stream_t stream) {
+    slr_path p;
+    const slr_status st = slr::validate(X, M, vals, meta, d_out, d_in, U, nullptr, r, Y, workspace, workspace_bytes,
+                                        path, true, true, false, &p);
+    if (st != SLR_OK || M == 0) return st;
+    return slr::run_combine(X, M, vals, meta, d_out, d_in, U, r, Y, workspace, p,
+                            reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SLR_OK
+               : SLR_ERR_CUDA;
+}
+
+slr_status slr_forward_with_path(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out,
+                                 int64_t d_in, const void *U, const void *V, int64_t r, void *Y, void *workspace,
+                                 size_t workspace_bytes, slr_path path, slr_stream_t stream) {
+    return slr::forward_impl(X, M, vals, meta, d_out, d_in, U, V, r, Y, workspace, workspace_bytes, path,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

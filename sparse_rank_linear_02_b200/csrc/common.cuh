@@ -1,0 +1,50 @@
+// common.cuh -- internal helpers shared by the kernels of libslr (not exported).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "slr.h"
+
+namespace slr {
+
+// bf16 bit pattern (low 16 bits of x) -> fp32, exact.
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t x) { return __uint_as_float(x << 16); }
+// bf16 bit pattern (high 16 bits of x) -> fp32, exact.
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+
+// fp32 -> bf16 bits, round to nearest even (the CUDA intrinsic).
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+    __nv_bfloat16_raw r = __nv_bfloat16_raw(__float2bfloat16_rn(f));
+    return r.x;
+}
+
+// Streaming 16-byte load that does not allocate in L1 (weights are read once).
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// ---------------------------------------------------------------- launchers
+// Each returns cudaSuccess or the launch error; arguments were validated by
+// the API layer.
+
+cudaError_t launch_pack_2to4(const uint16_t *W, int64_t d_out, int64_t d_in, int64_t ldw,
+                             uint16_t *vals, uint8_t *meta, cudaStream_t stream);
+
+// T = X * V^T for M tokens, written as fp32 [M, r] (T32, may be null) and/or
+// bf16 [M, r] (T16, may be null).
+cudaError_t launch_lowrank_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in,
+                                   int64_t r, float *T32, uint16_t *T16, cudaStream_t stream);
+
+// Small-M streaming forward: Y = X S^T + T U^T with T (fp32 [M, r]) precomputed.
+cudaError_t launch_decode_forward(const uint16_t *X, int64_t M, const uint16_t *vals,
+                                  const uint8_t *meta, int64_t d_out, int64_t d_in,
+                                  const uint16_t *U, const float *T32, int64_t r, uint16_t *Y,
+                                  cudaStream_t stream);
+
+}  // namespace slr

@@ -1,0 +1,118 @@
+// pack_2to4.cu -- 2:4 projection by magnitude and packing (values + 2-bit indices).
+//
+// Hard-thresholding onto the 2:4 pattern (HASSLE-free, section 4.1.1: the
+// data-free optimal sparse update keeps the largest magnitudes; 2:4 = two
+// nonzeros in each group of four, as on the 3BASiL page).  The magnitude key
+// is the bf16 bit pattern with its sign bit cleared, compared as an integer;
+// of two equal keys the lower index wins.
+//
+// Work unit = 8 consecutive bf16 of a row (two groups): one 16-byte load, one
+// 8-byte store of the four kept values and one metadata byte, so a warp moves
+// 512 B in, 256 B + 32 B out, all coalesced.  The kernel is HBM-bound at
+// 2 B read + 1.125 B written per weight; a grid-stride loop over
+// d_out * d_in / 8 units keeps the grid at a few waves of the 148 SMs.
+#include "common.cuh"
+
+namespace slr {
+namespace {
+
+// Select the two kept positions of a group given as two 32-bit words holding
+// bf16 values 0,1 (w01) and 2,3 (w23).  Returns the nibble idx0 | idx1 << 2 and
+// the two kept bit patterns packed low (idx0) / high (idx1).
+__device__ __forceinline__ uint32_t select_group(uint32_t w01, uint32_t w23, uint32_t *kept) {
+    const uint32_t k0 = w01 & 0x7FFFu, k1 = (w01 >> 16) & 0x7FFFu;
+    const uint32_t k2 = w23 & 0x7FFFu, k3 = (w23 >> 16) & 0x7FFFu;
+    // Position a beats position b (a < b) when key_a >= key_b.
+    const uint32_t b01 = k0 >= k1, b02 = k0 >= k2, b03 = k0 >= k3;
+    const uint32_t b12 = k1 >= k2, b13 = k1 >= k3, b23 = k2 >= k3;
+    // Number of positions that beat each position.
+    const uint32_t beat0 = (1u - b01) + (1u - b02) + (1u - b03);
+    const uint32_t beat1 = b01 + (1u - b12) + (1u - b13);
+    const uint32_t beat2 = b02 + b12 + (1u - b23);
+    const uint32_t beat3 = b03 + b13 + b23;
+    const uint32_t mask = (beat0 < 2u) | ((beat1 < 2u) << 1) | ((beat2 < 2u) << 2) | ((beat3 < 2u) << 3);
+    const uint32_t i0 = __ffs(mask) - 1;          // lowest kept position
+    const uint32_t i1 = 31 - __clz(mask);         // highest kept position
+    const uint32_t v0 = ((i0 & 2u) ? w23 : w01) >> ((i0 & 1u) * 16);
+    const uint32_t v1 = ((i1 & 2u) ? w23 : w01) >> ((i1 & 1u) * 16);
+    *kept = (v0 & 0xFFFFu) | (v1 << 16);
+    return i0 | (i1 << 2);
+}
+
+// Vectorised path: d_in % 8 == 0, ldw % 8 == 0, W 16-byte aligned.
+__global__ void __launch_bounds__(256) pack_2to4_v8_kernel(const uint16_t *__restrict__ W, int64_t d_out,
+                                                           int64_t d_in, int64_t ldw,
+                                                           uint16_t *__restrict__ vals,
+                                                           uint8_t *__restrict__ meta) {
+    const int64_t units_per_row = d_in / 8;
+    const int64_t meta_row = (d_in / 4 + 1) / 2;
+    const int64_t total = d_out * units_per_row;
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total;
+         u += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = u / units_per_row;
+        const int64_t c = u - row * units_per_row;
+        const uint4 w = ld_stream_v4(W + row * ldw + c * 8);
+        uint32_t kept0, kept1;
+        const uint32_t n0 = select_group(w.x, w.y, &kept0);
+        const uint32_t n1 = select_group(w.z, w.w, &kept1);
+        *reinterpret_cast<uint2 *>(vals + row * (d_in / 2) + c * 4) = make_uint2(kept0, kept1);
+        meta[row * meta_row + c] = (uint8_t)(n0 | (n1 << 4));
+    }
+}
+
+// General path: any alignment, d_in % 4 == 0.  Unit = one metadata byte
+// (two groups, or one for the last byte of a row with an odd group count).
+__global__ void __launch_bounds__(256) pack_2to4_any_kernel(const uint16_t *__restrict__ W, int64_t d_out,
+                                                            int64_t d_in, int64_t ldw,
+                                                            uint16_t *__restrict__ vals,
+                                                            uint8_t *__restrict__ meta) {
+    const int64_t groups = d_in / 4;
+    const int64_t meta_row = (groups + 1) / 2;
+    const int64_t total = d_out * meta_row;
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total;
+         u += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = u / meta_row;
+        const int64_t j = u - row * meta_row;
+        uint32_t byte = 0;
+        for (int h = 0; h < 2; ++h) {
+            const int64_t g = 2 * j + h;
+            if (g >= groups) break;
+            const uint16_t *src = W + row * ldw + 4 * g;
+            const uint32_t w01 = (uint32_t)src[0] | ((uint32_t)src[1] << 16);
+            const uint32_t w23 = (uint32_t)src[2] | ((uint32_t)src[3] << 16);
+            uint32_t kept;
+            const uint32_t nib = select_group(w01, w23, &kept);
+            uint16_t *dst = vals + row * (d_in / 2) + 2 * g;
+            dst[0] = (uint16_t)(kept & 0xFFFFu);
+            dst[1] = (uint16_t)(kept >> 16);
+            byte |= nib << (4 * h);
+        }
+        meta[row * meta_row + j] = (uint8_t)byte;
+    }
+}
+
+int grid_for(int64_t units, int threads) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (units + threads - 1) / threads;
+    const int64_t cap = (int64_t)sms * 8;  // 8 resident CTAs of 256 threads per SM
+    return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_pack_2to4(const uint16_t *W, int64_t d_out, int64_t d_in, int64_t ldw,
+                             uint16_t *vals, uint8_t *meta, cudaStream_t stream) {
+    const bool v8 = (d_in % 8 == 0) && (ldw % 8 == 0) && ((reinterpret_cast<uintptr_t>(W) & 15) == 0) &&
+                    ((reinterpret_cast<uintptr_t>(vals) & 7) == 0);
+    if (v8) {
+        const int64_t units = d_out * (d_in / 8);
+        pack_2to4_v8_kernel<<<grid_for(units, 256), 256, 0, stream>>>(W, d_out, d_in, ldw, vals, meta);
+    } else {
+        const int64_t units = d_out * ((d_in / 4 + 1) / 2);
+        pack_2to4_any_kernel<<<grid_for(units, 256), 256, 0, stream>>>(W, d_out, d_in, ldw, vals, meta);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace slr

@@ -1,0 +1,19 @@
+// tc_forward.cuh -- launcher of the 2:4 tcgen05 tensor-core forward (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace slr {
+
+// Y = X S^T + T U^T on the tensor cores.  T16 is bf16 [M, r] (may be null when
+// r == 0).  Requires d_in % 128 == 0, d_out % 8 == 0, r % 8 == 0.
+cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
+                              int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
+                              uint16_t *Y, cudaStream_t stream);
+
+// Reads and clears the device-side error word the tensor-core kernel sets when
+// a bounded wait expires (0 = none).  Synchronises the device.
+cudaError_t read_and_clear_kernel_error(unsigned *code);
+
+}  // namespace slr

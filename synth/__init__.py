@@ -8,8 +8,9 @@ Recipe (the workloads of the five benchmark configurations):
 
 * Gaussian draws in fp32 from numpy's PCG64 generator, one generator per
   tensor, seeded with ``1000*cfg + 10*sub + tensor_id`` where ``tensor_id`` is
-  X=1, W=2, U=3, V=4, outlier-permutation=5 and ``sub`` numbers the layer
-  shapes inside a configuration (0 when there is only one).
+  X=1, W=2, U=3, V=4, outlier-permutation=5.  ``sub`` numbers the layers
+  inside a configuration (0 when there is only one); W and X use the number
+  of the layer *shape* instead, so the rank variants of one shape share them.
 * Scale by the stated standard deviation, then round to bf16
   (round-to-nearest-even).  W is projected to 2:4 only after this rounding.
 * Outlier channels: ``round(0.01 * d_in)`` columns of X, chosen by a seeded
@@ -72,6 +73,7 @@ class Layer:
     r: int
     cfg: int
     sub: int = 0
+    shape_sub: int | None = None   # seeds of W and X; defaults to sub
     x_outliers: bool = False
     w_std: float = 0.02
     # "lowrank" selects the factor distributions:
@@ -87,8 +89,12 @@ class Layer:
             return 0.0
         return 1.0 / math.sqrt(self.r) if self.lowrank == "v_unit" else 0.02 / math.sqrt(self.r)
 
+    @property
+    def wsub(self) -> int:
+        return self.sub if self.shape_sub is None else self.shape_sub
+
     def weight(self) -> np.ndarray:
-        return gaussian_bf16((self.d_out, self.d_in), self.w_std, seed_for(self.cfg, TENSOR_W, self.sub))
+        return gaussian_bf16((self.d_out, self.d_in), self.w_std, seed_for(self.cfg, TENSOR_W, self.wsub))
 
     def factors(self) -> tuple[np.ndarray, np.ndarray]:
         U = gaussian_bf16((self.d_out, self.r), self.u_std(), seed_for(self.cfg, TENSOR_U, self.sub))
@@ -96,8 +102,8 @@ class Layer:
         return U, V
 
     def activations(self, M: int) -> np.ndarray:
-        out = seed_for(self.cfg, TENSOR_OUTLIER, self.sub) if self.x_outliers else None
-        return activations_bf16(M, self.d_in, seed_for(self.cfg, TENSOR_X, self.sub), out)
+        out = seed_for(self.cfg, TENSOR_OUTLIER, self.wsub) if self.x_outliers else None
+        return activations_bf16(M, self.d_in, seed_for(self.cfg, TENSOR_X, self.wsub), out)
 
 
 @dataclass(frozen=True)
@@ -118,9 +124,9 @@ def _cfg4_layers():
 def _cfg5_layers():
     out = []
     sub = 0
-    for name, do, di in (("up_proj_70b", 28672, 8192), ("down_proj_70b", 8192, 28672)):
+    for shape, (name, do, di) in enumerate((("up_proj_70b", 28672, 8192), ("down_proj_70b", 8192, 28672))):
         for r in (64, 128, 256):
-            out.append(Layer(f"{name}_r{r}", do, di, r, cfg=5, sub=sub, x_outliers=True,
+            out.append(Layer(f"{name}_r{r}", do, di, r, cfg=5, sub=sub, shape_sub=shape, x_outliers=True,
                              lowrank="both_small"))
             sub += 1
     return tuple(out)

@@ -256,6 +256,14 @@ def pin_forward_row_subset(o):
     Ys, Bs = o.forward(X, vals, meta, U, V, rows=rows)
     np.testing.assert_array_equal(Ys, Yall[rows])
     np.testing.assert_array_equal(Bs, Ball[rows])
+    outs = [11, 2, 2, 5]
+    Yo, Bo = o.forward(X, vals, meta, U, V, rows=rows, outs=outs)
+    np.testing.assert_array_equal(Yo, Yall[np.ix_(rows, outs)])
+    np.testing.assert_array_equal(Bo, Ball[np.ix_(rows, outs)])
+    # The subset entries also match the numpy definition directly.
+    S = _f64(o.unpack_2to4(vals, meta, 16))
+    Wp = S + _f64(U) @ _f64(V)
+    np.testing.assert_array_equal(Yo, (_f64(X) @ Wp.T)[np.ix_(rows, outs)])
 
 
 def pin_lowrank_project(o):

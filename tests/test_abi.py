@@ -1,0 +1,115 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+that include/slr.h declares, and rejects bad arguments on the host before any
+launch.  Fake pointer values are used only where validation fails before the
+device is touched."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "slr.h")
+
+import sparse_rank_linear_02_b200 as slr  # noqa: E402
+
+OK, NULL, SHAPE, ALIGN, WORKSPACE, DEVICE, CUDA, TIMEOUT, ARG = range(9)
+P = ctypes.c_void_p
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SLR_API\s+[\w\s\*]+?\b(slr_\w+)\s*\(", text)))
+
+
+def test_header_declares_api():
+    names = declared_functions()
+    for n in ["slr_pack_2to4", "slr_forward", "slr_forward_workspace_size", "slr_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(slr.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    for s in range(9):
+        assert slr.lib().slr_status_string(s).decode().startswith("SLR_")
+    assert slr.lib().slr_status_string(99) == b"SLR_ERR_UNKNOWN"
+
+
+def test_meta_row_bytes_and_workspace():
+    lib = slr.lib()
+    assert lib.slr_meta_row_bytes(4096) == 512
+    assert lib.slr_meta_row_bytes(12) == 2
+    assert lib.slr_meta_row_bytes(4) == 1
+    assert slr.workspace_size(16, 4096, 4096, 64) == 16 * 64 * 4
+    assert slr.workspace_size(2048, 14336, 4096, 64) == 2048 * 64 * 4
+    assert slr.workspace_size(8, 256, 256, 0) == 0
+    assert slr.workspace_size(0, 256, 256, 8) == 0
+
+
+def test_path_selection():
+    assert slr.select_path(1, 4096, 4096, 64) == "decode"
+    assert slr.select_path(16, 4096, 4096, 64) == "decode"
+    assert slr.select_path(2048, 14336, 4096, 64) == "tensor"
+    assert slr.select_path(2048, 100, 4096, 64) == "decode"   # d_out % 8 != 0
+
+
+def _fwd(X=0x1000, M=16, vals=0x2000, meta=0x3000, d_out=256, d_in=256, U=0x4000, V=0x5000, r=8,
+         Y=0x6000, ws=0x7000, ws_bytes=1 << 20, path=0):
+    return slr.lib().slr_forward_with_path(P(X), M, P(vals), P(meta), d_out, d_in, P(U), P(V), r, P(Y),
+                                           P(ws), ws_bytes, path, None)
+
+
+def test_forward_argument_errors():
+    assert _fwd(M=0, X=0, vals=0, meta=0, Y=0) == OK          # empty problem: no-op
+    assert _fwd(M=-1) == SHAPE
+    assert _fwd(r=-8) == SHAPE
+    assert _fwd(X=0) == NULL
+    assert _fwd(meta=0) == NULL
+    assert _fwd(Y=0) == NULL
+    assert _fwd(U=0) == NULL
+    assert _fwd(V=0, r=8) == NULL
+    assert _fwd(ws=0) == NULL
+    assert _fwd(d_in=200) == SHAPE             # not a multiple of 128
+    assert _fwd(d_in=0) == SHAPE
+    assert _fwd(r=12) == SHAPE                 # not a multiple of 8
+    assert _fwd(d_out=0) == SHAPE
+    assert _fwd(d_out=100, path=2) == SHAPE    # tensor path needs d_out % 8 == 0
+    assert _fwd(X=0x1008) == ALIGN
+    assert _fwd(vals=0x2004) == ALIGN
+    assert _fwd(meta=0x3001) == ALIGN
+    assert _fwd(U=0x4002) == ALIGN
+    assert _fwd(ws=0x7010) == ALIGN            # workspace needs 256-byte alignment
+    assert _fwd(ws_bytes=16) == WORKSPACE
+    assert _fwd(path=7) == ARG
+
+
+def test_forward_rank_zero_needs_no_factors_or_workspace():
+    # With r == 0 the factors and the workspace may be NULL; validation then
+    # reaches the device check (which fails here only when there is no GPU).
+    if torch.cuda.is_available():
+        pytest.skip("would launch with fake pointers on a GPU machine")
+    assert _fwd(U=0, V=0, r=0, ws=0, ws_bytes=0) == DEVICE
+
+
+def test_valid_arguments_without_gpu_report_device_error():
+    if torch.cuda.is_available():
+        pytest.skip("would launch with fake pointers on a GPU machine")
+    assert _fwd() == DEVICE
+    lib = slr.lib()
+    assert lib.slr_pack_2to4(P(0x1000), 4, 8, 8, P(0x2000), P(0x3000), None) == DEVICE
+
+
+def test_pack_argument_errors():
+    lib = slr.lib()
+    assert lib.slr_pack_2to4(P(0x1000), 4, 6, 6, P(0x2000), P(0x3000), None) == SHAPE   # d_in % 4
+    assert lib.slr_pack_2to4(P(0x1000), 4, 8, 4, P(0x2000), P(0x3000), None) == SHAPE   # ldw < d_in
+    assert lib.slr_pack_2to4(P(0x1000), -1, 8, 8, P(0x2000), P(0x3000), None) == SHAPE
+    assert lib.slr_pack_2to4(P(0), 4, 8, 8, P(0x2000), P(0x3000), None) == NULL
+    assert lib.slr_pack_2to4(P(0x1000), 4, 8, 8, P(0), P(0x3000), None) == NULL
+    assert lib.slr_pack_2to4(P(0), 0, 8, 8, P(0), P(0), None) == OK                    # empty

@@ -1,0 +1,180 @@
+"""GPU parity: the CUDA library (through the C ABI) against the fp64 oracle.
+
+Pack: bit-exact on every configuration shape and on adversarial inputs.
+Forward: the acceptance bounds (relative Frobenius <= 5e-3, per element
+|err| <= 1e-2 (|X||W'|^T) + 1e-3) on every configuration, on both execution
+paths, on seeded samples of (token, output) pairs at full size (all pairs for
+the small shapes), plus cases that isolate each term and the edge cases.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import (bits_to_f64, check_forward, from_dev, layer_activations, layer_weights,
+                      sample_indices, to_dev, to_dev_u8)
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import sparse_rank_linear_02_b200 as slr
+
+
+def _shapes():
+    seen, out = set(), []
+    for c in synth.CONFIGS.values():
+        for l in c.layers:
+            if (l.d_out, l.d_in) not in seen:
+                seen.add((l.d_out, l.d_in))
+                out.append((c.cfg, l.name))
+    return out
+
+
+# ----------------------------------------------------------------------------- pack
+
+@pytest.mark.parametrize("cfg,name", _shapes(), ids=lambda x: str(x))
+def test_pack_config_bit_exact(cfg, name):
+    layer, W, vals_ref, meta_ref, _, _ = layer_weights(cfg, name)
+    vals, meta = slr.pack_2to4(to_dev(W))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(from_dev(vals), vals_ref)
+    np.testing.assert_array_equal(meta.cpu().numpy(), meta_ref)
+
+
+def _adversarial(seed, rows, cols):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    W = rng.integers(0, 1 << 16, size=(rows, cols), dtype=np.uint32).astype(np.uint16)  # any bits, NaN too
+    W[:, : cols // 4] &= 0x8000 | 0x3F80          # many +-1.0 / +-0 ties
+    W[rows // 2:, cols // 2:] = rng.choice(np.array([0, 0x8000, 0x3F80, 0xBF80, 0x7F80, 0xFF80, 0x7FC0],
+                                                    dtype=np.uint16), size=(rows - rows // 2, cols - cols // 2))
+    return W
+
+
+@pytest.mark.parametrize("rows,cols", [(64, 256), (33, 72), (5, 12), (7, 4), (128, 4100)])
+def test_pack_adversarial_bit_exact(rows, cols):
+    W = _adversarial(rows * 1000 + cols, rows, cols)
+    vals_ref, meta_ref = oracle.pack_2to4(W)
+    vals, meta = slr.pack_2to4(to_dev(W))
+    np.testing.assert_array_equal(from_dev(vals), vals_ref)
+    np.testing.assert_array_equal(meta.cpu().numpy(), meta_ref)
+
+
+def test_pack_strided_and_unaligned():
+    """ldw > d_in (a column slice of a wider matrix) and W pointers that are not
+    16-byte aligned (8- and 2-byte offsets take the general kernel)."""
+    big = _adversarial(99, 40, 264)
+    Wd = to_dev(big)
+    for lo, hi in [(0, 256), (4, 260), (1, 253)]:
+        vals_ref, meta_ref = oracle.pack_2to4(np.ascontiguousarray(big[:, lo:hi]))
+        vals, meta = slr.pack_2to4(Wd[:, lo:hi])
+        np.testing.assert_array_equal(from_dev(vals), vals_ref)
+        np.testing.assert_array_equal(meta.cpu().numpy(), meta_ref)
+
+
+# ----------------------------------------------------------------------------- forward
+
+def _forward_case(cfg, name, M, path, k_rows=48, k_outs=384):
+    layer, W, vals, meta, U, V = layer_weights(cfg, name)
+    X = layer_activations(cfg, name, M)
+    Y = slr.forward(to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U), to_dev(V), path=path)
+    torch.cuda.synchronize()
+    slr.check_kernel_error()
+    rows = sample_indices(M, k_rows, seed=cfg * 7 + M)
+    outs = sample_indices(layer.d_out, k_outs, seed=cfg * 11 + layer.d_out)
+    Yref, Bref = oracle.forward(X, vals, meta, U, V, rows=rows, outs=outs)
+    Yg = from_dev(Y)[np.ix_(rows, outs)]
+    return check_forward(Yg, Yref, Bref, f"cfg{cfg} {name} M={M} path={path}")
+
+
+def _cases():
+    out = []
+    for c in synth.CONFIGS.values():
+        for l in c.layers:
+            for M in c.Ms:
+                out.append((c.cfg, l.name, M, "auto"))
+    # the other path on the decode and prefill shapes
+    for M in (1, 4, 16):
+        out.append((2, "q_proj", M, "tensor"))
+    out.append((1, "tiny", 8, "tensor"))
+    out.append((3, "gate_up", 2048, "decode"))
+    out.append((5, "up_proj_70b_r256", 128, "decode"))
+    return out
+
+
+@pytest.mark.parametrize("cfg,name,M,path", _cases(), ids=lambda x: str(x))
+def test_forward_config(cfg, name, M, path):
+    _forward_case(cfg, name, M, path)
+
+
+def _lowrank_only(d_out, d_in, r, M, path, seed):
+    """S = 0 and factors of unit scale: Y = (X V^T) U^T alone must meet the bounds
+    (the configured factor scales make the low-rank term too small to see)."""
+    X = synth.gaussian_bf16((M, d_in), 1.0, seed + 1)
+    U = synth.gaussian_bf16((d_out, r), 1.0, seed + 2)
+    V = synth.gaussian_bf16((r, d_in), 1.0 / np.sqrt(d_in), seed + 3)
+    vals = np.zeros((d_out, d_in // 2), dtype=np.uint16)
+    meta = np.full((d_out, d_in // 8), 0x44, dtype=np.uint8)
+    Y = slr.forward(to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U), to_dev(V), path=path)
+    rows = sample_indices(M, 40, seed)
+    outs = sample_indices(d_out, 300, seed + 5)
+    Yref, Bref = oracle.forward(X, vals, meta, U, V, rows=rows, outs=outs)
+    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, f"lowrank-only {d_out}x{d_in} r={r} M={M} {path}")
+
+
+@pytest.mark.parametrize("path", ["decode", "tensor"])
+@pytest.mark.parametrize("d_out,d_in,r,M", [(4096, 4096, 64, 16), (14336, 4096, 64, 300), (256, 256, 8, 8),
+                                            (1024, 8192, 256, 130), (512, 1024, 128, 1)])
+def test_forward_lowrank_only(d_out, d_in, r, M, path):
+    _lowrank_only(d_out, d_in, r, M, path, seed=d_out + d_in + r + M)
+
+
+@pytest.mark.parametrize("path", ["decode", "tensor"])
+def test_forward_one_hot_exact(path):
+    """U = 0 and X rows e_j: Y[m, :] = S[:, j] exactly (decodes the metadata of
+    every column of every row; any index, order or layout slip changes bits)."""
+    d_out, d_in = 384, 512
+    W = synth.gaussian_bf16((d_out, d_in), 0.02, 5151)
+    vals, meta = oracle.pack_2to4(W)
+    S = oracle.unpack_2to4(vals, meta, d_in)
+    X = np.zeros((d_in, d_in), dtype=np.uint16)
+    X[np.arange(d_in), np.arange(d_in)] = 0x3F80
+    U = np.zeros((d_out, 8), dtype=np.uint16)
+    V = synth.gaussian_bf16((8, d_in), 1.0, 5152)
+    Y = slr.forward(to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U), to_dev(V), path=path)
+    np.testing.assert_array_equal(bits_to_f64(from_dev(Y)), bits_to_f64(np.ascontiguousarray(S.T)))
+
+
+@pytest.mark.parametrize("path", ["decode", "tensor"])
+@pytest.mark.parametrize("d_out,d_in,r,M", [
+    (200, 256, 16, 37),      # ragged output tile, ragged token tile
+    (128, 128, 0, 1),        # one stage, no low-rank term
+    (136, 384, 8, 129),      # r = 8 pads to the MMA K step; M just over a tile
+    (256, 640, 128, 255),    # two rank steps on the tensor path
+    (264, 1024, 256, 20),    # four rank steps; decode with several token blocks
+])
+def test_forward_edges(d_out, d_in, r, M, path):
+    seed = d_out * 31 + d_in + r + M
+    X = synth.activations_bf16(M, d_in, seed, seed + 9)
+    W = synth.gaussian_bf16((d_out, d_in), 0.02, seed + 1)
+    vals, meta = oracle.pack_2to4(W)
+    U = synth.gaussian_bf16((d_out, r), 0.5, seed + 2)
+    V = synth.gaussian_bf16((r, d_in), 0.5 / np.sqrt(max(r, 1)), seed + 3)
+    Y = slr.forward(to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U) if r else None,
+                    to_dev(V) if r else None, path=path)
+    Yref, Bref = oracle.forward(X, vals, meta, U if r else None, V if r else None)
+    check_forward(from_dev(Y), Yref, Bref, f"edge {d_out}x{d_in} r={r} M={M} {path}")
+
+
+def test_forward_matches_between_paths():
+    """The two paths agree with each other as well as with the oracle."""
+    layer, W, vals, meta, U, V = layer_weights(2, "q_proj")
+    X = layer_activations(2, "q_proj", 16)
+    args = (to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U), to_dev(V))
+    Yd = bits_to_f64(from_dev(slr.forward(*args, path="decode")))
+    Yt = bits_to_f64(from_dev(slr.forward(*args, path="tensor")))
+    assert np.linalg.norm(Yd - Yt) / np.linalg.norm(Yd) < 5e-3
+
+
+def test_no_kernel_timeouts():
+    slr.check_kernel_error()
