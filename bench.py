@@ -49,7 +49,7 @@ SPARSE_RATIO = 2.0   # nominal 2:4 sparse / dense tensor throughput ratio
 
 # DRAM bytes per launch of the dominant kernel from the committed ncu capture
 # (profiles/); valid only for the kernel source it was taken on.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {"tc_forward": {"source_sha": "eafdd5bf5a7be4cd", "bytes_per_launch": 277621248}}
 
 
 def layer_of(cfg, name):
@@ -232,42 +232,24 @@ def run_ours(args, rank, world, dist):
                "project_ms": round(project_ms, 4), "combine_ms": round(combine_ms, 4)}
     clocks = clk.summary()
 
+    legs = set(args.only.split(","))
+    e2e = None
     # ------------------------------------------------ e2e through host buffers
-    X_pin = torch.from_numpy(Xh.view(np.int16)).view(torch.bfloat16).pin_memory()
-    Y_pin = torch.empty((M, d_out), dtype=torch.bfloat16).pin_memory()
-    s0 = sets[0]
-    for _ in range(2):
-        s0["X"].copy_(X_pin, non_blocking=True)
-        slr.forward(s0["X"], s0["vals"], s0["meta"], s0["U"], s0["V"], out=s0["Y"], workspace=s0["ws"])
-        Y_pin.copy_(s0["Y"], non_blocking=True)
-    Ke = max(3, K // 2)
-    barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for k in range(Ke):
-        s = sets[k % n_copies]
-        s["X"].copy_(X_pin, non_blocking=True)
-        slr.forward(s["X"], s["vals"], s["meta"], s["U"], s["V"], out=s["Y"], workspace=s["ws"])
-        Y_pin.copy_(s["Y"], non_blocking=True)
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / Ke
-    e2e = {"value": round(world * flops_dense / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-           "h2d_bytes_per_step": int(X_pin.numel() * 2), "d2h_bytes_per_step": int(Y_pin.numel() * 2),
-           "ms_per_step": round(e2e_ms, 4)}
-    del sets, s0
+    if "e2e" in legs:
+        e2e = run_e2e_leg(args, slr, torch, Xh, M, d_out, sets, n_copies, flops_dense, world, max_over_ranks,
+                          barrier)
+    del sets
 
     # ------------------------------------------------ decode leg (M = 1)
-    decode = run_decode_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier)
+    decode = run_decode_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier) if "decode" in legs else None
 
     # ------------------------------------------------ pack leg
-    pack = run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier)
+    pack = run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier) if "pack" in legs else None
     del W
 
     # ------------------------------------------------ CPU baseline (oracle), rank 0 at N = 1
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and "cpu" in legs:
         cpu = cpu_baseline_prefill(L, rows=args.cpu_rows)
 
     line = {
@@ -292,6 +274,34 @@ def run_ours(args, rank, world, dist):
         "kernel_source_sha": sha,
     }
     return line
+
+
+def run_e2e_leg(args, slr, torch, Xh, M, d_out, sets, n_copies, flops_dense, world, max_over_ranks, barrier):
+    """The same forward through the public API with host buffers: each step
+    copies X from pinned host memory, runs slr_forward and reads Y back."""
+    X_pin = torch.from_numpy(np.ascontiguousarray(Xh).view(np.int16)).view(torch.bfloat16).pin_memory()
+    Y_pin = torch.empty((M, d_out), dtype=torch.bfloat16).pin_memory()
+
+    def step(s):
+        s["X"].copy_(X_pin, non_blocking=True)
+        slr.forward(s["X"], s["vals"], s["meta"], s["U"], s["V"], out=s["Y"], workspace=s["ws"])
+        Y_pin.copy_(s["Y"], non_blocking=True)
+
+    for i in range(3):
+        step(sets[i % n_copies])
+    Ke = max(3, args.steps // 2)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for k in range(Ke):
+        step(sets[k % n_copies])
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / Ke
+    return {"value": round(world * flops_dense / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(X_pin.numel() * 2), "d2h_bytes_per_step": int(Y_pin.numel() * 2),
+            "ms_per_step": round(e2e_ms, 4), "steps": Ke}
 
 
 def run_decode_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier):
@@ -439,6 +449,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=64, help="token rows in the oracle CPU baseline sample")
     ap.add_argument("--ref-rows", type=int, default=8, help="token rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default="prefill,e2e,decode,pack,cpu",
+                    help="comma list of legs to run (profiling runs use one leg)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
