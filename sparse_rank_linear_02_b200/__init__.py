@@ -1,8 +1,8 @@
 """Python binding of libslr: the 2:4-sparse + low-rank linear layer on B200.
 
 Argument marshalling only.  Every step of the computation runs in the CUDA
-kernels of ``libslr.so`` (built in-tree by ``python -m
-sparse_rank_linear_02_b200.build``); there is no fallback of any kind, and the
+kernels of ``libslr.so`` (built in-tree by ``python
+sparse_rank_linear_02_b200/build.py``); there is no fallback of any kind, and the
 import fails if the library is missing.
 
 Functions mirror the C ABI in ``include/slr.h``:
@@ -43,7 +43,7 @@ class SlrError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing; build it with "
-                          f"`python -m sparse_rank_linear_02_b200.build`")
+                          f"`python sparse_rank_linear_02_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     i64, p, sz, st = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
     lib.slr_status_string.restype = ctypes.c_char_p

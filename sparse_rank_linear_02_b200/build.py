@@ -1,6 +1,7 @@
 """Build libslr.so in-tree with nvcc for sm_100a (B200).
 
-Usage: ``python -m sparse_rank_linear_02_b200.build [--force]``.  The library
+Usage: ``python sparse_rank_linear_02_b200/build.py [--force]`` (run it by
+path: importing the package loads the library this script builds).  The library
 statically links the CUDA runtime and resolves the one driver entry point it
 needs (tensor-map encoding) at run time, so it loads on a machine without a
 GPU driver (the exported symbols can be inspected there; compute calls then
