@@ -164,6 +164,40 @@ SLR_API slr_status slr_forward_combine(const void *X, int64_t M, const void *val
                                        const void *workspace, size_t workspace_bytes, slr_path path,
                                        slr_stream_t stream);
 
+/* --------------------------------------------------------------------------
+ * Small-M forward without a caller workspace.  (The pages have no
+ * counterpart to this entry point; it exists for callers of this library.)
+ *
+ * For callers that cannot allocate device memory where they run the layer,
+ * e.g. an inference engine that reserves the whole device heap at start-up
+ * and only hands out the tensors it manages, or a latency-critical decode loop
+ * that may not call cudaMalloc (which can synchronise the device).  It
+ * computes the same result as slr_forward_with_path(..., SLR_PATH_DECODE, ...),
+ * with the same argument layouts, but keeps the rank projection T = X V^T in an
+ * array built into the library instead of a workspace.
+ *
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - Capacity: M * r <= SLR_NOALLOC_MAX_T_ELEMS (fp32 entries, 64 KB); larger
+ *     problems return SLR_ERR_WORKSPACE with nothing queued.  r == 0 needs no
+ *     scratch and accepts any M.
+ *   - The array exists once per device that loads the library and stays
+ *     allocated until the process exits.
+ *   - The first call on a device does a one-time set-up (it looks up the
+ *     array's device address with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device uses the same array, which keeps the previous
+ *     call's contents; nothing in it needs to start at zero because each call
+ *     writes every entry it later reads.  Calls that can overlap on the GPU
+ *     (different streams, or host threads with no ordering between them) race
+ *     on the array: serialise them.
+ * Other requirements and errors are those of slr_forward (no workspace
+ * arguments).
+ * ------------------------------------------------------------------------ */
+#define SLR_NOALLOC_MAX_T_ELEMS 16384
+SLR_API slr_status slr_forward_decode_noalloc(const void *X, int64_t M, const void *vals, const void *meta,
+                                              int64_t d_out, int64_t d_in, const void *U, const void *V,
+                                              int64_t r, void *Y, slr_stream_t stream);
+
 /* Synchronises the current device, then reports (and clears) the error word
  * that the tensor-core kernel sets when one of its bounded waits expires:
  * SLR_ERR_TIMEOUT if any launch since the last check gave up, SLR_OK

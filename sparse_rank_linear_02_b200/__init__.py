@@ -67,6 +67,8 @@ def _load() -> ctypes.CDLL:
     lib.slr_forward_project.argtypes = [p, i64, p, i64, i64, i64, p, sz, st, p]
     lib.slr_forward_combine.restype = st
     lib.slr_forward_combine.argtypes = [p, i64, p, p, i64, i64, p, i64, p, p, sz, st, p]
+    lib.slr_forward_decode_noalloc.restype = st
+    lib.slr_forward_decode_noalloc.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, p]
     return lib
 
 
@@ -154,6 +156,24 @@ def forward_combine(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, U: 
     _check(_lib.slr_forward_combine(_ptr(X), M, _ptr(vals), _ptr(meta), d_out, d_in, _ptr(U), r, _ptr(out),
                                     _ptr(workspace), ws_bytes, PATHS[path], _stream()),
            "slr_forward_combine")
+    return out
+
+
+NOALLOC_MAX_T_ELEMS = 16384
+
+
+def forward_decode_noalloc(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, U: torch.Tensor | None,
+                           V: torch.Tensor | None, out: torch.Tensor) -> torch.Tensor:
+    """Small-M forward for callers that cannot allocate device memory
+    (``slr_forward_decode_noalloc``): no workspace; the rank projection lives in
+    a fixed array inside the library (M * r <= NOALLOC_MAX_T_ELEMS).  ``out``
+    must be provided."""
+    M, d_in = X.shape
+    d_out = vals.shape[0]
+    r = 0 if U is None else U.shape[1]
+    _check(_lib.slr_forward_decode_noalloc(_ptr(X), M, _ptr(vals), _ptr(meta), d_out, d_in, _ptr(U), _ptr(V), r,
+                                           _ptr(out), _stream()),
+           "slr_forward_decode_noalloc")
     return out
 
 
