@@ -90,7 +90,7 @@ cudaError_t run_project(const void *X, int64_t M, const void *V, int64_t d_in, i
     const uint16_t *x = static_cast<const uint16_t *>(X);
     const uint16_t *vv = static_cast<const uint16_t *>(V);
     if (p == SLR_PATH_DECODE) return launch_lowrank_project(x, M, vv, d_in, r, static_cast<float *>(workspace), nullptr, stream);
-    return launch_lowrank_project(x, M, vv, d_in, r, nullptr, static_cast<uint16_t *>(workspace), stream);
+    return launch_tc_project(x, M, vv, d_in, r, static_cast<uint16_t *>(workspace), stream);
 }
 
 // Stage 2: Y = X S^T + T U^T with T read from the workspace.

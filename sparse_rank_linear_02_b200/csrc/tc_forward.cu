@@ -35,10 +35,13 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
 #include "tc_forward.cuh"
+#include "tc_ptx.cuh"
 
 namespace slr {
 
@@ -49,212 +52,54 @@ namespace tc {
 constexpr int BM = 128;            // output rows per tile (MMA M)
 constexpr int BK = 128;            // logical K per pipeline stage
 constexpr int kThreads = 192;      // 6 warps
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kEcol = 256;    // metadata columns start after two accumulators
-constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at the boost clock
 
-template <int BN>
+constexpr uint32_t pow2_at_least(uint32_t x) {
+    uint32_t p = 32;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+// kSparse: the 2:4 forward (A = packed S tile, 128 logical K per stage, plus
+// rank stages).  !kSparse: the dense rank projection T^T = V X^T (A = V tile,
+// 64 K per stage, no metadata, no rank stages).
+template <int BN, bool kSparse>
 struct Cfg {
-    static constexpr int A_BYTES = BM * (BK / 2) * 2;   // 16 KB of packed values
-    static constexpr int B_HALF = BN * 64 * 2;          // one 128-byte-wide swizzle panel of X
-    static constexpr int B_BYTES = 2 * B_HALF;
-    static constexpr int E_BYTES = BM * BK / 8;         // 2 KB of metadata
-    static constexpr int STAGE = A_BYTES + B_BYTES + E_BYTES;
-    static constexpr int NS = (BN == 128) ? 4 : 6;
+    static constexpr int A_BYTES = BM * 64 * 2;         // 16 KB: 128 rows x one 128-byte swizzle panel
+    static constexpr int B_HALF = BN * 64 * 2;          // BN rows x one 128-byte swizzle panel of X
+    static constexpr int B_BYTES = kSparse ? 2 * B_HALF : B_HALF;
+    static constexpr int E_BYTES = kSparse ? BM * BK / 8 : 0;   // 2 KB of metadata
+    static constexpr int STAGE = ((A_BYTES + B_BYTES + E_BYTES + 1023) / 1024) * 1024;
     static constexpr int OUT_COLS = 32;                 // tokens per output chunk
     static constexpr int OUT_BYTES = OUT_COLS * BM * 2;
+    static constexpr int NS_FIT = (232448 - 2 * OUT_BYTES - 2048) / STAGE;
+    static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
+    static constexpr int K_PER_STAGE = kSparse ? BK : 64;
+    static constexpr uint32_t ECOL = 2 * BN;            // metadata columns after two accumulators
+    static constexpr uint32_t TMEM_COLS = pow2_at_least(2 * BN + (kSparse ? 4 : 0));
     static constexpr int RING = NS * STAGE;
     static constexpr int BAR_OFF = RING + 2 * OUT_BYTES;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;   // barriers + alignment slack
     static_assert(STAGE % 1024 == 0, "stage must keep 1024-byte alignment");
+    static_assert(NS >= 2, "need at least two stages");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-// ------------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait: false when the phase did not complete within kWaitCycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
-        if (clock64() - t0 > kWaitCycles) return false;
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint32_t dst, uint64_t *bar, int32_t c0,
-                                            int32_t c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
-            dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-        : "memory");
-}
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int32_t c0, int32_t c1) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(src), "r"(c0), "r"(c1)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Shared-memory matrix descriptor (tcgen05 "version 1" format): start address,
-// leading/stride byte offsets in 16-byte units, layout type in bits 61..63.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
-    d |= (uint64_t)layout << 61;
-    return d;
-}
-constexpr uint32_t kLayoutSW128 = 2;
-constexpr uint32_t kLayoutNone = 0;
-
-// K-major, 128-byte swizzled operand tile: 8-row groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) { return smem_desc(addr, 16, 1024, kLayoutSW128); }
-
-// Instruction descriptor, kind::f16 with bf16 inputs and fp32 accumulation,
-// both operands K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool sparse) {
-    return (sparse ? (1u << 2) : 0u)       // sparsity flag
-           | (1u << 4)                     // D format: f32
-           | (1u << 7)                     // A format: bf16
-           | (1u << 10)                    // B format: bf16
-           | ((uint32_t)(n >> 3) << 17)    // N / 8
-           | ((uint32_t)(m >> 4) << 24);   // M / 16
-}
-
-__device__ __forceinline__ void mma_sp(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t e_tmem, uint32_t idesc,
-                                       uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(e_tmem), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void mma_dense(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Permute one 2 KB metadata tile in place from the exported row-major layout
-// ([128 rows][16 bytes], byte j = groups 2j, 2j+1) into the tcgen05.cp source
-// layout.  Lane handles row pairs p = lane and lane + 32, p = m0 + 8*m2:
-// rows A = m0 + 16*m2 and B = A + 8 are read whole and rewritten as
-//   row A = [A.w0 B.w0 A.w2 B.w2 A.w4 B.w4 A.w6 B.w6]   (16-bit words)
-//   row B = [A.w1 B.w1 A.w3 B.w3 A.w5 B.w5 A.w7 B.w7]
-// Rows past d_out arrive zero-filled from TMA, i.e. with the index pair
-// (0, 0), which is not a valid 2:4 pattern; rewrite any nibble whose two
-// indices are equal to (0, 1).  The values there are zero, so the choice
-// does not change the result; it only keeps the hardware on defined input.
-__device__ __forceinline__ uint32_t sanitize_nibbles(uint32_t w) {
-    const uint32_t lo = w & 0x33333333u, hi = (w >> 2) & 0x33333333u;
-    const uint32_t same = ~(lo ^ hi);
-    const uint32_t eq = same & (same >> 1) & 0x11111111u;   // one bit per nibble with idx0 == idx1
-    return (w & ~(eq * 0xFu)) | (eq * 0x4u);
-}
-
-__device__ __forceinline__ void permute_meta_tile(uint8_t *e, int lane) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int p = lane + 32 * h;
-        const int rowA = (p & 7) + 16 * (p >> 3);
-        uint4 *ra = reinterpret_cast<uint4 *>(e + rowA * 16);
-        uint4 *rb = reinterpret_cast<uint4 *>(e + (rowA + 8) * 16);
-        uint4 a = *ra, b = *rb;
-        a.x = sanitize_nibbles(a.x); a.y = sanitize_nibbles(a.y); a.z = sanitize_nibbles(a.z); a.w = sanitize_nibbles(a.w);
-        b.x = sanitize_nibbles(b.x); b.y = sanitize_nibbles(b.y); b.z = sanitize_nibbles(b.z); b.w = sanitize_nibbles(b.w);
-        uint4 lo, hi;
-        lo.x = __byte_perm(a.x, b.x, 0x5410);
-        lo.y = __byte_perm(a.y, b.y, 0x5410);
-        lo.z = __byte_perm(a.z, b.z, 0x5410);
-        lo.w = __byte_perm(a.w, b.w, 0x5410);
-        hi.x = __byte_perm(a.x, b.x, 0x7632);
-        hi.y = __byte_perm(a.y, b.y, 0x7632);
-        hi.z = __byte_perm(a.z, b.z, 0x7632);
-        hi.w = __byte_perm(a.w, b.w, 0x7632);
-        *ra = lo;
-        *rb = hi;
-    }
-}
-
 struct Params {
-    int32_t M, d_out, d_in, r;
-    int32_t n_dtiles, n_tiles, nk, nlr;
+    int32_t M;          // tokens
+    int32_t n_ttiles;   // token tiles
+    int32_t n_tiles;    // output-row tiles x token tiles
+    int32_t nk, nlr;    // K stages, rank stages
 };
 
-template <int BN>
+// Tiles run output-row-tile major: the CTAs resident at one time share a few
+// S tiles and all token tiles, so X stays in L2 and S is fetched about once.
+template <int BN, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_forward_kernel(const __grid_constant__ CUtensorMap tm_vals, const __grid_constant__ CUtensorMap tm_meta,
                       const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_u,
                       const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_y,
                       const Params prm) {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, kSparse>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
@@ -282,12 +127,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(kTmemCols));
+                     "r"(C::TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (threadIdx.x == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_vals)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_meta)) : "memory");
+        if (kSparse) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_meta)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
     }
     tc_fence_before();
@@ -300,8 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             uint32_t s = 0, ph = 0;
             for (int tile = blockIdx.x; tile < prm.n_tiles && !*fail; tile += gridDim.x) {
-                const int tok0 = (tile / prm.n_dtiles) * BN;
-                const int d0 = (tile % prm.n_dtiles) * BM;
+                const int d0 = (tile / prm.n_ttiles) * BM;
+                const int tok0 = (tile % prm.n_ttiles) * BN;
                 for (int ks = 0; ks < prm.nk + prm.nlr; ++ks) {
                     if (!mbar_wait(&empty[s], ph ^ 1)) {
                         *fail = 1;
@@ -311,7 +156,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *st = smem + s * C::STAGE;
                     const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES),
                                    e = smem_u32(st + C::A_BYTES + C::B_BYTES);
-                    if (ks < prm.nk) {
+                    if (!kSparse) {
+                        mbar_expect_tx(&full[s], C::A_BYTES + C::B_HALF);
+                        tma_load_2d(&tm_vals, a, &full[s], ks * 64, d0);
+                        tma_load_2d(&tm_x, b, &full[s], ks * 64, tok0);
+                    } else if (ks < prm.nk) {
                         mbar_expect_tx(&full[s], C::A_BYTES + C::B_BYTES + C::E_BYTES);
                         tma_load_2d(&tm_vals, a, &full[s], ks * 64, d0);
                         tma_load_2d(&tm_x, b, &full[s], ks * BK, tok0);
@@ -334,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ MMA issue
         constexpr uint32_t kIdescSp = idesc_bf16(BM, BN, true);
         constexpr uint32_t kIdescDense = idesc_bf16(BM, BN, false);
-        const uint32_t e_tmem = tmem_base + kEcol;
+        const uint32_t e_tmem = tmem_base + C::ECOL;
         uint32_t s = 0, ph = 0;
         int it = 0;
         for (int tile = blockIdx.x; tile < prm.n_tiles && !*fail; tile += gridDim.x, ++it) {
@@ -355,7 +204,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 uint8_t *st = smem + s * C::STAGE;
                 const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES);
-                if (ks < prm.nk) {
+                if (!kSparse) {
+                    if (lane == 0) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            mma_dense(d_tmem, desc_sw128(a + 32 * c), desc_sw128(b + 32 * c), kIdescDense,
+                                      (ks | c) != 0);
+                        mma_commit(&empty[s]);
+                    }
+                } else if (ks < prm.nk) {
                     permute_meta_tile(st + C::A_BYTES + C::B_BYTES, lane);
                     fence_proxy_async_smem();
                     __syncwarp();
@@ -401,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t chunk = 0;
         int it = 0;
         for (int tile = blockIdx.x; tile < prm.n_tiles && !*fail; tile += gridDim.x, ++it) {
-            const int tok0 = (tile / prm.n_dtiles) * BN;
-            const int d0 = (tile % prm.n_dtiles) * BM;
+            const int d0 = (tile / prm.n_ttiles) * BM;
+            const int tok0 = (tile % prm.n_ttiles) * BN;
             const int buf = it & 1;
             const uint32_t use = (uint32_t)(it >> 1);
             if (!mbar_wait(&acc_full[buf], use & 1)) {
@@ -443,7 +301,317 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+    }
+}
+
+
+// =====================================================================================
+// 2-SM variant (cta_group::2).  A cluster of two CTAs on neighbouring SMs owns a
+// 256-row x BN-token tile of Y^T: CTA rank q stages rows 128q..128q+127 of the
+// S tile (values and metadata) and tokens (BN/2)q..(BN/2)q+BN/2-1 of the X tile.
+// The leader (rank 0) issues every tcgen05.cp / tcgen05.mma for the pair; each
+// operand descriptor names the same shared-memory offset in both CTAs.  Per
+// 128-K stage each SM moves 16 KB of S, 2 KB of metadata and BN/2*256 B of X
+// for an M=256 MMA: half the operand bytes per MMA cycle of the 1-SM tile.
+//
+// Warps: 0 TMA producer, 1 MMA issue (leader only), 2..5 epilogue, 6 metadata.
+// The metadata warp permutes each stage's metadata tile ahead of the MMA warp
+// and then signals the leader's ready[s]: in the leader with an arrive that
+// also expects 16 transaction bytes, in the follower with a 16-byte bulk copy
+// into the leader that completes those bytes.  The MMA warp therefore only
+// waits for ready[s] and issues.
+//
+// Accumulators: two TMEM buffers of BN columns.  When 2*BN + 4 exceeds the 512
+// columns (BN = 256) they overlap by OVL columns at the end of buffer 0 / start
+// of buffer 1, and the metadata takes the last 4 columns.  The epilogue drains
+// the overlapping 32-column chunk first and reports it (acc_ovl), so the next
+// tile's MMAs wait only for that chunk; acc_empty reports the whole buffer.
+//
+// Handshakes (all waits bounded):
+//   full[s]      local TMA completion (each CTA)
+//   ready[s]     leader: its metadata warp (count 1) + follower's 16 bytes
+//   empty[s]     leader's commit, multicast to both CTAs
+//   acc_full[b]  leader's commit, multicast
+//   acc_ovl[b]   8 epilogue warps (both CTAs) -> leader: overlap chunk drained
+//   acc_empty[b] 8 epilogue warps (both CTAs) -> leader: buffer drained
+template <int BN>
+struct Cfg2 {
+    static constexpr int HALF_N = BN / 2;               // tokens staged per CTA
+    static constexpr int A_BYTES = BM * 64 * 2;         // 16 KB of packed values
+    static constexpr int B_HALF = HALF_N * 64 * 2;      // one 128-byte-wide panel of this CTA's tokens
+    static constexpr int B_BYTES = 2 * B_HALF;
+    static constexpr int E_BYTES = BM * BK / 8;         // 2 KB of metadata
+    static constexpr int STAGE = ((A_BYTES + B_BYTES + E_BYTES + 1023) / 1024) * 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t OVL = (2 * BN + 4 > 512) ? (2 * BN + 4 - 512) : 0;
+    static constexpr uint32_t ACC1 = BN - OVL;          // column of accumulator 1
+    static constexpr uint32_t ECOL = (OVL > 0) ? 508 : 2 * BN;
+    static constexpr int OUT_COLS = 32;
+    static constexpr int OUT_BYTES = OUT_COLS * BM * 2; // one 32-token chunk of this CTA's rows
+    static constexpr int NS_FIT = (232448 - 2 * OUT_BYTES - 3072) / STAGE;
+    static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
+    static constexpr int RING = NS * STAGE;
+    static constexpr int BAR_OFF = RING + 2 * OUT_BYTES;
+    static constexpr int DUMMY_OFF = BAR_OFF + 512;     // 16-byte signal slots, one per stage
+    static constexpr int SMEM = DUMMY_OFF + 16 * 8 + 16 + 1024;
+    static_assert(NS >= 2, "need at least two stages");
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(ECOL + 4 <= TMEM_COLS && ACC1 + BN <= ECOL, "TMEM budget");
+    static_assert(OVL <= 32, "overlap must fit in one drained chunk");
+};
+
+constexpr int kThreads2 = 224;  // 7 warps
+
+template <int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
+    tc2_forward_kernel(const __grid_constant__ CUtensorMap tm_vals, const __grid_constant__ CUtensorMap tm_meta,
+                       const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_u,
+                       const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_y,
+                       const Params prm) {
+    using C = Cfg2<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *empty = full + C::NS;
+    uint64_t *ready = empty + C::NS;
+    uint64_t *acc_full = ready + C::NS;
+    uint64_t *acc_ovl = acc_full + 2;
+    uint64_t *acc_empty = acc_ovl + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    volatile uint32_t *fail = tmem_slot + 1;
+    uint8_t *dummy = smem + C::DUMMY_OFF;   // NS signal slots + 1 source slot
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+    const int nstages = prm.nk + prm.nlr;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&ready[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_ovl[b], 8);
+            mbar_init(&acc_empty[b], 8);
+        }
+        *fail = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    if (threadIdx.x == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_vals)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_meta)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
+    }
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs' barriers initialised and TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (each CTA)
+        if (lane == 0) {
+            uint32_t s = 0, ph = 0;
+            for (int tile = pair; tile < prm.n_tiles && !*fail; tile += npairs) {
+                const int d0 = (tile / prm.n_ttiles) * (2 * BM) + (int)rank * BM;
+                const int tok0 = (tile % prm.n_ttiles) * BN + (int)rank * C::HALF_N;
+                for (int ks = 0; ks < nstages; ++ks) {
+                    if (!mbar_wait_cluster(&empty[s], ph ^ 1)) {
+                        *fail = 1;
+                        atomicOr(&g_tc_error, 16u);
+                        break;
+                    }
+                    uint8_t *st = smem + s * C::STAGE;
+                    const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES),
+                                   e = smem_u32(st + C::A_BYTES + C::B_BYTES);
+                    if (ks < prm.nk) {
+                        mbar_expect_tx(&full[s], C::A_BYTES + C::B_BYTES + C::E_BYTES);
+                        tma_load_2d(&tm_vals, a, &full[s], ks * 64, d0);
+                        tma_load_2d(&tm_x, b, &full[s], ks * BK, tok0);
+                        tma_load_2d(&tm_x, b + C::B_HALF, &full[s], ks * BK + 64, tok0);
+                        tma_load_2d(&tm_meta, e, &full[s], ks * (BK / 8), d0);
+                    } else {
+                        const int j = ks - prm.nk;
+                        mbar_expect_tx(&full[s], C::A_BYTES + C::B_HALF);
+                        tma_load_2d(&tm_u, a, &full[s], j * 64, d0);
+                        tma_load_2d(&tm_t, b, &full[s], j * 64, tok0);
+                    }
+                    if (++s == (uint32_t)C::NS) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+            }
+        }
+    } else if (warp == 6) {
+        // ------------------------------------------------------------ metadata warp (each CTA)
+        const uint32_t src_slot = smem_u32(dummy + 16 * C::NS);
+        uint32_t s = 0, ph = 0;
+        for (int tile = pair; tile < prm.n_tiles && !*fail; tile += npairs) {
+            bool ok = true;
+            for (int ks = 0; ks < nstages; ++ks) {
+                if (!mbar_wait(&full[s], ph)) {
+                    ok = false;
+                    break;
+                }
+                if (ks < prm.nk) {
+                    permute_meta_tile(smem + s * C::STAGE + C::A_BYTES + C::B_BYTES, lane);
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    if (leader) {
+                        mbar_expect_tx(&ready[s], 16);
+                    } else {
+                        bulk_signal_peer(mapa_shared(smem_u32(dummy + 16 * s), 0), src_slot,
+                                         mapa_shared(smem_u32(&ready[s]), 0));
+                    }
+                }
+                __syncwarp();
+                if (++s == (uint32_t)C::NS) {
+                    s = 0;
+                    ph ^= 1;
+                }
+            }
+            if (!ok) {
+                *fail = 1;
+                atomicOr(&g_tc_error, 256u);
+                break;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issue (leader, one thread)
+        if (leader && lane == 0) {
+            constexpr uint32_t kIdescSp = idesc_bf16(2 * BM, BN, true);
+            constexpr uint32_t kIdescDense = idesc_bf16(2 * BM, BN, false);
+            const uint32_t e_tmem = tmem_base + C::ECOL;
+            uint32_t s = 0, ph = 0;
+            int it = 0;
+            for (int tile = pair; tile < prm.n_tiles && !*fail; tile += npairs, ++it) {
+                const int buf = it & 1;
+                const uint32_t use = (uint32_t)(it >> 1);
+                bool ok = mbar_wait_cluster(&acc_empty[buf], (use & 1) ^ 1);
+                if (ok && C::OVL > 0 && it > 0) ok = mbar_wait_cluster(&acc_ovl[buf ^ 1], ((uint32_t)((it - 1) >> 1)) & 1);
+                if (!ok) {
+                    *fail = 1;
+                    atomicOr(&g_tc_error, 32u);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (buf ? C::ACC1 : 0u);
+                for (int ks = 0; ks < nstages; ++ks) {
+                    if (!mbar_wait_cluster(&ready[s], ph)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint8_t *st = smem + s * C::STAGE;
+                    const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES);
+                    if (ks < prm.nk) {
+                        tmem_cp_pair_128x128b(e_tmem, smem_desc(smem_u32(st + C::A_BYTES + C::B_BYTES), 0, 128, kLayoutNone));
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const uint64_t adesc = desc_sw128(a + 32 * c);
+                            const uint64_t bdesc = desc_sw128(b + (c >> 1) * C::B_HALF + (c & 1) * 64);
+                            mma_sp_pair(d_tmem, adesc, bdesc, e_tmem + (uint32_t)(c & 2), kIdescSp | (uint32_t)(c & 1),
+                                        (ks | c) != 0);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            mma_dense_pair(d_tmem, desc_sw128(a + 32 * c), desc_sw128(b + 32 * c), kIdescDense, 1u);
+                    }
+                    mma_commit_pair(&empty[s]);
+                    if (++s == (uint32_t)C::NS) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                if (!ok) {
+                    *fail = 1;
+                    atomicOr(&g_tc_error, 64u);
+                    break;
+                }
+                mma_commit_pair(&acc_full[buf]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (each CTA, its 128 rows)
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const bool store_thread = (warp == 2 && lane == 0);
+        uint8_t *stage_out = smem + C::RING;
+        const uint32_t ovl_leader0 = mapa_shared(smem_u32(&acc_ovl[0]), 0);
+        const uint32_t empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
+        constexpr int NQ = BN / 32;
+        uint32_t chunk = 0;
+        int it = 0;
+        for (int tile = pair; tile < prm.n_tiles && !*fail; tile += npairs, ++it) {
+            const int d0 = (tile / prm.n_ttiles) * (2 * BM) + (int)rank * BM;
+            const int tok0 = (tile % prm.n_ttiles) * BN;
+            const int buf = it & 1;
+            const uint32_t use = (uint32_t)(it >> 1);
+            if (!mbar_wait_cluster(&acc_full[buf], use & 1)) {
+                *fail = 1;
+                atomicOr(&g_tc_error, 128u);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t acc_col = buf ? C::ACC1 : 0u;
+            // The chunk holding the overlap goes first: the last chunk of
+            // buffer 0, the first chunk of buffer 1.
+            const int first_q = (C::OVL > 0 && buf == 0) ? NQ - 1 : 0;
+#pragma unroll 1
+            for (int i = 0; i < NQ; ++i) {
+                const int q = (first_q + i) % NQ;
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc_col + (uint32_t)(q * 32), v);
+                if (i == 0 && C::OVL > 0) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote_relaxed(ovl_leader0 + (uint32_t)(buf * sizeof(uint64_t)));
+                }
+                if (i == NQ - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote_relaxed(empty_leader0 + (uint32_t)(buf * sizeof(uint64_t)));
+                }
+                if (tok0 + q * C::OUT_COLS >= prm.M) continue;  // uniform across the epilogue warps
+                const uint32_t sb = chunk & 1;
+                if (store_thread) bulk_wait_read1();
+                named_bar_sync(1, 128);
+                uint16_t *out = reinterpret_cast<uint16_t *>(stage_out + sb * C::OUT_BYTES);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) out[j * BM + row] = f32_to_bf16_bits(__uint_as_float(v[j]));
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (store_thread) {
+                    tma_store_2d(&tm_y, smem_u32(out), d0, tok0 + q * C::OUT_COLS);
+                    bulk_commit();
+                }
+                ++chunk;
+            }
+        }
+        if (store_thread) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    cluster_sync_all();  // the pair's MMAs, signals and stores are done before TMEM is freed
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
     }
 }
 
@@ -473,43 +641,97 @@ bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN>
-cudaError_t launch(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta, int64_t d_out,
-                   int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r, uint16_t *Y,
-                   cudaStream_t stream) {
-    using C = Cfg<BN>;
-    CUtensorMap m_vals, m_meta, m_x, m_u, m_t, m_y;
-    memset(&m_u, 0, sizeof m_u);
-    memset(&m_t, 0, sizeof m_t);
-    const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    bool ok = make_map(&m_vals, BF16, vals, d_in / 2, d_out, d_in, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map(&m_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, d_in / 8, d_out, d_in / 8, 16, BM,
-                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
-              make_map(&m_x, BF16, X, d_in, M, d_in * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map(&m_y, BF16, Y, d_out, M, d_out * 2, BM, C::OUT_COLS, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (ok && r > 0)
-        ok = make_map(&m_u, BF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_map(&m_t, BF16, T16, r, M, r * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (!ok) return cudaErrorInvalidValue;
-
+template <int BN, bool kSparse>
+cudaError_t run(const CUtensorMap &m_a, const CUtensorMap &m_meta, const CUtensorMap &m_x, const CUtensorMap &m_u,
+                const CUtensorMap &m_t, const CUtensorMap &m_out, int64_t rows, int64_t M, int nk, int nlr,
+                cudaStream_t stream) {
+    using C = Cfg<BN, kSparse>;
     Params prm;
     prm.M = (int32_t)M;
-    prm.d_out = (int32_t)d_out;
-    prm.d_in = (int32_t)d_in;
-    prm.r = (int32_t)r;
-    prm.n_dtiles = (int32_t)((d_out + BM - 1) / BM);
-    const int64_t n_ttiles = (M + BN - 1) / BN;
-    prm.n_tiles = (int32_t)(prm.n_dtiles * n_ttiles);
-    prm.nk = (int32_t)(d_in / BK);
-    prm.nlr = (int32_t)((r + 63) / 64);
-
+    prm.n_ttiles = (int32_t)((M + BN - 1) / BN);
+    prm.n_tiles = (int32_t)(((rows + BM - 1) / BM) * prm.n_ttiles);
+    prm.nk = nk;
+    prm.nlr = nlr;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaError_t err = cudaFuncSetAttribute(tc_forward_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t err =
+        cudaFuncSetAttribute(tc_forward_kernel<BN, kSparse>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (err != cudaSuccess) return err;
     const int grid = prm.n_tiles < sms ? prm.n_tiles : sms;
-    tc_forward_kernel<BN><<<grid, kThreads, C::SMEM, stream>>>(m_vals, m_meta, m_x, m_u, m_t, m_y, prm);
+    tc_forward_kernel<BN, kSparse><<<grid, kThreads, C::SMEM, stream>>>(m_a, m_meta, m_x, m_u, m_t, m_out, prm);
+    return cudaGetLastError();
+}
+
+constexpr auto kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+
+template <int BN>
+cudaError_t launch_sparse(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta, int64_t d_out,
+                          int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r, uint16_t *Y,
+                          cudaStream_t stream) {
+    CUtensorMap m_vals, m_meta, m_x, m_u, m_t, m_y;
+    memset(&m_u, 0, sizeof m_u);
+    memset(&m_t, 0, sizeof m_t);
+    bool ok = make_map(&m_vals, kBF16, vals, d_in / 2, d_out, d_in, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&m_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, d_in / 8, d_out, d_in / 8, 16, BM,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map(&m_x, kBF16, X, d_in, M, d_in * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&m_y, kBF16, Y, d_out, M, d_out * 2, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (ok && r > 0)
+        ok = make_map(&m_u, kBF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+             make_map(&m_t, kBF16, T16, r, M, r * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
+    return run<BN, true>(m_vals, m_meta, m_x, m_u, m_t, m_y, d_out, M, (int)(d_in / BK), (int)((r + 63) / 64),
+                         stream);
+}
+
+// T^T = V X^T: A = V (r rows, padded to 128 by TMA zero fill), B = X tile; the
+// epilogue stores D (r lanes x tokens) as T [M, r] row-major, the layout the
+// rank stages of the sparse kernel read.
+template <int BN>
+cudaError_t launch_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in, int64_t r, uint16_t *T16,
+                           cudaStream_t stream) {
+    CUtensorMap m_v, m_x, m_t, m_none;
+    memset(&m_none, 0, sizeof m_none);
+    bool ok = make_map(&m_v, kBF16, V, d_in, r, d_in * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&m_x, kBF16, X, d_in, M, d_in * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&m_t, kBF16, T16, r, M, r * 2, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return cudaErrorInvalidValue;
+    return run<BN, false>(m_v, m_none, m_x, m_none, m_none, m_t, r, M, (int)(d_in / 64), 0, stream);
+}
+
+
+template <int BN>
+cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
+                               int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
+                               uint16_t *Y, cudaStream_t stream) {
+    using C = Cfg2<BN>;
+    CUtensorMap m_vals, m_meta, m_x, m_u, m_t, m_y;
+    memset(&m_u, 0, sizeof m_u);
+    memset(&m_t, 0, sizeof m_t);
+    bool ok = make_map(&m_vals, kBF16, vals, d_in / 2, d_out, d_in, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&m_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, d_in / 8, d_out, d_in / 8, 16, BM,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map(&m_x, kBF16, X, d_in, M, d_in * 2, 64, C::HALF_N, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&m_y, kBF16, Y, d_out, M, d_out * 2, BM, C::OUT_COLS, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (ok && r > 0)
+        ok = make_map(&m_u, kBF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+             make_map(&m_t, kBF16, T16, r, M, r * 2, 64, C::HALF_N, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
+    Params prm;
+    prm.M = (int32_t)M;
+    prm.n_ttiles = (int32_t)((M + BN - 1) / BN);
+    prm.n_tiles = (int32_t)(((d_out + 2 * BM - 1) / (2 * BM)) * prm.n_ttiles);
+    prm.nk = (int32_t)(d_in / BK);
+    prm.nlr = (int32_t)((r + 63) / 64);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t err = cudaFuncSetAttribute(tc2_forward_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (err != cudaSuccess) return err;
+    const int max_pairs = sms / 2;
+    const int pairs = prm.n_tiles < max_pairs ? prm.n_tiles : max_pairs;
+    tc2_forward_kernel<BN><<<2 * pairs, kThreads2, C::SMEM, stream>>>(m_vals, m_meta, m_x, m_u, m_t, m_y, prm);
     return cudaGetLastError();
 }
 
@@ -520,7 +742,28 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
                               uint16_t *Y, cudaStream_t stream) {
     if (M <= 0) return cudaSuccess;
     if (M > INT32_MAX || d_out > INT32_MAX || d_in > INT32_MAX) return cudaErrorInvalidValue;
-    return tc::launch<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
+    // Variant: 2-SM pairs with 256-token tiles once there are enough tokens,
+    // 128-token pair tiles below that.  SLR_TC_KERNEL=1sm|2sm128|2sm256 forces
+    // one (used by the tests and for A/B measurements).
+    const char *force = getenv("SLR_TC_KERNEL");
+    if (force != nullptr) {
+        if (strcmp(force, "1sm") == 0) return tc::launch_sparse<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
+        if (strcmp(force, "2sm128") == 0)
+            return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
+        if (strcmp(force, "2sm256") == 0)
+            return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
+    }
+    if (M >= 192) return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
+    return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
+}
+
+cudaError_t launch_tc_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in, int64_t r,
+                              uint16_t *T16, cudaStream_t stream) {
+    if (M <= 0 || r <= 0) return cudaSuccess;
+    if (M > INT32_MAX || d_in > INT32_MAX || r > INT32_MAX) return cudaErrorInvalidValue;
+    if (M >= 4096) return tc::launch_project<128>(X, M, V, d_in, r, T16, stream);
+    if (M >= 1024) return tc::launch_project<64>(X, M, V, d_in, r, T16, stream);
+    return tc::launch_project<32>(X, M, V, d_in, r, T16, stream);
 }
 
 cudaError_t read_and_clear_kernel_error(unsigned *code) {

@@ -12,6 +12,11 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
                               int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
                               uint16_t *Y, cudaStream_t stream);
 
+// T = X V^T on the tensor cores, written as bf16 [M, r] (dense tcgen05 mode of
+// the same kernel).  Requires d_in % 64 == 0, r % 8 == 0.
+cudaError_t launch_tc_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in, int64_t r,
+                              uint16_t *T16, cudaStream_t stream);
+
 // Reads and clears the device-side error word the tensor-core kernel sets when
 // a bounded wait expires (0 = none).  Synchronises the device.
 cudaError_t read_and_clear_kernel_error(unsigned *code);

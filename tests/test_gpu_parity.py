@@ -178,3 +178,54 @@ def test_forward_matches_between_paths():
 
 def test_no_kernel_timeouts():
     slr.check_kernel_error()
+
+
+VARIANTS = ["1sm", "2sm128", "2sm256"]
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("d_out,d_in,r,M", [
+    (200, 256, 16, 37),      # ragged output rows (the pair's second CTA is partly outside d_out)
+    (136, 384, 8, 129),      # r = 8; M just over a 128-token tile
+    (512, 640, 128, 300),    # several pair tiles, two rank stages, ragged token tile
+    (1024, 1024, 256, 513),  # four rank stages; more tiles than one wave of pairs
+])
+def test_forward_tensor_variants(variant, d_out, d_in, r, M, monkeypatch):
+    """Every tensor-core kernel variant (1-SM, 2-SM with 128- and 256-token
+    tiles) against the oracle, selected through SLR_TC_KERNEL."""
+    monkeypatch.setenv("SLR_TC_KERNEL", variant)
+    seed = d_out * 7 + d_in + r + M
+    X = synth.activations_bf16(M, d_in, seed, seed + 9)
+    W = synth.gaussian_bf16((d_out, d_in), 0.02, seed + 1)
+    vals, meta = oracle.pack_2to4(W)
+    U = synth.gaussian_bf16((d_out, r), 0.5, seed + 2)
+    V = synth.gaussian_bf16((r, d_in), 0.5 / np.sqrt(r), seed + 3)
+    Y = slr.forward(to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U), to_dev(V), path="tensor")
+    torch.cuda.synchronize()
+    slr.check_kernel_error()
+    rows = sample_indices(M, 64, seed)
+    Yref, Bref = oracle.forward(X, vals, meta, U, V, rows=rows)
+    check_forward(from_dev(Y)[rows], Yref, Bref, f"{variant} {d_out}x{d_in} r={r} M={M}")
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_forward_tensor_variants_prefill(variant, monkeypatch):
+    """The gate/up prefill shape (14336 x 4096, r = 64, M = 2048) on each variant."""
+    monkeypatch.setenv("SLR_TC_KERNEL", variant)
+    _forward_case(3, "gate_up", 2048, "tensor")
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_forward_tensor_variants_one_hot(variant, monkeypatch):
+    """Exact metadata decoding on each variant (U = 0, X = identity rows)."""
+    monkeypatch.setenv("SLR_TC_KERNEL", variant)
+    d_out, d_in = 640, 256
+    W = synth.gaussian_bf16((d_out, d_in), 0.02, 6161)
+    vals, meta = oracle.pack_2to4(W)
+    S = oracle.unpack_2to4(vals, meta, d_in)
+    X = np.zeros((d_in, d_in), dtype=np.uint16)
+    X[np.arange(d_in), np.arange(d_in)] = 0x3F80
+    U = np.zeros((d_out, 8), dtype=np.uint16)
+    V = synth.gaussian_bf16((8, d_in), 1.0, 6162)
+    Y = slr.forward(to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U), to_dev(V), path="tensor")
+    np.testing.assert_array_equal(bits_to_f64(from_dev(Y)), bits_to_f64(np.ascontiguousarray(S.T)))
