@@ -95,7 +95,7 @@ cudaError_t run_project(const void *X, int64_t M, const void *V, int64_t d_in, i
 
 // Stage 2: Y = X S^T + T U^T with T read from the workspace.
 cudaError_t run_combine(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out, int64_t d_in,
-                        const void *U, int64_t r, void *Y, const void *workspace, slr_path p,
+                        const void *U, int64_t r, void *Y, const void *workspace, slr_path p, bool after_projection,
                         cudaStream_t stream) {
     const uint16_t *x = static_cast<const uint16_t *>(X);
     const uint16_t *v = static_cast<const uint16_t *>(vals);
@@ -104,9 +104,9 @@ cudaError_t run_combine(const void *X, int64_t M, const void *vals, const void *
     uint16_t *y = static_cast<uint16_t *>(Y);
     if (p == SLR_PATH_DECODE)
         return launch_decode_forward(x, M, v, m, d_out, d_in, u, r > 0 ? static_cast<const float *>(workspace) : nullptr,
-                                     r, y, stream);
+                                     r, y, after_projection, stream);
     return launch_tc_forward(x, M, v, m, d_out, d_in, u, r > 0 ? static_cast<const uint16_t *>(workspace) : nullptr,
-                             r, y, stream);
+                             r, y, after_projection, stream);
 }
 
 slr_status forward_impl(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out,
@@ -117,7 +117,7 @@ slr_status forward_impl(const void *X, int64_t M, const void *vals, const void *
                                    true, true, true, &p);
     if (st != SLR_OK || M == 0) return st;
     cudaError_t err = run_project(X, M, V, d_in, r, workspace, p, stream);
-    if (err == cudaSuccess) err = run_combine(X, M, vals, meta, d_out, d_in, U, r, Y, workspace, p, stream);
+    if (err == cudaSuccess) err = run_combine(X, M, vals, meta, d_out, d_in, U, r, Y, workspace, p, true, stream);
     return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
 }
 
@@ -207,7 +207,7 @@ slr_status slr_forward_combine(const void *X, int64_t M, const void *vals, const
     const slr_status st = slr::validate(X, M, vals, meta, d_out, d_in, U, nullptr, r, Y, workspace, workspace_bytes,
                                         path, true, true, false, &p);
     if (st != SLR_OK || M == 0) return st;
-    return slr::run_combine(X, M, vals, meta, d_out, d_in, U, r, Y, workspace, p,
+    return slr::run_combine(X, M, vals, meta, d_out, d_in, U, r, Y, workspace, p, false,
                             reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SLR_OK
                : SLR_ERR_CUDA;

@@ -42,9 +42,12 @@ cudaError_t launch_lowrank_project(const uint16_t *X, int64_t M, const uint16_t 
                                    int64_t r, float *T32, uint16_t *T16, cudaStream_t stream);
 
 // Small-M streaming forward: Y = X S^T + T U^T with T (fp32 [M, r]) precomputed.
+// after_projection: the projection kernel that writes T32 is the kernel
+// launched immediately before on `stream` (enables programmatic dependent
+// launch; must be false otherwise).
 cudaError_t launch_decode_forward(const uint16_t *X, int64_t M, const uint16_t *vals,
                                   const uint8_t *meta, int64_t d_out, int64_t d_in,
                                   const uint16_t *U, const float *T32, int64_t r, uint16_t *Y,
-                                  cudaStream_t stream);
+                                  bool after_projection, cudaStream_t stream);
 
 }  // namespace slr

@@ -19,7 +19,12 @@ namespace slr {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kUnroll = 4;
+constexpr int kBlocksPerSm = 4;
+// 16-byte chunks in flight per lane: a whole 4096-wide row per round trip for
+// one or two tokens; fewer with more tokens (their accumulators and X loads
+// need the registers).
+template <int MT>
+__host__ __device__ constexpr int unroll_for() { return MT == 1 ? 8 : 4; }
 
 // One group of four: kept values (low = lower index) in vv, nibble nib, the
 // four X values of the group in x01 (elements 0,1) and x23 (elements 2,3).
@@ -42,8 +47,10 @@ __device__ __forceinline__ float chunk_fma(uint4 v, uint32_t m16, uint4 xa, uint
     return acc;
 }
 
+// 4 resident CTAs per SM (<= 64 registers): 148 x 4 x 8 warps cover the 4096
+// rows of a Llama-3-8B projection in one wave.
 template <int MT>
-__global__ void __launch_bounds__(kWarps * 32) decode_forward_kernel(
+__global__ void __launch_bounds__(kWarps * 32, 4) decode_forward_kernel(
     const uint16_t *__restrict__ X, int64_t M, const uint16_t *__restrict__ vals,
     const uint8_t *__restrict__ meta, int64_t d_out, int64_t d_in, const uint16_t *__restrict__ U,
     const float *__restrict__ T32, int64_t r, uint16_t *__restrict__ Y) {
@@ -53,6 +60,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_forward_kernel(
     const int64_t chunks = d_in / 16;
     const int64_t nwarps = (int64_t)gridDim.x * kWarps;
     const uint16_t *xbase = X + m0 * d_in;
+    constexpr int kUnroll = unroll_for<MT>();
 
     for (int64_t row = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); row < d_out; row += nwarps) {
         float acc[MT];
@@ -91,6 +99,10 @@ __global__ void __launch_bounds__(kWarps * 32) decode_forward_kernel(
         }
 
         // Rank-r term: lanes split k, products land in the same partial sums.
+        // T comes from the projection kernel, which may still be running when
+        // this kernel starts (programmatic dependent launch): wait for it here,
+        // after the weight stream.
+        if (r > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
         for (int64_t k = lane; k < r; k += 32) {
             const float u = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(U) + row * r + k) << 16);
 #pragma unroll
@@ -118,28 +130,42 @@ __global__ void __launch_bounds__(kWarps * 32) decode_forward_kernel(
 template <int MT>
 cudaError_t launch_mt(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta, int64_t d_out,
                       int64_t d_in, const uint16_t *U, const float *T32, int64_t r, uint16_t *Y,
-                      cudaStream_t stream) {
+                      bool after_projection, cudaStream_t stream) {
     const int64_t tblocks = (M + MT - 1) / MT;
     if (tblocks > 65535) return cudaErrorInvalidConfiguration;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int64_t blocks = (d_out + kWarps - 1) / kWarps;
-    const int64_t cap = (int64_t)sms * 8;
+    const int64_t cap = (int64_t)sms * kBlocksPerSm;
     if (blocks > cap) blocks = cap;
-    dim3 grid((unsigned)blocks, (unsigned)tblocks);
-    decode_forward_kernel<MT><<<grid, kWarps * 32, 0, stream>>>(X, M, vals, meta, d_out, d_in, U, T32, r, Y);
-    return cudaGetLastError();
+    // Directly after the projection kernel on the same stream it is launched
+    // as a programmatic dependent: it may start streaming S before T is
+    // complete (it waits before reading T).  Otherwise it is an ordinary
+    // launch (a programmatic launch would also overlap an unrelated
+    // preceding kernel, e.g. the producer of X).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks, (unsigned)tblocks);
+    cfg.blockDim = dim3(kWarps * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_projection ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, decode_forward_kernel<MT>, X, M, vals, meta, d_out, d_in, U, T32, r, Y);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_forward(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                   int64_t d_out, int64_t d_in, const uint16_t *U, const float *T32, int64_t r,
-                                  uint16_t *Y, cudaStream_t stream) {
-    if (M <= 1) return launch_mt<1>(X, M, vals, meta, d_out, d_in, U, T32, r, Y, stream);
-    if (M <= 2) return launch_mt<2>(X, M, vals, meta, d_out, d_in, U, T32, r, Y, stream);
-    if (M <= 4) return launch_mt<4>(X, M, vals, meta, d_out, d_in, U, T32, r, Y, stream);
-    return launch_mt<8>(X, M, vals, meta, d_out, d_in, U, T32, r, Y, stream);
+                                  uint16_t *Y, bool after_projection, cudaStream_t stream) {
+    const bool pdl = after_projection && r > 0;
+    if (M <= 1) return launch_mt<1>(X, M, vals, meta, d_out, d_in, U, T32, r, Y, pdl, stream);
+    if (M <= 2) return launch_mt<2>(X, M, vals, meta, d_out, d_in, U, T32, r, Y, pdl, stream);
+    if (M <= 4) return launch_mt<4>(X, M, vals, meta, d_out, d_in, U, T32, r, Y, pdl, stream);
+    return launch_mt<8>(X, M, vals, meta, d_out, d_in, U, T32, r, Y, pdl, stream);
 }
 
 }  // namespace slr

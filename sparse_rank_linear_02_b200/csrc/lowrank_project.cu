@@ -36,6 +36,9 @@ __global__ void __launch_bounds__(kThreads) lowrank_project_kernel(const uint16_
                                                                    int64_t d_in, int64_t r,
                                                                    float *__restrict__ T32,
                                                                    uint16_t *__restrict__ T16) {
+    // Let the dependent streaming kernel launch now; it only reads T after
+    // its own griddepcontrol.wait, which waits for this grid to complete.
+    asm volatile("griddepcontrol.launch_dependents;");
     const int64_t k = blockIdx.x;
     const int64_t m0 = (int64_t)blockIdx.y * kTokens;
     const int nt = (int)((M - m0) < kTokens ? (M - m0) : kTokens);

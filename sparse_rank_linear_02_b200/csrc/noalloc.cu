@@ -98,6 +98,6 @@ extern "C" slr_status slr_forward_decode_noalloc(const void *X, int64_t M, const
     if (err == cudaSuccess)
         err = slr::launch_decode_forward(x, M, static_cast<const uint16_t *>(vals), static_cast<const uint8_t *>(meta),
                                          d_out, d_in, static_cast<const uint16_t *>(U), r > 0 ? T : nullptr, r,
-                                         static_cast<uint16_t *>(Y), s);
+                                         static_cast<uint16_t *>(Y), true, s);
     return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
 }

@@ -424,6 +424,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         // ------------------------------------------------------------ producer (each CTA)
         if (lane == 0) {
             uint32_t s = 0, ph = 0;
+            bool t_ready = false;
             for (int tile = pair; tile < prm.n_tiles && !*fail; tile += npairs) {
                 const int d0 = (tile / prm.n_ttiles) * (2 * BM) + (int)rank * BM;
                 const int tok0 = (tile % prm.n_ttiles) * BN + (int)rank * C::HALF_N;
@@ -444,6 +445,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
                         tma_load_2d(&tm_meta, e, &full[s], ks * (BK / 8), d0);
                     } else {
                         const int j = ks - prm.nk;
+                        if (!t_ready) {
+                            // T comes from the projection kernel, which may still
+                            // be running (programmatic dependent launch).
+                            asm volatile("griddepcontrol.wait;" ::: "memory");
+                            t_ready = true;
+                        }
                         mbar_expect_tx(&full[s], C::A_BYTES + C::B_HALF);
                         tma_load_2d(&tm_u, a, &full[s], j * 64, d0);
                         tma_load_2d(&tm_t, b, &full[s], j * 64, tok0);
@@ -704,7 +711,7 @@ cudaError_t launch_project(const uint16_t *X, int64_t M, const uint16_t *V, int6
 template <int BN>
 cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
-                               uint16_t *Y, cudaStream_t stream) {
+                               uint16_t *Y, bool after_projection, cudaStream_t stream) {
     using C = Cfg2<BN>;
     CUtensorMap m_vals, m_meta, m_x, m_u, m_t, m_y;
     memset(&m_u, 0, sizeof m_u);
@@ -731,15 +738,250 @@ cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *val
     if (err != cudaSuccess) return err;
     const int max_pairs = sms / 2;
     const int pairs = prm.n_tiles < max_pairs ? prm.n_tiles : max_pairs;
-    tc2_forward_kernel<BN><<<2 * pairs, kThreads2, C::SMEM, stream>>>(m_vals, m_meta, m_x, m_u, m_t, m_y, prm);
-    return cudaGetLastError();
+    // Directly after the projection kernel on this stream: programmatic
+    // dependent launch (the producer waits before it loads T).  Otherwise an
+    // ordinary launch, which must not overlap an unrelated preceding kernel.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(kThreads2);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (after_projection && r > 0) ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, tc2_forward_kernel<BN>, m_vals, m_meta, m_x, m_u, m_t, m_y, prm);
+}
+
+
+// =====================================================================================
+// Rank projection T = X V^T with split K (the first factor of the low-rank term,
+// LoSparse section 3.2).  A cluster of KS CTAs (KS <= 8) owns 128 tokens; CTA
+// rank q runs the q-th slice of the d_in stages with A = X tile (128 tokens,
+// M = 128) and B = V (N = RN >= r, rows past r zero-filled by TMA), so its TMEM
+// holds a partial T tile (lane = token, column = rank index).  The epilogue
+// warps write the partial to shared memory (fp32, padded rows), the cluster
+// synchronises, and each CTA sums its 128/KS tokens over all KS partials through
+// distributed shared memory and writes them to T [M, r] in bf16.  One kernel, no
+// atomics, no scratch outside shared memory.
+template <int RN>
+struct CfgP {
+    static constexpr int A_BYTES = BM * 64 * 2;          // 16 KB: 128 tokens x 64 K
+    static constexpr int B_BYTES = RN * 64 * 2;          // RN rows of V x 64 K
+    static constexpr int STAGE = ((A_BYTES + B_BYTES + 1023) / 1024) * 1024;
+    static constexpr int PROW = RN + 4;                  // padded fp32 row of the partial tile
+    static constexpr int P_BYTES = BM * PROW * 4;
+    // Up to ~110 KB of ring so that two CTAs fit on an SM when RN <= 128.
+    static constexpr int NS_FIT = (RN <= 128 ? 112640 : 230400) / STAGE;
+    static constexpr int NS = NS_FIT > 8 ? 8 : (NS_FIT < 2 ? 2 : NS_FIT);
+    static constexpr int RING = NS * STAGE;
+    static constexpr int BAR_OFF = (RING > P_BYTES ? RING : P_BYTES);
+    static constexpr int SMEM = BAR_OFF + 256 + 1024;
+    static constexpr uint32_t TMEM_COLS = pow2_at_least(RN);
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(RN % 16 == 0 && RN <= 256, "MMA N");
+};
+
+template <int RN>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_project_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_v,
+                      uint16_t *__restrict__ T16, int32_t M, int32_t r, int32_t nk_total) {
+    using C = CfgP<RN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *empty = full + C::NS;
+    uint64_t *acc_full = empty + C::NS;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    volatile uint32_t *fail = tmem_slot + 1;
+    float *part = reinterpret_cast<float *>(smem);      // reuses the ring after the K loop
+
+    // The fused forward kernel that consumes T may launch now (it waits for
+    // this grid before its first load of T).
+    asm volatile("griddepcontrol.launch_dependents;");
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    uint32_t ks_n, ks_q;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(ks_n));
+    ks_q = cluster_ctarank();
+    const int tile = blockIdx.x / (int)ks_n;
+    const int tok0 = tile * BM;
+    const int k_begin = (int)(((int64_t)nk_total * ks_q) / ks_n);
+    const int k_end = (int)(((int64_t)nk_total * (ks_q + 1)) / ks_n);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        *fail = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t s = 0, ph = 0;
+            for (int ks = k_begin; ks < k_end; ++ks) {
+                if (!mbar_wait(&empty[s], ph ^ 1)) {
+                    *fail = 1;
+                    atomicOr(&g_tc_error, 512u);
+                    break;
+                }
+                uint8_t *st = smem + s * C::STAGE;
+                mbar_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
+                tma_load_2d(&tm_x, smem_u32(st), &full[s], ks * 64, tok0);
+                tma_load_2d(&tm_v, smem_u32(st + C::A_BYTES), &full[s], ks * 64, 0);
+                if (++s == (uint32_t)C::NS) {
+                    s = 0;
+                    ph ^= 1;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t kIdesc = idesc_bf16(BM, RN, false);
+            uint32_t s = 0, ph = 0;
+            bool ok = true;
+            for (int ks = k_begin; ks < k_end; ++ks) {
+                if (!mbar_wait(&full[s], ph)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint8_t *st = smem + s * C::STAGE;
+                const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    mma_dense(tmem_base, desc_sw128(a + 32 * c), desc_sw128(b + 32 * c), kIdesc, (ks > k_begin) || c);
+                mma_commit(&empty[s]);
+                if (++s == (uint32_t)C::NS) {
+                    s = 0;
+                    ph ^= 1;
+                }
+            }
+            if (!ok) {
+                *fail = 1;
+                atomicOr(&g_tc_error, 1024u);
+            }
+            mma_commit(acc_full);  // also fires when this CTA had no stages
+        }
+    } else {
+        // epilogue: TMEM partial -> shared memory (fp32); an empty K slice
+        // contributes zeros
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;   // token within the tile
+        const bool have = k_end > k_begin;
+        if (mbar_wait(acc_full, 0)) {
+            tc_fence_after();
+            // 16 columns per load (RN is a multiple of 16)
+#pragma unroll 1
+            for (int q = 0; q < RN / 16; ++q) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(q * 16), v);
+                float4 *dst = reinterpret_cast<float4 *>(part + row * C::PROW + q * 16);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    dst[j] = have ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else {
+            *fail = 1;
+            atomicOr(&g_tc_error, 2048u);
+        }
+    }
+    tc_fence_before();
+    cluster_sync_all();  // every CTA's partial is in its shared memory
+
+    // Reduction: CTA q sums tokens [q*TPC, (q+1)*TPC) over the cluster's partials.
+    if (warp >= 2) {
+        const int tpc = BM / (int)ks_n;
+        const int items = tpc * (RN / 4);
+        const uint32_t part_addr = smem_u32(part);
+        for (int it = threadIdx.x - 64; it < items; it += 128) {
+            const int t = (int)ks_q * tpc + it / (RN / 4);
+            const int c = (it % (RN / 4)) * 4;
+            const uint32_t off = (uint32_t)((t * C::PROW + c) * 4);
+            // issue all remote loads before summing, so they are in flight together
+            float4 p[8];
+#pragma unroll
+            for (uint32_t q = 0; q < 8; ++q)
+                p[q] = q < ks_n ? ld_shared_cluster_v4(mapa_shared(part_addr + off, q)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 acc = p[0];
+#pragma unroll
+            for (int q = 1; q < 8; ++q) {
+                acc.x += p[q].x;
+                acc.y += p[q].y;
+                acc.z += p[q].z;
+                acc.w += p[q].w;
+            }
+            const int tok = tok0 + t;
+            if (tok < M && c < r) {
+                uint2 packed;
+                packed.x = (uint32_t)f32_to_bf16_bits(acc.x) | ((uint32_t)f32_to_bf16_bits(acc.y) << 16);
+                packed.y = (uint32_t)f32_to_bf16_bits(acc.z) | ((uint32_t)f32_to_bf16_bits(acc.w) << 16);
+                *reinterpret_cast<uint2 *>(T16 + (int64_t)tok * r + c) = packed;   // r % 8 == 0: 8-byte aligned
+            }
+        }
+    }
+    cluster_sync_all();  // no CTA leaves while its partial may still be read
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+    }
+}
+
+template <int RN>
+cudaError_t launch_project_splitk(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in, int64_t r,
+                                  uint16_t *T16, cudaStream_t stream) {
+    using C = CfgP<RN>;
+    CUtensorMap m_x, m_v;
+    if (!make_map(&m_x, kBF16, X, d_in, M, d_in * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&m_v, kBF16, V, d_in, r, d_in * 2, 64, RN, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int tiles = (int)((M + BM - 1) / BM);
+    const int nk = (int)(d_in / 64);
+    // Split K over a cluster of up to 4 CTAs (clusters of 8 large CTAs do not
+    // all fit at once), keeping the grid within about one wave.
+    int ks = 1;
+    while (ks < 4 && ks * 2 <= nk && tiles * ks * 2 <= 2 * sms) ks *= 2;
+    cudaError_t err = cudaFuncSetAttribute(tc_project_kernel<RN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles * ks));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, tc_project_kernel<RN>, m_x, m_v, T16, (int32_t)M, (int32_t)r, (int32_t)nk);
 }
 
 }  // namespace tc
 
 cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                               int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
-                              uint16_t *Y, cudaStream_t stream) {
+                              uint16_t *Y, bool after_projection, cudaStream_t stream) {
     if (M <= 0) return cudaSuccess;
     if (M > INT32_MAX || d_out > INT32_MAX || d_in > INT32_MAX) return cudaErrorInvalidValue;
     // Variant: 2-SM pairs with 256-token tiles once there are enough tokens,
@@ -749,18 +991,25 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
     if (force != nullptr) {
         if (strcmp(force, "1sm") == 0) return tc::launch_sparse<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
         if (strcmp(force, "2sm128") == 0)
-            return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
+            return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
         if (strcmp(force, "2sm256") == 0)
-            return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
+            return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     }
-    if (M >= 192) return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
-    return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
+    if (M >= 192)
+        return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+    return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
 }
 
 cudaError_t launch_tc_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in, int64_t r,
                               uint16_t *T16, cudaStream_t stream) {
     if (M <= 0 || r <= 0) return cudaSuccess;
     if (M > INT32_MAX || d_in > INT32_MAX || r > INT32_MAX) return cudaErrorInvalidValue;
+    // Split-K cluster kernel; ranks above 256 fall back to the persistent
+    // dense-mode kernel, which tiles r in 128-row steps.
+    if (r <= 16) return tc::launch_project_splitk<16>(X, M, V, d_in, r, T16, stream);
+    if (r <= 64) return tc::launch_project_splitk<64>(X, M, V, d_in, r, T16, stream);
+    if (r <= 128) return tc::launch_project_splitk<128>(X, M, V, d_in, r, T16, stream);
+    if (r <= 256) return tc::launch_project_splitk<256>(X, M, V, d_in, r, T16, stream);
     if (M >= 4096) return tc::launch_project<128>(X, M, V, d_in, r, T16, stream);
     if (M >= 1024) return tc::launch_project<64>(X, M, V, d_in, r, T16, stream);
     return tc::launch_project<32>(X, M, V, d_in, r, T16, stream);

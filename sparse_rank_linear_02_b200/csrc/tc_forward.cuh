@@ -8,9 +8,12 @@ namespace slr {
 
 // Y = X S^T + T U^T on the tensor cores.  T16 is bf16 [M, r] (may be null when
 // r == 0).  Requires d_in % 128 == 0, d_out % 8 == 0, r % 8 == 0.
+// after_projection: the kernel launched immediately before on `stream` is the
+// projection that writes T16 (enables programmatic dependent launch; must be
+// false otherwise).
 cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                               int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
-                              uint16_t *Y, cudaStream_t stream);
+                              uint16_t *Y, bool after_projection, cudaStream_t stream);
 
 // T = X V^T on the tensor cores, written as bf16 [M, r] (dense tcgen05 mode of
 // the same kernel).  Requires d_in % 64 == 0, r % 8 == 0.

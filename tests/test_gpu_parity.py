@@ -152,6 +152,7 @@ def test_forward_one_hot_exact(path):
     (136, 384, 8, 129),      # r = 8 pads to the MMA K step; M just over a tile
     (256, 640, 128, 255),    # two rank steps on the tensor path
     (264, 1024, 256, 20),    # four rank steps; decode with several token blocks
+    (256, 512, 264, 40),     # r > 256: the projection's persistent fallback, five rank steps
 ])
 def test_forward_edges(d_out, d_in, r, M, path):
     seed = d_out * 31 + d_in + r + M
