@@ -286,6 +286,9 @@ def run_ours(args, rank, world, dist):
     pack = run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier) if "pack" in legs else None
     del W
 
+    # ------------------------------------------------ the other configurations
+    sweep = run_sweep(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier, legs)
+
     # ------------------------------------------------ CPU baseline (oracle), rank 0 at N = 1
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and "cpu" in legs:
@@ -303,6 +306,7 @@ def run_ours(args, rank, world, dist):
                    "parallelism": f"dp{world} (independent token batches, no collective)"},
         "prefill": prefill,
         "decode_m1": decode,
+        **sweep,
         "pack": pack,
         "roofline": roofline,
         "e2e": e2e,
@@ -313,6 +317,154 @@ def run_ours(args, rank, world, dist):
         "kernel_source_sha": sha,
     }
     return line
+
+
+# ----------------------------------------------------------------------------- configuration sweep
+
+class LayerCache:
+    """Device copies of a layer's packed S and factors, shared by the sweep
+    points of one shape (the 70B rank variants share W)."""
+
+    def __init__(self, slr, torch, dev, to_dev):
+        self.slr, self.torch, self.dev, self.to_dev = slr, torch, dev, to_dev
+        self.packed = {}
+
+    def weights(self, L):
+        key = (L.cfg, L.wsub, L.d_out, L.d_in)
+        if key not in self.packed:
+            self.packed.clear()
+            self.torch.cuda.empty_cache()
+            W = self.to_dev(L.weight())
+            self.packed[key] = self.slr.pack_2to4(W)
+            del W
+        vals, meta = self.packed[key]
+        Uh, Vh = L.factors()
+        return vals, meta, self.to_dev(Uh), self.to_dev(Vh)
+
+
+def roofline_time(M, d_out, d_in, r, peaks):
+    bytes_ = algorithmic_bytes(M, d_out, d_in, r)
+    p_dense = peaks["bf16_tflops"] * 1e12
+    t_mem = bytes_ / (peaks["hbm_gbs"] * 1e9)
+    t_tc = 2.0 * M * d_out * d_in / (SPARSE_RATIO * p_dense) + 2.0 * M * r * (d_in + d_out) / p_dense
+    return max(t_mem, t_tc), ("hbm" if t_mem >= t_tc else "tensor"), bytes_
+
+
+def measure_point(slr, torch, dev, cache, L, M, K, peaks, max_over_ranks, barrier):
+    """One (layer, M) point: K forward steps in a CUDA graph over rotating
+    buffer sets (sized past L2); returns the metrics of the point."""
+    vals, meta, U, V = cache.weights(L)
+    d_out, d_in, r = L.d_out, L.d_in, L.r
+    path = slr.select_path(M, d_out, d_in, r)
+    ws_bytes = max(256, slr.workspace_size(M, d_out, d_in, r))
+    set_bytes = algorithmic_bytes(M, d_out, d_in, r)
+    n_copies = max(1, min(8, math.ceil(2.0 * L2_BYTES / set_bytes)))
+    Xh = L.activations(M)
+    sets = []
+    for c in range(n_copies):
+        sets.append(dict(X=cache.to_dev(Xh), vals=vals if c == 0 else vals.clone(), meta=meta if c == 0 else meta.clone(),
+                         U=U, V=V, Y=torch.empty((M, d_out), dtype=torch.bfloat16, device=dev),
+                         ws=torch.empty(ws_bytes, dtype=torch.uint8, device=dev)))
+
+    def fwd(s):
+        slr.forward(s["X"], s["vals"], s["meta"], s["U"], s["V"], out=s["Y"], workspace=s["ws"], path=path)
+
+    for i in range(3):
+        fwd(sets[i % n_copies])
+    barrier()
+    ms = max_over_ranks(graph_time_ms(torch, [lambda s=sets[k % n_copies]: fwd(s) for k in range(K)])) / K
+    t_roof, bound, bytes_ = roofline_time(M, d_out, d_in, r, peaks)
+    del sets
+    return {"layer": L.name, "d_out": d_out, "d_in": d_in, "r": r, "M": M, "path": path, "ms": round(ms, 5),
+            "tflops_dense_equiv": round(2.0 * M * d_out * d_in / (ms * 1e-3) / 1e12, 2),
+            "gbs": round(bytes_ / (ms * 1e-3) / 1e9, 1), "bound": bound,
+            "frac_of_roofline": round(t_roof / (ms * 1e-3), 4),
+            "l2": f"{n_copies} rotating sets of {set_bytes / 1e6:.1f} MB"}
+
+
+def run_sweep(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier, legs):
+    cache = LayerCache(slr, torch, dev, to_dev)
+    out = {}
+    if "cfg2" in legs:
+        L = layer_of(2, "q_proj")
+        out["cfg2_decode"] = [measure_point(slr, torch, dev, cache, L, M, max(20, args.steps), peaks,
+                                            max_over_ranks, barrier) for M in (1, 4, 16)]
+    if "cfg4" in legs:
+        out["cfg4_block"] = run_block(args, slr, torch, dev, cache, peaks, max_over_ranks, barrier)
+    if "cfg5" in legs:
+        pts = []
+        for L in synth.CONFIGS[5].layers:
+            for M in synth.CONFIGS[5].Ms:
+                K = 5 if M >= 1024 else 10
+                pts.append(measure_point(slr, torch, dev, cache, L, M, K, peaks, max_over_ranks, barrier))
+        out["cfg5_sweep"] = pts
+        # Crossover between the memory-bound plateau and the compute-bound
+        # regime: measured as plateau time / per-token time at the largest M,
+        # and the same quantity from the roofline model with the measured peaks.
+        cross = []
+        for L in synth.CONFIGS[5].layers:
+            mine = [p for p in pts if p["layer"] == L.name]
+            plateau = min(p["ms"] for p in mine if p["M"] <= 128)
+            big = max(mine, key=lambda p: p["M"])
+            t_mem = roofline_time(1, L.d_out, L.d_in, L.r, peaks)[0]
+            per_tok = roofline_time(big["M"], L.d_out, L.d_in, L.r, peaks)[0] / big["M"]
+            cross.append({"layer": L.name, "measured_M": round(plateau / (big["ms"] / big["M"]), 1),
+                          "roofline_M": round(t_mem / per_tok, 1)})
+        out["cfg5_crossover"] = cross
+    return out
+
+
+def run_block(args, slr, torch, dev, cache, peaks, max_over_ranks, barrier):
+    """The seven Llama-3-8B block linears at M = 4096, back to back in one
+    graph, and the 2:4 pack of the seven dense weights."""
+    M = 4096
+    layers = synth.CONFIGS[4].layers
+    data = []
+    for L in layers:
+        W = cache.to_dev(L.weight())
+        vals, meta = slr.pack_2to4(W)
+        Uh, Vh = L.factors()
+        data.append(dict(L=L, W=W, vals=vals, meta=meta, U=cache.to_dev(Uh), V=cache.to_dev(Vh),
+                         X=cache.to_dev(L.activations(M)),
+                         Y=torch.empty((M, L.d_out), dtype=torch.bfloat16, device=dev),
+                         ws=torch.empty(max(256, slr.workspace_size(M, L.d_out, L.d_in, L.r)), dtype=torch.uint8,
+                                        device=dev)))
+
+    def fwd(d):
+        slr.forward(d["X"], d["vals"], d["meta"], d["U"], d["V"], out=d["Y"], workspace=d["ws"])
+
+    lib = slr.lib()
+
+    def pack(d):
+        st = lib.slr_pack_2to4(slr._ptr(d["W"]), d["L"].d_out, d["L"].d_in, d["L"].d_in, slr._ptr(d["vals"]),
+                               slr._ptr(d["meta"]), slr._stream())
+        assert st == 0, st
+
+    for d in data:
+        fwd(d)
+    K = max(3, args.steps // 5)
+    barrier()
+    ms = max_over_ranks(graph_time_ms(torch, [lambda d=d: fwd(d) for _ in range(K) for d in data])) / K
+    per = []
+    for d in data:
+        t = graph_time_ms(torch, [lambda d=d: fwd(d) for _ in range(K)]) / K
+        L = d["L"]
+        t_roof, bound, _ = roofline_time(M, L.d_out, L.d_in, L.r, peaks)
+        per.append({"layer": L.name, "d_out": L.d_out, "d_in": L.d_in, "ms": round(t, 5),
+                    "frac_of_roofline": round(t_roof / (t * 1e-3), 4)})
+    flops = sum(2.0 * M * d["L"].d_out * d["L"].d_in for d in data)
+    t_roof_all = sum(roofline_time(M, d["L"].d_out, d["L"].d_in, d["L"].r, peaks)[0] for d in data)
+    pack_bytes = sum(d["L"].d_out * d["L"].d_in * 3.125 for d in data)
+    pack_ms = graph_time_ms(torch, [lambda d=d: pack(d) for _ in range(K) for d in data]) / K
+    del data
+    torch.cuda.empty_cache()
+    return {"workload": "seven Llama-3-8B block linears (q, k, v, o, gate, up, down), r = 64, M = 4096, "
+                        "back to back in one CUDA graph", "ms": round(ms, 4),
+            "tflops_dense_equiv": round(flops / (ms * 1e-3) / 1e12, 1),
+            "frac_of_roofline": round(t_roof_all / (ms * 1e-3), 4), "layers": per,
+            "pack_all_seven": {"ms": round(pack_ms, 4), "gbs": round(pack_bytes / (pack_ms * 1e-3) / 1e9, 1),
+                               "frac": round(pack_bytes / (pack_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                               "note": "working set larger than L2 (682 MB read + written)"}}
 
 
 def run_e2e_leg(args, slr, torch, Xh, M, d_out, sets, n_copies, flops_dense, world, max_over_ranks, barrier):
@@ -479,7 +631,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024, help="token rows in the oracle CPU baseline sample")
     ap.add_argument("--ref-rows", type=int, default=64, help="token rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="prefill,e2e,decode,pack,cpu",
+    ap.add_argument("--only", default="prefill,e2e,decode,pack,cpu,cfg2,cfg4,cfg5",
                     help="comma list of legs to run (profiling runs use one leg)")
     args = ap.parse_args()
     if args.warmup < 3:

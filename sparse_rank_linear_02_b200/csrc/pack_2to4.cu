@@ -39,7 +39,23 @@ __device__ __forceinline__ uint32_t select_group(uint32_t w01, uint32_t w23, uin
     return i0 | (i1 << 2);
 }
 
-// Vectorised path: d_in % 8 == 0, ldw % 8 == 0, W 16-byte aligned.
+// Vectorised path: d_in % 8 == 0, ldw % 8 == 0, W 16-byte aligned.  Each
+// thread keeps kPackUnroll 16-byte loads in flight (units u, u + stride, ...,
+// coalesced across the warp for each step) before selecting and storing.
+constexpr int kPackUnroll = 4;
+
+__device__ __forceinline__ void pack_unit(uint4 w, int64_t u, int64_t units_per_row, int64_t d_in,
+                                          int64_t meta_row, uint16_t *__restrict__ vals,
+                                          uint8_t *__restrict__ meta) {
+    const int64_t row = u / units_per_row;
+    const int64_t c = u - row * units_per_row;
+    uint32_t kept0, kept1;
+    const uint32_t n0 = select_group(w.x, w.y, &kept0);
+    const uint32_t n1 = select_group(w.z, w.w, &kept1);
+    *reinterpret_cast<uint2 *>(vals + row * (d_in / 2) + c * 4) = make_uint2(kept0, kept1);
+    meta[row * meta_row + c] = (uint8_t)(n0 | (n1 << 4));
+}
+
 __global__ void __launch_bounds__(256) pack_2to4_v8_kernel(const uint16_t *__restrict__ W, int64_t d_out,
                                                            int64_t d_in, int64_t ldw,
                                                            uint16_t *__restrict__ vals,
@@ -47,16 +63,22 @@ __global__ void __launch_bounds__(256) pack_2to4_v8_kernel(const uint16_t *__res
     const int64_t units_per_row = d_in / 8;
     const int64_t meta_row = (d_in / 4 + 1) / 2;
     const int64_t total = d_out * units_per_row;
-    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total;
-         u += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t row = u / units_per_row;
-        const int64_t c = u - row * units_per_row;
-        const uint4 w = ld_stream_v4(W + row * ldw + c * 8);
-        uint32_t kept0, kept1;
-        const uint32_t n0 = select_group(w.x, w.y, &kept0);
-        const uint32_t n1 = select_group(w.z, w.w, &kept1);
-        *reinterpret_cast<uint2 *>(vals + row * (d_in / 2) + c * 4) = make_uint2(kept0, kept1);
-        meta[row * meta_row + c] = (uint8_t)(n0 | (n1 << 4));
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t u0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u0 < total; u0 += kPackUnroll * stride) {
+        uint4 w[kPackUnroll];
+#pragma unroll
+        for (int i = 0; i < kPackUnroll; ++i) {
+            const int64_t u = u0 + i * stride;
+            if (u < total) {
+                const int64_t row = u / units_per_row;
+                w[i] = ld_stream_v4(W + row * ldw + (u - row * units_per_row) * 8);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kPackUnroll; ++i) {
+            const int64_t u = u0 + i * stride;
+            if (u < total) pack_unit(w[i], u, units_per_row, d_in, meta_row, vals, meta);
+        }
     }
 }
 

@@ -977,6 +977,268 @@ cudaError_t launch_project_splitk(const uint16_t *X, int64_t M, const uint16_t *
     return cudaLaunchKernelEx(&cfg, tc_project_kernel<RN>, m_x, m_v, T16, (int32_t)M, (int32_t)r, (int32_t)nk);
 }
 
+
+// =====================================================================================
+// Small-M forward (M <= 64 tokens): Y = X S^T + T U^T when the layer is bound by
+// the bytes of S.  One cluster of KS CTAs (KS <= 4) owns a 128-row x BN-token
+// tile and splits its K stages (the 2:4 stages, then the rank stages) across
+// its CTAs, so that all SMs stream S at once even when d_out / 128 is small.
+// Each CTA accumulates its partial Y^T tile in TMEM (2:4 tcgen05.mma.sp with
+// the same metadata permute as the large-M kernels, N = BN), writes it to
+// shared memory in fp32, and after a cluster barrier CTA q sums rows
+// [q*128/KS, (q+1)*128/KS) over the KS partials through distributed shared
+// memory and stores them to Y in bf16 (RNE).
+template <int BN>
+struct CfgS {
+    static constexpr int A_BYTES = BM * 64 * 2;          // 16 KB of packed values (128 logical K)
+    static constexpr int B_HALF = BN * 64 * 2;           // BN tokens x one 128-byte panel
+    static constexpr int B_BYTES = 2 * B_HALF;
+    static constexpr int E_BYTES = BM * BK / 8;          // 2 KB of metadata
+    static constexpr int STAGE = ((A_BYTES + B_BYTES + E_BYTES + 1023) / 1024) * 1024;
+    static constexpr int PROW = BN + 4;                  // padded fp32 row of the partial tile
+    static constexpr int P_BYTES = BM * PROW * 4;
+    static constexpr int NS_FIT = 102400 / STAGE;        // about 100 KB: two CTAs per SM
+    static constexpr int NS = NS_FIT > 8 ? 8 : (NS_FIT < 2 ? 2 : NS_FIT);
+    static constexpr int RING = NS * STAGE;
+    static constexpr int BAR_OFF = (RING > P_BYTES ? RING : P_BYTES);
+    static constexpr int SMEM = BAR_OFF + 256 + 1024;
+    static constexpr uint32_t ECOL = BN;
+    static constexpr uint32_t TMEM_COLS = pow2_at_least(BN + 4);
+    static_assert(SMEM <= 116736, "two CTAs per SM");
+    static_assert(BN % 16 == 0 && BN <= 64, "MMA N");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 2)
+    tc_small_kernel(const __grid_constant__ CUtensorMap tm_vals, const __grid_constant__ CUtensorMap tm_meta,
+                    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_u,
+                    const __grid_constant__ CUtensorMap tm_t, uint16_t *__restrict__ Y, int32_t M, int32_t d_out,
+                    int32_t n_ttiles, int32_t nk, int32_t nlr) {
+    using C = CfgS<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *empty = full + C::NS;
+    uint64_t *acc_full = empty + C::NS;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    float *part = reinterpret_cast<float *>(smem);      // reuses the ring after the K loop
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    uint32_t ks_n;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(ks_n));
+    const uint32_t ks_q = cluster_ctarank();
+    const int work = blockIdx.x / (int)ks_n;
+    const int d0 = (work / n_ttiles) * BM;
+    const int tok0 = (work % n_ttiles) * BN;
+    const int total = nk + nlr;
+    const int k_begin = (int)(((int64_t)total * ks_q) / ks_n);
+    const int k_end = (int)(((int64_t)total * (ks_q + 1)) / ks_n);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t s = 0, ph = 0;
+            bool t_ready = false;
+            for (int ks = k_begin; ks < k_end; ++ks) {
+                if (!mbar_wait(&empty[s], ph ^ 1)) {
+                    atomicOr(&g_tc_error, 4096u);
+                    break;
+                }
+                uint8_t *st = smem + s * C::STAGE;
+                const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES),
+                               e = smem_u32(st + C::A_BYTES + C::B_BYTES);
+                if (ks < nk) {
+                    mbar_expect_tx(&full[s], C::A_BYTES + C::B_BYTES + C::E_BYTES);
+                    tma_load_2d(&tm_vals, a, &full[s], ks * 64, d0);
+                    tma_load_2d(&tm_x, b, &full[s], ks * BK, tok0);
+                    tma_load_2d(&tm_x, b + C::B_HALF, &full[s], ks * BK + 64, tok0);
+                    tma_load_2d(&tm_meta, e, &full[s], ks * (BK / 8), d0);
+                } else {
+                    if (!t_ready) {
+                        // T may still be in production (programmatic dependent launch)
+                        asm volatile("griddepcontrol.wait;" ::: "memory");
+                        t_ready = true;
+                    }
+                    const int j = ks - nk;
+                    mbar_expect_tx(&full[s], C::A_BYTES + C::B_HALF);
+                    tma_load_2d(&tm_u, a, &full[s], j * 64, d0);
+                    tma_load_2d(&tm_t, b, &full[s], j * 64, tok0);
+                }
+                if (++s == (uint32_t)C::NS) {
+                    s = 0;
+                    ph ^= 1;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        constexpr uint32_t kIdescSp = idesc_bf16(BM, BN, true);
+        constexpr uint32_t kIdescDense = idesc_bf16(BM, BN, false);
+        const uint32_t e_tmem = tmem_base + C::ECOL;
+        uint32_t s = 0, ph = 0;
+        bool ok = true;
+        for (int ks = k_begin; ks < k_end; ++ks) {
+            if (!mbar_wait(&full[s], ph)) {
+                ok = false;
+                break;
+            }
+            uint8_t *st = smem + s * C::STAGE;
+            const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES);
+            const uint32_t first = (ks == k_begin) ? 1u : 0u;
+            if (ks < nk) {
+                permute_meta_tile(st + C::A_BYTES + C::B_BYTES, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tc_fence_after();
+                    tmem_cp_128x128b(e_tmem, smem_desc(smem_u32(st + C::A_BYTES + C::B_BYTES), 0, 128, kLayoutNone));
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint64_t adesc = desc_sw128(a + 32 * c);
+                        const uint64_t bdesc = desc_sw128(b + (c >> 1) * C::B_HALF + (c & 1) * 64);
+                        mma_sp(tmem_base, adesc, bdesc, e_tmem + (uint32_t)(c & 2), kIdescSp | (uint32_t)(c & 1),
+                               !(first && c == 0));
+                    }
+                    mma_commit(&empty[s]);
+                }
+            } else if (lane == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    mma_dense(tmem_base, desc_sw128(a + 32 * c), desc_sw128(b + 32 * c), kIdescDense,
+                              !(first && c == 0));
+                mma_commit(&empty[s]);
+            }
+            __syncwarp();
+            if (++s == (uint32_t)C::NS) {
+                s = 0;
+                ph ^= 1;
+            }
+        }
+        if (!ok && lane == 0) atomicOr(&g_tc_error, 8192u);
+        if (lane == 0) mma_commit(acc_full);  // fires at once when this CTA had no stages
+        __syncwarp();
+    } else {
+        // TMEM partial (lane = output row, column = token) -> shared memory
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const bool have = k_end > k_begin;
+        if (mbar_wait(acc_full, 0)) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int q = 0; q < BN / 16; ++q) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(q * 16), v);
+                float4 *dst = reinterpret_cast<float4 *>(part + row * C::PROW + q * 16);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    dst[j] = have ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else {
+            atomicOr(&g_tc_error, 16384u);
+        }
+    }
+    tc_fence_before();
+    cluster_sync_all();  // every CTA's partial is in its shared memory
+
+    // CTA q: rows [q*RPC, (q+1)*RPC) of the tile, all BN tokens, summed over
+    // the cluster; thread -> (row, group of 4 tokens), rows fastest so that
+    // the bf16 stores of one token are contiguous in Y.
+    if (warp >= 2) {
+        const int rpc = BM / (int)ks_n;
+        const int items = rpc * (BN / 4);
+        const uint32_t part_addr = smem_u32(part);
+        for (int it = threadIdx.x - 64; it < items; it += 128) {
+            const int row = (int)ks_q * rpc + it % rpc;
+            const int tg = it / rpc;
+            const uint32_t off = (uint32_t)((row * C::PROW + 4 * tg) * 4);
+            float4 p[4];
+#pragma unroll
+            for (uint32_t q = 0; q < 4; ++q)
+                p[q] = q < ks_n ? ld_shared_cluster_v4(mapa_shared(part_addr + off, q)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float sum[4] = {p[0].x + p[1].x + p[2].x + p[3].x, p[0].y + p[1].y + p[2].y + p[3].y,
+                                  p[0].z + p[1].z + p[2].z + p[3].z, p[0].w + p[1].w + p[2].w + p[3].w};
+            const int out_row = d0 + row;
+            if (out_row < d_out) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int tok = tok0 + 4 * tg + j;
+                    if (tok < M) Y[(int64_t)tok * d_out + out_row] = f32_to_bf16_bits(sum[j]);
+                }
+            }
+        }
+    }
+    cluster_sync_all();  // no CTA leaves while its partial may still be read
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+    }
+}
+
+template <int BN>
+cudaError_t launch_sparse_small(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
+                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
+                                uint16_t *Y, bool after_projection, cudaStream_t stream) {
+    using C = CfgS<BN>;
+    CUtensorMap m_vals, m_meta, m_x, m_u, m_t;
+    memset(&m_u, 0, sizeof m_u);
+    memset(&m_t, 0, sizeof m_t);
+    bool ok = make_map(&m_vals, kBF16, vals, d_in / 2, d_out, d_in, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&m_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, d_in / 8, d_out, d_in / 8, 16, BM,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map(&m_x, kBF16, X, d_in, M, d_in * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (ok && r > 0)
+        ok = make_map(&m_u, kBF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+             make_map(&m_t, kBF16, T16, r, M, r * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int n_ttiles = (int)((M + BN - 1) / BN);
+    const int work = (int)((d_out + BM - 1) / BM) * n_ttiles;
+    const int nk = (int)(d_in / BK), nlr = (int)((r + 63) / 64);
+    int ks = 1;
+    while (ks < 4 && ks * 2 <= nk + nlr && work * ks * 2 <= 2 * sms) ks *= 2;
+    cudaError_t err = cudaFuncSetAttribute(tc_small_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(work * ks));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (after_projection && r > 0) ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, tc_small_kernel<BN>, m_vals, m_meta, m_x, m_u, m_t, Y, (int32_t)M,
+                              (int32_t)d_out, (int32_t)n_ttiles, (int32_t)nk, (int32_t)nlr);
+}
+
 }  // namespace tc
 
 cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
@@ -994,7 +1256,17 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
             return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
         if (strcmp(force, "2sm256") == 0)
             return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+        if (strcmp(force, "small") == 0 && M <= 64) {
+            if (M <= 16) return tc::launch_sparse_small<16>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+            if (M <= 32) return tc::launch_sparse_small<32>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+            return tc::launch_sparse_small<64>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+        }
     }
+    // Up to 64 tokens the layer streams S: the split-K small-M kernel.  Then
+    // 2-SM pair tiles of 128 tokens, and of 256 tokens from 192 tokens on.
+    if (M <= 16) return tc::launch_sparse_small<16>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+    if (M <= 32) return tc::launch_sparse_small<32>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+    if (M <= 64) return tc::launch_sparse_small<64>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     if (M >= 192)
         return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);

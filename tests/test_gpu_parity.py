@@ -181,7 +181,7 @@ def test_no_kernel_timeouts():
     slr.check_kernel_error()
 
 
-VARIANTS = ["1sm", "2sm128", "2sm256"]
+VARIANTS = ["1sm", "2sm128", "2sm256", "small"]
 
 
 @pytest.mark.parametrize("variant", VARIANTS)
@@ -190,6 +190,10 @@ VARIANTS = ["1sm", "2sm128", "2sm256"]
     (136, 384, 8, 129),      # r = 8; M just over a 128-token tile
     (512, 640, 128, 300),    # several pair tiles, two rank stages, ragged token tile
     (1024, 1024, 256, 513),  # four rank stages; more tiles than one wave of pairs
+    (384, 512, 64, 5),       # small M: split K over a cluster, ragged token tile
+    (1024, 2048, 128, 16),   # small M, 16-token tile, two rank stages
+    (256, 4096, 64, 33),     # small M, 64-token tile
+    (4096, 4096, 64, 1),     # one token, 32 row tiles x 4-CTA clusters
 ])
 def test_forward_tensor_variants(variant, d_out, d_in, r, M, monkeypatch):
     """Every tensor-core kernel variant (1-SM, 2-SM with 128- and 256-token
