@@ -49,7 +49,7 @@ SPARSE_RATIO = 2.0   # nominal 2:4 sparse / dense tensor throughput ratio
 
 # DRAM bytes per launch of the dominant kernel from the committed ncu capture
 # (profiles/); valid only for the kernel source it was taken on.
-NCU_TRAFFIC = {"tc_forward": {"source_sha": "eafdd5bf5a7be4cd", "bytes_per_launch": 277621248}}
+NCU_TRAFFIC = {"tc_forward": {"source_sha": "91fd9f0d9f8ada5c", "bytes_per_launch": 119750400}}
 
 
 def layer_of(cfg, name):
@@ -254,7 +254,7 @@ def run_ours(args, rank, world, dist):
     sha = kernel_source_sha()
     traffic = NCU_TRAFFIC.get("tc_forward", {})
     traffic_bytes = traffic.get("bytes_per_launch") if traffic.get("source_sha") == sha else None
-    roofline = {"bound": "tensor", "kernel": "tc_forward_kernel (2:4 tcgen05.mma.sp + rank-r tcgen05.mma)",
+    roofline = {"bound": "tensor", "kernel": "tc2_forward_kernel<256> (2-SM 2:4 tcgen05.mma.sp + rank-r tcgen05.mma)",
                 "achieved": round(achieved_k, 1), "peak": round(peak_k, 1), "unit": "TFLOP/s",
                 "frac": round(achieved_k / peak_k, 4), "traffic": traffic_bytes,
                 "algorithmic_flops_per_launch": k_flops_sp + k_flops_lr,

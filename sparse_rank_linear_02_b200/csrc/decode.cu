@@ -18,8 +18,8 @@
 namespace slr {
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kBlocksPerSm = 4;
+constexpr int kWarps = 4;
+constexpr int kBlocksPerSm = 7;
 // 16-byte chunks in flight per lane: a whole 4096-wide row per round trip for
 // one or two tokens; fewer with more tokens (their accumulators and X loads
 // need the registers).
@@ -47,10 +47,10 @@ __device__ __forceinline__ float chunk_fma(uint4 v, uint32_t m16, uint4 xa, uint
     return acc;
 }
 
-// 4 resident CTAs per SM (<= 64 registers): 148 x 4 x 8 warps cover the 4096
-// rows of a Llama-3-8B projection in one wave.
+// 7 resident CTAs of 4 warps per SM (<= 73 registers): 148 x 7 x 4 warps cover
+// the 4096 rows of a Llama-3-8B projection, one row per warp, in one wave.
 template <int MT>
-__global__ void __launch_bounds__(kWarps * 32, 4) decode_forward_kernel(
+__global__ void __launch_bounds__(kWarps * 32, kBlocksPerSm) decode_forward_kernel(
     const uint16_t *__restrict__ X, int64_t M, const uint16_t *__restrict__ vals,
     const uint8_t *__restrict__ meta, int64_t d_out, int64_t d_in, const uint16_t *__restrict__ U,
     const float *__restrict__ T32, int64_t r, uint16_t *__restrict__ Y) {
@@ -68,6 +68,28 @@ __global__ void __launch_bounds__(kWarps * 32, 4) decode_forward_kernel(
         for (int t = 0; t < MT; ++t) acc[t] = 0.f;
         const uint16_t *vrow = vals + row * (d_in / 2);
         const uint8_t *mrow = meta + row * (d_in / 8);
+        // The rank-r operands of this row: U now (it does not depend on the
+        // projection), T after griddepcontrol.wait once the first weight
+        // chunks are in flight, so neither load adds a round trip at the end.
+        constexpr int kRk = 2;   // r <= 32 * kRk handled from registers
+        float ur[kRk];
+        float tr[kRk][MT];
+#pragma unroll
+        for (int j = 0; j < kRk; ++j) {
+            const int64_t k = lane + 32 * j;
+            ur[j] = k < r ? __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(U) + row * r + k) << 16) : 0.f;
+        }
+        bool t_loaded = false;
+        auto load_t = [&]() {
+            t_loaded = true;
+            if (r > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+#pragma unroll
+            for (int j = 0; j < kRk; ++j) {
+                const int64_t k = lane + 32 * j;
+#pragma unroll
+                for (int t = 0; t < MT; ++t) tr[j][t] = (k < r && t < nt) ? __ldg(T32 + (m0 + t) * r + k) : 0.f;
+            }
+        };
 
         for (int64_t c0 = lane; c0 < chunks; c0 += 32 * kUnroll) {
             uint4 v[kUnroll];
@@ -83,6 +105,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4) decode_forward_kernel(
                     mm[u] = 0x4444u;  // valid nibbles for the zero padding
                 }
             }
+            if (!t_loaded) load_t();   // the first weight chunks are in flight
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 const int64_t c = c0 + 32 * u;
@@ -98,12 +121,16 @@ __global__ void __launch_bounds__(kWarps * 32, 4) decode_forward_kernel(
             }
         }
 
+        if (!t_loaded) load_t();   // lanes that had no weight chunk
         // Rank-r term: lanes split k, products land in the same partial sums.
         // T comes from the projection kernel, which may still be running when
-        // this kernel starts (programmatic dependent launch): wait for it here,
-        // after the weight stream.
-        if (r > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
-        for (int64_t k = lane; k < r; k += 32) {
+        // this kernel starts (programmatic dependent launch); it was loaded
+        // after griddepcontrol.wait above.  Ranks beyond 32 * kRk continue here.
+#pragma unroll
+        for (int j = 0; j < kRk; ++j)
+#pragma unroll
+            for (int t = 0; t < MT; ++t) acc[t] = fmaf(ur[j], tr[j][t], acc[t]);
+        for (int64_t k = lane + 32 * kRk; k < r; k += 32) {
             const float u = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(U) + row * r + k) << 16);
 #pragma unroll
             for (int t = 0; t < MT; ++t)

@@ -39,45 +39,40 @@ __device__ __forceinline__ uint32_t select_group(uint32_t w01, uint32_t w23, uin
     return i0 | (i1 << 2);
 }
 
-// Vectorised path: d_in % 8 == 0, ldw % 8 == 0, W 16-byte aligned.  Each
-// thread keeps kPackUnroll 16-byte loads in flight (units u, u + stride, ...,
-// coalesced across the warp for each step) before selecting and storing.
+// Vectorised path: d_in % 8 == 0, ldw % 8 == 0, W 16-byte aligned.  Rows are
+// distributed over the grid; the CTA's threads sweep a row in 16-byte units,
+// keeping kPackUnroll loads in flight per thread (coalesced across the CTA for
+// each step).  No integer division on the index path.
 constexpr int kPackUnroll = 4;
-
-__device__ __forceinline__ void pack_unit(uint4 w, int64_t u, int64_t units_per_row, int64_t d_in,
-                                          int64_t meta_row, uint16_t *__restrict__ vals,
-                                          uint8_t *__restrict__ meta) {
-    const int64_t row = u / units_per_row;
-    const int64_t c = u - row * units_per_row;
-    uint32_t kept0, kept1;
-    const uint32_t n0 = select_group(w.x, w.y, &kept0);
-    const uint32_t n1 = select_group(w.z, w.w, &kept1);
-    *reinterpret_cast<uint2 *>(vals + row * (d_in / 2) + c * 4) = make_uint2(kept0, kept1);
-    meta[row * meta_row + c] = (uint8_t)(n0 | (n1 << 4));
-}
 
 __global__ void __launch_bounds__(256) pack_2to4_v8_kernel(const uint16_t *__restrict__ W, int64_t d_out,
                                                            int64_t d_in, int64_t ldw,
                                                            uint16_t *__restrict__ vals,
                                                            uint8_t *__restrict__ meta) {
-    const int64_t units_per_row = d_in / 8;
+    const int units = (int)(d_in / 8);
     const int64_t meta_row = (d_in / 4 + 1) / 2;
-    const int64_t total = d_out * units_per_row;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t u0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u0 < total; u0 += kPackUnroll * stride) {
-        uint4 w[kPackUnroll];
+    for (int64_t row = blockIdx.x; row < d_out; row += gridDim.x) {
+        const uint16_t *wrow = W + row * ldw;
+        uint2 *vrow = reinterpret_cast<uint2 *>(vals + row * (d_in / 2));
+        uint8_t *mrow = meta + row * meta_row;
+        for (int c0 = threadIdx.x; c0 < units; c0 += kPackUnroll * blockDim.x) {
+            uint4 w[kPackUnroll];
 #pragma unroll
-        for (int i = 0; i < kPackUnroll; ++i) {
-            const int64_t u = u0 + i * stride;
-            if (u < total) {
-                const int64_t row = u / units_per_row;
-                w[i] = ld_stream_v4(W + row * ldw + (u - row * units_per_row) * 8);
+            for (int i = 0; i < kPackUnroll; ++i) {
+                const int c = c0 + i * blockDim.x;
+                if (c < units) w[i] = ld_stream_v4(wrow + (int64_t)c * 8);
             }
-        }
 #pragma unroll
-        for (int i = 0; i < kPackUnroll; ++i) {
-            const int64_t u = u0 + i * stride;
-            if (u < total) pack_unit(w[i], u, units_per_row, d_in, meta_row, vals, meta);
+            for (int i = 0; i < kPackUnroll; ++i) {
+                const int c = c0 + i * blockDim.x;
+                if (c < units) {
+                    uint32_t kept0, kept1;
+                    const uint32_t n0 = select_group(w[i].x, w[i].y, &kept0);
+                    const uint32_t n1 = select_group(w[i].z, w[i].w, &kept1);
+                    vrow[c] = make_uint2(kept0, kept1);
+                    mrow[c] = (uint8_t)(n0 | (n1 << 4));
+                }
+            }
         }
     }
 }
@@ -128,8 +123,11 @@ cudaError_t launch_pack_2to4(const uint16_t *W, int64_t d_out, int64_t d_in, int
     const bool v8 = (d_in % 8 == 0) && (ldw % 8 == 0) && ((reinterpret_cast<uintptr_t>(W) & 15) == 0) &&
                     ((reinterpret_cast<uintptr_t>(vals) & 7) == 0);
     if (v8) {
-        const int64_t units = d_out * (d_in / 8);
-        pack_2to4_v8_kernel<<<grid_for(units, 256), 256, 0, stream>>>(W, d_out, d_in, ldw, vals, meta);
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t cap = (int64_t)sms * 8;
+        const int grid = (int)(d_out < cap ? d_out : cap);
+        pack_2to4_v8_kernel<<<grid, 256, 0, stream>>>(W, d_out, d_in, ldw, vals, meta);
     } else {
         const int64_t units = d_out * ((d_in / 4 + 1) / 2);
         pack_2to4_any_kernel<<<grid_for(units, 256), 256, 0, stream>>>(W, d_out, d_in, ldw, vals, meta);
