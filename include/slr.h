@@ -210,6 +210,17 @@ SLR_API slr_status slr_forward_decode_noalloc(const void *X, int64_t M, const vo
  * their resources and return, so the CUDA context stays usable. */
 SLR_API slr_status slr_check_kernel_error(void);
 
+/* Failure-detection self-test (no counterpart on the pages; it checks this
+ * library's own error path).  Launches, on `stream`, one thread that waits with
+ * the same bounded mbarrier wait the tensor-core kernels use, but with a limit
+ * of `limit_cycles` SM clock cycles (1 <= limit_cycles < 2^31; 2e6 is about a
+ * millisecond), on a barrier that nothing completes.  The wait expires, the
+ * kernel records a timeout in the library's error word and returns, so the
+ * next slr_check_kernel_error() reports SLR_ERR_TIMEOUT and the context stays
+ * usable.  Returns SLR_ERR_ARG for a limit out of range, SLR_ERR_DEVICE
+ * without an sm_100 device, SLR_ERR_CUDA if the launch fails. */
+SLR_API slr_status slr_selftest_wait_timeout(int64_t limit_cycles, slr_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -69,6 +69,8 @@ def _load() -> ctypes.CDLL:
     lib.slr_forward_combine.argtypes = [p, i64, p, p, i64, i64, p, i64, p, p, sz, st, p]
     lib.slr_forward_decode_noalloc.restype = st
     lib.slr_forward_decode_noalloc.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, p]
+    lib.slr_selftest_wait_timeout.restype = st
+    lib.slr_selftest_wait_timeout.argtypes = [i64, p]
     return lib
 
 
@@ -180,3 +182,10 @@ def forward_decode_noalloc(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tens
 def check_kernel_error() -> None:
     """Synchronise and raise if a tensor-core kernel reported a bounded-wait timeout."""
     _check(_lib.slr_check_kernel_error(), "slr_check_kernel_error")
+
+
+def selftest_wait_timeout(limit_cycles: int = 2_000_000) -> None:
+    """Launch the failure-detection self-test (``slr_selftest_wait_timeout``): a
+    bounded wait that expires after ``limit_cycles`` SM cycles and records a
+    timeout that the next :func:`check_kernel_error` raises."""
+    _check(_lib.slr_selftest_wait_timeout(int(limit_cycles), _stream()), "slr_selftest_wait_timeout")

@@ -185,6 +185,15 @@ slr_status slr_check_kernel_error(void) {
     return code ? SLR_ERR_TIMEOUT : SLR_OK;
 }
 
+slr_status slr_selftest_wait_timeout(int64_t limit_cycles, slr_stream_t stream) {
+    if (limit_cycles < 1 || limit_cycles > INT32_MAX) return SLR_ERR_ARG;
+    if (slr::check_device() != SLR_OK) return SLR_ERR_DEVICE;
+    return slr::launch_wait_timeout_selftest((long long)limit_cycles, reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? SLR_OK
+               : SLR_ERR_CUDA;
+}
+
 slr_status slr_forward(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out, int64_t d_in,
                        const void *U, const void *V, int64_t r, void *Y, void *workspace, size_t workspace_bytes,
                        slr_stream_t stream) {

@@ -307,80 +307,221 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
 // =====================================================================================
-// 2-SM variant (cta_group::2).  A cluster of two CTAs on neighbouring SMs owns a
-// 256-row x BN-token tile of Y^T: CTA rank q stages rows 128q..128q+127 of the
-// S tile (values and metadata) and tokens (BN/2)q..(BN/2)q+BN/2-1 of the X tile.
-// The leader (rank 0) issues every tcgen05.cp / tcgen05.mma for the pair; each
-// operand descriptor names the same shared-memory offset in both CTAs.  Per
-// 128-K stage each SM moves 16 KB of S, 2 KB of metadata and BN/2*256 B of X
-// for an M=256 MMA: half the operand bytes per MMA cycle of the 1-SM tile.
+// 2-SM variant (cta_group::2).  A cluster of two CTAs on neighbouring SMs computes
+// 256-row x n-token pieces of Y^T ("chunks", n <= BN, n a multiple of 16): CTA
+// rank q stages rows 128q..128q+127 of the S tile (values and metadata) and
+// tokens q*n/2..q*n/2+n/2-1 of the chunk's X rows.  The leader (rank 0) issues
+// every tcgen05.cp / tcgen05.mma for the pair; each operand descriptor names the
+// same shared-memory offset in both CTAs.  Per 128-K stage each SM moves 16 KB
+// of S, 2 KB of metadata and n/2*256 B of X for an M=256 MMA: half the operand
+// bytes per MMA cycle of a 1-SM tile.
+//
+// Work partition (a data-parallel phase, then a balanced tail): the output is
+// cut into 256-row tiles and each tile's tokens into 16-token units; a row's
+// units form `ttiles` token tiles of near-equal width (<= BN tokens).
+//  * Cyclic phase: for `cyc` rounds, round j deals tiles j*P .. j*P+P-1
+//    (row-tile major) to the P pairs, rotated by j so that no pair always gets
+//    the same token column.  The pairs of one round share a few S row tiles
+//    and all of X, so both stay in L2 and S is read from HBM about once.
+//  * Tail: the remaining units (between one and two rounds of tiles), in
+//    row-tile-major order, are split into contiguous ranges, one per pair,
+//    sized on the host so that every pair ends with the same number of
+//    units.  A range is cut into chunks of at most BN/16 units that do not
+//    cross a row tile (a segment is split into near-equal chunks); even pairs
+//    walk their range forwards and odd pairs backwards, so the two pairs that
+//    share a row tile at a range boundary read it at about the same time.
+// Against whole tiles dealt out in rounds this removes the idle pairs of the
+// last round (448 tiles of 256 x 256 on 74 pairs is 7 rounds for 6.05 rounds
+// of work on the Llama-3-8B gate/up layer at M = 2048).  X rows are loaded in
+// boxes of 64/32/16/8 rows (or one box of BN/2 rows for a full chunk), so a
+// narrow chunk moves only its own tokens.
 //
 // Warps: 0 TMA producer, 1 MMA issue (leader only), 2..5 epilogue, 6 metadata.
-// The metadata warp permutes each stage's metadata tile ahead of the MMA warp
-// and then signals the leader's ready[s]: in the leader with an arrive that
-// also expects 16 transaction bytes, in the follower with a 16-byte bulk copy
-// into the leader that completes those bytes.  The MMA warp therefore only
-// waits for ready[s] and issues.
+// Operand stages: both CTAs' TMA loads of a stage (S values and X, or U and
+// T) complete on the LEADER's full[s] barrier (cp.async.bulk.tensor with
+// .cta_group::2, no multicast), so the MMA warp learns from one barrier that
+// the pair's stage has landed.  Metadata takes a separate, deeper ring: the
+// metadata warp of each CTA loads the tile MLEAD sparse stages ahead, permutes
+// it into the TMEM layout and signals the leader's mready[m] (the leader with
+// an arrive that expects 16 transaction bytes, the follower with a 16-byte
+// bulk copy into the leader that completes them), so the permute is off the
+// path from a stage's arrival to its MMAs.  The producer and MMA warps walk
+// their loops with the whole warp (every branch warp-uniform) and one elected
+// lane issues.
 //
-// Accumulators: two TMEM buffers of BN columns.  When 2*BN + 4 exceeds the 512
-// columns (BN = 256) they overlap by OVL columns at the end of buffer 0 / start
-// of buffer 1, and the metadata takes the last 4 columns.  The epilogue drains
-// the overlapping 32-column chunk first and reports it (acc_ovl), so the next
-// tile's MMAs wait only for that chunk; acc_empty reports the whole buffer.
+// Accumulators: two TMEM buffers of BN columns (2*BN + 4 <= 512 columns; the
+// metadata takes 4 columns after them), so the epilogue of one chunk overlaps
+// the MMAs of the next.
 //
 // Handshakes (all waits bounded):
-//   full[s]      local TMA completion (each CTA)
-//   ready[s]     leader: its metadata warp (count 1) + follower's 16 bytes
+//   full[s]      leader: its producer's arrive (both CTAs' bytes) + TMA bytes
 //   empty[s]     leader's commit, multicast to both CTAs
+//   mfull[m]     local metadata TMA completion (each CTA)
+//   mready[m]    leader: its metadata warp (count 1) + follower's 16 bytes
+//   mempty[m]    leader's commit after the MMAs that read slot m, multicast
 //   acc_full[b]  leader's commit, multicast
-//   acc_ovl[b]   8 epilogue warps (both CTAs) -> leader: overlap chunk drained
 //   acc_empty[b] 8 epilogue warps (both CTAs) -> leader: buffer drained
 template <int BN>
 struct Cfg2 {
-    static constexpr int HALF_N = BN / 2;               // tokens staged per CTA
+    static constexpr int HALF_N = BN / 2;               // most tokens staged per CTA
+    static constexpr int CHU = BN / 16;                 // most 16-token units per chunk
     static constexpr int A_BYTES = BM * 64 * 2;         // 16 KB of packed values
     static constexpr int B_HALF = HALF_N * 64 * 2;      // one 128-byte-wide panel of this CTA's tokens
     static constexpr int B_BYTES = 2 * B_HALF;
     static constexpr int E_BYTES = BM * BK / 8;         // 2 KB of metadata
-    static constexpr int STAGE = ((A_BYTES + B_BYTES + E_BYTES + 1023) / 1024) * 1024;
+    static constexpr int STAGE = ((A_BYTES + B_BYTES + 1023) / 1024) * 1024;
+    static constexpr int MS = 8;                        // metadata slots
+    static constexpr int MLEAD = 4;                     // metadata loads ahead of use (even: per-warp parity)
+    static constexpr int PF = 12;                       // S tiles prefetched into L2 this many stages ahead
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t OVL = (2 * BN + 4 > 512) ? (2 * BN + 4 - 512) : 0;
-    static constexpr uint32_t ACC1 = BN - OVL;          // column of accumulator 1
-    static constexpr uint32_t ECOL = (OVL > 0) ? 508 : 2 * BN;
+    static constexpr uint32_t ACC1 = BN;                // column of accumulator 1
+    static constexpr uint32_t ECOL = 2 * BN;            // metadata columns
     static constexpr int OUT_COLS = 32;
-    static constexpr int OUT_BYTES = OUT_COLS * BM * 2; // one 32-token chunk of this CTA's rows
-    static constexpr int NS_FIT = (232448 - 2 * OUT_BYTES - 3072) / STAGE;
+    static constexpr int OUT_BYTES = OUT_COLS * BM * 2; // one 32-token piece of this CTA's rows
+    static constexpr int FIXED1 = MS * E_BYTES + 1024 + 16 * MS + 16;
+    static constexpr int AVAIL = 232448 - 1024 - FIXED1;
+    // Two output staging buffers unless dropping one buys another stage.
+    static constexpr int NOUT = ((AVAIL - 2 * OUT_BYTES) / STAGE < (AVAIL - OUT_BYTES) / STAGE) ? 1 : 2;
+    static constexpr int NS_FIT = (AVAIL - NOUT * OUT_BYTES) / STAGE;
     static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
     static constexpr int RING = NS * STAGE;
-    static constexpr int BAR_OFF = RING + 2 * OUT_BYTES;
-    static constexpr int DUMMY_OFF = BAR_OFF + 512;     // 16-byte signal slots, one per stage
-    static constexpr int SMEM = DUMMY_OFF + 16 * 8 + 16 + 1024;
+    static constexpr int META_OFF = RING;
+    static constexpr int OUT_OFF = META_OFF + MS * E_BYTES;
+    static constexpr int BAR_OFF = OUT_OFF + NOUT * OUT_BYTES;
+    static constexpr int DUMMY_OFF = BAR_OFF + 1024;    // 16-byte signal slots, one per metadata slot
+    static constexpr int SMEM = DUMMY_OFF + 16 * MS + 16 + 1024;
+    static_assert(BN % 16 == 0 && BN <= 224, "chunk width");
+    static_assert(B_HALF % 1024 == 0, "SW128 panels start on 1 KB");
     static_assert(NS >= 2, "need at least two stages");
+    static_assert(MLEAD < MS && MLEAD % 2 == 0 && MS % 2 == 0, "metadata lead");
     static_assert(SMEM <= 232448, "shared memory budget");
-    static_assert(ECOL + 4 <= TMEM_COLS && ACC1 + BN <= ECOL, "TMEM budget");
-    static_assert(OVL <= 32, "overlap must fit in one drained chunk");
+    static_assert(ECOL + 4 <= TMEM_COLS, "TMEM budget");
+    static_assert((2 * NS + 3 * MS + 4) * 8 + 8 <= 1024, "barrier area");
 };
 
-constexpr int kThreads2 = 224;  // 7 warps
+// Tensor maps of the 2-SM kernel.  xs[i] loads box_rows(i) rows of X for both
+// 64-element K panels of a stage in one copy (a 3-D view of X: element, row,
+// panel), landing as panel 0's rows then panel 1's rows; ts[i] loads
+// box_rows(i) rows of T (one panel).  A chunk uses the smallest box that holds
+// its rows; rows past the chunk are loaded but not read by the MMA.
+struct Maps2 {
+    CUtensorMap vals, meta, u, y32, y16;
+    CUtensorMap xs[5];
+    CUtensorMap ts[5];
+};
+
+__host__ __device__ constexpr int box_rows(int i, int half_n) { return i < 4 ? (8 << i) : half_n; }
+__host__ __device__ constexpr int pick_box(int rows) { return rows <= 8 ? 0 : rows <= 16 ? 1 : rows <= 32 ? 2 : rows <= 64 ? 3 : 4; }
+
+constexpr int kMaxPairs = 128;
+
+struct Params2 {
+    int32_t M;          // tokens
+    int32_t d_out;      // output rows
+    int32_t nk, nlr;    // K stages, rank stages
+    int32_t ut;         // 16-token units per row tile
+    int32_t ttiles;     // token tiles per row tile
+    int32_t wu, wr;     // token tile tt has wu + (tt < wr) units
+    int32_t cyc;        // rounds of the cyclic phase
+    int64_t tail[kMaxPairs + 1];  // pair p's tail units are [tail[p], tail[p+1])
+};
+
+struct Chunk {
+    int32_t d0;         // first output row of the pair's 256-row tile
+    int32_t tok0;       // first token
+    int32_t n;          // tokens (multiple of 16)
+};
+
+// The chunk sequence of one pair; every warp role of the pair walks the same
+// sequence.  All partition parameters are copied into registers when the
+// iterator is built, so the loops never read the kernel parameters again.
+struct ChunkIter {
+    int32_t j, cyc, ut, ttiles, wu, wr, pair, npairs;
+    int64_t lo, hi;
+
+    __device__ __forceinline__ ChunkIter(const Params2 &prm, int pair_, int npairs_)
+        : j(0), cyc(prm.cyc), ut(prm.ut), ttiles(prm.ttiles), wu(prm.wu), wr(prm.wr), pair(pair_), npairs(npairs_),
+          lo(prm.tail[pair_]), hi(prm.tail[pair_ + 1]) {}
+
+    __device__ __forceinline__ bool next(int32_t chu, Chunk &c) {
+        if (j < cyc) {
+            const int64_t tile = (int64_t)j * npairs + (pair + j) % npairs;
+            const int64_t rt = tile / ttiles;
+            const int32_t tt = (int32_t)(tile - rt * ttiles);
+            const int32_t u0 = tt * wu + (tt < wr ? tt : wr);
+            c.d0 = (int32_t)(rt * (2 * BM));
+            c.tok0 = u0 * 16;
+            c.n = (wu + (tt < wr ? 1 : 0)) * 16;
+            ++j;
+            return true;
+        }
+        if (lo >= hi) return false;
+        if ((pair & 1) == 0) {
+            const int64_t rt = lo / ut;
+            const int32_t ui = (int32_t)(lo - rt * ut);
+            const int64_t left = hi - lo, to_end = ut - ui;
+            const int32_t seg = (int32_t)(left < to_end ? left : to_end);
+            const int32_t pieces = (seg + chu - 1) / chu;
+            const int32_t nu = (seg + pieces - 1) / pieces;
+            c.d0 = (int32_t)(rt * (2 * BM));
+            c.tok0 = ui * 16;
+            c.n = nu * 16;
+            lo += nu;
+        } else {
+            const int64_t rt = (hi - 1) / ut;
+            const int64_t start = rt * ut;
+            const int64_t left = hi - lo, to_start = hi - start;
+            const int32_t seg = (int32_t)(left < to_start ? left : to_start);
+            const int32_t pieces = (seg + chu - 1) / chu;
+            const int32_t nu = (seg + pieces - 1) / pieces;
+            c.d0 = (int32_t)(rt * (2 * BM));
+            c.tok0 = (int32_t)(hi - nu - start) * 16;
+            c.n = nu * 16;
+            hi -= nu;
+        }
+        return true;
+    }
+};
+
+// Cursor over a pair's sparse stages (chunk by chunk, nk stages each), for the
+// metadata warp.
+struct SparseCursor {
+    ChunkIter iter;
+    Chunk ch;
+    int32_t ks, nk;
+    bool valid;
+
+    __device__ __forceinline__ SparseCursor(const Params2 &prm, int pair, int npairs, int nk_, int32_t chu)
+        : iter(prm, pair, npairs), ks(0), nk(nk_) {
+        valid = iter.next(chu, ch);
+    }
+    __device__ __forceinline__ void advance(int32_t chu) {
+        if (++ks == nk) {
+            ks = 0;
+            valid = iter.next(chu, ch);
+        }
+    }
+};
+
+constexpr int kThreads2 = 256;  // 8 warps
 
 template <int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
-    tc2_forward_kernel(const __grid_constant__ CUtensorMap tm_vals, const __grid_constant__ CUtensorMap tm_meta,
-                       const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_u,
-                       const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_y,
-                       const Params prm) {
+    tc2_forward_kernel(const __grid_constant__ Maps2 maps, const __grid_constant__ Params2 prm) {
     using C = Cfg2<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
     uint64_t *empty = full + C::NS;
-    uint64_t *ready = empty + C::NS;
-    uint64_t *acc_full = ready + C::NS;
-    uint64_t *acc_ovl = acc_full + 2;
-    uint64_t *acc_empty = acc_ovl + 2;
+    uint64_t *mfull = empty + C::NS;
+    uint64_t *mready = mfull + C::MS;
+    uint64_t *mempty = mready + C::MS;
+    uint64_t *acc_full = mempty + C::MS;
+    uint64_t *acc_empty = acc_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
     volatile uint32_t *fail = tmem_slot + 1;
-    uint8_t *dummy = smem + C::DUMMY_OFF;   // NS signal slots + 1 source slot
+    uint8_t *meta_ring = smem + C::META_OFF;
+    uint8_t *dummy = smem + C::DUMMY_OFF;   // MS signal slots + 1 source slot
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -388,17 +529,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     const bool leader = rank == 0;
     const int pair = blockIdx.x >> 1;
     const int npairs = gridDim.x >> 1;
-    const int nstages = prm.nk + prm.nlr;
+    const int nk = prm.nk;
+    const int nstages = nk + prm.nlr;
+    const int M = prm.M;
+    const int d_out = prm.d_out;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&ready[s], 1);
+        }
+        for (int m = 0; m < C::MS; ++m) {
+            mbar_init(&mfull[m], 1);
+            mbar_init(&mready[m], 1);
+            mbar_init(&mempty[m], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_ovl[b], 8);
             mbar_init(&acc_empty[b], 8);
         }
         *fail = 0;
@@ -411,9 +558,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
     }
     if (threadIdx.x == 0) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_vals)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_meta)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.vals)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.meta)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.xs[4])) : "memory");
     }
     tc_fence_before();
     cluster_sync_all();  // both CTAs' barriers initialised and TMEM allocated
@@ -422,68 +569,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (each CTA)
-        if (lane == 0) {
-            uint32_t s = 0, ph = 0;
-            bool t_ready = false;
-            for (int tile = pair; tile < prm.n_tiles && !*fail; tile += npairs) {
-                const int d0 = (tile / prm.n_ttiles) * (2 * BM) + (int)rank * BM;
-                const int tok0 = (tile % prm.n_ttiles) * BN + (int)rank * C::HALF_N;
-                for (int ks = 0; ks < nstages; ++ks) {
-                    if (!mbar_wait_cluster(&empty[s], ph ^ 1)) {
+        const uint32_t full_leader0 = mapa_shared(smem_u32(&full[0]), 0);
+        uint32_t s = 0, ph = 0;
+        bool t_ready = false;
+        ChunkIter iter(prm, pair, npairs);
+        Chunk ch;
+        while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(C::CHU, ch)) {
+            const int d0 = ch.d0 + (int)rank * BM;
+            const int rows = ch.n / 2;
+            const int tok = ch.tok0 + (int)rank * rows;
+            const int bi = pick_box(rows);
+            const uint32_t brows = (uint32_t)box_rows(bi, C::HALF_N);
+            const CUtensorMap *xmap = &maps.xs[bi];
+            const CUtensorMap *tmap = &maps.ts[bi];
+            for (int ks = 0; ks < nstages; ++ks) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(&empty[s], ph ^ 1))) {
+                    if (lane == 0) {
                         *fail = 1;
                         atomicOr(&g_tc_error, 16u);
-                        break;
                     }
-                    uint8_t *st = smem + s * C::STAGE;
-                    const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES),
-                                   e = smem_u32(st + C::A_BYTES + C::B_BYTES);
-                    if (ks < prm.nk) {
-                        mbar_expect_tx(&full[s], C::A_BYTES + C::B_BYTES + C::E_BYTES);
-                        tma_load_2d(&tm_vals, a, &full[s], ks * 64, d0);
-                        tma_load_2d(&tm_x, b, &full[s], ks * BK, tok0);
-                        tma_load_2d(&tm_x, b + C::B_HALF, &full[s], ks * BK + 64, tok0);
-                        tma_load_2d(&tm_meta, e, &full[s], ks * (BK / 8), d0);
-                    } else {
-                        const int j = ks - prm.nk;
-                        if (!t_ready) {
-                            // T comes from the projection kernel, which may still
-                            // be running (programmatic dependent launch).
-                            asm volatile("griddepcontrol.wait;" ::: "memory");
-                            t_ready = true;
-                        }
-                        mbar_expect_tx(&full[s], C::A_BYTES + C::B_HALF);
-                        tma_load_2d(&tm_u, a, &full[s], j * 64, d0);
-                        tma_load_2d(&tm_t, b, &full[s], j * 64, tok0);
-                    }
-                    if (++s == (uint32_t)C::NS) {
-                        s = 0;
-                        ph ^= 1;
-                    }
-                }
-            }
-        }
-    } else if (warp == 6) {
-        // ------------------------------------------------------------ metadata warp (each CTA)
-        const uint32_t src_slot = smem_u32(dummy + 16 * C::NS);
-        uint32_t s = 0, ph = 0;
-        for (int tile = pair; tile < prm.n_tiles && !*fail; tile += npairs) {
-            bool ok = true;
-            for (int ks = 0; ks < nstages; ++ks) {
-                if (!mbar_wait(&full[s], ph)) {
-                    ok = false;
                     break;
                 }
-                if (ks < prm.nk) {
-                    permute_meta_tile(smem + s * C::STAGE + C::A_BYTES + C::B_BYTES, lane);
-                    fence_proxy_async_smem();
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    if (leader) {
-                        mbar_expect_tx(&ready[s], 16);
-                    } else {
-                        bulk_signal_peer(mapa_shared(smem_u32(dummy + 16 * s), 0), src_slot,
-                                         mapa_shared(smem_u32(&ready[s]), 0));
+                uint8_t *st = smem + s * C::STAGE;
+                const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES);
+                const uint32_t bar = full_leader0 + s * (uint32_t)sizeof(uint64_t);
+                if (ks < nk) {
+                    if (elect_one()) {
+                        if (leader) mbar_expect_tx(&full[s], 2u * (C::A_BYTES + brows * 256u));
+                        tma_load_2d_pair(&maps.vals, a, bar, ks * 64, d0);
+                        tma_load_3d_pair(xmap, b, bar, 0, tok, ks * 2);
+                        // Bring the S tile of a later stage into L2 now, so that
+                        // its load does not wait on HBM.
+                        if (ks + C::PF < nk) {
+                            tma_prefetch_2d(&maps.vals, (ks + C::PF) * 64, d0);
+                            tma_prefetch_2d(&maps.meta, (ks + C::PF) * (BK / 8), d0);
+                        }
+                    }
+                } else {
+                    const int j = ks - nk;
+                    if (!t_ready) {
+                        // T comes from the projection kernel, which may still
+                        // be running (programmatic dependent launch).
+                        asm volatile("griddepcontrol.wait;" ::: "memory");
+                        t_ready = true;
+                    }
+                    if (elect_one()) {
+                        if (leader) mbar_expect_tx(&full[s], 2u * (C::A_BYTES + brows * 128u));
+                        tma_load_2d_pair(&maps.u, a, bar, j * 64, d0);
+                        tma_load_2d_pair(tmap, b, bar, j * 64, tok);
                     }
                 }
                 __syncwarp();
@@ -492,66 +625,150 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
                     ph ^= 1;
                 }
             }
-            if (!ok) {
-                *fail = 1;
-                atomicOr(&g_tc_error, 256u);
+        }
+    } else if (warp >= 6) {
+        // ------------------------------------------------------------ metadata warps (each CTA)
+        // Warp 6 takes the even sparse stages, warp 7 the odd ones; each loads
+        // its tiles MLEAD stages ahead into slots of its own parity.
+        const int par = warp - 6;
+        const uint32_t src_slot = smem_u32(dummy + 16 * C::MS);
+        SparseCursor ld(prm, pair, npairs, nk, C::CHU), use(prm, pair, npairs, nk, C::CHU);
+        if (par) {
+            ld.advance(C::CHU);
+            use.advance(C::CHU);
+        }
+        auto issue = [&](int slot) {
+            if (elect_one()) {
+                mbar_expect_tx(&mfull[slot], C::E_BYTES);
+                tma_load_2d(&maps.meta, smem_u32(meta_ring + slot * C::E_BYTES), &mfull[slot], ld.ks * (BK / 8),
+                            ld.ch.d0 + (int)rank * BM);
+            }
+            __syncwarp();
+            ld.advance(C::CHU);
+            if (ld.valid) ld.advance(C::CHU);
+        };
+        int64_t n_ld = par;
+        for (; n_ld < C::MLEAD && ld.valid; n_ld += 2) issue((int)(n_ld % C::MS));
+        int64_t k = par;
+        while (use.valid && !__any_sync(0xFFFFFFFFu, *fail != 0)) {
+            const int slot = (int)(k % C::MS);
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&mfull[slot], (uint32_t)((k / C::MS) & 1)))) {
+                if (lane == 0) {
+                    *fail = 1;
+                    atomicOr(&g_tc_error, 256u);
+                }
                 break;
             }
+            // Zero-filled rows past d_out carry (0,0) index pairs; only tiles
+            // that reach past d_out need them rewritten.
+            if (use.ch.d0 + (int)rank * BM + BM > d_out)
+                permute_meta_tile<true>(meta_ring + slot * C::E_BYTES, lane);
+            else
+                permute_meta_tile<false>(meta_ring + slot * C::E_BYTES, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (elect_one()) {
+                if (leader) {
+                    mbar_expect_tx(&mready[slot], 16);
+                } else {
+                    bulk_signal_peer(mapa_shared(smem_u32(dummy + 16 * slot), 0), src_slot + 0,
+                                     mapa_shared(smem_u32(&mready[slot]), 0));
+                }
+            }
+            __syncwarp();
+            if (ld.valid) {
+                // The slot of stage n_ld last held stage n_ld - MS; the MMAs
+                // that read it must be done before it is refilled.
+                const int s2 = (int)(n_ld % C::MS);
+                if (n_ld >= C::MS &&
+                    !__all_sync(0xFFFFFFFFu,
+                                mbar_wait_cluster(&mempty[s2], (uint32_t)(((n_ld - C::MS) / C::MS) & 1)))) {
+                    if (lane == 0) {
+                        *fail = 1;
+                        atomicOr(&g_tc_error, 512u);
+                    }
+                    break;
+                }
+                issue(s2);
+                n_ld += 2;
+            }
+            use.advance(C::CHU);
+            if (use.valid) use.advance(C::CHU);
+            k += 2;
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issue (leader, one thread)
-        if (leader && lane == 0) {
-            constexpr uint32_t kIdescSp = idesc_bf16(2 * BM, BN, true);
-            constexpr uint32_t kIdescDense = idesc_bf16(2 * BM, BN, false);
+        // ------------------------------------------------------------ MMA issue (leader CTA)
+        if (leader) {
             const uint32_t e_tmem = tmem_base + C::ECOL;
             uint32_t s = 0, ph = 0;
             int it = 0;
-            for (int tile = pair; tile < prm.n_tiles && !*fail; tile += npairs, ++it) {
+            int64_t k = 0;   // sparse stages consumed (metadata slot sequence)
+            ChunkIter iter(prm, pair, npairs);
+            Chunk ch;
+            while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(C::CHU, ch)) {
+                const uint32_t idesc_sp = idesc_bf16(2 * BM, ch.n, true);
+                const uint32_t idesc_dense = idesc_bf16(2 * BM, ch.n, false);
+                const uint32_t panel = (uint32_t)box_rows(pick_box(ch.n / 2), C::HALF_N) * 128u;
                 const int buf = it & 1;
                 const uint32_t use = (uint32_t)(it >> 1);
-                bool ok = mbar_wait_cluster(&acc_empty[buf], (use & 1) ^ 1);
-                if (ok && C::OVL > 0 && it > 0) ok = mbar_wait_cluster(&acc_ovl[buf ^ 1], ((uint32_t)((it - 1) >> 1)) & 1);
+                bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_cluster(&acc_empty[buf], (use & 1) ^ 1));
                 if (!ok) {
-                    *fail = 1;
-                    atomicOr(&g_tc_error, 32u);
+                    if (lane == 0) {
+                        *fail = 1;
+                        atomicOr(&g_tc_error, 32u);
+                    }
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (buf ? C::ACC1 : 0u);
                 for (int ks = 0; ks < nstages; ++ks) {
-                    if (!mbar_wait_cluster(&ready[s], ph)) {
+                    const bool sparse = ks < nk;
+                    const int m = (int)(k % C::MS);
+                    bool got = mbar_wait_cluster(&full[s], ph);
+                    if (got && sparse) got = mbar_wait_cluster(&mready[m], (uint32_t)((k / C::MS) & 1));
+                    if (!__all_sync(0xFFFFFFFFu, got)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     uint8_t *st = smem + s * C::STAGE;
                     const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES);
-                    if (ks < prm.nk) {
-                        tmem_cp_pair_128x128b(e_tmem, smem_desc(smem_u32(st + C::A_BYTES + C::B_BYTES), 0, 128, kLayoutNone));
+                    if (elect_one()) {
+                        if (sparse) {
+                            tmem_cp_pair_128x128b(e_tmem,
+                                                  smem_desc(smem_u32(meta_ring + m * C::E_BYTES), 0, 128, kLayoutNone));
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const uint64_t adesc = desc_sw128(a + 32 * c);
-                            const uint64_t bdesc = desc_sw128(b + (c >> 1) * C::B_HALF + (c & 1) * 64);
-                            mma_sp_pair(d_tmem, adesc, bdesc, e_tmem + (uint32_t)(c & 2), kIdescSp | (uint32_t)(c & 1),
-                                        (ks | c) != 0);
+                            for (int c = 0; c < 4; ++c) {
+                                const uint64_t adesc = desc_sw128(a + 32 * c);
+                                const uint64_t bdesc = desc_sw128(b + (c >> 1) * panel + (c & 1) * 64);
+                                mma_sp_pair(d_tmem, adesc, bdesc, e_tmem + (uint32_t)(c & 2),
+                                            idesc_sp | (uint32_t)(c & 1), (ks | c) != 0);
+                            }
+                            mma_commit_pair(&mempty[m]);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                mma_dense_pair(d_tmem, desc_sw128(a + 32 * c), desc_sw128(b + 32 * c), idesc_dense, 1u);
                         }
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            mma_dense_pair(d_tmem, desc_sw128(a + 32 * c), desc_sw128(b + 32 * c), kIdescDense, 1u);
+                        mma_commit_pair(&empty[s]);
                     }
-                    mma_commit_pair(&empty[s]);
+                    __syncwarp();
+                    if (sparse) ++k;
                     if (++s == (uint32_t)C::NS) {
                         s = 0;
                         ph ^= 1;
                     }
                 }
                 if (!ok) {
-                    *fail = 1;
-                    atomicOr(&g_tc_error, 64u);
+                    if (lane == 0) {
+                        *fail = 1;
+                        atomicOr(&g_tc_error, 64u);
+                    }
                     break;
                 }
-                mma_commit_pair(&acc_full[buf]);
+                if (elect_one()) mma_commit_pair(&acc_full[buf]);
+                __syncwarp();
+                ++it;
             }
         }
     } else {
@@ -559,15 +776,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const bool store_thread = (warp == 2 && lane == 0);
-        uint8_t *stage_out = smem + C::RING;
-        const uint32_t ovl_leader0 = mapa_shared(smem_u32(&acc_ovl[0]), 0);
+        uint8_t *stage_out = smem + C::OUT_OFF;
         const uint32_t empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
-        constexpr int NQ = BN / 32;
-        uint32_t chunk = 0;
+        uint32_t piece = 0;
         int it = 0;
-        for (int tile = pair; tile < prm.n_tiles && !*fail; tile += npairs, ++it) {
-            const int d0 = (tile / prm.n_ttiles) * (2 * BM) + (int)rank * BM;
-            const int tok0 = (tile % prm.n_ttiles) * BN;
+        ChunkIter iter(prm, pair, npairs);
+        Chunk ch;
+        while (!*fail && iter.next(C::CHU, ch)) {
+            const int d0 = ch.d0 + (int)rank * BM;
             const int buf = it & 1;
             const uint32_t use = (uint32_t)(it >> 1);
             if (!mbar_wait_cluster(&acc_full[buf], use & 1)) {
@@ -576,40 +792,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
                 break;
             }
             tc_fence_after();
-            const uint32_t acc_col = buf ? C::ACC1 : 0u;
-            // The chunk holding the overlap goes first: the last chunk of
-            // buffer 0, the first chunk of buffer 1.
-            const int first_q = (C::OVL > 0 && buf == 0) ? NQ - 1 : 0;
+            const uint32_t acc = tmem_base + ((uint32_t)(quarter * 32) << 16) + (buf ? C::ACC1 : 0u);
+            const int nq = (ch.n + 31) / 32;
 #pragma unroll 1
-            for (int i = 0; i < NQ; ++i) {
-                const int q = (first_q + i) % NQ;
+            for (int q = 0; q < nq; ++q) {
+                const bool wide = ch.n - q * 32 >= 32;   // else a 16-token piece
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc_col + (uint32_t)(q * 32), v);
-                if (i == 0 && C::OVL > 0) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_remote_relaxed(ovl_leader0 + (uint32_t)(buf * sizeof(uint64_t)));
+                if (wide) {
+                    tmem_ld_32x32b_x32(acc + (uint32_t)(q * 32), v);
+                } else {
+                    uint32_t h[16];
+                    tmem_ld_32x32b_x16(acc + (uint32_t)(q * 32), h);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] = h[j];
                 }
-                if (i == NQ - 1) {
+                if (q == nq - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_remote_relaxed(empty_leader0 + (uint32_t)(buf * sizeof(uint64_t)));
                 }
-                if (tok0 + q * C::OUT_COLS >= prm.M) continue;  // uniform across the epilogue warps
-                const uint32_t sb = chunk & 1;
-                if (store_thread) bulk_wait_read1();
+                const int tq = ch.tok0 + q * C::OUT_COLS;
+                if (tq >= M) continue;  // uniform across the epilogue warps
+                const uint32_t sb = C::NOUT == 2 ? (piece & 1) : 0u;
+                if (store_thread) {
+                    if (C::NOUT == 2)
+                        bulk_wait_read1();
+                    else
+                        bulk_wait_read0();
+                }
                 named_bar_sync(1, 128);
                 uint16_t *out = reinterpret_cast<uint16_t *>(stage_out + sb * C::OUT_BYTES);
+                if (wide) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) out[j * BM + row] = f32_to_bf16_bits(__uint_as_float(v[j]));
+                    for (int j = 0; j < 32; ++j) out[j * BM + row] = f32_to_bf16_bits(__uint_as_float(v[j]));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) out[j * BM + row] = f32_to_bf16_bits(__uint_as_float(v[j]));
+                }
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
                 if (store_thread) {
-                    tma_store_2d(&tm_y, smem_u32(out), d0, tok0 + q * C::OUT_COLS);
+                    tma_store_2d(wide ? &maps.y32 : &maps.y16, smem_u32(out), d0, tq);
                     bulk_commit();
                 }
-                ++chunk;
+                ++piece;
             }
+            ++it;
         }
         if (store_thread) bulk_wait_all();
     }
@@ -646,6 +874,21 @@ bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// X [M, d_in] bf16 seen as (element in panel, row, panel) with panels of 64
+// elements: one copy brings `rows` rows of two adjacent 128-byte panels, laid
+// out panel after panel, each in the 128-byte swizzle.
+bool make_map_panels(CUtensorMap *map, const void *X, uint64_t d_in, uint64_t M, uint32_t rows) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[3] = {64, M, d_in / 64};
+    const cuuint64_t strides[2] = {d_in * 2, 128};
+    const cuuint32_t box[3] = {64, rows, 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(X), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int BN, bool kSparse>
@@ -708,36 +951,81 @@ cudaError_t launch_project(const uint16_t *X, int64_t M, const uint16_t *V, int6
 }
 
 
+// Host side of the 2-SM work partition (see the kernel's description): token
+// tiles, the cyclic rounds and the tail ranges, sized so that every pair gets
+// the same number of units in total when the cyclic phase allows it.
+void plan_pairs(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int chu, int max_pairs, Params2 *prm,
+                int *pairs_out) {
+    memset(prm, 0, sizeof *prm);
+    prm->M = (int32_t)M;
+    prm->d_out = (int32_t)d_out;
+    prm->nk = (int32_t)(d_in / BK);
+    prm->nlr = (int32_t)((r + 63) / 64);
+    const int64_t ut = (M + 15) / 16;
+    const int64_t rows = (d_out + 2 * BM - 1) / (2 * BM);
+    const int64_t units = rows * ut;
+    const int64_t ttiles = (ut + chu - 1) / chu;
+    prm->ut = (int32_t)ut;
+    prm->ttiles = (int32_t)ttiles;
+    prm->wu = (int32_t)(ut / ttiles);
+    prm->wr = (int32_t)(ut % ttiles);
+    const int P = (int)(units < max_pairs ? units : max_pairs);
+    const int64_t rounds = rows * ttiles / P;
+    const int64_t cyc = rounds >= 2 ? rounds - 1 : 0;
+    prm->cyc = (int32_t)cyc;
+    const int64_t c_tiles = cyc * P;
+    const int64_t rt_c = c_tiles / ttiles, tt_c = c_tiles % ttiles;
+    const int64_t u_c = rt_c * ut + tt_c * prm->wu + (tt_c < prm->wr ? tt_c : prm->wr);
+    // Units each pair already has from the cyclic phase (bounded work: the
+    // exact sizing is skipped for very long cyclic phases).
+    int64_t cyc_units[kMaxPairs] = {0};
+    bool exact = cyc * P <= (int64_t)1 << 16;
+    for (int p = 0; p < P && exact; ++p)
+        for (int64_t j = 0; j < cyc; ++j) {
+            const int64_t tt = (j * P + (p + j) % P) % ttiles;
+            cyc_units[p] += prm->wu + (tt < prm->wr ? 1 : 0);
+        }
+    int64_t share[kMaxPairs];
+    for (int p = 0; p < P && exact; ++p) {
+        const int64_t target = units * (p + 1) / P - units * p / P;
+        share[p] = target - cyc_units[p];
+        if (share[p] < 0) exact = false;
+    }
+    prm->tail[0] = u_c;
+    for (int p = 0; p < P; ++p)
+        prm->tail[p + 1] = exact ? prm->tail[p] + share[p] : u_c + (units - u_c) * (p + 1) / P;
+    *pairs_out = P;
+}
+
 template <int BN>
 cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
                                uint16_t *Y, bool after_projection, cudaStream_t stream) {
     using C = Cfg2<BN>;
-    CUtensorMap m_vals, m_meta, m_x, m_u, m_t, m_y;
-    memset(&m_u, 0, sizeof m_u);
-    memset(&m_t, 0, sizeof m_t);
-    bool ok = make_map(&m_vals, kBF16, vals, d_in / 2, d_out, d_in, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map(&m_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, d_in / 8, d_out, d_in / 8, 16, BM,
+    Maps2 maps;
+    memset(&maps, 0, sizeof maps);
+    bool ok = make_map(&maps.vals, kBF16, vals, d_in / 2, d_out, d_in, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&maps.meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, d_in / 8, d_out, d_in / 8, 16, BM,
                        CU_TENSOR_MAP_SWIZZLE_NONE) &&
-              make_map(&m_x, kBF16, X, d_in, M, d_in * 2, 64, C::HALF_N, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map(&m_y, kBF16, Y, d_out, M, d_out * 2, BM, C::OUT_COLS, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (ok && r > 0)
-        ok = make_map(&m_u, kBF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_map(&m_t, kBF16, T16, r, M, r * 2, 64, C::HALF_N, CU_TENSOR_MAP_SWIZZLE_128B);
+              make_map(&maps.y32, kBF16, Y, d_out, M, d_out * 2, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map(&maps.y16, kBF16, Y, d_out, M, d_out * 2, BM, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+    for (int i = 0; i < 5 && ok; ++i)
+        ok = make_map_panels(&maps.xs[i], X, d_in, M, (uint32_t)box_rows(i, C::HALF_N));
+    if (ok && r > 0) {
+        ok = make_map(&maps.u, kBF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+        for (int i = 0; i < 5 && ok; ++i)
+            ok = make_map(&maps.ts[i], kBF16, T16, r, M, r * 2, 64, (uint32_t)box_rows(i, C::HALF_N),
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+    }
     if (!ok) return cudaErrorInvalidValue;
-    Params prm;
-    prm.M = (int32_t)M;
-    prm.n_ttiles = (int32_t)((M + BN - 1) / BN);
-    prm.n_tiles = (int32_t)(((d_out + 2 * BM - 1) / (2 * BM)) * prm.n_ttiles);
-    prm.nk = (int32_t)(d_in / BK);
-    prm.nlr = (int32_t)((r + 63) / 64);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaError_t err = cudaFuncSetAttribute(tc2_forward_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (err != cudaSuccess) return err;
-    const int max_pairs = sms / 2;
-    const int pairs = prm.n_tiles < max_pairs ? prm.n_tiles : max_pairs;
+    Params2 prm;
+    int pairs = 0;
+    plan_pairs(M, d_out, d_in, r, C::CHU, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, &prm, &pairs);
     // Directly after the projection kernel on this stream: programmatic
     // dependent launch (the producer waits before it loads T).  Otherwise an
     // ordinary launch, which must not overlap an unrelated preceding kernel.
@@ -751,7 +1039,7 @@ cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *val
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = (after_projection && r > 0) ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, tc2_forward_kernel<BN>, m_vals, m_meta, m_x, m_u, m_t, m_y, prm);
+    return cudaLaunchKernelEx(&cfg, tc2_forward_kernel<BN>, maps, prm);
 }
 
 
@@ -1246,16 +1534,16 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
                               uint16_t *Y, bool after_projection, cudaStream_t stream) {
     if (M <= 0) return cudaSuccess;
     if (M > INT32_MAX || d_out > INT32_MAX || d_in > INT32_MAX) return cudaErrorInvalidValue;
-    // Variant: 2-SM pairs with 256-token tiles once there are enough tokens,
-    // 128-token pair tiles below that.  SLR_TC_KERNEL=1sm|2sm128|2sm256 forces
-    // one (used by the tests and for A/B measurements).
+    // Variant: 2-SM pairs with chunks of up to 192 tokens once there are
+    // enough tokens, up to 128 below that.  SLR_TC_KERNEL=1sm|2sm128|2sm192|small
+    // forces one (used by the tests and for A/B measurements).
     const char *force = getenv("SLR_TC_KERNEL");
     if (force != nullptr) {
         if (strcmp(force, "1sm") == 0) return tc::launch_sparse<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
         if (strcmp(force, "2sm128") == 0)
             return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
-        if (strcmp(force, "2sm256") == 0)
-            return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+        if (strcmp(force, "2sm192") == 0)
+            return tc::launch_sparse_pair<192>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
         if (strcmp(force, "small") == 0 && M <= 64) {
             if (M <= 16) return tc::launch_sparse_small<16>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
             if (M <= 32) return tc::launch_sparse_small<32>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
@@ -1263,12 +1551,13 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
         }
     }
     // Up to 64 tokens the layer streams S: the split-K small-M kernel.  Then
-    // 2-SM pair tiles of 128 tokens, and of 256 tokens from 192 tokens on.
+    // 2-SM pairs with chunks of up to 128 tokens, and of up to 192 tokens from
+    // 192 tokens on.
     if (M <= 16) return tc::launch_sparse_small<16>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     if (M <= 32) return tc::launch_sparse_small<32>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     if (M <= 64) return tc::launch_sparse_small<64>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     if (M >= 192)
-        return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+        return tc::launch_sparse_pair<192>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
 }
 
@@ -1285,6 +1574,26 @@ cudaError_t launch_tc_project(const uint16_t *X, int64_t M, const uint16_t *V, i
     if (M >= 4096) return tc::launch_project<128>(X, M, V, d_in, r, T16, stream);
     if (M >= 1024) return tc::launch_project<64>(X, M, V, d_in, r, T16, stream);
     return tc::launch_project<32>(X, M, V, d_in, r, T16, stream);
+}
+
+namespace tc {
+// Failure-detection self-test: one thread waits, with the kernels' bounded
+// mbarrier wait, on a barrier whose phase nothing completes; when the limit
+// expires it sets bit 12 of the error word and the kernel returns.
+__global__ void wait_timeout_kernel(long long limit_cycles) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait_for(&bar, 0, limit_cycles)) atomicOr(&g_tc_error, 1u << 12);
+}
+}  // namespace tc
+
+cudaError_t launch_wait_timeout_selftest(long long limit_cycles, cudaStream_t stream) {
+    tc::wait_timeout_kernel<<<1, 32, 0, stream>>>(limit_cycles);
+    return cudaGetLastError();
 }
 
 cudaError_t read_and_clear_kernel_error(unsigned *code) {

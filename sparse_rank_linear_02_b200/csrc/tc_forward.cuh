@@ -20,6 +20,10 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
 cudaError_t launch_tc_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in, int64_t r,
                               uint16_t *T16, cudaStream_t stream);
 
+// Launches the failure-detection self-test kernel (a bounded wait that is
+// made to expire after limit_cycles SM clock cycles).
+cudaError_t launch_wait_timeout_selftest(long long limit_cycles, cudaStream_t stream);
+
 // Reads and clears the device-side error word the tensor-core kernel sets when
 // a bounded wait expires (0 = none).  Synchronises the device.
 cudaError_t read_and_clear_kernel_error(unsigned *code);

@@ -37,16 +37,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: false when the phase did not complete within kWaitCycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// Bounded wait: false when the phase did not complete within `limit` SM
+// clock cycles (kWaitCycles in the kernels).
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (clock64() - t0 > kWaitCycles) return false;
+        if (clock64() - t0 > limit) return false;
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    return mbar_wait_for(bar, parity, kWaitCycles);
+}
+
+// One elected lane of a converged warp (the lowest active lane).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
 }
 
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint32_t dst, uint64_t *bar, int32_t c0,
@@ -56,6 +71,36 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint32_t dst
             dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
         : "memory");
+}
+// Tiled load by one CTA of a 2-SM pair whose completion is counted on an
+// mbarrier that may sit in the peer CTA (`bar` is a shared::cluster address):
+// the data land in the executing CTA's shared memory.  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t dst, uint32_t bar, int32_t c0,
+                                                 int32_t c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(const CUtensorMap *map, uint32_t dst, uint32_t bar, int32_t c0,
+                                                 int32_t c1, int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+// L2 prefetch of a tensor tile (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int32_t c0, int32_t c1, int32_t c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
 }
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int32_t c0, int32_t c1) {
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
@@ -171,6 +216,7 @@ __device__ __forceinline__ uint32_t sanitize_nibbles(uint32_t w) {
     return (w & ~(eq * 0xFu)) | (eq * 0x4u);
 }
 
+template <bool kSanitize = true>
 __device__ __forceinline__ void permute_meta_tile(uint8_t *e, int lane) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -179,8 +225,10 @@ __device__ __forceinline__ void permute_meta_tile(uint8_t *e, int lane) {
         uint4 *ra = reinterpret_cast<uint4 *>(e + rowA * 16);
         uint4 *rb = reinterpret_cast<uint4 *>(e + (rowA + 8) * 16);
         uint4 a = *ra, b = *rb;
-        a.x = sanitize_nibbles(a.x); a.y = sanitize_nibbles(a.y); a.z = sanitize_nibbles(a.z); a.w = sanitize_nibbles(a.w);
-        b.x = sanitize_nibbles(b.x); b.y = sanitize_nibbles(b.y); b.z = sanitize_nibbles(b.z); b.w = sanitize_nibbles(b.w);
+        if (kSanitize) {
+            a.x = sanitize_nibbles(a.x); a.y = sanitize_nibbles(a.y); a.z = sanitize_nibbles(a.z); a.w = sanitize_nibbles(a.w);
+            b.x = sanitize_nibbles(b.x); b.y = sanitize_nibbles(b.y); b.z = sanitize_nibbles(b.z); b.w = sanitize_nibbles(b.w);
+        }
         uint4 lo, hi;
         lo.x = __byte_perm(a.x, b.x, 0x5410);
         lo.y = __byte_perm(a.y, b.y, 0x5410);

@@ -116,3 +116,12 @@ def test_pack_argument_errors():
     assert lib.slr_pack_2to4(P(0), 4, 8, 8, P(0x2000), P(0x3000), None) == NULL
     assert lib.slr_pack_2to4(P(0x1000), 4, 8, 8, P(0), P(0x3000), None) == NULL
     assert lib.slr_pack_2to4(P(0), 0, 8, 8, P(0), P(0), None) == OK                    # empty
+
+
+def test_selftest_wait_timeout_arguments():
+    lib = slr.lib()
+    assert lib.slr_selftest_wait_timeout(0, None) == ARG
+    assert lib.slr_selftest_wait_timeout(-1, None) == ARG
+    assert lib.slr_selftest_wait_timeout(1 << 31, None) == ARG
+    if not torch.cuda.is_available():
+        assert lib.slr_selftest_wait_timeout(1000, None) == DEVICE

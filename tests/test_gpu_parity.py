@@ -181,7 +181,7 @@ def test_no_kernel_timeouts():
     slr.check_kernel_error()
 
 
-VARIANTS = ["1sm", "2sm128", "2sm256", "small"]
+VARIANTS = ["1sm", "2sm128", "2sm192", "small"]
 
 
 @pytest.mark.parametrize("variant", VARIANTS)
