@@ -254,7 +254,7 @@ def run_ours(args, rank, world, dist):
     sha = kernel_source_sha()
     traffic = NCU_TRAFFIC.get("tc_forward", {})
     traffic_bytes = traffic.get("bytes_per_launch") if traffic.get("source_sha") == sha else None
-    roofline = {"bound": "tensor", "kernel": "tc2_forward_kernel<192> (2-SM 2:4 tcgen05.mma.sp + rank-r tcgen05.mma, balanced token chunks)",
+    roofline = {"bound": "tensor", "kernel": "tc2t_forward_kernel<240> (2-SM pairs on 512-row tiles: 2:4 tcgen05.mma.sp + rank-r tcgen05.mma)",
                 "achieved": round(achieved_k, 1), "peak": round(peak_k, 1), "unit": "TFLOP/s",
                 "frac": round(achieved_k / peak_k, 4), "traffic": traffic_bytes,
                 "algorithmic_flops_per_launch": k_flops_sp + k_flops_lr,

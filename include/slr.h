@@ -135,7 +135,8 @@ typedef enum slr_path {
                             for one or two tokens)                                  */
     SLR_PATH_TENSOR = 2  /* 2:4 tcgen05 tensor-core kernels with the rank-r term
                             fused: split-K streaming kernel for M <= 64, 2-SM
-                            256-row tiles above                                     */
+                            pairs on 256-row tiles above, on 512-row tiles once
+                            those fill a round of pairs                             */
 } slr_path;
 
 /* The path SLR_PATH_AUTO takes for this problem. */

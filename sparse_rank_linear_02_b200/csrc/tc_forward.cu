@@ -374,8 +374,11 @@ struct Cfg2 {
     static constexpr int MLEAD = 4;                     // metadata loads ahead of use (even: per-warp parity)
     static constexpr int PF = 12;                       // S tiles prefetched into L2 this many stages ahead
     static constexpr uint32_t TMEM_COLS = 512;
+    // Two accumulators when they fit beside the metadata (the epilogue of one
+    // chunk then overlaps the MMAs of the next), else one (BN = 256).
+    static constexpr int NACC = (2 * BN + 4 <= 512) ? 2 : 1;
     static constexpr uint32_t ACC1 = BN;                // column of accumulator 1
-    static constexpr uint32_t ECOL = 2 * BN;            // metadata columns
+    static constexpr uint32_t ECOL = NACC * BN;         // metadata columns
     static constexpr int OUT_COLS = 32;
     static constexpr int OUT_BYTES = OUT_COLS * BM * 2; // one 32-token piece of this CTA's rows
     static constexpr int FIXED1 = MS * E_BYTES + 1024 + 16 * MS + 16;
@@ -390,7 +393,7 @@ struct Cfg2 {
     static constexpr int BAR_OFF = OUT_OFF + NOUT * OUT_BYTES;
     static constexpr int DUMMY_OFF = BAR_OFF + 1024;    // 16-byte signal slots, one per metadata slot
     static constexpr int SMEM = DUMMY_OFF + 16 * MS + 16 + 1024;
-    static_assert(BN % 16 == 0 && BN <= 224, "chunk width");
+    static_assert(BN % 16 == 0 && BN <= 256, "chunk width");
     static_assert(B_HALF % 1024 == 0, "SW128 panels start on 1 KB");
     static_assert(NS >= 2, "need at least two stages");
     static_assert(MLEAD < MS && MLEAD % 2 == 0 && MS % 2 == 0, "metadata lead");
@@ -418,11 +421,13 @@ constexpr int kMaxPairs = 128;
 struct Params2 {
     int32_t M;          // tokens
     int32_t d_out;      // output rows
+    int32_t tile_rows;  // output rows per pair tile (256 or 512)
     int32_t nk, nlr;    // K stages, rank stages
     int32_t ut;         // 16-token units per row tile
     int32_t ttiles;     // token tiles per row tile
     int32_t wu, wr;     // token tile tt has wu + (tt < wr) units
     int32_t cyc;        // rounds of the cyclic phase
+    int64_t n_tiles;    // tiles dealt in the cyclic phase (a last round may be partial)
     int64_t tail[kMaxPairs + 1];  // pair p's tail units are [tail[p], tail[p+1])
 };
 
@@ -436,20 +441,20 @@ struct Chunk {
 // sequence.  All partition parameters are copied into registers when the
 // iterator is built, so the loops never read the kernel parameters again.
 struct ChunkIter {
-    int32_t j, cyc, ut, ttiles, wu, wr, pair, npairs;
-    int64_t lo, hi;
+    int32_t j, cyc, ut, ttiles, wu, wr, pair, npairs, tile_rows;
+    int64_t n_tiles, lo, hi;
 
-    __device__ __forceinline__ ChunkIter(const Params2 &prm, int pair_, int npairs_)
+    __host__ __device__ __forceinline__ ChunkIter(const Params2 &prm, int pair_, int npairs_)
         : j(0), cyc(prm.cyc), ut(prm.ut), ttiles(prm.ttiles), wu(prm.wu), wr(prm.wr), pair(pair_), npairs(npairs_),
-          lo(prm.tail[pair_]), hi(prm.tail[pair_ + 1]) {}
+          tile_rows(prm.tile_rows), n_tiles(prm.n_tiles), lo(prm.tail[pair_]), hi(prm.tail[pair_ + 1]) {}
 
-    __device__ __forceinline__ bool next(int32_t chu, Chunk &c) {
-        if (j < cyc) {
-            const int64_t tile = (int64_t)j * npairs + (pair + j) % npairs;
+    __host__ __device__ __forceinline__ bool next(int32_t chu, Chunk &c) {
+        const int64_t tile = (int64_t)j * npairs + (pair + j) % npairs;
+        if (j < cyc && tile < n_tiles) {
             const int64_t rt = tile / ttiles;
             const int32_t tt = (int32_t)(tile - rt * ttiles);
             const int32_t u0 = tt * wu + (tt < wr ? tt : wr);
-            c.d0 = (int32_t)(rt * (2 * BM));
+            c.d0 = (int32_t)(rt * tile_rows);
             c.tok0 = u0 * 16;
             c.n = (wu + (tt < wr ? 1 : 0)) * 16;
             ++j;
@@ -463,7 +468,7 @@ struct ChunkIter {
             const int32_t seg = (int32_t)(left < to_end ? left : to_end);
             const int32_t pieces = (seg + chu - 1) / chu;
             const int32_t nu = (seg + pieces - 1) / pieces;
-            c.d0 = (int32_t)(rt * (2 * BM));
+            c.d0 = (int32_t)(rt * tile_rows);
             c.tok0 = ui * 16;
             c.n = nu * 16;
             lo += nu;
@@ -474,7 +479,7 @@ struct ChunkIter {
             const int32_t seg = (int32_t)(left < to_start ? left : to_start);
             const int32_t pieces = (seg + chu - 1) / chu;
             const int32_t nu = (seg + pieces - 1) / pieces;
-            c.d0 = (int32_t)(rt * (2 * BM));
+            c.d0 = (int32_t)(rt * tile_rows);
             c.tok0 = (int32_t)(hi - nu - start) * 16;
             c.n = nu * 16;
             hi -= nu;
@@ -709,8 +714,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
                 const uint32_t idesc_sp = idesc_bf16(2 * BM, ch.n, true);
                 const uint32_t idesc_dense = idesc_bf16(2 * BM, ch.n, false);
                 const uint32_t panel = (uint32_t)box_rows(pick_box(ch.n / 2), C::HALF_N) * 128u;
-                const int buf = it & 1;
-                const uint32_t use = (uint32_t)(it >> 1);
+                const int buf = C::NACC == 2 ? (it & 1) : 0;
+                const uint32_t use = (uint32_t)(C::NACC == 2 ? (it >> 1) : it);
                 bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_cluster(&acc_empty[buf], (use & 1) ^ 1));
                 if (!ok) {
                     if (lane == 0) {
@@ -784,8 +789,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         Chunk ch;
         while (!*fail && iter.next(C::CHU, ch)) {
             const int d0 = ch.d0 + (int)rank * BM;
-            const int buf = it & 1;
-            const uint32_t use = (uint32_t)(it >> 1);
+            const int buf = C::NACC == 2 ? (it & 1) : 0;
+            const uint32_t use = (uint32_t)(C::NACC == 2 ? (it >> 1) : it);
             if (!mbar_wait_cluster(&acc_full[buf], use & 1)) {
                 *fail = 1;
                 atomicOr(&g_tc_error, 128u);
@@ -836,6 +841,403 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
                     bulk_commit();
                 }
                 ++piece;
+            }
+            ++it;
+        }
+        if (store_thread) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    cluster_sync_all();  // the pair's MMAs, signals and stores are done before TMEM is freed
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+    }
+}
+
+// =====================================================================================
+// Tall 2-SM variant for large M: a pair computes 512 output rows (two 256-row
+// halves, each one M=256 cta_group::2 MMA) x n tokens, and both halves read
+// the same staged X tile.  Against 256-row pair tiles this halves the number
+// of times X crosses from L2 into shared memory (the kernel is bound by that
+// traffic: with 256 x 192 tiles on the Llama-3-8B gate/up layer, X is read
+// once per 256-row tile, 56 times in all).  CTA rank q stages rows
+// 256h + 128q .. +127 of half h of the S tile and tokens q*n/2 .. of X.
+//
+// TMEM: accumulator h at columns h*BN (2*BN + 8 <= 512, no double
+// buffering), metadata of half h at 2*BN + 4h.  The epilogue (8 warps, four
+// per half) drains both accumulators after a chunk's last stage; the next
+// chunk's MMAs wait for that drain.  Everything else follows the 256-row
+// kernel: stage loads of both CTAs complete on the leader's full[s], the
+// metadata ring (4 KB per stage: both halves) is loaded MLEAD stages ahead
+// and permuted by two warps (even / odd stages), and the producer and MMA
+// warps run converged with one elected lane issuing.
+template <int BN>
+struct CfgT {
+    static constexpr int HALF_N = BN / 2;               // most tokens staged per CTA
+    static constexpr int CHU = BN / 16;                 // most 16-token units per chunk
+    static constexpr int A_BYTES = BM * 64 * 2;         // 16 KB of packed values per half
+    static constexpr int B_HALF = HALF_N * 64 * 2;      // one 128-byte-wide panel of this CTA's tokens
+    static constexpr int B_BYTES = 2 * B_HALF;
+    static constexpr int B_OFF = 2 * A_BYTES;
+    static constexpr int E_BYTES = BM * BK / 8;         // 2 KB of metadata per half
+    static constexpr int STAGE = ((2 * A_BYTES + B_BYTES + 1023) / 1024) * 1024;
+    static constexpr int MS = 5;                        // metadata slots (both halves each)
+    static constexpr int MLEAD = 2;                     // metadata loads ahead of use (even: per-warp parity)
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t ECOL = 2 * BN;            // metadata columns (4 per half)
+    static constexpr int OUT_COLS = 32;
+    static constexpr int OUT_BYTES = OUT_COLS * BM * 2; // one 32-token piece of one half's rows
+    static constexpr int FIXED = MS * 2 * E_BYTES + 2 * OUT_BYTES + 1024 + 16 * MS + 16;
+    static constexpr int NS_FIT = (232448 - 1024 - FIXED) / STAGE;
+    static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
+    static constexpr int RING = NS * STAGE;
+    static constexpr int META_OFF = RING;
+    static constexpr int OUT_OFF = META_OFF + MS * 2 * E_BYTES;
+    static constexpr int BAR_OFF = OUT_OFF + 2 * OUT_BYTES;
+    static constexpr int DUMMY_OFF = BAR_OFF + 1024;
+    static constexpr int SMEM = DUMMY_OFF + 16 * MS + 16 + 1024;
+    static_assert(BN % 16 == 0 && 2 * BN + 8 <= 512, "TMEM budget");
+    static_assert(B_HALF % 1024 == 0, "SW128 panels start on 1 KB");
+    static_assert(NS >= 2, "need at least two stages");
+    static_assert(MLEAD < MS && MLEAD % 2 == 0, "metadata lead");
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert((2 * NS + 3 * MS + 4) * 8 + 8 <= 1024, "barrier area");
+};
+
+constexpr int kThreadsT = 384;  // 12 warps
+
+template <int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
+    tc2t_forward_kernel(const __grid_constant__ Maps2 maps, const __grid_constant__ Params2 prm) {
+    using C = CfgT<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *empty = full + C::NS;
+    uint64_t *mfull = empty + C::NS;
+    uint64_t *mready = mfull + C::MS;
+    uint64_t *mempty = mready + C::MS;
+    uint64_t *acc_full = mempty + C::MS;
+    uint64_t *acc_empty = acc_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
+    volatile uint32_t *fail = tmem_slot + 1;
+    uint8_t *meta_ring = smem + C::META_OFF;
+    uint8_t *dummy = smem + C::DUMMY_OFF;   // MS signal slots + 1 source slot
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+    const int nk = prm.nk;
+    const int nstages = nk + prm.nlr;
+    const int M = prm.M;
+    const int d_out = prm.d_out;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int m = 0; m < C::MS; ++m) {
+            mbar_init(&mfull[m], 1);
+            mbar_init(&mready[m], 1);
+            mbar_init(&mempty[m], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 16);
+        *fail = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    if (threadIdx.x == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.vals)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.meta)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.xs[4])) : "memory");
+    }
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs' barriers initialised and TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (each CTA)
+        const uint32_t full_leader0 = mapa_shared(smem_u32(&full[0]), 0);
+        uint32_t s = 0, ph = 0;
+        bool t_ready = false;
+        ChunkIter iter(prm, pair, npairs);
+        Chunk ch;
+        while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(C::CHU, ch)) {
+            const int d0 = ch.d0 + (int)rank * BM;        // half 0 rows of this CTA; half 1 at +256
+            const int rows = ch.n / 2;
+            const int tok = ch.tok0 + (int)rank * rows;
+            const int bi = pick_box(rows);
+            const uint32_t brows = (uint32_t)box_rows(bi, C::HALF_N);
+            const CUtensorMap *xmap = &maps.xs[bi];
+            const CUtensorMap *tmap = &maps.ts[bi];
+            for (int ks = 0; ks < nstages; ++ks) {
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(&empty[s], ph ^ 1))) {
+                    if (lane == 0) {
+                        *fail = 1;
+                        atomicOr(&g_tc_error, 16u);
+                    }
+                    break;
+                }
+                uint8_t *st = smem + s * C::STAGE;
+                const uint32_t a = smem_u32(st), b = smem_u32(st + C::B_OFF);
+                const uint32_t bar = full_leader0 + s * (uint32_t)sizeof(uint64_t);
+                if (ks < nk) {
+                    if (elect_one()) {
+                        if (leader) mbar_expect_tx(&full[s], 2u * (2u * C::A_BYTES + brows * 256u));
+                        tma_load_2d_pair(&maps.vals, a, bar, ks * 64, d0);
+                        tma_load_2d_pair(&maps.vals, a + C::A_BYTES, bar, ks * 64, d0 + 2 * BM);
+                        tma_load_3d_pair(xmap, b, bar, 0, tok, ks * 2);
+                    }
+                } else {
+                    const int j = ks - nk;
+                    if (!t_ready) {
+                        // T comes from the projection kernel, which may still
+                        // be running (programmatic dependent launch).
+                        asm volatile("griddepcontrol.wait;" ::: "memory");
+                        t_ready = true;
+                    }
+                    if (elect_one()) {
+                        if (leader) mbar_expect_tx(&full[s], 2u * (2u * C::A_BYTES + brows * 128u));
+                        tma_load_2d_pair(&maps.u, a, bar, j * 64, d0);
+                        tma_load_2d_pair(&maps.u, a + C::A_BYTES, bar, j * 64, d0 + 2 * BM);
+                        tma_load_2d_pair(tmap, b, bar, j * 64, tok);
+                    }
+                }
+                __syncwarp();
+                if (++s == (uint32_t)C::NS) {
+                    s = 0;
+                    ph ^= 1;
+                }
+            }
+        }
+    } else if (warp >= 10) {
+        // ------------------------------------------------------------ metadata warps (each CTA)
+        // Warp 10 takes the even sparse stages, warp 11 the odd ones; a slot
+        // holds both halves' tiles (2 x 2 KB).
+        const int par = warp - 10;
+        const uint32_t src_slot = smem_u32(dummy + 16 * C::MS);
+        SparseCursor ld(prm, pair, npairs, nk, C::CHU), use(prm, pair, npairs, nk, C::CHU);
+        if (par) {
+            ld.advance(C::CHU);
+            use.advance(C::CHU);
+        }
+        auto issue = [&](int slot) {
+            if (elect_one()) {
+                uint8_t *e = meta_ring + slot * 2 * C::E_BYTES;
+                mbar_expect_tx(&mfull[slot], 2 * C::E_BYTES);
+                const int r0 = ld.ch.d0 + (int)rank * BM;
+                tma_load_2d(&maps.meta, smem_u32(e), &mfull[slot], ld.ks * (BK / 8), r0);
+                tma_load_2d(&maps.meta, smem_u32(e + C::E_BYTES), &mfull[slot], ld.ks * (BK / 8), r0 + 2 * BM);
+            }
+            __syncwarp();
+            ld.advance(C::CHU);
+            if (ld.valid) ld.advance(C::CHU);
+        };
+        int64_t n_ld = par;
+        for (; n_ld < C::MLEAD && ld.valid; n_ld += 2) issue((int)(n_ld % C::MS));
+        int64_t k = par;
+        while (use.valid && !__any_sync(0xFFFFFFFFu, *fail != 0)) {
+            const int slot = (int)(k % C::MS);
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&mfull[slot], (uint32_t)((k / C::MS) & 1)))) {
+                if (lane == 0) {
+                    *fail = 1;
+                    atomicOr(&g_tc_error, 256u);
+                }
+                break;
+            }
+            uint8_t *e = meta_ring + slot * 2 * C::E_BYTES;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                // Zero-filled rows past d_out carry (0,0) index pairs; only
+                // tiles that reach past d_out need them rewritten.
+                if (use.ch.d0 + h * 2 * BM + (int)rank * BM + BM > d_out)
+                    permute_meta_tile<true>(e + h * C::E_BYTES, lane);
+                else
+                    permute_meta_tile<false>(e + h * C::E_BYTES, lane);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (elect_one()) {
+                if (leader) {
+                    mbar_expect_tx(&mready[slot], 16);
+                } else {
+                    bulk_signal_peer(mapa_shared(smem_u32(dummy + 16 * slot), 0), src_slot,
+                                     mapa_shared(smem_u32(&mready[slot]), 0));
+                }
+            }
+            __syncwarp();
+            if (ld.valid) {
+                // The slot of stage n_ld last held stage n_ld - MS; the MMAs
+                // that read it must be done before it is refilled.
+                const int s2 = (int)(n_ld % C::MS);
+                if (n_ld >= C::MS &&
+                    !__all_sync(0xFFFFFFFFu,
+                                mbar_wait_cluster(&mempty[s2], (uint32_t)(((n_ld - C::MS) / C::MS) & 1)))) {
+                    if (lane == 0) {
+                        *fail = 1;
+                        atomicOr(&g_tc_error, 512u);
+                    }
+                    break;
+                }
+                issue(s2);
+                n_ld += 2;
+            }
+            use.advance(C::CHU);
+            if (use.valid) use.advance(C::CHU);
+            k += 2;
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issue (leader CTA)
+        if (leader) {
+            const uint32_t e_tmem = tmem_base + C::ECOL;
+            uint32_t s = 0, ph = 0;
+            int it = 0;
+            int64_t k = 0;   // sparse stages consumed (metadata slot sequence)
+            ChunkIter iter(prm, pair, npairs);
+            Chunk ch;
+            while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(C::CHU, ch)) {
+                const uint32_t idesc_sp = idesc_bf16(2 * BM, ch.n, true);
+                const uint32_t idesc_dense = idesc_bf16(2 * BM, ch.n, false);
+                const uint32_t panel = (uint32_t)box_rows(pick_box(ch.n / 2), C::HALF_N) * 128u;
+                bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_cluster(acc_empty, (uint32_t)((it & 1) ^ 1)));
+                if (!ok) {
+                    if (lane == 0) {
+                        *fail = 1;
+                        atomicOr(&g_tc_error, 32u);
+                    }
+                    break;
+                }
+                tc_fence_after();
+                for (int ks = 0; ks < nstages; ++ks) {
+                    const bool sparse = ks < nk;
+                    const int m = (int)(k % C::MS);
+                    bool got = mbar_wait_cluster(&full[s], ph);
+                    if (got && sparse) got = mbar_wait_cluster(&mready[m], (uint32_t)((k / C::MS) & 1));
+                    if (!__all_sync(0xFFFFFFFFu, got)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint8_t *st = smem + s * C::STAGE;
+                    const uint32_t a = smem_u32(st), b = smem_u32(st + C::B_OFF);
+                    if (elect_one()) {
+                        if (sparse) {
+                            const uint32_t e = smem_u32(meta_ring + m * 2 * C::E_BYTES);
+                            tmem_cp_pair_128x128b(e_tmem, smem_desc(e, 0, 128, kLayoutNone));
+                            tmem_cp_pair_128x128b(e_tmem + 4, smem_desc(e + C::E_BYTES, 0, 128, kLayoutNone));
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                                for (int c = 0; c < 4; ++c) {
+                                    const uint64_t adesc = desc_sw128(a + h * C::A_BYTES + 32 * c);
+                                    const uint64_t bdesc = desc_sw128(b + (c >> 1) * panel + (c & 1) * 64);
+                                    mma_sp_pair(tmem_base + h * BN, adesc, bdesc, e_tmem + 4 * h + (uint32_t)(c & 2),
+                                                idesc_sp | (uint32_t)(c & 1), (ks | c) != 0);
+                                }
+                            mma_commit_pair(&mempty[m]);
+                        } else {
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                                for (int c = 0; c < 4; ++c)
+                                    mma_dense_pair(tmem_base + h * BN, desc_sw128(a + h * C::A_BYTES + 32 * c),
+                                                   desc_sw128(b + 32 * c), idesc_dense, 1u);
+                        }
+                        mma_commit_pair(&empty[s]);
+                    }
+                    __syncwarp();
+                    if (sparse) ++k;
+                    if (++s == (uint32_t)C::NS) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                if (!ok) {
+                    if (lane == 0) {
+                        *fail = 1;
+                        atomicOr(&g_tc_error, 64u);
+                    }
+                    break;
+                }
+                if (elect_one()) mma_commit_pair(acc_full);
+                __syncwarp();
+                ++it;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2..9)
+        // Warps 2..5 drain accumulator 0, warps 6..9 accumulator 1; each warp
+        // reads the TMEM lanes of its quadrant (warp % 4), one output row per
+        // thread.  The drain is on the critical path (the next chunk's MMAs
+        // wait for both accumulators), so a thread first moves its row of the
+        // chunk from TMEM into registers as packed bf16 (RNE) and releases the
+        // accumulators; the stores (32-token pieces staged in shared memory,
+        // TMA-stored) then overlap the next chunk's main loop.
+        constexpr int kPieces = BN / 16;
+        const int grp = (warp - 2) >> 2;
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const bool store_thread = ((warp - 2) % 4 == 0 && lane == 0);
+        uint16_t *out = reinterpret_cast<uint16_t *>(smem + C::OUT_OFF + grp * C::OUT_BYTES);
+        const uint32_t empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+        int it = 0;
+        ChunkIter iter(prm, pair, npairs);
+        Chunk ch;
+        while (!*fail && iter.next(C::CHU, ch)) {
+            const int d0 = ch.d0 + grp * 2 * BM + (int)rank * BM;
+            if (!mbar_wait_cluster(acc_full, (uint32_t)(it & 1))) {
+                *fail = 1;
+                atomicOr(&g_tc_error, 128u);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t acc = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(grp * BN);
+            uint32_t packed[kPieces * 8];
+#pragma unroll
+            for (int q = 0; q < kPieces; ++q) {
+                if (q * 16 < ch.n) {
+                    uint32_t h[16];
+                    tmem_ld_32x32b_x16(acc + (uint32_t)(q * 16), h);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        packed[q * 8 + j] = (uint32_t)f32_to_bf16_bits(__uint_as_float(h[2 * j])) |
+                                            ((uint32_t)f32_to_bf16_bits(__uint_as_float(h[2 * j + 1])) << 16);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote_relaxed(empty_leader);
+#pragma unroll
+            for (int p = 0; p < (kPieces + 1) / 2; ++p) {
+                const int tq = ch.tok0 + 32 * p;
+                if (32 * p < ch.n && tq < M) {          // uniform across the group's warps
+                    const bool wide = ch.n - 32 * p >= 32;
+                    if (store_thread) bulk_wait_read0();
+                    named_bar_sync(1 + grp, 128);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if (2 * p + (j >> 4) < kPieces && (wide || j < 16))
+                            out[j * BM + row] = (uint16_t)(packed[(2 * p + (j >> 4)) * 8 + ((j & 15) >> 1)] >> (16 * (j & 1)));
+                    }
+                    fence_proxy_async_smem();
+                    named_bar_sync(1 + grp, 128);
+                    if (store_thread) {
+                        tma_store_2d(wide ? &maps.y32 : &maps.y16, smem_u32(out), d0, tq);
+                        bulk_commit();
+                    }
+                }
             }
             ++it;
         }
@@ -954,15 +1356,16 @@ cudaError_t launch_project(const uint16_t *X, int64_t M, const uint16_t *V, int6
 // Host side of the 2-SM work partition (see the kernel's description): token
 // tiles, the cyclic rounds and the tail ranges, sized so that every pair gets
 // the same number of units in total when the cyclic phase allows it.
-void plan_pairs(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int chu, int max_pairs, Params2 *prm,
-                int *pairs_out) {
+void plan_pairs(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int chu, int tile_rows, int max_pairs,
+                bool split_tail, Params2 *prm, int *pairs_out) {
     memset(prm, 0, sizeof *prm);
     prm->M = (int32_t)M;
     prm->d_out = (int32_t)d_out;
+    prm->tile_rows = tile_rows;
     prm->nk = (int32_t)(d_in / BK);
     prm->nlr = (int32_t)((r + 63) / 64);
     const int64_t ut = (M + 15) / 16;
-    const int64_t rows = (d_out + 2 * BM - 1) / (2 * BM);
+    const int64_t rows = (d_out + tile_rows - 1) / tile_rows;
     const int64_t units = rows * ut;
     const int64_t ttiles = (ut + chu - 1) / chu;
     prm->ut = (int32_t)ut;
@@ -970,37 +1373,74 @@ void plan_pairs(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int chu, int 
     prm->wu = (int32_t)(ut / ttiles);
     prm->wr = (int32_t)(ut % ttiles);
     const int P = (int)(units < max_pairs ? units : max_pairs);
-    const int64_t rounds = rows * ttiles / P;
-    const int64_t cyc = rounds >= 2 ? rounds - 1 : 0;
+    // Whole rounds of tiles first.  With split_tail the tiles of the last,
+    // partial round are then split among all pairs, each pair taking one
+    // piece of one tile (a piece never crosses a tile, so no pair gets an
+    // extra chunk); without it the last round is dealt as whole tiles too.
+    const int64_t T = rows * ttiles;
+    prm->n_tiles = T;
+    if (!split_tail) {
+        prm->cyc = (int32_t)((T + P - 1) / P);
+        for (int p = 0; p <= P; ++p) prm->tail[p] = units;
+        *pairs_out = P;
+        return;
+    }
+    const int64_t cyc = T / P;
     prm->cyc = (int32_t)cyc;
     const int64_t c_tiles = cyc * P;
-    const int64_t rt_c = c_tiles / ttiles, tt_c = c_tiles % ttiles;
-    const int64_t u_c = rt_c * ut + tt_c * prm->wu + (tt_c < prm->wr ? tt_c : prm->wr);
-    // Units each pair already has from the cyclic phase (bounded work: the
-    // exact sizing is skipped for very long cyclic phases).
-    int64_t cyc_units[kMaxPairs] = {0};
-    bool exact = cyc * P <= (int64_t)1 << 16;
-    for (int p = 0; p < P && exact; ++p)
-        for (int64_t j = 0; j < cyc; ++j) {
-            const int64_t tt = (j * P + (p + j) % P) % ttiles;
-            cyc_units[p] += prm->wu + (tt < prm->wr ? 1 : 0);
+    const int64_t rem = T - c_tiles;                   // tiles left, fewer than P
+    auto tile_u0 = [&](int64_t tile) {                 // first unit of a tile, row-major unit order
+        const int64_t rt = tile / ttiles, tt = tile % ttiles;
+        return rt * ut + tt * prm->wu + (tt < prm->wr ? tt : prm->wr);
+    };
+    prm->tail[0] = rem > 0 ? tile_u0(c_tiles) : units;
+    if (rem == 0) {
+        for (int p = 0; p < P; ++p) prm->tail[p + 1] = units;
+    } else {
+        // Pairs [first(i), first(i+1)) share tile c_tiles + i.
+        int p = 0;
+        for (int64_t i = 0; i < rem; ++i) {
+            const int first = (int)(i * P / rem), last = (int)((i + 1) * P / rem);
+            const int g = last - first;
+            const int64_t u0 = tile_u0(c_tiles + i);
+            const int64_t nu = (c_tiles + i + 1 < T) ? tile_u0(c_tiles + i + 1) - u0 : units - u0;
+            for (int k = 1; k <= g; ++k, ++p) prm->tail[p + 1] = u0 + nu * k / g;
         }
-    int64_t share[kMaxPairs];
-    for (int p = 0; p < P && exact; ++p) {
-        const int64_t target = units * (p + 1) / P - units * p / P;
-        share[p] = target - cyc_units[p];
-        if (share[p] < 0) exact = false;
     }
-    prm->tail[0] = u_c;
-    for (int p = 0; p < P; ++p)
-        prm->tail[p + 1] = exact ? prm->tail[p] + share[p] : u_c + (units - u_c) * (p + 1) / P;
     *pairs_out = P;
+}
+
+// Estimated cycles of the slowest pair for a plan: per chunk, its stages at
+// the larger of the MMA time and the operand bytes over the shared-memory fill
+// rate one SM sustains (about 44 B per cycle measured on B200 for these TMA
+// tiles), plus a fixed cost per chunk (the accumulator drain of the 512-row
+// kernel is not overlapped).  Only used to rank plans.
+double plan_cycles(const Params2 &prm, int pairs, int chu, int half_n, int mode) {
+    // mode 0: 256-row tiles, two accumulators; 1: 256-row, one accumulator;
+    // 2: 512-row tiles (one accumulator per half).
+    const int nstages = prm.nk + prm.nlr;
+    const bool tall = mode == 2;
+    const double overhead = mode == 0 ? 800.0 : 3000.0;
+    double worst = 0;
+    for (int p = 0; p < pairs; ++p) {
+        ChunkIter it(prm, p, pairs);
+        Chunk ch;
+        double cyc = 0;
+        while (it.next(chu, ch)) {
+            const double brows = box_rows(pick_box(ch.n / 2), half_n);
+            const double bytes = tall ? 2.0 * 16384 + brows * 256 + 4096 : 16384 + brows * 256 + 2048;
+            const double mma = (tall ? 4.0 : 2.0) * ch.n;
+            cyc += nstages * (mma > bytes / 44.0 ? mma : bytes / 44.0) + overhead;
+        }
+        if (cyc > worst) worst = cyc;
+    }
+    return worst;
 }
 
 template <int BN>
 cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
-                               uint16_t *Y, bool after_projection, cudaStream_t stream) {
+                               uint16_t *Y, bool after_projection, bool split_tail, cudaStream_t stream) {
     using C = Cfg2<BN>;
     Maps2 maps;
     memset(&maps, 0, sizeof maps);
@@ -1025,7 +1465,7 @@ cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *val
     if (err != cudaSuccess) return err;
     Params2 prm;
     int pairs = 0;
-    plan_pairs(M, d_out, d_in, r, C::CHU, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, &prm, &pairs);
+    plan_pairs(M, d_out, d_in, r, C::CHU, 2 * BM, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, split_tail, &prm, &pairs);
     // Directly after the projection kernel on this stream: programmatic
     // dependent launch (the producer waits before it loads T).  Otherwise an
     // ordinary launch, which must not overlap an unrelated preceding kernel.
@@ -1040,6 +1480,51 @@ cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *val
     cfg.attrs = attr;
     cfg.numAttrs = (after_projection && r > 0) ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, tc2_forward_kernel<BN>, maps, prm);
+}
+
+template <int BN>
+cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
+                               int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
+                               uint16_t *Y, bool after_projection, bool split_tail, cudaStream_t stream) {
+    using C = CfgT<BN>;
+    Maps2 maps;
+    memset(&maps, 0, sizeof maps);
+    bool ok = make_map(&maps.vals, kBF16, vals, d_in / 2, d_out, d_in, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&maps.meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, d_in / 8, d_out, d_in / 8, 16, BM,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map(&maps.y32, kBF16, Y, d_out, M, d_out * 2, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map(&maps.y16, kBF16, Y, d_out, M, d_out * 2, BM, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+    for (int i = 0; i < 5 && ok; ++i)
+        ok = make_map_panels(&maps.xs[i], X, d_in, M, (uint32_t)box_rows(i, C::HALF_N));
+    if (ok && r > 0) {
+        ok = make_map(&maps.u, kBF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+        for (int i = 0; i < 5 && ok; ++i)
+            ok = make_map(&maps.ts[i], kBF16, T16, r, M, r * 2, 64, (uint32_t)box_rows(i, C::HALF_N),
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t err = cudaFuncSetAttribute(tc2t_forward_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (err != cudaSuccess) return err;
+    Params2 prm;
+    int pairs = 0;
+    plan_pairs(M, d_out, d_in, r, C::CHU, 4 * BM, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, split_tail, &prm, &pairs);
+    // Directly after the projection kernel on this stream: programmatic
+    // dependent launch (the producer waits before it loads T).  Otherwise an
+    // ordinary launch, which must not overlap an unrelated preceding kernel.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(kThreadsT);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (after_projection && r > 0) ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, tc2t_forward_kernel<BN>, maps, prm);
 }
 
 
@@ -1244,10 +1729,11 @@ cudaError_t launch_project_splitk(const uint16_t *X, int64_t M, const uint16_t *
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int tiles = (int)((M + BM - 1) / BM);
     const int nk = (int)(d_in / 64);
-    // Split K over a cluster of up to 4 CTAs (clusters of 8 large CTAs do not
-    // all fit at once), keeping the grid within about one wave.
+    // Split K over a cluster of up to 8 CTAs, keeping the grid within one
+    // SM's worth of CTAs per SM (clusters of 8 only when few token tiles make
+    // the K loop long per CTA).
     int ks = 1;
-    while (ks < 4 && ks * 2 <= nk && tiles * ks * 2 <= 2 * sms) ks *= 2;
+    while (ks < 8 && ks * 2 <= nk && tiles * ks * 2 <= (ks >= 4 ? sms : 2 * sms)) ks *= 2;
     cudaError_t err = cudaFuncSetAttribute(tc_project_kernel<RN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -1534,31 +2020,69 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
                               uint16_t *Y, bool after_projection, cudaStream_t stream) {
     if (M <= 0) return cudaSuccess;
     if (M > INT32_MAX || d_out > INT32_MAX || d_in > INT32_MAX) return cudaErrorInvalidValue;
-    // Variant: 2-SM pairs with chunks of up to 192 tokens once there are
-    // enough tokens, up to 128 below that.  SLR_TC_KERNEL=1sm|2sm128|2sm192|small
-    // forces one (used by the tests and for A/B measurements).
+    // SLR_TC_KERNEL=1sm|2sm128[w]|2sm240[w]|2smtall[w]|small forces one kernel
+    // (a trailing w deals whole tiles only); used by the tests and for A/B
+    // measurements.
     const char *force = getenv("SLR_TC_KERNEL");
     if (force != nullptr) {
         if (strcmp(force, "1sm") == 0) return tc::launch_sparse<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
-        if (strcmp(force, "2sm128") == 0)
-            return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
-        if (strcmp(force, "2sm192") == 0)
-            return tc::launch_sparse_pair<192>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+        const bool whole = force[0] != 0 && force[strlen(force) - 1] == 'w';
+        if (strncmp(force, "2sm128", 6) == 0)
+            return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, !whole, stream);
+        if (strncmp(force, "2sm256", 6) == 0)
+            return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, !whole, stream);
+        if (strncmp(force, "2sm240", 6) == 0)
+            return tc::launch_sparse_pair<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, !whole, stream);
+        if (strncmp(force, "2smtall", 7) == 0)
+            return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, !whole, stream);
         if (strcmp(force, "small") == 0 && M <= 64) {
             if (M <= 16) return tc::launch_sparse_small<16>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
             if (M <= 32) return tc::launch_sparse_small<32>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
             return tc::launch_sparse_small<64>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
         }
     }
-    // Up to 64 tokens the layer streams S: the split-K small-M kernel.  Then
-    // 2-SM pairs with chunks of up to 128 tokens, and of up to 192 tokens from
-    // 192 tokens on.
+    // Up to 64 tokens the layer streams S: the split-K small-M kernel.  Above,
+    // 2-SM pairs: on 256-row tiles with chunks of up to 128 tokens (M < 192) or
+    // 240 tokens, or on 512-row tiles, which move X into shared memory half as
+    // often but drain their accumulators between chunks; each with the last
+    // round split among all pairs or dealt as whole tiles.  The plan with the
+    // smallest estimated time of its slowest pair is launched.
     if (M <= 16) return tc::launch_sparse_small<16>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     if (M <= 32) return tc::launch_sparse_small<32>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     if (M <= 64) return tc::launch_sparse_small<64>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
-    if (M >= 192)
-        return tc::launch_sparse_pair<192>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
-    return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int maxp = sms / 2 < tc::kMaxPairs ? sms / 2 : tc::kMaxPairs;
+    struct Cand {
+        int kind;  // 0: 256-row, 128-token chunks; 1: 256-row, 240; 2: 512-row, 240; 3: 256-row, 256
+        bool split;
+    };
+    const Cand cands[8] = {{0, true}, {0, false}, {1, true}, {1, false}, {2, true}, {2, false}, {3, true}, {3, false}};
+    int best = -1;
+    double best_cost = 0;
+    for (int i = 0; i < 8; ++i) {
+        const Cand &c = cands[i];
+        if (c.kind == 0 && M >= 192) continue;
+        if (c.kind != 0 && M < 192) continue;
+        const int chu = c.kind == 0 ? tc::Cfg2<128>::CHU : c.kind == 3 ? tc::Cfg2<256>::CHU : tc::Cfg2<240>::CHU;
+        const int half_n = chu * 8;
+        tc::Params2 plan;
+        int pairs = 0;
+        tc::plan_pairs(M, d_out, d_in, r, chu, c.kind == 2 ? 4 * tc::BM : 2 * tc::BM, maxp, c.split, &plan, &pairs);
+        const double cost = tc::plan_cycles(plan, pairs, chu, half_n, c.kind == 2 ? 2 : c.kind == 3 ? 1 : 0);
+        if (best < 0 || cost < best_cost) {
+            best = i;
+            best_cost = cost;
+        }
+    }
+    const Cand &c = cands[best];
+    if (c.kind == 0)
+        return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream);
+    if (c.kind == 1)
+        return tc::launch_sparse_pair<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream);
+    if (c.kind == 3)
+        return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream);
+    return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream);
 }
 
 cudaError_t launch_tc_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in, int64_t r,

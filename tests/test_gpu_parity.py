@@ -181,7 +181,7 @@ def test_no_kernel_timeouts():
     slr.check_kernel_error()
 
 
-VARIANTS = ["1sm", "2sm128", "2sm192", "small"]
+VARIANTS = ["1sm", "2sm128", "2sm240", "2sm256", "2smtall", "2smtallw", "small"]
 
 
 @pytest.mark.parametrize("variant", VARIANTS)
@@ -196,8 +196,9 @@ VARIANTS = ["1sm", "2sm128", "2sm192", "small"]
     (4096, 4096, 64, 1),     # one token, 32 row tiles x 4-CTA clusters
 ])
 def test_forward_tensor_variants(variant, d_out, d_in, r, M, monkeypatch):
-    """Every tensor-core kernel variant (1-SM, 2-SM with 128- and 256-token
-    tiles) against the oracle, selected through SLR_TC_KERNEL."""
+    """Every tensor-core kernel variant (1-SM; 2-SM pairs on 256-row tiles with
+    chunks of up to 128 or 240 tokens; 2-SM pairs on 512-row tiles; the split-K
+    small-M kernel) against the oracle, selected through SLR_TC_KERNEL."""
     monkeypatch.setenv("SLR_TC_KERNEL", variant)
     seed = d_out * 7 + d_in + r + M
     X = synth.activations_bf16(M, d_in, seed, seed + 9)
