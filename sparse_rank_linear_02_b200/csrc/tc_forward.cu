@@ -427,6 +427,7 @@ struct Params2 {
     int32_t ttiles;     // token tiles per row tile
     int32_t wu, wr;     // token tile tt has wu + (tt < wr) units
     int32_t cyc;        // rounds of the cyclic phase
+    int32_t chu;        // most 16-token units per chunk (<= the kernel's BN / 16)
     int64_t n_tiles;    // tiles dealt in the cyclic phase (a last round may be partial)
     int64_t tail[kMaxPairs + 1];  // pair p's tail units are [tail[p], tail[p+1])
 };
@@ -579,7 +580,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         bool t_ready = false;
         ChunkIter iter(prm, pair, npairs);
         Chunk ch;
-        while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(C::CHU, ch)) {
+        while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(prm.chu, ch)) {
             const int d0 = ch.d0 + (int)rank * BM;
             const int rows = ch.n / 2;
             const int tok = ch.tok0 + (int)rank * rows;
@@ -637,10 +638,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         // its tiles MLEAD stages ahead into slots of its own parity.
         const int par = warp - 6;
         const uint32_t src_slot = smem_u32(dummy + 16 * C::MS);
-        SparseCursor ld(prm, pair, npairs, nk, C::CHU), use(prm, pair, npairs, nk, C::CHU);
+        SparseCursor ld(prm, pair, npairs, nk, prm.chu), use(prm, pair, npairs, nk, prm.chu);
         if (par) {
-            ld.advance(C::CHU);
-            use.advance(C::CHU);
+            ld.advance(prm.chu);
+            use.advance(prm.chu);
         }
         auto issue = [&](int slot) {
             if (elect_one()) {
@@ -649,8 +650,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
                             ld.ch.d0 + (int)rank * BM);
             }
             __syncwarp();
-            ld.advance(C::CHU);
-            if (ld.valid) ld.advance(C::CHU);
+            ld.advance(prm.chu);
+            if (ld.valid) ld.advance(prm.chu);
         };
         int64_t n_ld = par;
         for (; n_ld < C::MLEAD && ld.valid; n_ld += 2) issue((int)(n_ld % C::MS));
@@ -697,8 +698,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
                 issue(s2);
                 n_ld += 2;
             }
-            use.advance(C::CHU);
-            if (use.valid) use.advance(C::CHU);
+            use.advance(prm.chu);
+            if (use.valid) use.advance(prm.chu);
             k += 2;
         }
     } else if (warp == 1) {
@@ -710,7 +711,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
             int64_t k = 0;   // sparse stages consumed (metadata slot sequence)
             ChunkIter iter(prm, pair, npairs);
             Chunk ch;
-            while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(C::CHU, ch)) {
+            while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(prm.chu, ch)) {
                 const uint32_t idesc_sp = idesc_bf16(2 * BM, ch.n, true);
                 const uint32_t idesc_dense = idesc_bf16(2 * BM, ch.n, false);
                 const uint32_t panel = (uint32_t)box_rows(pick_box(ch.n / 2), C::HALF_N) * 128u;
@@ -787,7 +788,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         int it = 0;
         ChunkIter iter(prm, pair, npairs);
         Chunk ch;
-        while (!*fail && iter.next(C::CHU, ch)) {
+        while (!*fail && iter.next(prm.chu, ch)) {
             const int d0 = ch.d0 + (int)rank * BM;
             const int buf = C::NACC == 2 ? (it & 1) : 0;
             const uint32_t use = (uint32_t)(C::NACC == 2 ? (it >> 1) : it);
@@ -974,7 +975,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
         bool t_ready = false;
         ChunkIter iter(prm, pair, npairs);
         Chunk ch;
-        while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(C::CHU, ch)) {
+        while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(prm.chu, ch)) {
             const int d0 = ch.d0 + (int)rank * BM;        // half 0 rows of this CTA; half 1 at +256
             const int rows = ch.n / 2;
             const int tok = ch.tok0 + (int)rank * rows;
@@ -1028,10 +1029,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
         // holds both halves' tiles (2 x 2 KB).
         const int par = warp - 10;
         const uint32_t src_slot = smem_u32(dummy + 16 * C::MS);
-        SparseCursor ld(prm, pair, npairs, nk, C::CHU), use(prm, pair, npairs, nk, C::CHU);
+        SparseCursor ld(prm, pair, npairs, nk, prm.chu), use(prm, pair, npairs, nk, prm.chu);
         if (par) {
-            ld.advance(C::CHU);
-            use.advance(C::CHU);
+            ld.advance(prm.chu);
+            use.advance(prm.chu);
         }
         auto issue = [&](int slot) {
             if (elect_one()) {
@@ -1042,8 +1043,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
                 tma_load_2d(&maps.meta, smem_u32(e + C::E_BYTES), &mfull[slot], ld.ks * (BK / 8), r0 + 2 * BM);
             }
             __syncwarp();
-            ld.advance(C::CHU);
-            if (ld.valid) ld.advance(C::CHU);
+            ld.advance(prm.chu);
+            if (ld.valid) ld.advance(prm.chu);
         };
         int64_t n_ld = par;
         for (; n_ld < C::MLEAD && ld.valid; n_ld += 2) issue((int)(n_ld % C::MS));
@@ -1094,8 +1095,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
                 issue(s2);
                 n_ld += 2;
             }
-            use.advance(C::CHU);
-            if (use.valid) use.advance(C::CHU);
+            use.advance(prm.chu);
+            if (use.valid) use.advance(prm.chu);
             k += 2;
         }
     } else if (warp == 1) {
@@ -1107,7 +1108,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
             int64_t k = 0;   // sparse stages consumed (metadata slot sequence)
             ChunkIter iter(prm, pair, npairs);
             Chunk ch;
-            while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(C::CHU, ch)) {
+            while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(prm.chu, ch)) {
                 const uint32_t idesc_sp = idesc_bf16(2 * BM, ch.n, true);
                 const uint32_t idesc_dense = idesc_bf16(2 * BM, ch.n, false);
                 const uint32_t panel = (uint32_t)box_rows(pick_box(ch.n / 2), C::HALF_N) * 128u;
@@ -1195,7 +1196,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
         int it = 0;
         ChunkIter iter(prm, pair, npairs);
         Chunk ch;
-        while (!*fail && iter.next(C::CHU, ch)) {
+        while (!*fail && iter.next(prm.chu, ch)) {
             const int d0 = ch.d0 + grp * 2 * BM + (int)rank * BM;
             if (!mbar_wait_cluster(acc_full, (uint32_t)(it & 1))) {
                 *fail = 1;
@@ -1362,6 +1363,7 @@ void plan_pairs(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int chu, int 
     prm->M = (int32_t)M;
     prm->d_out = (int32_t)d_out;
     prm->tile_rows = tile_rows;
+    prm->chu = chu;
     prm->nk = (int32_t)(d_in / BK);
     prm->nlr = (int32_t)((r + 63) / 64);
     const int64_t ut = (M + 15) / 16;
@@ -1437,10 +1439,64 @@ double plan_cycles(const Params2 &prm, int pairs, int chu, int half_n, int mode)
     return worst;
 }
 
+// The plan of the pair kernels for one problem shape: kernel kind (0: 256-row
+// tiles, chunks of up to 128 tokens; 1: 256-row, 240; 2: 512-row, 240;
+// 3: 256-row, 256), chunk width cap and whether the last round is split.
+// Chosen by the smallest plan_cycles estimate over the kinds that apply and
+// chunk caps of the kind's maximum and up to five units less (narrower token
+// tiles can make the tile count fit the pairs better); cached per shape.
+struct PlanChoice {
+    int kind, chu;
+    bool split;
+};
+
+PlanChoice choose_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int sms) {
+    struct Key {
+        int64_t M, d_out, d_in, r;
+        int sms;
+    };
+    static std::mutex mu;
+    static Key keys[64];
+    static PlanChoice vals[64];
+    static int n_cached = 0, next_slot = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < n_cached; ++i)
+            if (keys[i].M == M && keys[i].d_out == d_out && keys[i].d_in == d_in && keys[i].r == r && keys[i].sms == sms)
+                return vals[i];
+    }
+    const int maxp = sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs;
+    PlanChoice best{-1, 0, true};
+    double best_cost = 0;
+    for (int kind = 0; kind < 4; ++kind) {
+        if ((kind == 0) != (M < 192)) continue;
+        const int cap = kind == 0 ? Cfg2<128>::CHU : kind == 3 ? Cfg2<256>::CHU : Cfg2<240>::CHU;
+        const int half_n = cap * 8;
+        for (int chu = cap; chu >= cap - 5 && chu >= 1; --chu) {
+            for (int sp = 0; sp < 2; ++sp) {
+                Params2 plan;
+                int pairs = 0;
+                plan_pairs(M, d_out, d_in, r, chu, kind == 2 ? 4 * BM : 2 * BM, maxp, sp == 0, &plan, &pairs);
+                const double cost = plan_cycles(plan, pairs, chu, half_n, kind == 2 ? 2 : kind == 3 ? 1 : 0);
+                if (best.kind < 0 || cost < best_cost) {
+                    best = PlanChoice{kind, chu, sp == 0};
+                    best_cost = cost;
+                }
+            }
+        }
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    keys[next_slot] = Key{M, d_out, d_in, r, sms};
+    vals[next_slot] = best;
+    next_slot = (next_slot + 1) % 64;
+    if (n_cached < 64) ++n_cached;
+    return best;
+}
+
 template <int BN>
 cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
-                               uint16_t *Y, bool after_projection, bool split_tail, cudaStream_t stream) {
+                               uint16_t *Y, bool after_projection, bool split_tail, cudaStream_t stream, int chu = 0) {
     using C = Cfg2<BN>;
     Maps2 maps;
     memset(&maps, 0, sizeof maps);
@@ -1465,7 +1521,8 @@ cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *val
     if (err != cudaSuccess) return err;
     Params2 prm;
     int pairs = 0;
-    plan_pairs(M, d_out, d_in, r, C::CHU, 2 * BM, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, split_tail, &prm, &pairs);
+    if (chu <= 0 || chu > C::CHU) chu = C::CHU;
+    plan_pairs(M, d_out, d_in, r, chu, 2 * BM, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, split_tail, &prm, &pairs);
     // Directly after the projection kernel on this stream: programmatic
     // dependent launch (the producer waits before it loads T).  Otherwise an
     // ordinary launch, which must not overlap an unrelated preceding kernel.
@@ -1485,7 +1542,7 @@ cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *val
 template <int BN>
 cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
-                               uint16_t *Y, bool after_projection, bool split_tail, cudaStream_t stream) {
+                               uint16_t *Y, bool after_projection, bool split_tail, cudaStream_t stream, int chu = 0) {
     using C = CfgT<BN>;
     Maps2 maps;
     memset(&maps, 0, sizeof maps);
@@ -1510,7 +1567,8 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
     if (err != cudaSuccess) return err;
     Params2 prm;
     int pairs = 0;
-    plan_pairs(M, d_out, d_in, r, C::CHU, 4 * BM, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, split_tail, &prm, &pairs);
+    if (chu <= 0 || chu > C::CHU) chu = C::CHU;
+    plan_pairs(M, d_out, d_in, r, chu, 4 * BM, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, split_tail, &prm, &pairs);
     // Directly after the projection kernel on this stream: programmatic
     // dependent launch (the producer waits before it loads T).  Otherwise an
     // ordinary launch, which must not overlap an unrelated preceding kernel.
@@ -2052,37 +2110,14 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
     if (M <= 64) return tc::launch_sparse_small<64>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int maxp = sms / 2 < tc::kMaxPairs ? sms / 2 : tc::kMaxPairs;
-    struct Cand {
-        int kind;  // 0: 256-row, 128-token chunks; 1: 256-row, 240; 2: 512-row, 240; 3: 256-row, 256
-        bool split;
-    };
-    const Cand cands[8] = {{0, true}, {0, false}, {1, true}, {1, false}, {2, true}, {2, false}, {3, true}, {3, false}};
-    int best = -1;
-    double best_cost = 0;
-    for (int i = 0; i < 8; ++i) {
-        const Cand &c = cands[i];
-        if (c.kind == 0 && M >= 192) continue;
-        if (c.kind != 0 && M < 192) continue;
-        const int chu = c.kind == 0 ? tc::Cfg2<128>::CHU : c.kind == 3 ? tc::Cfg2<256>::CHU : tc::Cfg2<240>::CHU;
-        const int half_n = chu * 8;
-        tc::Params2 plan;
-        int pairs = 0;
-        tc::plan_pairs(M, d_out, d_in, r, chu, c.kind == 2 ? 4 * tc::BM : 2 * tc::BM, maxp, c.split, &plan, &pairs);
-        const double cost = tc::plan_cycles(plan, pairs, chu, half_n, c.kind == 2 ? 2 : c.kind == 3 ? 1 : 0);
-        if (best < 0 || cost < best_cost) {
-            best = i;
-            best_cost = cost;
-        }
-    }
-    const Cand &c = cands[best];
+    const tc::PlanChoice c = tc::choose_plan(M, d_out, d_in, r, sms);
     if (c.kind == 0)
-        return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream);
+        return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream, c.chu);
     if (c.kind == 1)
-        return tc::launch_sparse_pair<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream);
+        return tc::launch_sparse_pair<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream, c.chu);
     if (c.kind == 3)
-        return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream);
-    return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream);
+        return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream, c.chu);
+    return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream, c.chu);
 }
 
 cudaError_t launch_tc_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in, int64_t r,
