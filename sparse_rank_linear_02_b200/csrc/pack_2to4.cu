@@ -19,23 +19,26 @@ namespace {
 // Select the two kept positions of a group given as two 32-bit words holding
 // bf16 values 0,1 (w01) and 2,3 (w23).  Returns the nibble idx0 | idx1 << 2 and
 // the two kept bit patterns packed low (idx0) / high (idx1).
+//
+// Each position p gets the sort key (magnitude bits << 2) | (3 - p): a larger
+// magnitude wins and, of two equal magnitudes, the lower position.  The two
+// largest keys of four come from a max/min network (max of the pair maxima,
+// then the larger of the smaller pair maximum and the larger pair minimum),
+// and one byte permute gathers the two kept values.
 __device__ __forceinline__ uint32_t select_group(uint32_t w01, uint32_t w23, uint32_t *kept) {
-    const uint32_t k0 = w01 & 0x7FFFu, k1 = (w01 >> 16) & 0x7FFFu;
-    const uint32_t k2 = w23 & 0x7FFFu, k3 = (w23 >> 16) & 0x7FFFu;
-    // Position a beats position b (a < b) when key_a >= key_b.
-    const uint32_t b01 = k0 >= k1, b02 = k0 >= k2, b03 = k0 >= k3;
-    const uint32_t b12 = k1 >= k2, b13 = k1 >= k3, b23 = k2 >= k3;
-    // Number of positions that beat each position.
-    const uint32_t beat0 = (1u - b01) + (1u - b02) + (1u - b03);
-    const uint32_t beat1 = b01 + (1u - b12) + (1u - b13);
-    const uint32_t beat2 = b02 + b12 + (1u - b23);
-    const uint32_t beat3 = b03 + b13 + b23;
-    const uint32_t mask = (beat0 < 2u) | ((beat1 < 2u) << 1) | ((beat2 < 2u) << 2) | ((beat3 < 2u) << 3);
-    const uint32_t i0 = __ffs(mask) - 1;          // lowest kept position
-    const uint32_t i1 = 31 - __clz(mask);         // highest kept position
-    const uint32_t v0 = ((i0 & 2u) ? w23 : w01) >> ((i0 & 1u) * 16);
-    const uint32_t v1 = ((i1 & 2u) ? w23 : w01) >> ((i1 & 1u) * 16);
-    *kept = (v0 & 0xFFFFu) | (v1 << 16);
+    const uint32_t e0 = ((w01 & 0x7FFFu) << 2) | 3u;
+    const uint32_t e1 = ((w01 >> 14) & 0x1FFFCu) | 2u;
+    const uint32_t e2 = ((w23 & 0x7FFFu) << 2) | 1u;
+    const uint32_t e3 = (w23 >> 14) & 0x1FFFCu;
+    const uint32_t m01 = max(e0, e1), n01 = min(e0, e1);
+    const uint32_t m23 = max(e2, e3), n23 = min(e2, e3);
+    const uint32_t first = max(m01, m23);
+    const uint32_t second = max(min(m01, m23), max(n01, n23));
+    const uint32_t pa = 3u - (first & 3u), pb = 3u - (second & 3u);
+    const uint32_t i0 = min(pa, pb), i1 = max(pa, pb);
+    // Position p sits in bytes 2p, 2p+1 of (w01, w23).
+    const uint32_t sel = (i0 * 2u) * 0x11u + 0x10u + (((i1 * 2u) * 0x11u + 0x10u) << 8);
+    *kept = __byte_perm(w01, w23, sel);
     return i0 | (i1 << 2);
 }
 
