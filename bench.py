@@ -265,9 +265,18 @@ def run_ours(args, rank, world, dist):
     step_bytes = algorithmic_bytes(M, d_out, d_in, r)
     t_roof_step = max(step_bytes / (peaks["hbm_gbs"] * 1e9),
                       flops_dense / (p_sparse * 1e12) + flops_lr / (p_dense * 1e12))
+    # The step is timed after an untimed preheat, at the clocks a long run
+    # settles to under the power cap: the sustained measured peak is its
+    # denominator (the burst-peak fraction is kept beside it).
+    p_dense_s = peaks["bf16_tflops_sustained"]
+    t_roof_step_s = max(step_bytes / (peaks["hbm_gbs"] * 1e9),
+                        flops_dense / (SPARSE_RATIO * p_dense_s * 1e12) + flops_lr / (p_dense_s * 1e12))
     prefill = {"tflops_dense_equiv": round(value / world, 1), "tflops_executed": round(flops_exec / (ms_per_step * 1e-3) / 1e12, 1),
                "gbs": round(step_bytes / (ms_per_step * 1e-3) / 1e9, 1),
                "frac_of_roofline": round(t_roof_step / (ms_per_step * 1e-3), 4),
+               "frac_of_roofline_sustained_peak": round(t_roof_step_s / (ms_per_step * 1e-3), 4),
+               "peak_note": "frac_of_roofline uses the burst bf16 peak; the step runs after a 0.5 s preheat "
+                            "at sustained clocks, for which the sustained measured peak is the denominator",
                "project_ms": round(project_ms, 4), "combine_ms": round(combine_ms, 4)}
     clocks = clk.summary()
 
