@@ -1206,15 +1206,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
             tc_fence_after();
             const uint32_t acc = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(grp * BN);
             uint32_t packed[kPieces * 8];
+            // Two 16-column pieces per TMEM round trip (a piece past the
+            // chunk re-reads the last valid one; its values are not used).
 #pragma unroll
-            for (int q = 0; q < kPieces; ++q) {
+            for (int q = 0; q < kPieces; q += 2) {
                 if (q * 16 < ch.n) {
-                    uint32_t h[16];
-                    tmem_ld_32x32b_x16(acc + (uint32_t)(q * 16), h);
+                    const int q2 = (q + 1 < kPieces && (q + 1) * 16 < ch.n) ? q + 1 : q;
+                    uint32_t h[32];
+                    tmem_ld_32x32b_2x16(acc + (uint32_t)(q * 16), acc + (uint32_t)(q2 * 16), h);
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
                         packed[q * 8 + j] = (uint32_t)f32_to_bf16_bits(__uint_as_float(h[2 * j])) |
                                             ((uint32_t)f32_to_bf16_bits(__uint_as_float(h[2 * j + 1])) << 16);
+                    if (q + 1 < kPieces) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            packed[(q + 1) * 8 + j] = (uint32_t)f32_to_bf16_bits(__uint_as_float(h[16 + 2 * j])) |
+                                                      ((uint32_t)f32_to_bf16_bits(__uint_as_float(h[17 + 2 * j])) << 16);
+                    }
                 }
             }
             tc_fence_before();
