@@ -167,6 +167,31 @@ def test_forward_edges(d_out, d_in, r, M, path):
     check_forward(from_dev(Y), Yref, Bref, f"edge {d_out}x{d_in} r={r} M={M} {path}")
 
 
+@pytest.mark.parametrize("d_out,d_in,r,M", [
+    (4096, 4096, 64, 256),    # mid M: 256-row tiles, chunk cap below the kernel's maximum
+    (4096, 4096, 64, 512),
+    (1024, 4096, 64, 4096),   # few row tiles, many tokens
+    (2048, 8192, 64, 1000),   # 512-row tiles, ragged token count
+    (3072, 4096, 128, 700),   # d_out not a multiple of 512
+])
+def test_forward_plan_shapes(d_out, d_in, r, M):
+    """Default dispatch on shapes where the pair-kernel plan choice matters
+    (kernel kind, chunk-width cap, split or whole last round)."""
+    seed = d_out + 3 * d_in + 5 * r + 7 * M
+    X = synth.activations_bf16(M, d_in, seed, seed + 9)
+    W = synth.gaussian_bf16((d_out, d_in), 0.02, seed + 1)
+    vals, meta = oracle.pack_2to4(W)
+    U = synth.gaussian_bf16((d_out, r), 0.5, seed + 2)
+    V = synth.gaussian_bf16((r, d_in), 0.5 / np.sqrt(r), seed + 3)
+    Y = slr.forward(to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U), to_dev(V), path="tensor")
+    torch.cuda.synchronize()
+    slr.check_kernel_error()
+    rows = sample_indices(M, 48, seed)
+    outs = sample_indices(d_out, 512, seed + 1)
+    Yref, Bref = oracle.forward(X, vals, meta, U, V, rows=rows, outs=outs)
+    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, f"plan {d_out}x{d_in} r={r} M={M}")
+
+
 def test_forward_matches_between_paths():
     """The two paths agree with each other as well as with the oracle."""
     layer, W, vals, meta, U, V = layer_weights(2, "q_proj")
