@@ -1885,15 +1885,22 @@ __global__ void __launch_bounds__(kThreads, 2)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async_smem();
     }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(C::TMEM_COLS));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    // The producer needs no TMEM: warp 0 arrives on the start barrier and
+    // streams at once; the other warps wait there for the TMEM allocation.
+    uint32_t tmem_base = 0;
+    if (warp == 0) {
+        asm volatile("bar.arrive 1, %0;" ::"r"(kThreads) : "memory");
+    } else {
+        if (warp == 1) {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                         "r"(C::TMEM_COLS));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        }
+        tc_fence_before();
+        asm volatile("bar.sync 1, %0;" ::"r"(kThreads) : "memory");
+        tc_fence_after();
+        tmem_base = *tmem_slot;
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
         if (lane == 0) {
