@@ -28,12 +28,14 @@ __host__ __device__ constexpr int unroll_for() { return MT == 1 ? 8 : 4; }
 
 // One group of four: kept values (low = lower index) in vv, nibble nib, the
 // four X values of the group in x01 (elements 0,1) and x23 (elements 2,3).
+// One byte permute gathers the two X values the kept weights multiply (byte
+// selectors 2*idx, 2*idx+1 for each index); bf16 -> fp32 is a 16-bit shift
+// or a mask.
 __device__ __forceinline__ float group_fma(uint32_t vv, uint32_t nib, uint32_t x01, uint32_t x23, float acc) {
-    const uint32_t i0 = nib & 3u, i1 = nib >> 2;
-    const uint32_t a = ((i0 & 2u) ? x23 : x01) >> ((i0 & 1u) * 16);
-    const uint32_t b = ((i1 & 2u) ? x23 : x01) >> ((i1 & 1u) * 16);
-    acc = fmaf(bf16lo_to_f32(vv), bf16lo_to_f32(a), acc);
-    acc = fmaf(bf16hi_to_f32(vv), bf16lo_to_f32(b), acc);
+    const uint32_t sel = ((nib & 3u) | ((nib & 0xCu) << 6)) * 0x22u + 0x1010u;
+    const uint32_t xs = __byte_perm(x01, x23, sel);
+    acc = fmaf(bf16lo_to_f32(vv), bf16lo_to_f32(xs), acc);
+    acc = fmaf(bf16hi_to_f32(vv), bf16hi_to_f32(xs), acc);
     return acc;
 }
 
