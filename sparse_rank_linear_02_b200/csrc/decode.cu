@@ -73,24 +73,23 @@ __global__ void __launch_bounds__(kWarps * 32, kBlocksPerSm) decode_forward_kern
         // The rank-r operands of this row: U now (it does not depend on the
         // projection), T after griddepcontrol.wait once the first weight
         // chunks are in flight, so neither load adds a round trip at the end.
-        constexpr int kRk = 2;   // r <= 32 * kRk handled from registers
-        float ur[kRk];
-        float tr[kRk][MT];
-#pragma unroll
-        for (int j = 0; j < kRk; ++j) {
-            const int64_t k = lane + 32 * j;
-            ur[j] = k < r ? __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(U) + row * r + k) << 16) : 0.f;
+        // Lane l holds rank pair k = 2l, 2l + 1 (r % 8 == 0, so the pair is
+        // 4-byte aligned in U and 8-byte aligned in T): one load each.
+        const bool rk = 2 * lane < r;
+        float ur0 = 0.f, ur1 = 0.f;
+        if (rk) {
+            const uint32_t u2 = __ldg(reinterpret_cast<const unsigned int *>(U + row * r) + lane);
+            ur0 = bf16lo_to_f32(u2);
+            ur1 = bf16hi_to_f32(u2);
         }
+        float2 tr[MT];
         bool t_loaded = false;
         auto load_t = [&]() {
             t_loaded = true;
             if (r > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
-            for (int j = 0; j < kRk; ++j) {
-                const int64_t k = lane + 32 * j;
-#pragma unroll
-                for (int t = 0; t < MT; ++t) tr[j][t] = (k < r && t < nt) ? __ldg(T32 + (m0 + t) * r + k) : 0.f;
-            }
+            for (int t = 0; t < MT; ++t)
+                tr[t] = (rk && t < nt) ? __ldg(reinterpret_cast<const float2 *>(T32 + (m0 + t) * r) + lane) : make_float2(0.f, 0.f);
         };
 
         for (int64_t c0 = lane; c0 < chunks; c0 += 32 * kUnroll) {
@@ -127,12 +126,10 @@ __global__ void __launch_bounds__(kWarps * 32, kBlocksPerSm) decode_forward_kern
         // Rank-r term: lanes split k, products land in the same partial sums.
         // T comes from the projection kernel, which may still be running when
         // this kernel starts (programmatic dependent launch); it was loaded
-        // after griddepcontrol.wait above.  Ranks beyond 32 * kRk continue here.
+        // after griddepcontrol.wait above.  Ranks past 64 continue here.
 #pragma unroll
-        for (int j = 0; j < kRk; ++j)
-#pragma unroll
-            for (int t = 0; t < MT; ++t) acc[t] = fmaf(ur[j], tr[j][t], acc[t]);
-        for (int64_t k = lane + 32 * kRk; k < r; k += 32) {
+        for (int t = 0; t < MT; ++t) acc[t] = fmaf(ur1, tr[t].y, fmaf(ur0, tr[t].x, acc[t]));
+        for (int64_t k = lane + 64; k < r; k += 32) {
             const float u = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(U) + row * r + k) << 16);
 #pragma unroll
             for (int t = 0; t < MT; ++t)
