@@ -79,6 +79,10 @@ class Oracle:
         lib.oracle_lowrank_project.restype = ctypes.c_int
         lib.oracle_lowrank_project.argtypes = [p, i64, p, i64, i64, p]
         lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_pack_2to4_scaled.restype = ctypes.c_int
+        lib.oracle_pack_2to4_scaled.argtypes = [p, i64, i64, i64, p, p, p]
+        lib.oracle_column_norms.restype = ctypes.c_int
+        lib.oracle_column_norms.argtypes = [p, i64, i64, p]
         self._lib = lib
         self.path = lib_path
 
@@ -102,6 +106,31 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle_pack_2to4 rejected shape {W.shape} (rc={rc})")
         return vals, meta
+
+    def pack_2to4_scaled(self, W: np.ndarray, scale: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+        """Activation-aware 2:4 projection: weights of column j ranked by the
+        float32 product |w| * |scale[j]| (HASSLE-free, section 4.1.2, diagonal
+        Hessian); same packed format as :meth:`pack_2to4`."""
+        W = _u16(W)
+        d_out, d_in = W.shape
+        scale = np.ascontiguousarray(scale, dtype=np.float32).reshape(-1)
+        if scale.shape[0] != d_in:
+            raise ValueError("scale must hold one float per input column")
+        vals = np.zeros((d_out, d_in // 2), dtype=np.uint16)
+        meta = np.zeros((d_out, self.meta_row_bytes(d_in)), dtype=np.uint8)
+        rc = self._lib.oracle_pack_2to4_scaled(_ptr(W), d_out, d_in, d_in, _ptr(scale), _ptr(vals), _ptr(meta))
+        if rc != 0:
+            raise ValueError(f"oracle_pack_2to4_scaled rejected shape {W.shape} (rc={rc})")
+        return vals, meta
+
+    def column_norms(self, X: np.ndarray) -> np.ndarray:
+        """fp64 norms of the columns of bf16 ``X`` [M, d_in]."""
+        X = _u16(X)
+        M, d_in = X.shape
+        out = np.zeros(d_in, dtype=np.float64)
+        if self._lib.oracle_column_norms(_ptr(X), M, d_in, _ptr(out)) != 0:
+            raise ValueError("oracle_column_norms rejected its arguments")
+        return out
 
     def unpack_2to4(self, vals: np.ndarray, meta: np.ndarray, d_in: int) -> np.ndarray:
         """Dense bf16 bits [d_out, d_in] of a packed 2:4 matrix (zeros elsewhere)."""
@@ -186,6 +215,14 @@ def meta_row_bytes(d_in: int) -> int:
 
 def max_threads() -> int:
     return default().max_threads()
+
+
+def pack_2to4_scaled(W, scale):
+    return default().pack_2to4_scaled(W, scale)
+
+
+def column_norms(X):
+    return default().column_norms(X)
 
 
 def pack_2to4(W):

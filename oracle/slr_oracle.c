@@ -21,6 +21,16 @@
  *      order; metadata byte j of a row holds group 2j in its low nibble and
  *      group 2j+1 in its high nibble, nibble = idx0 | idx1 << 2.
  *
+ *   1b. The activation-aware 2:4 projection.  HASSLE-free, section 4.1.2:
+ *      with a diagonal Hessian the optimal sparse update is a scaled
+ *      hard-thresholding (the Wanda-style score |w_ij| * s_j, s_j the norm of
+ *      input column j, s_j^2 the Hessian diagonal).  The score of a weight is
+ *      the single-precision product |w| * |s| (round to nearest); any NaN
+ *      product scores 0x7FFFFFFF; keys are compared as unsigned integers
+ *      (the bits of a non-negative float), ties go to the lower index, and the
+ *      packed format is the one above.  The column norms s_j = ||X[:, j]||_2
+ *      are computed in fp64.
+ *
  *   2. The forward pass.  LoSparse (arXiv 2306.11222), section 3 and
  *      section 3.2: the compressed layer replaces X*W by the sum of a sparse
  *      term and a low-rank term, run in parallel.  In the d_out x d_in
@@ -116,6 +126,80 @@ int oracle_pack_2to4(const uint16_t *W, int64_t d_out, int64_t d_in, int64_t ldw
             unsigned nib = (unsigned)a | ((unsigned)b << 2);
             meta[i * mrow + g / 2] |= (uint8_t)(nib << (4 * (g % 2)));
         }
+    }
+    return 0;
+}
+
+/* Score key of one weight under the activation-aware projection: the bits
+ * of the float product |w| * |s| (IEEE single, round to nearest, one multiply;
+ * both factors are non-negative, so the sign bit is clear and the bits order
+ * like the values); a NaN product scores 0x7FFFFFFF. */
+static uint32_t scaled_key(uint16_t w, float s)
+{
+    uint32_t u = ((uint32_t)(w & 0x7FFFu)) << 16;
+    float aw;
+    memcpy(&aw, &u, sizeof aw);
+    volatile float prod = aw * fabsf(s);
+    if (isnan(prod)) return 0x7FFFFFFFu;
+    float pf = prod;
+    uint32_t k;
+    memcpy(&k, &pf, sizeof k);
+    return k;
+}
+
+/* As choose_two, on the scaled keys of the four positions. */
+static void choose_two_keys(const uint32_t key[4], int *idx0, int *idx1)
+{
+    int kept[2];
+    int n = 0;
+    for (int p = 0; p < 4; ++p) {
+        int rank = 0;
+        for (int q = 0; q < 4; ++q)
+            if (key[q] > key[p] || (key[q] == key[p] && q < p)) ++rank;
+        if (rank < 2) kept[n++] = p;
+    }
+    *idx0 = kept[0];
+    *idx1 = kept[1];
+}
+
+/* Activation-aware 2:4 projection and packing: as oracle_pack_2to4, with the
+ * weights of column j ranked by the scaled key of (w_ij, scale[j]).
+ *   scale : d_in floats. */
+int oracle_pack_2to4_scaled(const uint16_t *W, int64_t d_out, int64_t d_in, int64_t ldw, const float *scale,
+                            uint16_t *vals, uint8_t *meta)
+{
+    if (d_in % 4 != 0 || ldw < d_in || d_out < 0) return -1;
+    int64_t groups = d_in / 4;
+    int64_t mrow = oracle_meta_row_bytes(d_in);
+    for (int64_t i = 0; i < d_out; ++i) {
+        memset(meta + i * mrow, 0, (size_t)mrow);
+        for (int64_t g = 0; g < groups; ++g) {
+            const uint16_t *w = W + i * ldw + 4 * g;
+            uint32_t key[4];
+            for (int p = 0; p < 4; ++p) key[p] = scaled_key(w[p], scale[4 * g + p]);
+            int a, b;
+            choose_two_keys(key, &a, &b);
+            vals[i * (d_in / 2) + 2 * g + 0] = w[a];
+            vals[i * (d_in / 2) + 2 * g + 1] = w[b];
+            unsigned nib = (unsigned)a | ((unsigned)b << 2);
+            meta[i * mrow + g / 2] |= (uint8_t)(nib << (4 * (g % 2)));
+        }
+    }
+    return 0;
+}
+
+/* Column norms of X (M x d_in, bf16 bits): out[j] = sqrt(sum_m X[m][j]^2) in
+ * fp64, the sum taken in row order. */
+int oracle_column_norms(const uint16_t *X, int64_t M, int64_t d_in, double *out)
+{
+    if (M < 0 || d_in < 0) return -1;
+    for (int64_t j = 0; j < d_in; ++j) {
+        double acc = 0.0;
+        for (int64_t m = 0; m < M; ++m) {
+            double x = bf16_bits_to_double(X[m * d_in + j]);
+            acc += x * x;
+        }
+        out[j] = sqrt(acc);
     }
     return 0;
 }

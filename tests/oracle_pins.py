@@ -271,9 +271,152 @@ def pin_lowrank_project(o):
     np.testing.assert_array_equal(o.lowrank_project(X, V), _f64(X) @ _f64(V).T)
 
 
+# --------------------------------------------------------------------------- activation-aware pack pins
+#
+# HASSLE-free, section 4.1.2: with the diagonal Hessian D^2 (D = diag of the
+# input column norms) the sparse step hard-thresholds W D, i.e. weight w_ij is
+# ranked by |w_ij| * s_j.  The pins below check the oracle's fp32 score against
+# exact arithmetic where the product is exact, against the weighted objective,
+# and against the unscaled projection where the scale is uniform.
+
+def _pow2_scales(rng, n, lo=-6, hi=7):
+    return np.ldexp(1.0, rng.integers(lo, hi, size=n)).astype(np.float32)
+
+
+def _bf16_scales(rng, n):
+    """Positive scales with 8-bit significands, so |w| * s (bf16 w) is exact in fp32."""
+    return synth.bf16_bits_to_f32(_bf16(rng.uniform(0.25, 4.0, size=n))).astype(np.float32)
+
+
+def pin_scaled_uniform_equals_unscaled(o):
+    """scale == c (any power of two, either sign) reduces to the plain 2:4 projection."""
+    W = synth.gaussian_bf16((48, 128), 0.02, 21)
+    v0, m0 = o.pack_2to4(W)
+    for c in (1.0, 0.5, -8.0, 2.0 ** -20):
+        v1, m1 = o.pack_2to4_scaled(W, np.full(128, c, dtype=np.float32))
+        np.testing.assert_array_equal(v1, v0)
+        np.testing.assert_array_equal(m1, m0)
+
+
+def pin_scaled_bruteforce_exact(o, seed: int = 22):
+    """Exact products (bf16 weights times 8-bit-significand scales) ranked by
+    enumeration of the six pairs; the narrow weight alphabet makes many ties."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    d_in = 32
+    sign = rng.integers(0, 2, size=(200, d_in)).astype(np.uint16) << 15
+    expo = rng.integers(125, 129, size=(200, d_in)).astype(np.uint16) << 7
+    mant = rng.integers(0, 4, size=(200, d_in)).astype(np.uint16) << 5
+    W = (sign | expo | mant).astype(np.uint16)
+    for scale in (_pow2_scales(rng, d_in), _bf16_scales(rng, d_in), -_pow2_scales(rng, d_in, -2, 3)):
+        vals, meta = o.pack_2to4_scaled(W, scale)
+        score = np.abs(_f64(W)) * np.abs(scale.astype(np.float64))
+        for i in range(W.shape[0]):
+            pairs = decode_meta(meta[i], d_in // 4)
+            for g in range(d_in // 4):
+                a, b = brute_force_pair(score[i, 4 * g:4 * g + 4])
+                assert pairs[g] == (a, b), (i, g, pairs[g], (a, b))
+                assert vals[i, 2 * g] == W[i, 4 * g + a] and vals[i, 2 * g + 1] == W[i, 4 * g + b]
+
+
+def pin_scaled_minimises_weighted_error(o, seed: int = 23):
+    """The kept pair minimises the diagonal-Hessian error sum_j s_j^2 w_j^2 over
+    the dropped positions of each group, among all six 2-of-4 masks (fp64,
+    with slack for the fp32 rounding of the score)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    W = synth.gaussian_bf16((64, 64), 0.02, seed)
+    scale = np.exp(rng.normal(0.0, 1.5, size=64)).astype(np.float32)
+    vals, meta = o.pack_2to4_scaled(W, scale)
+    S = _f64(o.unpack_2to4(vals, meta, 64))
+    Wf, s2 = _f64(W), scale.astype(np.float64) ** 2
+    for i in range(64):
+        for g in range(16):
+            w, ss = Wf[i, 4 * g:4 * g + 4], s2[4 * g:4 * g + 4]
+            err = np.sum(ss * (w - S[i, 4 * g:4 * g + 4]) ** 2)
+            best = min(np.sum([ss[p] * w[p] ** 2 for p in range(4) if p not in pair])
+                       for pair in itertools.combinations(range(4), 2))
+            assert err <= best * (1 + 2.0 ** -20) + 1e-300, (i, g, err, best)
+
+
+def pin_scaled_hand_examples(o):
+    """Worked by hand: weights 1,2,3,4 with scales 4,2,1,1/2 score 4,4,3,2
+    (keep 0 and 1); scores 1,3,2,3 keep 1 and 3; an all-equal score keeps 0, 1."""
+    W = _bf16([[1, 2, 3, 4, 1, 1, 1, 1, 2, 1, 1, 2, -3, 0.5, 2, -1]])
+    scale = np.array([4, 2, 1, 0.5, 1, 3, 2, 3, 1, 2, 2, 1, -1, 8, -0.75, 2], dtype=np.float32)
+    vals, meta = o.pack_2to4_scaled(W, scale)
+    # group 3 scores 3, 4, 1.5, 2 -> keep 0, 1
+    np.testing.assert_array_equal(vals, _bf16([[1, 2, 1, 1, 2, 1, -3, 0.5]]))
+    assert int(meta[0, 0]) == ((0 | 1 << 2) | ((1 | 3 << 2) << 4))
+    assert int(meta[0, 1]) == ((0 | 1 << 2) | ((0 | 1 << 2) << 4))
+    # The unscaled projection of the same row differs in groups 0 and 3.
+    v0, _ = o.pack_2to4(W)
+    np.testing.assert_array_equal(v0[0, [0, 1, 6, 7]], _bf16([3, 4, -3, 2]))
+
+
+def pin_scaled_specials(o):
+    """Stated readings: a NaN score (NaN weight, or 0 times an infinite scale)
+    ranks above every number; an infinite score ranks above every finite one;
+    a zero scale makes all four scores +0, so the lower index wins."""
+    W = np.array([[0x3F80, 0x7FC0, 0x4000, 0x4040,      # NaN weight kept with the 3
+                   0x0000, 0x3F80, 0x4000, 0x4040,      # 0 * Inf = NaN, kept with the 3 (Inf)
+                   0x4040, 0x4000, 0x3F80, 0xC080]],    # zero scales: keep positions 0, 1
+                 dtype=np.uint16)
+    scale = np.array([1, 1, 1, 1, np.inf, 1, 1, np.inf, 0, 0, 0, 0], dtype=np.float32)
+    vals, meta = o.pack_2to4_scaled(W, scale)
+    np.testing.assert_array_equal(vals, [[0x7FC0, 0x4040, 0x0000, 0x4040, 0x4040, 0x4000]])
+    assert int(meta[0, 0]) == ((1 | 3 << 2) | ((0 | 3 << 2) << 4))
+    assert int(meta[0, 1]) == (0 | 1 << 2)
+
+
+def pin_scaled_group_locality(o, seed: int = 24):
+    """A group's choice depends on its own four scales only, and on their ratios:
+    multiplying one group's scales by a power of two changes nothing, and
+    permuting groups (weights and scales together) permutes the output."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    W = synth.gaussian_bf16((16, 48), 0.02, seed)
+    scale = np.exp(rng.normal(0.0, 1.0, size=48)).astype(np.float32)
+    vals, meta = o.pack_2to4_scaled(W, scale)
+    s2 = scale.copy()
+    s2[8:12] *= 64.0
+    s2[20:24] *= 2.0 ** -9
+    v2, m2 = o.pack_2to4_scaled(W, s2)
+    np.testing.assert_array_equal(v2, vals)
+    np.testing.assert_array_equal(m2, meta)
+    perm = rng.permutation(12)
+    cols = (4 * perm[:, None] + np.arange(4)).reshape(-1)
+    vp, mp = o.pack_2to4_scaled(W[:, cols], scale[cols])
+    pv = (2 * perm[:, None] + np.arange(2)).reshape(-1)
+    np.testing.assert_array_equal(vp, vals[:, pv])
+    for i in range(16):
+        assert decode_meta(mp[i], 12) == [decode_meta(meta[i], 12)[k] for k in perm]
+
+
+def pin_column_norms(o):
+    """Closed forms: a constant column c over M = 16 rows has norm 4|c|; a
+    one-hot column has norm |x|; a 3-4-5 column has norm 5; random columns
+    agree with the library 2-norm."""
+    M = 16
+    X = np.zeros((M, 8), dtype=np.uint16)
+    X[:, 0] = _bf16([-1.5] * M)
+    X[:, 1] = _bf16([2.0 ** -10] * M)
+    X[5, 2] = _bf16([-7.0])[0]
+    X[0, 3], X[9, 3] = _bf16([3.0, -4.0])
+    X[:, 5] = _bf16(np.arange(M) - 7.5)
+    X[:, 6] = 0x8000                                     # -0 everywhere
+    X[:, 7] = _bf16(np.where(np.arange(M) % 2 == 0, 1.0, -1.0))
+    n = o.column_norms(X)
+    assert n[0] == 6.0 and n[1] == 4 * 2.0 ** -10 and n[2] == 7.0 and n[3] == 5.0
+    assert n[4] == 0.0 and n[6] == 0.0 and n[7] == 4.0
+    assert abs(n[5] - np.sqrt(np.sum((np.arange(M) - 7.5) ** 2))) <= 1e-15 * n[5]
+    Xr = synth.gaussian_bf16((37, 24), 1.0, 25)
+    np.testing.assert_allclose(o.column_norms(Xr), np.linalg.norm(_f64(Xr), axis=0), rtol=1e-14)
+    assert o.column_norms(np.zeros((0, 5), dtype=np.uint16)).tolist() == [0.0] * 5
+
+
 ALL_PINS = [
     pin_pack_golden, pin_pack_exhaustive_alphabet, pin_pack_random_bruteforce,
     pin_pack_invariants, pin_pack_roundtrip, pin_pack_specials, pin_pack_odd_groups,
     pin_forward_golden, pin_forward_identity_exact, pin_forward_numpy, pin_forward_one_hot,
     pin_forward_sparse_only, pin_forward_row_subset, pin_lowrank_project,
+    pin_scaled_uniform_equals_unscaled, pin_scaled_bruteforce_exact, pin_scaled_minimises_weighted_error,
+    pin_scaled_hand_examples, pin_scaled_specials, pin_scaled_group_locality, pin_column_norms,
 ]

@@ -33,10 +33,10 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "slr_oracle.c")
 MUTANTS = [
     ("tie_to_higher_index", "(kq == kp && q < p)", "(kq == kp && q > p)", 1),
     ("signed_key", " & 0x7FFFu;", ";", 2),
-    ("smallest_magnitude", "if (rank < 2) kept[n++] = p;", "if (rank >= 2) kept[n++] = p;", 1),
-    ("kept_order_swapped", "*idx0 = kept[0];\n    *idx1 = kept[1];", "*idx0 = kept[1];\n    *idx1 = kept[0];", 1),
-    ("nibble_fields_swapped", "(unsigned)a | ((unsigned)b << 2)", "(unsigned)b | ((unsigned)a << 2)", 1),
-    ("nibble_position_swapped", "nib << (4 * (g % 2))", "nib << (4 * ((g + 1) % 2))", 1),
+    ("smallest_magnitude", "if (rank < 2) kept[n++] = p;", "if (rank >= 2) kept[n++] = p;", 2),
+    ("kept_order_swapped", "*idx0 = kept[0];\n    *idx1 = kept[1];", "*idx0 = kept[1];\n    *idx1 = kept[0];", 2),
+    ("nibble_fields_swapped", "(unsigned)a | ((unsigned)b << 2)", "(unsigned)b | ((unsigned)a << 2)", 2),
+    ("nibble_position_swapped", "nib << (4 * (g % 2))", "nib << (4 * ((g + 1) % 2))", 2),
     ("lowrank_sign", "row[j] += lr;", "row[j] -= lr;", 1),
     ("lowrank_dropped", "row[j] += lr;", "(void)lr;", 1),
     ("V_transposed", "V[k * d_in + j]", "V[j * r + k]", 2),
@@ -45,6 +45,16 @@ MUTANTS = [
     ("bound_signed", "fabs(xr[j]) * fabs(row[j])", "xr[j] * row[j]", 1),
     ("sparse_vals_swapped", "row[4 * g + a] = bf16_bits_to_double(vals[i * (d_in / 2) + 2 * g + 0]);",
      "row[4 * g + a] = bf16_bits_to_double(vals[i * (d_in / 2) + 2 * g + 1]);", 1),
+    ("scaled_tie_to_higher_index", "(key[q] == key[p] && q < p)", "(key[q] == key[p] && q > p)", 1),
+    ("scaled_signed_scale", "aw * fabsf(s)", "aw * s", 1),
+    ("scaled_nan_lowest", "if (isnan(prod)) return 0x7FFFFFFFu;", "if (isnan(prod)) return 0u;", 1),
+    ("scaled_wrong_column", "scale[4 * g + p]", "scale[p]", 1),
+    ("scaled_scale_ignored", "key[p] = scaled_key(w[p], scale[4 * g + p]);",
+     "key[p] = scaled_key(w[p], 1.0f);", 1),
+    ("norm_no_sqrt", "out[j] = sqrt(acc);", "out[j] = acc;", 1),
+    ("norm_abs_sum", "acc += x * x;", "acc += fabs(x);", 1),
+    ("norm_wrong_column", "double x = bf16_bits_to_double(X[m * d_in + j]);",
+     "double x = bf16_bits_to_double(X[m * d_in]);", 1),
 ]
 
 
