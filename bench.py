@@ -293,6 +293,8 @@ def run_ours(args, rank, world, dist):
 
     # ------------------------------------------------ pack leg
     pack = run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier) if "pack" in legs else None
+    calibrate = run_calibrate_leg(args, slr, torch, dev, W, to_dev, peaks, max_over_ranks, barrier) \
+        if "calibrate" in legs else None
     del W
 
     # ------------------------------------------------ the other configurations
@@ -317,6 +319,7 @@ def run_ours(args, rank, world, dist):
         "decode_m1": decode,
         **sweep,
         "pack": pack,
+        "calibrate": calibrate,
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": 2 * K,
@@ -608,6 +611,60 @@ def run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier):
             "frac": round(gbs / peaks["hbm_gbs"], 4)}
 
 
+def run_calibrate_leg(args, slr, torch, dev, W, to_dev, peaks, max_over_ranks, barrier):
+    """Activation-aware 2:4 projection (HASSLE-free section 4.1.2): the column
+    norms of a batch of calibration tokens, then the projection of the
+    gate/up weight scaled by them.  Each kernel is timed alone over rotating
+    buffers larger than L2; GB/s counts the algorithmic bytes (X read once and
+    d_in norms written; W read, vals + meta written, d_in scales read)."""
+    d_out, d_in = W.shape
+    L = layer_of(PREFILL["cfg"], PREFILL["name"])
+    Mc = 16384
+    Xh = L.activations(Mc)
+    x_bytes = Mc * d_in * 2 + d_in * (8 + 8 + 4)
+    n_x = max(2, math.ceil(2.0 * L2_BYTES / x_bytes))
+    Xs = [to_dev(Xh) for _ in range(n_x)]
+    ws_need = max(slr.column_norms_workspace_size(Mc, d_in), 16)
+    ws = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    sumsq = torch.zeros(d_in, dtype=torch.float64, device=dev)
+    norms = torch.empty(d_in, dtype=torch.float32, device=dev)
+    lib = slr.lib()
+
+    def norm(i):
+        st = lib.slr_column_norms(slr._ptr(Xs[i % n_x]), Mc, d_in, d_in, slr._ptr(sumsq), slr._ptr(norms),
+                                  slr._ptr(ws), ws_need, slr._stream())
+        assert st == 0, st
+
+    p_bytes = d_out * d_in * 2 + d_out * d_in + d_out * d_in // 8 + d_in * 4
+    n_w = max(2, math.ceil(2.0 * L2_BYTES / p_bytes))
+    Ws = [W if i == 0 else W.clone() for i in range(n_w)]
+    outs = [(torch.empty((d_out, d_in // 2), dtype=torch.bfloat16, device=dev),
+             torch.empty((d_out, d_in // 8), dtype=torch.uint8, device=dev)) for _ in range(n_w)]
+
+    def pack(i):
+        v, m = outs[i % n_w]
+        st = lib.slr_pack_2to4_scaled(slr._ptr(Ws[i % n_w]), d_out, d_in, d_in, slr._ptr(norms), slr._ptr(v),
+                                      slr._ptr(m), slr._stream())
+        assert st == 0, st
+
+    for i in range(3):
+        norm(i)
+        pack(i)
+    K = max(10, args.steps)
+    barrier()
+    ms_n = max_over_ranks(graph_time_ms(torch, [lambda k=k: norm(k) for k in range(K)])) / K
+    ms_p = max_over_ranks(graph_time_ms(torch, [lambda k=k: pack(k) for k in range(K)])) / K
+    gbs_n = x_bytes / (ms_n * 1e-3) / 1e9
+    gbs_p = p_bytes / (ms_p * 1e-3) / 1e9
+    hbm = peaks["hbm_gbs"]
+    return {"workload": f"column norms of {Mc} calibration tokens x {d_in}, then the activation-aware 2:4 "
+                        f"projection of the {d_out}x{d_in} gate/up weight",
+            "column_norms": {"value": round(gbs_n, 1), "unit": "GB/s", "ms_per_call": round(ms_n, 5),
+                             "bytes_per_call": x_bytes, "frac": round(gbs_n / hbm, 4), "launches_per_call": 2},
+            "pack_scaled": {"value": round(gbs_p, 1), "unit": "GB/s", "ms_per_launch": round(ms_p, 5),
+                            "bytes_per_launch": p_bytes, "frac": round(gbs_p / hbm, 4)}}
+
+
 def cpu_baseline_prefill(L, rows: int):
     import oracle
     W = L.weight()
@@ -670,7 +727,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024, help="token rows in the oracle CPU baseline sample")
     ap.add_argument("--ref-rows", type=int, default=64, help="token rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="prefill,e2e,decode,pack,cpu,cfg2,cfg4,cfg5",
+    ap.add_argument("--only", default="prefill,e2e,decode,pack,calibrate,cpu,cfg2,cfg4,cfg5",
                     help="comma list of legs to run (profiling runs use one leg)")
     args = ap.parse_args()
     if args.warmup < 3:

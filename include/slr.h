@@ -92,6 +92,63 @@ SLR_API slr_status slr_pack_2to4(const void *W, int64_t d_out, int64_t d_in, int
 SLR_API int64_t slr_meta_row_bytes(int64_t d_in);
 
 /* --------------------------------------------------------------------------
+ * Activation-aware 2:4 projection and packing.
+ *
+ * HASSLE-free, section 4.1.2: with the diagonal Hessian approximation
+ * H = diag(X^T X) the sparse step hard-thresholds W D, D = diag of the input
+ * column norms, which is Wanda's score.  The weight w_ij is ranked by the
+ * fp32 product |w_ij| * |scale[j]| (one IEEE multiply, round to nearest); a
+ * NaN product ranks above every number; equal products keep the lower index.
+ * The kept values are the unscaled weights; the output format is the one of
+ * slr_pack_2to4, so slr_forward consumes it unchanged.  With every scale equal
+ * to the same power of two the result equals slr_pack_2to4's.
+ *
+ *   W      device, bf16 [d_out, ldw] (ldw >= d_in), read only.
+ *   scale  device, fp32 [d_in], read only: the column scales (the sign is
+ *          ignored), e.g. the norms from slr_column_norms.
+ *   vals, meta  as for slr_pack_2to4.
+ *
+ * Requirements: as slr_pack_2to4, and scale non-NULL unless d_out * d_in == 0.
+ * Any alignment is accepted; 16-byte aligned W and scale with d_in and ldw
+ * multiples of 8 take the vectorised path.  Bit-exact and deterministic.
+ * ------------------------------------------------------------------------ */
+SLR_API slr_status slr_pack_2to4_scaled(const void *W, int64_t d_out, int64_t d_in, int64_t ldw,
+                                const float *scale, void *vals, void *meta, slr_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Column norms of calibration activations (the scale of the projection above).
+ *
+ * HASSLE-free, section 4.1.2 (diagonal Hessian) and section 5.1 (the Hessian
+ * is gathered over many token segments): each call adds one batch X
+ * (M tokens x d_in) to a running per-column sum of squares and can emit the
+ * norms, so a calibration set is streamed batch by batch.
+ *
+ *   X        device, bf16 [M, ldx] (ldx >= d_in), read only.
+ *   sumsq    device, fp64 [d_in], in/out: sumsq[j] += sum_m X[m][j]^2.  Zero it
+ *            before the first batch.
+ *   norms    device, fp32 [d_in], out, or NULL: norms[j] = sqrt(sumsq[j]) (after
+ *            the update; fp64 square root rounded to nearest fp32).
+ *   workspace / workspace_bytes: device scratch of at least
+ *            slr_column_norms_workspace_size(M, d_in) bytes; clobbered.
+ *
+ * Arithmetic: squares are summed in fp32 over at most 64 rows per thread and
+ * 8 threads per column, partial sums are then added in fp64 in a fixed order
+ * (which depends on M and d_in only: deterministic on any device).  Relative
+ * error of a batch's sum of squares <= 80 * 2^-24 for M <= 2^25 (tested
+ * against fp64).
+ *
+ * Requirements: M >= 0, d_in >= 0, d_in % 8 == 0, ldx >= d_in, ldx % 8 == 0;
+ * when d_in > 0: sumsq non-NULL and 8-byte aligned, norms 4-byte aligned, and
+ * when also M > 0: X non-NULL and 16-byte aligned, workspace large enough.
+ * M == 0 only (re)writes norms from sumsq; d_in == 0 does nothing.
+ * ------------------------------------------------------------------------ */
+SLR_API slr_status slr_column_norms(const void *X, int64_t M, int64_t d_in, int64_t ldx, double *sumsq,
+                            float *norms, void *workspace, size_t workspace_bytes, slr_stream_t stream);
+
+/* Scratch bytes slr_column_norms needs for a batch of M tokens (0 when none). */
+SLR_API size_t slr_column_norms_workspace_size(int64_t M, int64_t d_in);
+
+/* --------------------------------------------------------------------------
  * Forward pass  Y = X * S^T + (X * V^T) * U^T.
  *
  * LoSparse, section 3.2: the compressed layer computes the low-rank and sparse

@@ -8,6 +8,8 @@ import fails if the library is missing.
 Functions mirror the C ABI in ``include/slr.h``:
 
 * ``pack_2to4(W) -> (vals, meta)``  -- ``slr_pack_2to4``
+* ``pack_2to4_scaled(W, scale) -> (vals, meta)``  -- ``slr_pack_2to4_scaled``
+* ``column_norms(X, sumsq=None) -> (norms, sumsq)``  -- ``slr_column_norms``
 * ``forward(X, vals, meta, U, V) -> Y``  -- ``slr_forward`` /
   ``slr_forward_with_path``
 * ``workspace_size``, ``select_path``, ``check_kernel_error``
@@ -53,6 +55,12 @@ def _load() -> ctypes.CDLL:
     lib.slr_pack_2to4.argtypes = [p, i64, i64, i64, p, p, p]
     lib.slr_meta_row_bytes.restype = i64
     lib.slr_meta_row_bytes.argtypes = [i64]
+    lib.slr_pack_2to4_scaled.restype = st
+    lib.slr_pack_2to4_scaled.argtypes = [p, i64, i64, i64, p, p, p, p]
+    lib.slr_column_norms.restype = st
+    lib.slr_column_norms.argtypes = [p, i64, i64, i64, p, p, p, sz, p]
+    lib.slr_column_norms_workspace_size.restype = sz
+    lib.slr_column_norms_workspace_size.argtypes = [i64, i64]
     lib.slr_forward.restype = st
     lib.slr_forward.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, p, sz, p]
     lib.slr_forward_with_path.restype = st
@@ -109,6 +117,47 @@ def pack_2to4(W: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
     _check(_lib.slr_pack_2to4(_ptr(W), d_out, d_in, W.stride(0), _ptr(vals), _ptr(meta), _stream()),
            "slr_pack_2to4")
     return vals, meta
+
+
+def pack_2to4_scaled(W: torch.Tensor, scale: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+    """Activation-aware 2:4 projection of bf16 ``W`` [d_out, d_in]: weights of
+    column j ranked by |w| * |scale[j]| (fp32 ``scale`` [d_in])."""
+    if W.dtype != torch.bfloat16 or W.dim() != 2 or not W.is_cuda or W.stride(1) != 1:
+        raise ValueError("W must be a 2-D CUDA bf16 tensor with unit column stride")
+    d_out, d_in = W.shape
+    if scale.dtype != torch.float32 or scale.shape != (d_in,) or not scale.is_contiguous() or \
+            scale.device != W.device:
+        raise ValueError("scale must be a contiguous fp32 tensor of d_in elements on W's device")
+    vals = torch.empty((d_out, d_in // 2), dtype=torch.bfloat16, device=W.device)
+    meta = torch.empty((d_out, meta_row_bytes(d_in)), dtype=torch.uint8, device=W.device)
+    _check(_lib.slr_pack_2to4_scaled(_ptr(W), d_out, d_in, W.stride(0), _ptr(scale), _ptr(vals), _ptr(meta),
+                                     _stream()), "slr_pack_2to4_scaled")
+    return vals, meta
+
+
+def column_norms_workspace_size(M: int, d_in: int) -> int:
+    return int(_lib.slr_column_norms_workspace_size(M, d_in))
+
+
+def column_norms(X: torch.Tensor, sumsq: torch.Tensor | None = None, *, want_norms: bool = True,
+                 workspace: torch.Tensor | None = None) -> tuple[torch.Tensor | None, torch.Tensor]:
+    """Add the column sums of squares of bf16 ``X`` [M, d_in] to the fp64
+    running sum ``sumsq`` (a new zero sum when None) and return
+    ``(norms, sumsq)``, norms = fp32 sqrt(sumsq) (None unless ``want_norms``)."""
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or not X.is_cuda or X.stride(1) != 1:
+        raise ValueError("X must be a 2-D CUDA bf16 tensor with unit column stride")
+    M, d_in = X.shape
+    if sumsq is None:
+        sumsq = torch.zeros(d_in, dtype=torch.float64, device=X.device)
+    elif sumsq.dtype != torch.float64 or sumsq.shape != (d_in,) or not sumsq.is_contiguous():
+        raise ValueError("sumsq must be a contiguous fp64 tensor of d_in elements")
+    norms = torch.empty(d_in, dtype=torch.float32, device=X.device) if want_norms else None
+    need = column_norms_workspace_size(M, d_in)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
+    _check(_lib.slr_column_norms(_ptr(X), M, d_in, X.stride(0), _ptr(sumsq), _ptr(norms), _ptr(workspace),
+                                 workspace.numel(), _stream()), "slr_column_norms")
+    return norms, sumsq
 
 
 def workspace_size(M: int, d_out: int, d_in: int, r: int) -> int:

@@ -162,6 +162,42 @@ slr_status slr_pack_2to4(const void *W, int64_t d_out, int64_t d_in, int64_t ldw
     return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
 }
 
+slr_status slr_pack_2to4_scaled(const void *W, int64_t d_out, int64_t d_in, int64_t ldw, const float *scale,
+                                void *vals, void *meta, slr_stream_t stream) {
+    if (d_out < 0 || d_in < 0 || d_in % 4 != 0 || ldw < d_in) return SLR_ERR_SHAPE;
+    if (d_out == 0 || d_in == 0) return SLR_OK;
+    if (W == nullptr || scale == nullptr || vals == nullptr || meta == nullptr) return SLR_ERR_NULL;
+    const slr_status dev = slr::check_device();
+    if (dev != SLR_OK) return dev;
+    const cudaError_t err = slr::launch_pack_2to4_scaled(
+        static_cast<const uint16_t *>(W), d_out, d_in, ldw, scale, static_cast<uint16_t *>(vals),
+        static_cast<uint8_t *>(meta), reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
+}
+
+size_t slr_column_norms_workspace_size(int64_t M, int64_t d_in) {
+    if (M <= 0 || d_in <= 0 || d_in % 8 != 0) return 0;
+    const slr::NormPlan p = slr::column_norms_plan(M, d_in);
+    return slr::round_up((size_t)p.splits * (size_t)d_in * sizeof(float), slr::kAlign);
+}
+
+slr_status slr_column_norms(const void *X, int64_t M, int64_t d_in, int64_t ldx, double *sumsq, float *norms,
+                            void *workspace, size_t workspace_bytes, slr_stream_t stream) {
+    if (M < 0 || d_in < 0 || d_in % 8 != 0 || ldx < d_in || ldx % 8 != 0) return SLR_ERR_SHAPE;
+    if (d_in == 0) return SLR_OK;
+    if (sumsq == nullptr || (M > 0 && (X == nullptr || workspace == nullptr))) return SLR_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(sumsq) & 7) != 0 || (reinterpret_cast<uintptr_t>(norms) & 3) != 0 ||
+        (M > 0 && (!slr::aligned16(X) || !slr::aligned16(workspace))))
+        return SLR_ERR_ALIGN;
+    if (workspace_bytes < slr_column_norms_workspace_size(M, d_in)) return SLR_ERR_WORKSPACE;
+    const slr_status dev = slr::check_device();
+    if (dev != SLR_OK) return dev;
+    const cudaError_t err = slr::launch_column_norms(static_cast<const uint16_t *>(X), M, d_in, ldx, sumsq, norms,
+                                                     static_cast<float *>(workspace),
+                                                     reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
+}
+
 size_t slr_forward_workspace_size(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
     (void)d_out;
     (void)d_in;

@@ -36,6 +36,25 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
 cudaError_t launch_pack_2to4(const uint16_t *W, int64_t d_out, int64_t d_in, int64_t ldw,
                              uint16_t *vals, uint8_t *meta, cudaStream_t stream);
 
+// Activation-aware 2:4 projection: as launch_pack_2to4 with the weights of
+// column j ranked by |w| * |scale[j]| (fp32).
+cudaError_t launch_pack_2to4_scaled(const uint16_t *W, int64_t d_out, int64_t d_in, int64_t ldw,
+                                    const float *scale, uint16_t *vals, uint8_t *meta, cudaStream_t stream);
+
+// Row split of the column-norm reduction: `splits` row ranges of
+// `rows_per_split` rows, each leaving d_in fp32 partial sums in the workspace.
+struct NormPlan {
+    int64_t rows_per_split;
+    int64_t splits;
+};
+NormPlan column_norms_plan(int64_t M, int64_t d_in);
+
+// sumsq[j] += sum_m X[m][j]^2; norms[j] = sqrt(sumsq[j]) rounded to fp32 when
+// norms is not null.  partial: splits * d_in floats of scratch (d_in >= 1,
+// d_in % 8 == 0, ldx % 8 == 0, X 16-byte aligned).
+cudaError_t launch_column_norms(const uint16_t *X, int64_t M, int64_t d_in, int64_t ldx, double *sumsq,
+                                float *norms, float *partial, cudaStream_t stream);
+
 // T = X * V^T for M tokens, written as fp32 [M, r] (T32, may be null) and/or
 // bf16 [M, r] (T16, may be null).
 cudaError_t launch_lowrank_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in,

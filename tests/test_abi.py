@@ -125,3 +125,37 @@ def test_selftest_wait_timeout_arguments():
     assert lib.slr_selftest_wait_timeout(1 << 31, None) == ARG
     if not torch.cuda.is_available():
         assert lib.slr_selftest_wait_timeout(1000, None) == DEVICE
+
+
+def test_pack_scaled_argument_errors():
+    lib = slr.lib()
+    f = lib.slr_pack_2to4_scaled
+    assert f(P(0x1000), 4, 6, 6, P(0x4000), P(0x2000), P(0x3000), None) == SHAPE   # d_in % 4
+    assert f(P(0x1000), 4, 8, 4, P(0x4000), P(0x2000), P(0x3000), None) == SHAPE   # ldw < d_in
+    assert f(P(0x1000), 4, 8, 8, P(0), P(0x2000), P(0x3000), None) == NULL         # scale
+    assert f(P(0), 0, 8, 8, P(0), P(0), P(0), None) == OK                           # empty
+    if not torch.cuda.is_available():
+        assert f(P(0x1000), 4, 8, 8, P(0x4000), P(0x2000), P(0x3000), None) == DEVICE
+
+
+def test_column_norms_argument_errors_and_workspace():
+    lib = slr.lib()
+    f = lib.slr_column_norms
+    assert f(P(0x1000), 4, 12, 12, P(0x2000), None, P(0x3000), 1 << 20, None) == SHAPE  # d_in % 8
+    assert f(P(0x1000), 4, 16, 8, P(0x2000), None, P(0x3000), 1 << 20, None) == SHAPE   # ldx < d_in
+    assert f(P(0x1000), 4, 16, 20, P(0x2000), None, P(0x3000), 1 << 20, None) == SHAPE  # ldx % 8
+    assert f(P(0x1000), -1, 16, 16, P(0x2000), None, P(0x3000), 1 << 20, None) == SHAPE
+    assert f(P(0x1000), 4, 16, 16, P(0), None, P(0x3000), 1 << 20, None) == NULL       # sumsq
+    assert f(P(0), 4, 16, 16, P(0x2000), None, P(0x3000), 1 << 20, None) == NULL       # X
+    assert f(P(0x1008), 4, 16, 16, P(0x2000), None, P(0x3000), 1 << 20, None) == ALIGN  # X 16 B
+    assert f(P(0x1000), 4, 16, 16, P(0x2004), None, P(0x3000), 1 << 20, None) == ALIGN  # sumsq 8 B
+    assert f(P(0x1000), 4, 16, 16, P(0x2000), None, P(0x3000), 0, None) == WORKSPACE
+    assert f(P(0), 4, 0, 0, P(0), None, P(0), 0, None) == OK                           # d_in == 0
+    if not torch.cuda.is_available():
+        assert f(P(0), 0, 16, 16, P(0x2000), P(0x4000), P(0), 0, None) == DEVICE     # M == 0: norms only
+    ws = slr.column_norms_workspace_size
+    assert ws(0, 4096) == 0 and ws(16, 0) == 0
+    # 2048 tokens x 4096 columns: 16 strips x 64 splits of 32 rows = 1024 CTAs.
+    assert ws(2048, 4096) == 64 * 4096 * 4
+    # Very tall batches cap a split at 512 rows.
+    assert ws(1 << 20, 4096) == (1 << 20) // 512 * 4096 * 4
