@@ -144,9 +144,10 @@ def column_norms(X: torch.Tensor, sumsq: torch.Tensor | None = None, *, want_nor
     """Add the column sums of squares of bf16 ``X`` [M, d_in] to the fp64
     running sum ``sumsq`` (a new zero sum when None) and return
     ``(norms, sumsq)``, norms = fp32 sqrt(sumsq) (None unless ``want_norms``)."""
-    if X.dtype != torch.bfloat16 or X.dim() != 2 or not X.is_cuda or X.stride(1) != 1:
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or not X.is_cuda or (X.numel() > 0 and X.stride(1) != 1):
         raise ValueError("X must be a 2-D CUDA bf16 tensor with unit column stride")
     M, d_in = X.shape
+    ldx = X.stride(0) if X.numel() > 0 else d_in
     if sumsq is None:
         sumsq = torch.zeros(d_in, dtype=torch.float64, device=X.device)
     elif sumsq.dtype != torch.float64 or sumsq.shape != (d_in,) or not sumsq.is_contiguous():
@@ -155,7 +156,7 @@ def column_norms(X: torch.Tensor, sumsq: torch.Tensor | None = None, *, want_nor
     need = column_norms_workspace_size(M, d_in)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
-    _check(_lib.slr_column_norms(_ptr(X), M, d_in, X.stride(0), _ptr(sumsq), _ptr(norms), _ptr(workspace),
+    _check(_lib.slr_column_norms(_ptr(X), M, d_in, ldx, _ptr(sumsq), _ptr(norms), _ptr(workspace),
                                  workspace.numel(), _stream()), "slr_column_norms")
     return norms, sumsq
 

@@ -9,16 +9,19 @@
 // runs over batches: every call adds one batch's squares to a running fp64 sum.
 //
 // Two kernels, HBM-bound on reading X once (2 bytes per element):
-//  (1) partial sums.  Grid = (strips of 256 columns) x (row splits).  Lane l
-//      of a warp owns 8 columns (one 16-byte load per row, so a warp reads
-//      512 contiguous bytes of a row); the 8 warps of a CTA take interleaved
-//      rows of the split, kNormRows rows in flight per thread; each thread
+//  (1) partial sums.  Grid = (strips of 256 columns) x (row splits), sized
+//      to one wave of 6 resident CTAs on each of 148 SMs.  Lane l of a warp
+//      owns 8 columns (one 16-byte load per row, so a warp reads 512
+//      contiguous bytes of a row); the 8 warps of a CTA take interleaved rows
+//      of the split, kNormRows rows in flight per thread; each thread
 //      accumulates its 8 columns in fp32; the 8 warp sums of a column are then
 //      added in warp order through shared memory and written to row `split`
 //      of the workspace.
-//  (2) finish.  One thread per column adds the split sums in split order in
-//      fp64 to the running sum and, when asked, writes the norm: the fp64
-//      square root rounded to fp32.
+//  (2) finish, launched as a programmatic dependent of (1) so that its launch
+//      overlaps (1)'s tail.  Four threads per column each add every fourth
+//      split in fp64, the four sums are added in a fixed order, the total is
+//      added to the running sum and, when asked, the norm is written: the
+//      fp64 square root rounded to fp32.
 // The split count depends on (M, d_in) only, so the result is deterministic
 // and the same on every device.
 #include "common.cuh"
@@ -29,11 +32,12 @@ namespace {
 constexpr int kNormThreads = 256;     // 8 warps
 constexpr int kNormStripCols = 256;   // 32 lanes x 8 columns
 constexpr int kNormRows = 4;          // rows in flight per thread
-constexpr int64_t kNormTargetCtas = 1184;  // 8 CTAs on each of 148 SMs
+constexpr int kNormCtasPerSm = 6;
+constexpr int64_t kNormTargetCtas = 148 * kNormCtasPerSm;  // one wave on B200
 constexpr int64_t kNormMinRows = 32;  // one step of 8 warps x kNormRows
 constexpr int64_t kNormMaxRows = 512; // caps a thread's serial fp32 sum at 64 terms
 
-__global__ void __launch_bounds__(kNormThreads) column_sumsq_partial_kernel(const uint16_t *__restrict__ X,
+__global__ void __launch_bounds__(kNormThreads, kNormCtasPerSm) column_sumsq_partial_kernel(const uint16_t *__restrict__ X,
                                                                             int64_t M, int64_t d_in, int64_t ldx,
                                                                             int64_t rows_per_split,
                                                                             float *__restrict__ partial) {
@@ -68,6 +72,9 @@ __global__ void __launch_bounds__(kNormThreads) column_sumsq_partial_kernel(cons
             }
         }
     }
+    // The finish kernel may be scheduled now; it waits for this grid's
+    // completion (and memory flush) before reading the partial sums.
+    asm volatile("griddepcontrol.launch_dependents;");
 #pragma unroll
     for (int k = 0; k < 8; ++k) red[warp][lane * 9 + k] = acc[k];
     __syncthreads();
@@ -81,16 +88,26 @@ __global__ void __launch_bounds__(kNormThreads) column_sumsq_partial_kernel(cons
     }
 }
 
+// Block = 64 columns x 4 split classes; thread (q, c) adds splits q, q+4, ...
 __global__ void __launch_bounds__(256) column_norms_finish_kernel(const float *__restrict__ partial, int64_t splits,
                                                                   int64_t d_in, double *__restrict__ sumsq,
                                                                   float *__restrict__ norms) {
-    const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (j >= d_in) return;
+    __shared__ double red[4][64];
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int q = threadIdx.x >> 6, cl = threadIdx.x & 63;
+    const int64_t j = (int64_t)blockIdx.x * 64 + cl;
     double s = 0.0;
-    for (int64_t k = 0; k < splits; ++k) s += (double)partial[k * d_in + j];
-    const double total = sumsq[j] + s;
-    sumsq[j] = total;
-    if (norms != nullptr) norms[j] = __double2float_rn(sqrt(total));
+    if (j < d_in) {
+#pragma unroll 8
+        for (int64_t k = q; k < splits; k += 4) s += (double)partial[k * d_in + j];
+    }
+    red[q][cl] = s;
+    __syncthreads();
+    if (q == 0 && j < d_in) {
+        const double total = sumsq[j] + (((red[0][cl] + red[1][cl]) + red[2][cl]) + red[3][cl]);
+        sumsq[j] = total;
+        if (norms != nullptr) norms[j] = __double2float_rn(sqrt(total));
+    }
 }
 
 }  // namespace
@@ -117,9 +134,21 @@ cudaError_t launch_column_norms(const uint16_t *X, int64_t M, int64_t d_in, int6
         column_sumsq_partial_kernel<<<dim3((unsigned)strips, (unsigned)p.splits), kNormThreads, 0, stream>>>(
             X, M, d_in, ldx, p.rows_per_split, partial);
     }
-    column_norms_finish_kernel<<<(unsigned)((d_in + 255) / 256), 256, 0, stream>>>(partial, p.splits, d_in, sumsq,
-                                                                                    norms);
-    return cudaGetLastError();
+    if (p.splits == 0) {
+        column_norms_finish_kernel<<<(unsigned)((d_in + 63) / 64), 256, 0, stream>>>(partial, 0, d_in, sumsq, norms);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((d_in + 63) / 64));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, column_norms_finish_kernel, (const float *)partial, p.splits, d_in, sumsq, norms);
 }
 
 }  // namespace slr

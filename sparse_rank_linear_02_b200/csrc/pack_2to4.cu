@@ -64,21 +64,38 @@ __device__ __forceinline__ uint32_t select_group(uint32_t w01, uint32_t w23, uin
 // nearest (an explicit _rn multiply, never contracted), sign cleared; a NaN
 // product takes the largest key 0x7FFFFFFF.  Non-negative floats order like
 // their bit patterns, so the keys compare as unsigned integers.
-__device__ __forceinline__ uint64_t scaled_key(uint32_t mag_hi, float a, uint32_t low) {
-    uint32_t k = __float_as_uint(__fmul_rn(__uint_as_float(mag_hi), a)) & 0x7FFFFFFFu;
-    k = k > 0x7F800000u ? 0x7FFFFFFFu : k;
-    return ((uint64_t)k << 2) | low;
+__device__ __forceinline__ uint32_t scaled_key(uint32_t mag_hi, float a) {
+    const uint32_t k = __float_as_uint(__fmul_rn(__uint_as_float(mag_hi), a)) & 0x7FFFFFFFu;
+    return k > 0x7F800000u ? 0x7FFFFFFFu : k;
 }
 
 // Activation-aware projection of one group; a0..a3 are the absolute scales
-// of its four columns.
+// of its four columns.  The keys use all 32 bits, so the position tie-break
+// is explicit: a tournament of (0,1) and (2,3), where a tie keeps the lower
+// position; the overall first is the better of the two pair winners (ties to
+// the (0,1) side, whose positions are lower); the second is the better of the
+// winning pair's loser and the losing pair's winner (again ties to the lower
+// position, which is the one from (0,1)).
 __device__ __forceinline__ uint32_t select_group_scaled(uint32_t w01, uint32_t w23, float a0, float a1, float a2,
                                                         float a3, uint32_t *kept) {
-    const uint64_t e0 = scaled_key((w01 & 0x7FFFu) << 16, a0, 3u);
-    const uint64_t e1 = scaled_key(w01 & 0x7FFF0000u, a1, 2u);
-    const uint64_t e2 = scaled_key((w23 & 0x7FFFu) << 16, a2, 1u);
-    const uint64_t e3 = scaled_key(w23 & 0x7FFF0000u, a3, 0u);
-    const uint32_t nib = top_two_nibble(e0, e1, e2, e3);
+    const uint32_t k0 = scaled_key((w01 & 0x7FFFu) << 16, a0);
+    const uint32_t k1 = scaled_key(w01 & 0x7FFF0000u, a1);
+    const uint32_t k2 = scaled_key((w23 & 0x7FFFu) << 16, a2);
+    const uint32_t k3 = scaled_key(w23 & 0x7FFF0000u, a3);
+    const bool b01 = k0 >= k1, b23 = k2 >= k3;
+    const uint32_t hi01 = max(k0, k1), lo01 = min(k0, k1);
+    const uint32_t hi23 = max(k2, k3), lo23 = min(k2, k3);
+    const uint32_t win01 = b01 ? 0u : 1u, los01 = b01 ? 1u : 0u;
+    const uint32_t win23 = b23 ? 2u : 3u, los23 = b23 ? 3u : 2u;
+    uint32_t first, second;
+    if (hi01 >= hi23) {
+        first = win01;
+        second = lo01 >= hi23 ? los01 : win23;
+    } else {
+        first = win23;
+        second = hi01 >= lo23 ? win01 : los23;
+    }
+    const uint32_t nib = min(first, second) | (max(first, second) << 2);
     *kept = gather_kept(nib, w01, w23);
     return nib;
 }

@@ -155,7 +155,8 @@ def test_column_norms_argument_errors_and_workspace():
         assert f(P(0), 0, 16, 16, P(0x2000), P(0x4000), P(0), 0, None) == DEVICE     # M == 0: norms only
     ws = slr.column_norms_workspace_size
     assert ws(0, 4096) == 0 and ws(16, 0) == 0
-    # 2048 tokens x 4096 columns: 16 strips x 64 splits of 32 rows = 1024 CTAs.
-    assert ws(2048, 4096) == 64 * 4096 * 4
+    # 2048 tokens x 4096 columns: 16 strips; one wave of 888 CTAs wants 37 rows
+    # per split, rounded up to 64: 32 splits.
+    assert ws(2048, 4096) == 32 * 4096 * 4
     # Very tall batches cap a split at 512 rows.
     assert ws(1 << 20, 4096) == (1 << 20) // 512 * 4096 * 4
