@@ -81,6 +81,10 @@ class Oracle:
         lib.oracle_max_threads.restype = ctypes.c_int
         lib.oracle_pack_2to4_scaled.restype = ctypes.c_int
         lib.oracle_pack_2to4_scaled.argtypes = [p, i64, i64, i64, p, p, p]
+        lib.oracle_pack_2to8.restype = ctypes.c_int
+        lib.oracle_pack_2to8.argtypes = [p, i64, i64, i64, p, p]
+        lib.oracle_unpack_2to8.restype = ctypes.c_int
+        lib.oracle_unpack_2to8.argtypes = [p, p, i64, i64, p]
         lib.oracle_column_norms.restype = ctypes.c_int
         lib.oracle_column_norms.argtypes = [p, i64, i64, p]
         self._lib = lib
@@ -122,6 +126,39 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle_pack_2to4_scaled rejected shape {W.shape} (rc={rc})")
         return vals, meta
+
+    def pack_2to8(self, W: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+        """2:8 projection by magnitude: (vals [d_out, d_in/4], meta [d_out, d_in/8]),
+        meta byte = idx0 | idx1 << 3."""
+        W = _u16(W)
+        d_out, d_in = W.shape
+        vals = np.zeros((d_out, d_in // 4), dtype=np.uint16)
+        meta = np.zeros((d_out, d_in // 8), dtype=np.uint8)
+        rc = self._lib.oracle_pack_2to8(_ptr(W), d_out, d_in, d_in, _ptr(vals), _ptr(meta))
+        if rc != 0:
+            raise ValueError(f"oracle_pack_2to8 rejected shape {W.shape} (rc={rc})")
+        return vals, meta
+
+    def unpack_2to8(self, vals: np.ndarray, meta: np.ndarray, d_in: int) -> np.ndarray:
+        """Dense bf16 bits [d_out, d_in] of a 2:8 packing (+0 elsewhere)."""
+        vals = _u16(vals)
+        meta = np.ascontiguousarray(meta, dtype=np.uint8)
+        d_out = vals.shape[0]
+        S = np.zeros((d_out, d_in), dtype=np.uint16)
+        if self._lib.oracle_unpack_2to8(_ptr(vals), _ptr(meta), d_out, d_in, _ptr(S)) != 0:
+            raise ValueError("oracle_unpack_2to8 rejected its arguments")
+        return S
+
+    def as_2to4(self, vals8: np.ndarray, meta8: np.ndarray, d_in: int) -> tuple[np.ndarray, np.ndarray]:
+        """The 2:4 packing of a 2:8 matrix (lossless: every half-group of four
+        holds at most two of the kept positions)."""
+        return self.pack_2to4(self.unpack_2to8(vals8, meta8, d_in))
+
+    def forward_2to8(self, X, vals8, meta8, U, V, rows=None, outs=None):
+        """Forward of a 2:8 layer: the forward of its 2:4 packing."""
+        d_in = _u16(X).shape[1]
+        vals, meta = self.as_2to4(vals8, meta8, d_in)
+        return self.forward(X, vals, meta, U, V, rows=rows, outs=outs)
 
     def column_norms(self, X: np.ndarray) -> np.ndarray:
         """fp64 norms of the columns of bf16 ``X`` [M, d_in]."""
@@ -223,6 +260,22 @@ def pack_2to4_scaled(W, scale):
 
 def column_norms(X):
     return default().column_norms(X)
+
+
+def pack_2to8(W):
+    return default().pack_2to8(W)
+
+
+def unpack_2to8(vals, meta, d_in):
+    return default().unpack_2to8(vals, meta, d_in)
+
+
+def as_2to4(vals8, meta8, d_in):
+    return default().as_2to4(vals8, meta8, d_in)
+
+
+def forward_2to8(X, vals8, meta8, U, V, rows=None, outs=None):
+    return default().forward_2to8(X, vals8, meta8, U, V, rows=rows, outs=outs)
 
 
 def pack_2to4(W):

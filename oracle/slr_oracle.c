@@ -31,6 +31,17 @@
  *      packed format is the one above.  The column norms s_j = ||X[:, j]||_2
  *      are computed in fp64.
  *
+ *   1c. The 2:8 projection (the "2:8 plus rank-64" configuration of the
+ *      3BASiL summary page, "Faster compression and gains that survive LoRA"
+ *      and "Weigh the gap reduction against the configuration"): at most two
+ *      nonzeros in every aligned run of eight weights along d_in, kept by the
+ *      same hard-thresholding rule (largest magnitude keys, ties to the lower
+ *      index).  Packed densely: two values per group of eight in ascending
+ *      index order, and one metadata byte per group, idx0 | idx1 << 3.  Every
+ *      2:8 matrix is also a 2:4 matrix (each half-group of four holds at most
+ *      two nonzeros), so the forward of a 2:8 layer is the forward of its
+ *      2:4 packing (oracle_pack_2to4 of the unpacked matrix).
+ *
  *   2. The forward pass.  LoSparse (arXiv 2306.11222), section 3 and
  *      section 3.2: the compressed layer replaces X*W by the sum of a sparse
  *      term and a low-rank term, run in parallel.  In the d_out x d_in
@@ -183,6 +194,60 @@ int oracle_pack_2to4_scaled(const uint16_t *W, int64_t d_out, int64_t d_in, int6
             vals[i * (d_in / 2) + 2 * g + 1] = w[b];
             unsigned nib = (unsigned)a | ((unsigned)b << 2);
             meta[i * mrow + g / 2] |= (uint8_t)(nib << (4 * (g % 2)));
+        }
+    }
+    return 0;
+}
+
+/* 2:8 projection and packing.
+ *   W    : d_out rows, row stride ldw elements (ldw >= d_in), bf16 bits.
+ *   vals : d_out x (d_in/4) bf16 bits: the two kept values of group g (columns
+ *          8g..8g+7) at 2g, 2g+1, lower index first.
+ *   meta : d_out x (d_in/8) bytes: byte g = idx0 | idx1 << 3, idx0 < idx1.
+ * The two kept positions of a group are those whose magnitude key (bf16 bits
+ * without the sign) is beaten by fewer than two others, where q beats p when
+ * its key is larger, or equal with q < p.
+ * Returns 0, or -1 when d_in is not a multiple of 8 or ldw < d_in. */
+int oracle_pack_2to8(const uint16_t *W, int64_t d_out, int64_t d_in, int64_t ldw,
+                     uint16_t *vals, uint8_t *meta)
+{
+    if (d_in % 8 != 0 || ldw < d_in || d_out < 0) return -1;
+    int64_t groups = d_in / 8;
+    for (int64_t i = 0; i < d_out; ++i) {
+        for (int64_t g = 0; g < groups; ++g) {
+            const uint16_t *w = W + i * ldw + 8 * g;
+            int kept[2];
+            int n = 0;
+            for (int p = 0; p < 8; ++p) {
+                unsigned kp = w[p] & 0x7FFFu;
+                int beaten = 0;
+                for (int q = 0; q < 8; ++q) {
+                    unsigned kq = w[q] & 0x7FFFu;
+                    if (kq > kp || (kq == kp && q < p)) ++beaten;
+                }
+                if (beaten < 2) kept[n++] = p;
+            }
+            vals[i * (d_in / 4) + 2 * g + 0] = w[kept[0]];
+            vals[i * (d_in / 4) + 2 * g + 1] = w[kept[1]];
+            meta[i * groups + g] = (uint8_t)(kept[0] | (kept[1] << 3));
+        }
+    }
+    return 0;
+}
+
+/* Expand a 2:8 packing back to the dense d_out x d_in matrix (+0.0 at the
+ * positions that were not kept). */
+int oracle_unpack_2to8(const uint16_t *vals, const uint8_t *meta, int64_t d_out, int64_t d_in, uint16_t *S)
+{
+    if (d_in % 8 != 0 || d_out < 0) return -1;
+    int64_t groups = d_in / 8;
+    for (int64_t i = 0; i < d_out; ++i) {
+        for (int64_t j = 0; j < d_in; ++j) S[i * d_in + j] = 0;
+        for (int64_t g = 0; g < groups; ++g) {
+            unsigned byte = meta[i * groups + g];
+            int a = (int)(byte & 7u), b = (int)((byte >> 3) & 7u);
+            S[i * d_in + 8 * g + a] = vals[i * (d_in / 4) + 2 * g + 0];
+            S[i * d_in + 8 * g + b] = vals[i * (d_in / 4) + 2 * g + 1];
         }
     }
     return 0;

@@ -412,6 +412,109 @@ def pin_column_norms(o):
     assert o.column_norms(np.zeros((0, 5), dtype=np.uint16)).tolist() == [0.0] * 5
 
 
+# --------------------------------------------------------------------------- 2:8 pins
+#
+# The 2:8 projection keeps the two largest magnitudes of each aligned group of
+# eight (ties to the lower index); a 2:8 matrix is also a 2:4 matrix.
+
+_PAIRS8 = list(itertools.combinations(range(8), 2))
+
+
+def brute_force_pairs8(absg: np.ndarray) -> np.ndarray:
+    """For each row of ``absg`` [G, 8], the lexicographically first pair (a, b)
+    whose kept magnitudes are all >= every dropped one (enumeration of the 28
+    pairs, vectorised over the groups).  Returns [G, 2]."""
+    G = absg.shape[0]
+    best = np.full((G, 2), -1, dtype=np.int64)
+    for a, b in _PAIRS8:
+        dropped = np.delete(absg, [a, b], axis=1).max(axis=1)
+        ok = (np.minimum(absg[:, a], absg[:, b]) >= dropped) & (best[:, 0] < 0)
+        best[ok] = (a, b)
+    assert np.all(best >= 0)
+    return best
+
+
+def _check_pack28(W, vals, meta):
+    d_out, d_in = W.shape
+    G = d_in // 8
+    absg = np.abs(_f64(W)).reshape(d_out * G, 8)
+    want = brute_force_pairs8(absg)
+    got = np.stack([meta.reshape(-1) & 7, meta.reshape(-1) >> 3], axis=1).astype(np.int64)
+    np.testing.assert_array_equal(got, want)
+    Wg = W.reshape(d_out * G, 8)
+    idx = np.arange(d_out * G)
+    np.testing.assert_array_equal(vals.reshape(-1, 2)[:, 0], Wg[idx, want[:, 0]])
+    np.testing.assert_array_equal(vals.reshape(-1, 2)[:, 1], Wg[idx, want[:, 1]])
+
+
+def pin_pack28_exhaustive_alphabet(o):
+    """Every group of eight over {+0, -1, 1, 2} (4^8 groups, many ties)."""
+    alpha = _bf16([0.0, -1.0, 1.0, 2.0])
+    groups = np.array(list(itertools.product(range(4), repeat=8)), dtype=np.int64)
+    W = alpha[groups].reshape(-1, 64)               # eight groups per row
+    vals, meta = o.pack_2to8(W)
+    _check_pack28(W, vals, meta)
+
+
+def pin_pack28_random_bruteforce(o, seed: int = 61):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    sign = rng.integers(0, 2, size=(200, 48)).astype(np.uint16) << 15
+    expo = rng.integers(125, 129, size=(200, 48)).astype(np.uint16) << 7
+    mant = rng.integers(0, 4, size=(200, 48)).astype(np.uint16) << 5
+    W = (sign | expo | mant).astype(np.uint16)
+    vals, meta = o.pack_2to8(W)
+    _check_pack28(W, vals, meta)
+    Wg = synth.gaussian_bf16((64, 256), 0.02, seed)
+    v2, m2 = o.pack_2to8(Wg)
+    _check_pack28(Wg, v2, m2)
+
+
+def pin_pack28_hand_and_specials(o):
+    """Worked by hand: |1 5 3 -7 2 0 6 4| keeps -7 (3) and 6 (6); all zeros keep
+    positions 0 and 1; NaN above Inf above finite; equal magnitudes of either
+    sign tie and go to the lower index."""
+    W = np.concatenate([_bf16([[1, 5, 3, -7, 2, 0, 6, 4, 0, 0, 0, 0, 0, 0, 0, 0]]),
+                        np.array([[0x3F80, 0x7F80, 0x4000, 0x7FC0, 0, 0, 0, 0,
+                                   0xBF80, 0x3F80, 0x3F80, 0xBF80, 0x3F80, 0, 0, 0]], dtype=np.uint16)], axis=1)
+    vals, meta = o.pack_2to8(W)
+    np.testing.assert_array_equal(meta, [[3 | 6 << 3, 0 | 1 << 3, 1 | 3 << 3, 0 | 1 << 3]])
+    np.testing.assert_array_equal(vals, np.concatenate([_bf16([[-7, 6, 0, 0]]),
+                                                       [[0x7F80, 0x7FC0, 0xBF80, 0x3F80]]], axis=1))
+
+
+def pin_pack28_is_2to4(o):
+    """A 2:8 matrix packs losslessly as 2:4, and the kept positions of each
+    group of eight are among the 2:4 choices of their half-groups."""
+    W = synth.gaussian_bf16((48, 192), 0.02, 62)
+    v8, m8 = o.pack_2to8(W)
+    S8 = o.unpack_2to8(v8, m8, 192)
+    assert np.all(np.count_nonzero(S8.reshape(48, -1, 4) & 0x7FFF, axis=2) <= 2)
+    v4, m4 = o.as_2to4(v8, m8, 192)
+    np.testing.assert_array_equal(o.unpack_2to4(v4, m4, 192), S8)
+    _, mw = o.pack_2to4(W)
+    for i in range(48):
+        pairs4 = decode_meta(mw[i], 48)
+        for g in range(24):
+            a, b = int(m8[i, g]) & 7, int(m8[i, g]) >> 3
+            for p in (a, b):
+                assert p % 4 in pairs4[2 * g + p // 4], (i, g, p)
+    # Idempotent on its own output.
+    v8b, m8b = o.pack_2to8(S8)
+    np.testing.assert_array_equal(v8b, v8)
+    np.testing.assert_array_equal(m8b, m8)
+
+
+def pin_forward_2to8_identity(o):
+    """X S8^T + (X V^T) U^T with small integers, exactly, through the 2:4 packing."""
+    X, W, U, V = _small_int_problem(63, 6, 10, 32, 3)
+    v8, m8 = o.pack_2to8(W)
+    S = _f64(o.unpack_2to8(v8, m8, 32))
+    Xf = _f64(X)
+    Y, B = o.forward_2to8(X, v8, m8, U, V)
+    np.testing.assert_array_equal(Y, Xf @ S.T + (Xf @ _f64(V).T) @ _f64(U).T)
+    np.testing.assert_array_equal(B, np.abs(Xf) @ np.abs(S + _f64(U) @ _f64(V)).T)
+
+
 ALL_PINS = [
     pin_pack_golden, pin_pack_exhaustive_alphabet, pin_pack_random_bruteforce,
     pin_pack_invariants, pin_pack_roundtrip, pin_pack_specials, pin_pack_odd_groups,
@@ -419,4 +522,6 @@ ALL_PINS = [
     pin_forward_sparse_only, pin_forward_row_subset, pin_lowrank_project,
     pin_scaled_uniform_equals_unscaled, pin_scaled_bruteforce_exact, pin_scaled_minimises_weighted_error,
     pin_scaled_hand_examples, pin_scaled_specials, pin_scaled_group_locality, pin_column_norms,
+    pin_pack28_exhaustive_alphabet, pin_pack28_random_bruteforce, pin_pack28_hand_and_specials,
+    pin_pack28_is_2to4, pin_forward_2to8_identity,
 ]

@@ -31,8 +31,8 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "slr_oracle.c")
 
 # (name, text to replace, replacement, expected number of occurrences)
 MUTANTS = [
-    ("tie_to_higher_index", "(kq == kp && q < p)", "(kq == kp && q > p)", 1),
-    ("signed_key", " & 0x7FFFu;", ";", 2),
+    ("tie_to_higher_index", "(kq == kp && q < p)", "(kq == kp && q > p)", 2),
+    ("signed_key", " & 0x7FFFu;", ";", 4),
     ("smallest_magnitude", "if (rank < 2) kept[n++] = p;", "if (rank >= 2) kept[n++] = p;", 2),
     ("kept_order_swapped", "*idx0 = kept[0];\n    *idx1 = kept[1];", "*idx0 = kept[1];\n    *idx1 = kept[0];", 2),
     ("nibble_fields_swapped", "(unsigned)a | ((unsigned)b << 2)", "(unsigned)b | ((unsigned)a << 2)", 2),
@@ -53,6 +53,10 @@ MUTANTS = [
      "key[p] = scaled_key(w[p], 1.0f);", 1),
     ("norm_no_sqrt", "out[j] = sqrt(acc);", "out[j] = acc;", 1),
     ("norm_abs_sum", "acc += x * x;", "acc += fabs(x);", 1),
+    ("pack28_meta_shift", "(uint8_t)(kept[0] | (kept[1] << 3))", "(uint8_t)(kept[0] | (kept[1] << 2))", 1),
+    ("pack28_vals_swapped", "vals[i * (d_in / 4) + 2 * g + 0] = w[kept[0]];", "vals[i * (d_in / 4) + 2 * g + 0] = w[kept[1]];", 1),
+    ("pack28_group_stride", "const uint16_t *w = W + i * ldw + 8 * g;", "const uint16_t *w = W + i * ldw + 4 * g;", 1),
+    ("unpack28_meta_field", "(int)((byte >> 3) & 7u)", "(int)((byte >> 4) & 7u)", 1),
     ("norm_wrong_column", "double x = bf16_bits_to_double(X[m * d_in + j]);",
      "double x = bf16_bits_to_double(X[m * d_in]);", 1),
 ]
