@@ -293,6 +293,8 @@ def run_ours(args, rank, world, dist):
 
     # ------------------------------------------------ pack leg
     pack = run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier) if "pack" in legs else None
+    sparse28 = run_2to8_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier) \
+        if "2to8" in legs else None
     calibrate = run_calibrate_leg(args, slr, torch, dev, W, to_dev, peaks, max_over_ranks, barrier) \
         if "calibrate" in legs else None
     del W
@@ -320,6 +322,7 @@ def run_ours(args, rank, world, dist):
         **sweep,
         "pack": pack,
         "calibrate": calibrate,
+        "sparse_2to8": sparse28,
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": 2 * K,
@@ -585,6 +588,54 @@ def run_decode_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier
             "l2": f"rotating {n_copies} buffer sets of {nbytes / 1e6:.1f} MB"}
 
 
+def run_2to8_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier):
+    """2:8 + rank-64 decode (the 3BASiL summary page's 2:8 configuration) on
+    the Llama-3-70B MLP up projection: the dense 2:8 packing through the 2:8
+    streaming forward, against the 2:4 packing of the same matrix through
+    slr_forward.  GB/s counts X + vals8 + meta8 + U + V + Y."""
+    L = layer_of(5, "up_proj_70b_r64")
+    d_out, d_in, r = L.d_out, L.d_in, L.r
+    W = to_dev(L.weight())
+    v8, m8, v4, m4 = slr.pack_2to8(W)
+    del W
+    Uh, Vh = L.factors()
+    U, V = to_dev(Uh), to_dev(Vh)
+    copies28 = [(v8, m8), (v8.clone(), m8.clone())]      # 2 x 147 MB > L2
+    copies24 = [(v4, m4), (v4.clone(), m4.clone())]      # 2 x 264 MB
+    K = max(50, 10 * args.steps)
+    res = {"workload": f"Llama-3-70B MLP up projection {d_out}x{d_in}, 2:8 sparse + rank {r}, decode",
+           "unit": "GB/s"}
+    for M in (1, 2):
+        Xh = L.activations(M)
+        X = to_dev(Xh)
+        Y = torch.empty((M, d_out), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(slr.workspace_size(M, d_out, d_in, r), 256), dtype=torch.uint8, device=dev)
+        bytes28 = 2 * M * d_in + d_out * d_in * 5 // 8 + 2 * r * (d_out + d_in) + 2 * M * d_out
+
+        def f28(k):
+            a, b = copies28[k % 2]
+            slr.forward_2to8(X, a, b, U, V, out=Y, workspace=ws)
+
+        def f24(k):
+            a, b = copies24[k % 2]
+            slr.forward(X, a, b, U, V, out=Y, workspace=ws)
+
+        for i in range(max(args.warmup, 5)):
+            f28(i)
+            f24(i)
+        slr.check_kernel_error()
+        barrier()
+        ms28 = max_over_ranks(graph_time_ms(torch, [lambda k=k: f28(k) for k in range(K)])) / K
+        ms24 = max_over_ranks(graph_time_ms(torch, [lambda k=k: f24(k) for k in range(K)])) / K
+        gbs = bytes28 / (ms28 * 1e-3) / 1e9
+        res[f"M{M}"] = {"value": round(gbs, 1), "ms_per_step": round(ms28, 5), "algorithmic_bytes": bytes28,
+                        "frac": round(gbs / peaks["hbm_gbs"], 4),
+                        "ms_2to4_packing_same_matrix": round(ms24, 5), "speedup_vs_2to4": round(ms24 / ms28, 3),
+                        "path_2to4": slr.select_path(M, d_out, d_in, r)}
+    del copies28, copies24
+    return res
+
+
 def run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier):
     d_out, d_in = W.shape
     nbytes = d_out * d_in * 2 + d_out * d_in + d_out * d_in // 8   # read W, write vals + meta
@@ -727,7 +778,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024, help="token rows in the oracle CPU baseline sample")
     ap.add_argument("--ref-rows", type=int, default=64, help="token rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="prefill,e2e,decode,pack,calibrate,cpu,cfg2,cfg4,cfg5",
+    ap.add_argument("--only", default="prefill,e2e,decode,pack,calibrate,2to8,cpu,cfg2,cfg4,cfg5",
                     help="comma list of legs to run (profiling runs use one leg)")
     args = ap.parse_args()
     if args.warmup < 3:

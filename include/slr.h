@@ -149,6 +149,54 @@ SLR_API slr_status slr_column_norms(const void *X, int64_t M, int64_t d_in, int6
 SLR_API size_t slr_column_norms_workspace_size(int64_t M, int64_t d_in);
 
 /* --------------------------------------------------------------------------
+ * 2:8 projection and packing.
+ *
+ * The 2:8 configuration (3BASiL summary page, "Faster compression and gains
+ * that survive LoRA": 2:8 sparse plus rank 64): at most two nonzeros in every
+ * aligned run of eight weights along d_in, chosen by the same rule as
+ * slr_pack_2to4 (largest magnitude bits, ties to the lower index, exactly two
+ * positions kept per group).  One pass over W writes either or both of:
+ *
+ *   vals8  device, bf16 [d_out, d_in/4]: the two kept values of group g
+ *          (columns 8g..8g+7) at 2g, 2g+1, lower index first.  4-byte aligned.
+ *   meta8  device, uint8 [d_out, d_in/8]: byte g = idx0 | idx1 << 3.
+ *   vals4, meta4  the slr_pack_2to4 format of the projected matrix (positions
+ *          not kept hold +0), bit-identical to slr_pack_2to4 applied to it;
+ *          for slr_forward.  vals4 8-byte aligned.
+ *
+ * Pass NULL for both members of a pair to skip it (not both pairs).
+ * Requirements: d_out >= 0, d_in >= 0, d_in % 8 == 0, ldw >= d_in; W any
+ * alignment (16-byte aligned W with ldw % 8 == 0 takes the vectorised path).
+ * Bit-exact and deterministic.
+ * ------------------------------------------------------------------------ */
+SLR_API slr_status slr_pack_2to8(const void *W, int64_t d_out, int64_t d_in, int64_t ldw, void *vals8,
+                         void *meta8, void *vals4, void *meta4, slr_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Forward pass of a 2:8-packed layer (small M).
+ *
+ * Y = X * S^T + (X * V^T) * U^T with S in the dense 2:8 packing of
+ * slr_pack_2to8 (vals8, meta8): 0.625 B per weight instead of 1.125 B, so the
+ * byte-bound decode of one or two tokens moves ~45% fewer bytes than
+ * slr_forward on the 2:4 packing.  CUDA cores, one streaming kernel after the
+ * rank projection T = X V^T (fp32).  For many tokens use slr_forward on the
+ * 2:4 packing of the same matrix (vals4, meta4), which runs on the tensor
+ * cores.
+ *
+ * Arguments as slr_forward, with vals8 [d_out, d_in/4] and meta8
+ * [d_out, d_in/8]; workspace of at least slr_forward_workspace_size(M, d_out,
+ * d_in, r) bytes.  Arithmetic: fp32 products and sums (T in fp32), one bf16
+ * rounding of Y; same accuracy contract as slr_forward.
+ *
+ * Requirements: 0 <= M < 2^18 (M == 0 returns SLR_OK), d_out >= 1, d_in >= 32
+ * with d_in % 32 == 0, r >= 0 with r % 8 == 0, d_out, d_in < 2^31, all
+ * pointers 16-byte aligned (workspace 256-byte aligned).
+ * ------------------------------------------------------------------------ */
+SLR_API slr_status slr_forward_2to8(const void *X, int64_t M, const void *vals8, const void *meta8,
+                            int64_t d_out, int64_t d_in, const void *U, const void *V, int64_t r,
+                            void *Y, void *workspace, size_t workspace_bytes, slr_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * Forward pass  Y = X * S^T + (X * V^T) * U^T.
  *
  * LoSparse, section 3.2: the compressed layer computes the low-rank and sparse

@@ -10,6 +10,8 @@ Functions mirror the C ABI in ``include/slr.h``:
 * ``pack_2to4(W) -> (vals, meta)``  -- ``slr_pack_2to4``
 * ``pack_2to4_scaled(W, scale) -> (vals, meta)``  -- ``slr_pack_2to4_scaled``
 * ``column_norms(X, sumsq=None) -> (norms, sumsq)``  -- ``slr_column_norms``
+* ``pack_2to8(W, dense=True, as_2to4=True)``  -- ``slr_pack_2to8``
+* ``forward_2to8(X, vals8, meta8, U, V) -> Y``  -- ``slr_forward_2to8``
 * ``forward(X, vals, meta, U, V) -> Y``  -- ``slr_forward`` /
   ``slr_forward_with_path``
 * ``workspace_size``, ``select_path``, ``check_kernel_error``
@@ -57,6 +59,10 @@ def _load() -> ctypes.CDLL:
     lib.slr_meta_row_bytes.argtypes = [i64]
     lib.slr_pack_2to4_scaled.restype = st
     lib.slr_pack_2to4_scaled.argtypes = [p, i64, i64, i64, p, p, p, p]
+    lib.slr_pack_2to8.restype = st
+    lib.slr_pack_2to8.argtypes = [p, i64, i64, i64, p, p, p, p, p]
+    lib.slr_forward_2to8.restype = st
+    lib.slr_forward_2to8.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, p, sz, p]
     lib.slr_column_norms.restype = st
     lib.slr_column_norms.argtypes = [p, i64, i64, i64, p, p, p, sz, p]
     lib.slr_column_norms_workspace_size.restype = sz
@@ -159,6 +165,41 @@ def column_norms(X: torch.Tensor, sumsq: torch.Tensor | None = None, *, want_nor
     _check(_lib.slr_column_norms(_ptr(X), M, d_in, ldx, _ptr(sumsq), _ptr(norms), _ptr(workspace),
                                  workspace.numel(), _stream()), "slr_column_norms")
     return norms, sumsq
+
+
+def pack_2to8(W: torch.Tensor, *, dense: bool = True, as_2to4: bool = True):
+    """2:8 projection of bf16 ``W`` [d_out, d_in]: returns ``(vals8, meta8,
+    vals4, meta4)``, the dense 2:8 packing and the 2:4 packing of the same
+    projected matrix (an unrequested pair is ``None``)."""
+    if W.dtype != torch.bfloat16 or W.dim() != 2 or not W.is_cuda or W.stride(1) != 1:
+        raise ValueError("W must be a 2-D CUDA bf16 tensor with unit column stride")
+    d_out, d_in = W.shape
+    dev = W.device
+    vals8 = torch.empty((d_out, d_in // 4), dtype=torch.bfloat16, device=dev) if dense else None
+    meta8 = torch.empty((d_out, d_in // 8), dtype=torch.uint8, device=dev) if dense else None
+    vals4 = torch.empty((d_out, d_in // 2), dtype=torch.bfloat16, device=dev) if as_2to4 else None
+    meta4 = torch.empty((d_out, meta_row_bytes(d_in)), dtype=torch.uint8, device=dev) if as_2to4 else None
+    _check(_lib.slr_pack_2to8(_ptr(W), d_out, d_in, W.stride(0), _ptr(vals8), _ptr(meta8), _ptr(vals4),
+                              _ptr(meta4), _stream()), "slr_pack_2to8")
+    return vals8, meta8, vals4, meta4
+
+
+def forward_2to8(X: torch.Tensor, vals8: torch.Tensor, meta8: torch.Tensor, U: torch.Tensor | None,
+                 V: torch.Tensor | None, *, out: torch.Tensor | None = None,
+                 workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """``Y = X @ S.T + (X @ V.T) @ U.T`` with S in the dense 2:8 packing."""
+    M, d_in = X.shape
+    d_out = vals8.shape[0]
+    r = 0 if U is None else U.shape[1]
+    if out is None:
+        out = torch.empty((M, d_out), dtype=torch.bfloat16, device=X.device)
+    need = workspace_size(M, d_out, d_in, r)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.slr_forward_2to8(_ptr(X), M, _ptr(vals8), _ptr(meta8), d_out, d_in, _ptr(U), _ptr(V), r,
+                                 _ptr(out), _ptr(workspace), ws_bytes, _stream()), "slr_forward_2to8")
+    return out
 
 
 def workspace_size(M: int, d_out: int, d_in: int, r: int) -> int:

@@ -175,6 +175,56 @@ slr_status slr_pack_2to4_scaled(const void *W, int64_t d_out, int64_t d_in, int6
     return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
 }
 
+slr_status slr_pack_2to8(const void *W, int64_t d_out, int64_t d_in, int64_t ldw, void *vals8, void *meta8,
+                         void *vals4, void *meta4, slr_stream_t stream) {
+    if (d_out < 0 || d_in < 0 || d_in % 8 != 0 || ldw < d_in) return SLR_ERR_SHAPE;
+    if ((vals8 == nullptr) != (meta8 == nullptr) || (vals4 == nullptr) != (meta4 == nullptr) ||
+        (vals8 == nullptr && vals4 == nullptr))
+        return SLR_ERR_NULL;
+    if (d_out == 0 || d_in == 0) return SLR_OK;
+    if (W == nullptr) return SLR_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(vals8) & 3) != 0 || (reinterpret_cast<uintptr_t>(vals4) & 7) != 0)
+        return SLR_ERR_ALIGN;
+    const slr_status dev = slr::check_device();
+    if (dev != SLR_OK) return dev;
+    const cudaError_t err = slr::launch_pack_2to8(
+        static_cast<const uint16_t *>(W), d_out, d_in, ldw, static_cast<uint16_t *>(vals8),
+        static_cast<uint8_t *>(meta8), static_cast<uint16_t *>(vals4), static_cast<uint8_t *>(meta4),
+        reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
+}
+
+slr_status slr_forward_2to8(const void *X, int64_t M, const void *vals8, const void *meta8, int64_t d_out,
+                            int64_t d_in, const void *U, const void *V, int64_t r, void *Y, void *workspace,
+                            size_t workspace_bytes, slr_stream_t stream) {
+    if (M < 0 || d_out < 0 || d_in < 0 || r < 0) return SLR_ERR_SHAPE;
+    if (M == 0) return SLR_OK;
+    const size_t need = slr::workspace_bytes_for(M, r, SLR_PATH_DECODE);
+    if (X == nullptr || vals8 == nullptr || meta8 == nullptr || Y == nullptr) return SLR_ERR_NULL;
+    if (r > 0 && (U == nullptr || V == nullptr)) return SLR_ERR_NULL;
+    if (need > 0 && workspace == nullptr) return SLR_ERR_NULL;
+    if (d_out < 1 || d_in < 32 || d_in % 32 != 0 || r % 8 != 0) return SLR_ERR_SHAPE;
+    if (M >= (int64_t(1) << 18) || d_out > INT32_MAX || d_in > INT32_MAX) return SLR_ERR_SHAPE;
+    if (!slr::aligned16(X) || !slr::aligned16(vals8) || !slr::aligned16(meta8) || !slr::aligned16(Y))
+        return SLR_ERR_ALIGN;
+    if (r > 0 && (!slr::aligned16(U) || !slr::aligned16(V))) return SLR_ERR_ALIGN;
+    if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) % slr::kAlign) != 0) return SLR_ERR_ALIGN;
+    if (workspace_bytes < need) return SLR_ERR_WORKSPACE;
+    const slr_status dev = slr::check_device();
+    if (dev != SLR_OK) return dev;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const uint16_t *x = static_cast<const uint16_t *>(X);
+    float *T32 = r > 0 ? static_cast<float *>(workspace) : nullptr;
+    cudaError_t err = cudaSuccess;
+    if (r > 0) err = slr::launch_lowrank_project(x, M, static_cast<const uint16_t *>(V), d_in, r, T32, nullptr, st);
+    if (err == cudaSuccess)
+        err = slr::launch_decode28_forward(x, M, static_cast<const uint16_t *>(vals8),
+                                           static_cast<const uint8_t *>(meta8), d_out, d_in,
+                                           static_cast<const uint16_t *>(U), T32, r, static_cast<uint16_t *>(Y),
+                                           r > 0, st);
+    return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
+}
+
 size_t slr_column_norms_workspace_size(int64_t M, int64_t d_in) {
     if (M <= 0 || d_in <= 0 || d_in % 8 != 0) return 0;
     const slr::NormPlan p = slr::column_norms_plan(M, d_in);

@@ -41,6 +41,18 @@ cudaError_t launch_pack_2to4(const uint16_t *W, int64_t d_out, int64_t d_in, int
 cudaError_t launch_pack_2to4_scaled(const uint16_t *W, int64_t d_out, int64_t d_in, int64_t ldw,
                                     const float *scale, uint16_t *vals, uint8_t *meta, cudaStream_t stream);
 
+// 2:8 projection; any of the two output pairs may be null (both members of a
+// pair together).  vals8 4-byte aligned, vals4 8-byte aligned; d_in % 8 == 0.
+cudaError_t launch_pack_2to8(const uint16_t *W, int64_t d_out, int64_t d_in, int64_t ldw, uint16_t *vals8,
+                             uint8_t *meta8, uint16_t *vals4, uint8_t *meta4, cudaStream_t stream);
+
+// Small-M streaming forward of a 2:8-packed layer: Y = X S^T + T U^T, T fp32
+// [M, r] precomputed (after_projection as for launch_decode_forward).
+// d_in % 32 == 0, all pointers 16-byte aligned.
+cudaError_t launch_decode28_forward(const uint16_t *X, int64_t M, const uint16_t *vals8, const uint8_t *meta8,
+                                    int64_t d_out, int64_t d_in, const uint16_t *U, const float *T32, int64_t r,
+                                    uint16_t *Y, bool after_projection, cudaStream_t stream);
+
 // Row split of the column-norm reduction: `splits` row ranges of
 // `rows_per_split` rows, each leaving d_in fp32 partial sums in the workspace.
 struct NormPlan {

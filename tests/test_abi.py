@@ -160,3 +160,34 @@ def test_column_norms_argument_errors_and_workspace():
     assert ws(2048, 4096) == 32 * 4096 * 4
     # Very tall batches cap a split at 512 rows.
     assert ws(1 << 20, 4096) == (1 << 20) // 512 * 4096 * 4
+
+
+def test_pack_2to8_argument_errors():
+    f = slr.lib().slr_pack_2to8
+    a, b, c, d = P(0x2000), P(0x3000), P(0x4000), P(0x5000)
+    assert f(P(0x1000), 4, 12, 12, a, b, c, d, None) == SHAPE          # d_in % 8
+    assert f(P(0x1000), 4, 16, 8, a, b, c, d, None) == SHAPE           # ldw < d_in
+    assert f(P(0x1000), 4, 16, 16, a, P(0), c, d, None) == NULL        # half a pair
+    assert f(P(0x1000), 4, 16, 16, P(0), P(0), P(0), P(0), None) == NULL  # no output
+    assert f(P(0), 4, 16, 16, a, b, None, None, None) == NULL          # W
+    assert f(P(0x1000), 4, 16, 16, P(0x2002), b, None, None, None) == ALIGN   # vals8 4 B
+    assert f(P(0x1000), 4, 16, 16, None, None, P(0x4004), d, None) == ALIGN   # vals4 8 B
+    assert f(P(0), 0, 16, 16, a, b, None, None, None) == OK            # empty
+    if not torch.cuda.is_available():
+        assert f(P(0x1000), 4, 16, 16, a, b, c, d, None) == DEVICE
+
+
+def test_forward_2to8_argument_errors():
+    f = slr.lib().slr_forward_2to8
+    x, v, m, u, vv, y, ws = (P(0x10000 * k) for k in range(1, 8))
+    assert f(x, 0, None, None, 8, 64, None, None, 0, None, None, 0, None) == OK        # M == 0
+    assert f(x, 1, v, m, 8, 48, u, vv, 8, y, ws, 1 << 20, None) == SHAPE               # d_in % 32
+    assert f(x, 1, v, m, 8, 64, u, vv, 4, y, ws, 1 << 20, None) == SHAPE               # r % 8
+    assert f(x, 1 << 18, v, m, 8, 64, u, vv, 8, y, ws, 1 << 30, None) == SHAPE         # M too large
+    assert f(x, 1, P(0), m, 8, 64, u, vv, 8, y, ws, 1 << 20, None) == NULL
+    assert f(x, 1, v, m, 8, 64, P(0), vv, 8, y, ws, 1 << 20, None) == NULL             # U with r > 0
+    assert f(P(0x10008), 1, v, m, 8, 64, u, vv, 8, y, ws, 1 << 20, None) == ALIGN
+    assert f(x, 2, v, m, 8, 64, u, vv, 8, y, ws, 16, None) == WORKSPACE
+    if not torch.cuda.is_available():
+        assert f(x, 1, v, m, 8, 64, u, vv, 8, y, ws, 1 << 20, None) == DEVICE
+        assert f(x, 1, v, m, 8, 64, None, None, 0, y, None, 0, None) == DEVICE        # r == 0: no factors
