@@ -266,9 +266,10 @@ slr_path slr_forward_select_path(int64_t M, int64_t d_out, int64_t d_in, int64_t
 slr_status slr_check_kernel_error(void) {
     if (slr::check_device() != SLR_OK) return SLR_ERR_DEVICE;
     if (cudaDeviceSynchronize() != cudaSuccess) return SLR_ERR_CUDA;
-    unsigned code = 0;
+    unsigned code = 0, code28 = 0;
     if (slr::read_and_clear_kernel_error(&code) != cudaSuccess) return SLR_ERR_CUDA;
-    return code ? SLR_ERR_TIMEOUT : SLR_OK;
+    if (slr::read_and_clear_decode28_error(&code28) != cudaSuccess) return SLR_ERR_CUDA;
+    return (code | code28) ? SLR_ERR_TIMEOUT : SLR_OK;
 }
 
 slr_status slr_selftest_wait_timeout(int64_t limit_cycles, slr_stream_t stream) {

@@ -53,6 +53,9 @@ cudaError_t launch_decode28_forward(const uint16_t *X, int64_t M, const uint16_t
                                     int64_t d_out, int64_t d_in, const uint16_t *U, const float *T32, int64_t r,
                                     uint16_t *Y, bool after_projection, cudaStream_t stream);
 
+// Reads and clears the error word of the 2:8 ring kernel's bounded waits.
+cudaError_t read_and_clear_decode28_error(unsigned *code);
+
 // Row split of the column-norm reduction: `splits` row ranges of
 // `rows_per_split` rows, each leaving d_in fp32 partial sums in the workspace.
 struct NormPlan {

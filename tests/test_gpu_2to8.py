@@ -111,11 +111,14 @@ def test_forward_2to8(cfg, name, M):
     _forward_case(_layer(cfg, name), M, seed=M * 31 + cfg)
 
 
+@pytest.mark.parametrize("kernel", ["ring", "regs"])
 @pytest.mark.parametrize("rw", ["1", "2", "4"])
-def test_forward_2to8_rows_per_warp_variants(rw, monkeypatch):
-    """Every rows-per-warp instantiation on a shape with a ragged last group
-    (d_out = 4100 rows is not a multiple of 4) and both token blocks."""
+def test_forward_2to8_rows_per_warp_variants(kernel, rw, monkeypatch):
+    """Both kernels (shared-memory ring, registers), every rows-per-thread
+    instantiation, on a shape with a ragged last row block (d_out = 4100) and
+    every token-block size."""
     monkeypatch.setenv("SLR_DECODE28_RW", rw)
+    monkeypatch.setenv("SLR_DECODE28_KERNEL", kernel)
     d_out, d_in, r = 4100, 1024, 64
     W = synth.gaussian_bf16((d_out, d_in), 0.02, 71)
     U = synth.gaussian_bf16((d_out, r), 0.5, 72)
@@ -130,8 +133,10 @@ def test_forward_2to8_rows_per_warp_variants(rw, monkeypatch):
 
 
 def test_forward_2to8_rank_variants_and_edges():
-    """r = 0 (sparse term alone, exact small integers), r = 128 (ranks past 64
-    take the loop), d_in = 32 (one chunk: most lanes idle), M = 0."""
+    """r = 0 (sparse term alone, exact small integers), r = 128 with 32 threads
+    per row slot (ranks past 64 take the loop), d_in = 32 (register kernel: one
+    chunk, most lanes idle), d_in = 1152 and 128 (ring, partial thread use),
+    d_in = 16640 (ring, five segments of 3328 columns), M = 0."""
     rng = np.random.Generator(np.random.PCG64(81))
     d_out, d_in = 96, 64
     Wi = synth.f32_to_bf16_bits(rng.integers(-4, 5, size=(d_out, d_in)).astype(np.float32))
@@ -141,7 +146,8 @@ def test_forward_2to8_rank_variants_and_edges():
     S = synth.bf16_bits_to_f32(oracle.unpack_2to8(v8, m8, d_in)).astype(np.float64)
     exact = synth.bf16_bits_to_f32(Xi).astype(np.float64) @ S.T      # integers, exact in fp32
     np.testing.assert_array_equal(from_dev(Y), synth.f32_to_bf16_bits(exact.astype(np.float32)))
-    for (d_out, d_in, r, M) in [(200, 256, 128, 2), (64, 32, 8, 1), (300, 32, 16, 4)]:
+    for (d_out, d_in, r, M) in [(200, 256, 128, 2), (64, 32, 8, 1), (300, 32, 16, 4), (300, 1152, 64, 3),
+                                (40, 128, 64, 1), (260, 16640, 64, 2)]:
         W = synth.gaussian_bf16((d_out, d_in), 0.05, d_out + d_in)
         U = synth.gaussian_bf16((d_out, r), 0.5, r + 1)
         V = synth.gaussian_bf16((r, d_in), 0.5 / np.sqrt(d_in), r + 2)
