@@ -7,3 +7,12 @@ from oracle_pins import ALL_PINS
 @pytest.mark.parametrize("pin", ALL_PINS, ids=[p.__name__ for p in ALL_PINS])
 def test_oracle_pin(pin, oracle_lib):
     pin(oracle_lib)
+
+
+from oracle_pins import AM_PINS  # noqa: E402
+
+
+@pytest.mark.parametrize("pin", AM_PINS, ids=[p.__name__ for p in AM_PINS])
+def test_oracle_am_pin(pin):
+    import oracle.datafree_am as am
+    pin(am)

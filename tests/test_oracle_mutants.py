@@ -5,6 +5,7 @@ import os
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 import oracle
@@ -74,3 +75,39 @@ def test_mutant_is_caught(name, old, new, count, tmp_path):
     caught = [l.split()[1] for l in proc.stdout.splitlines() if l.startswith("CAUGHT")]
     # A crash of the mutant also counts as detection, but say so.
     assert caught or proc.returncode != 0, f"no pin caught mutant {name}: {proc.stderr[-500:]}"
+
+
+# Planted mistakes in the alternating-minimisation oracle (numpy): each copy is
+# imported from a temporary file and must fail at least one AM pin.
+AM_SRC = os.path.join(os.path.dirname(oracle.__file__), "datafree_am.py")
+AM_MUTANTS = [
+    ("am_tie_to_higher", "            if q < p:\n", "            if q > p:\n", 1),
+    ("am_keep_three", "keep = (beaten < 2)", "keep = (beaten < 3)", 1),
+    ("am_truncation_one_more", "return (Uz[:, :r] * sz[:r]) @ Vz[:r, :]", "return (Uz[:, :r + 1] * sz[:r + 1]) @ Vz[:r + 1, :]", 1),
+    ("am_smallest_singular", "return (Uz[:, :r] * sz[:r]) @ Vz[:r, :]", "return (Uz[:, -r:] * sz[-r:]) @ Vz[-r:, :]", 1),
+    ("am_threshold_signed", "g = np.abs(R).reshape", "g = R.reshape", 1),
+    ("am_p2_uses_w", "L = truncated_svd(Wf - S, r)", "L = truncated_svd(Wf, r)", 1),
+    ("am_p1_ignores_l", "S = hard_threshold_2to4(Wf - L)\n        objs", "S = hard_threshold_2to4(Wf)\n        objs", 1),
+]
+
+
+@pytest.mark.parametrize("name,old,new,count", AM_MUTANTS, ids=[m[0] for m in AM_MUTANTS])
+def test_am_mutant_is_caught(name, old, new, count, tmp_path):
+    import importlib.util
+    import sys as _sys
+    _sys.path.insert(0, TESTS)
+    from oracle_pins import AM_PINS
+    text = open(AM_SRC).read()
+    assert text.count(old) == count, f"mutation site for {name} not found"
+    path = tmp_path / f"{name}.py"
+    path.write_text(text.replace(old, new))
+    spec = importlib.util.spec_from_file_location(f"am_{name}", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    caught = []
+    for pin in AM_PINS:
+        try:
+            pin(mod)
+        except (AssertionError, ValueError, IndexError, np.linalg.LinAlgError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught mutant {name}"
