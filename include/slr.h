@@ -197,6 +197,41 @@ SLR_API slr_status slr_forward_2to8(const void *X, int64_t M, const void *vals8,
                             void *Y, void *workspace, size_t workspace_bytes, slr_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * Data-free decomposition W ~ S + U V by alternating minimisation.
+ *
+ * HASSLE-free, section 4 (data-free variant: identity Hessian), started as in
+ * LoSparse, section 3.2 (the low-rank part from the top-r singular subspace
+ * of W).  After the start, each of `iters` iterations solves
+ *   P2: U V = C_r(W - S)   (rank-r truncated SVD, HASSLE-free section 4.2.1)
+ *   P1: S = 2:4 hard threshold of W - U V  (largest |.| of each group of four,
+ *       ties to the lower index; HASSLE-free section 4.1.1).
+ * C_r is computed by subspace iteration on W - S (power_first steps at the
+ * start, from the caller's random Q0, then `power` steps warm-started from the
+ * previous subspace, CholeskyQR2 orthonormalisation), in fp32.
+ *
+ *   W          device, bf16 [d_out, d_in], read only.
+ *   Q0         device, fp32 [d_in, r]: the random start (e.g. Gaussian).
+ *   vals, meta device: S in the slr_pack_2to4 format (values = W - U V at the
+ *              kept positions, rounded to bf16).
+ *   U          device, bf16 [d_out, r];  V  device, bf16 [r, d_in].
+ *   objective  device, fp64 [iters + 1], or NULL: ||W - S - U V||_F (fp32 U V,
+ *              unrounded S) after the start and after every iteration.
+ *   workspace  device scratch of slr_decompose_workspace_size() bytes.
+ *
+ * Requirements: d_out >= 1, d_in >= 8 with d_in % 8 == 0, 8 <= r <= 128 with
+ * r % 8 == 0 and r <= min(d_out, d_in), 0 <= iters <= 10000,
+ * 1 <= power_first, power <= 1000; all pointers 16-byte aligned (objective
+ * 8-byte aligned).  Deterministic for a given Q0.
+ * ------------------------------------------------------------------------ */
+SLR_API slr_status slr_decompose_datafree(const void *W, int64_t d_out, int64_t d_in, int64_t r, int iters,
+                                  int power_first, int power, const float *Q0, void *vals, void *meta,
+                                  void *U, void *V, double *objective, void *workspace,
+                                  size_t workspace_bytes, slr_stream_t stream);
+
+/* Scratch bytes of slr_decompose_datafree (about 4 * d_out * d_in + O((d_out + d_in) * r)). */
+SLR_API size_t slr_decompose_workspace_size(int64_t d_out, int64_t d_in, int64_t r);
+
+/* --------------------------------------------------------------------------
  * Forward pass  Y = X * S^T + (X * V^T) * U^T.
  *
  * LoSparse, section 3.2: the compressed layer computes the low-rank and sparse

@@ -12,6 +12,8 @@ Functions mirror the C ABI in ``include/slr.h``:
 * ``column_norms(X, sumsq=None) -> (norms, sumsq)``  -- ``slr_column_norms``
 * ``pack_2to8(W, dense=True, as_2to4=True)``  -- ``slr_pack_2to8``
 * ``forward_2to8(X, vals8, meta8, U, V) -> Y``  -- ``slr_forward_2to8``
+* ``decompose_datafree(W, r, iters, ...) -> (vals, meta, U, V, objective)``  --
+  ``slr_decompose_datafree``
 * ``forward(X, vals, meta, U, V) -> Y``  -- ``slr_forward`` /
   ``slr_forward_with_path``
 * ``workspace_size``, ``select_path``, ``check_kernel_error``
@@ -63,6 +65,11 @@ def _load() -> ctypes.CDLL:
     lib.slr_pack_2to8.argtypes = [p, i64, i64, i64, p, p, p, p, p]
     lib.slr_forward_2to8.restype = st
     lib.slr_forward_2to8.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, p, sz, p]
+    lib.slr_decompose_datafree.restype = st
+    lib.slr_decompose_datafree.argtypes = [p, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, p, p, p, p,
+                                           p, p, p, sz, p]
+    lib.slr_decompose_workspace_size.restype = sz
+    lib.slr_decompose_workspace_size.argtypes = [i64, i64, i64]
     lib.slr_column_norms.restype = st
     lib.slr_column_norms.argtypes = [p, i64, i64, i64, p, p, p, sz, p]
     lib.slr_column_norms_workspace_size.restype = sz
@@ -200,6 +207,33 @@ def forward_2to8(X: torch.Tensor, vals8: torch.Tensor, meta8: torch.Tensor, U: t
     _check(_lib.slr_forward_2to8(_ptr(X), M, _ptr(vals8), _ptr(meta8), d_out, d_in, _ptr(U), _ptr(V), r,
                                  _ptr(out), _ptr(workspace), ws_bytes, _stream()), "slr_forward_2to8")
     return out
+
+
+def decompose_datafree(W: torch.Tensor, r: int, iters: int, *, power_first: int = 8, power: int = 2,
+                       Q0: torch.Tensor | None = None, seed: int = 0):
+    """Data-free alternating minimisation W ~ S + U V (S 2:4, rank r): returns
+    ``(vals, meta, U, V, objective)`` with ``objective`` an fp64 CUDA tensor of
+    ``iters + 1`` values.  ``Q0`` (fp32 [d_in, r]) is the random start of the
+    subspace iteration; by default a standard normal one from ``seed``."""
+    if W.dtype != torch.bfloat16 or W.dim() != 2 or not W.is_cuda or not W.is_contiguous():
+        raise ValueError("W must be a contiguous 2-D CUDA bf16 tensor")
+    d_out, d_in = W.shape
+    dev = W.device
+    if Q0 is None:
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        Q0 = torch.randn((d_in, r), generator=g, device=dev, dtype=torch.float32)
+    vals = torch.empty((d_out, d_in // 2), dtype=torch.bfloat16, device=dev)
+    meta = torch.empty((d_out, meta_row_bytes(d_in)), dtype=torch.uint8, device=dev)
+    U = torch.empty((d_out, r), dtype=torch.bfloat16, device=dev)
+    V = torch.empty((r, d_in), dtype=torch.bfloat16, device=dev)
+    obj = torch.empty(iters + 1, dtype=torch.float64, device=dev)
+    need = int(_lib.slr_decompose_workspace_size(d_out, d_in, r))
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(_lib.slr_decompose_datafree(_ptr(W), d_out, d_in, r, iters, power_first, power, _ptr(Q0), _ptr(vals),
+                                       _ptr(meta), _ptr(U), _ptr(V), _ptr(obj), _ptr(ws), ws.numel(), _stream()),
+           "slr_decompose_datafree")
+    return vals, meta, U, V, obj
 
 
 def workspace_size(M: int, d_out: int, d_in: int, r: int) -> int:

@@ -225,6 +225,38 @@ slr_status slr_forward_2to8(const void *X, int64_t M, const void *vals8, const v
     return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
 }
 
+size_t slr_decompose_workspace_size(int64_t d_out, int64_t d_in, int64_t r) {
+    if (d_out < 1 || d_in < 8 || r < 8 || r > 128) return 0;
+    return (size_t)slr::am_plan(d_out, d_in, r).bytes;
+}
+
+slr_status slr_decompose_datafree(const void *W, int64_t d_out, int64_t d_in, int64_t r, int iters,
+                                  int power_first, int power, const float *Q0, void *vals, void *meta, void *U,
+                                  void *V, double *objective, void *workspace, size_t workspace_bytes,
+                                  slr_stream_t stream) {
+    if (d_out < 1 || d_in < 8 || d_in % 8 != 0 || r < 8 || r > 128 || r % 8 != 0 || r > d_out || r > d_in ||
+        d_out > INT32_MAX || d_in > INT32_MAX)
+        return SLR_ERR_SHAPE;
+    if (iters < 0 || iters > 10000 || power_first < 1 || power_first > 1000 || power < 1 || power > 1000)
+        return SLR_ERR_ARG;
+    if (W == nullptr || Q0 == nullptr || vals == nullptr || meta == nullptr || U == nullptr || V == nullptr ||
+        workspace == nullptr)
+        return SLR_ERR_NULL;
+    if (!slr::aligned16(W) || !slr::aligned16(Q0) || !slr::aligned16(vals) || !slr::aligned16(meta) ||
+        !slr::aligned16(U) || !slr::aligned16(V) || !slr::aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(objective) & 7) != 0)
+        return SLR_ERR_ALIGN;
+    if (workspace_bytes < slr_decompose_workspace_size(d_out, d_in, r)) return SLR_ERR_WORKSPACE;
+    const slr_status dev = slr::check_device();
+    if (dev != SLR_OK) return dev;
+    const cudaError_t err = slr::launch_am_datafree(
+        static_cast<const uint16_t *>(W), d_out, d_in, (int)r, iters, power_first, power, Q0,
+        static_cast<uint16_t *>(vals), static_cast<uint8_t *>(meta), static_cast<uint16_t *>(U),
+        static_cast<uint16_t *>(V), objective, static_cast<uint8_t *>(workspace),
+        reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
+}
+
 size_t slr_column_norms_workspace_size(int64_t M, int64_t d_in) {
     if (M <= 0 || d_in <= 0 || d_in % 8 != 0) return 0;
     const slr::NormPlan p = slr::column_norms_plan(M, d_in);

@@ -56,6 +56,22 @@ cudaError_t launch_decode28_forward(const uint16_t *X, int64_t M, const uint16_t
 // Reads and clears the error word of the 2:8 ring kernel's bounded waits.
 cudaError_t read_and_clear_decode28_error(unsigned *code);
 
+// Data-free alternating minimisation: workspace layout (byte offsets) and the
+// split counts of its products.
+struct AmPlan {
+    int64_t split_nn, split_tn, split_gram, split_mul;
+    int64_t tiles_res;
+    int64_t off_Z, off_Q, off_Q2, off_P, off_M, off_part, off_obj, bytes;
+};
+AmPlan am_plan(int64_t d_out, int64_t d_in, int64_t r);
+
+// W (bf16 d_out x d_in) -> packed 2:4 S (vals, meta), U (bf16 d_out x r),
+// V (bf16 r x d_in); objective (device, iters + 1 doubles) may be null.
+// Q0: fp32 d_in x r start of the subspace iteration.  ws: am_plan().bytes.
+cudaError_t launch_am_datafree(const uint16_t *W, int64_t d_out, int64_t d_in, int r, int iters, int power0,
+                               int power, const float *Q0, uint16_t *vals, uint8_t *meta, uint16_t *U, uint16_t *V,
+                               double *objective, uint8_t *ws, cudaStream_t st);
+
 // Row split of the column-norm reduction: `splits` row ranges of
 // `rows_per_split` rows, each leaving d_in fp32 partial sums in the workspace.
 struct NormPlan {

@@ -191,3 +191,22 @@ def test_forward_2to8_argument_errors():
     if not torch.cuda.is_available():
         assert f(x, 1, v, m, 8, 64, u, vv, 8, y, ws, 1 << 20, None) == DEVICE
         assert f(x, 1, v, m, 8, 64, None, None, 0, y, None, 0, None) == DEVICE        # r == 0: no factors
+
+
+def test_decompose_argument_errors():
+    f = slr.lib().slr_decompose_datafree
+    w, q, v, m, u, vv, ws = (P(0x10000 * k) for k in range(1, 8))
+    big = 1 << 30
+    assert f(w, 64, 64, 12, 1, 1, 1, q, v, m, u, vv, None, ws, big, None) == SHAPE     # r % 8
+    assert f(w, 64, 60, 8, 1, 1, 1, q, v, m, u, vv, None, ws, big, None) == SHAPE     # d_in % 8
+    assert f(w, 64, 64, 136, 1, 1, 1, q, v, m, u, vv, None, ws, big, None) == SHAPE   # r > 128
+    assert f(w, 8, 64, 16, 1, 1, 1, q, v, m, u, vv, None, ws, big, None) == SHAPE     # r > d_out
+    assert f(w, 64, 64, 8, -1, 1, 1, q, v, m, u, vv, None, ws, big, None) == ARG
+    assert f(w, 64, 64, 8, 1, 0, 1, q, v, m, u, vv, None, ws, big, None) == ARG
+    assert f(w, 64, 64, 8, 1, 1, 1, P(0), v, m, u, vv, None, ws, big, None) == NULL   # Q0
+    assert f(w, 64, 64, 8, 1, 1, 1, q, v, m, u, vv, P(0x80004), ws, big, None) == ALIGN
+    assert f(w, 64, 64, 8, 1, 1, 1, q, v, m, u, vv, None, ws, 16, None) == WORKSPACE
+    need = slr.lib().slr_decompose_workspace_size(14336, 4096, 64)
+    assert need >= 14336 * 4096 * 4
+    if not torch.cuda.is_available():
+        assert f(w, 64, 64, 8, 1, 1, 1, q, v, m, u, vv, None, ws, big, None) == DEVICE

@@ -1,0 +1,112 @@
+"""GPU parity of the data-free alternating minimisation W ~ S + U V (HASSLE-free
+section 4, identity Hessian; LoSparse section 3.2 start) against the fp64
+oracle (oracle/datafree_am.py: exact SVD, exact hard threshold).
+
+The GPU computes C_r by subspace iteration in fp32 and rounds S, U, V to bf16
+for storage, so trajectories are compared through what is unique: the
+objective ||W - S - U V||_F after the start and after every iteration
+(relative 2e-3 once the subspace iteration has converged), its monotone
+decrease, the 2:4 structure of S, and the consistency of the returned
+factors with the reported objective.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.datafree_am as am
+import synth
+from gpu_util import bits_to_f64, from_dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import sparse_rank_linear_02_b200 as slr
+
+
+def _q0(d_in, r, seed):
+    return torch.from_numpy(np.random.Generator(np.random.PCG64(seed)).standard_normal((d_in, r))
+                            .astype(np.float32)).cuda()
+
+
+def _dense_S(vals, meta, d_in):
+    import oracle
+    return bits_to_f64(oracle.unpack_2to4(from_dev(vals), meta.cpu().numpy(), d_in))
+
+
+def _check_structure(vals, meta, d_out, d_in):
+    m = meta.cpu().numpy().astype(np.int64)
+    nib = np.stack([m & 0xF, m >> 4], axis=-1).reshape(d_out, -1)[:, : d_in // 4]
+    lo, hi = nib & 3, nib >> 2
+    assert np.all(lo < hi), "metadata nibbles must name two ascending positions"
+
+
+@pytest.mark.parametrize("d_out,d_in,r,iters", [(256, 128, 8, 4), (192, 320, 16, 3)])
+def test_decompose_matches_oracle_objectives(d_out, d_in, r, iters):
+    W = synth.gaussian_bf16((d_out, d_in), 0.02, d_out + d_in)
+    vals, meta, U, V, obj = slr.decompose_datafree(to_dev(W), r, iters, power_first=80, power=30,
+                                                    Q0=_q0(d_in, r, 5))
+    torch.cuda.synchronize()
+    obj = obj.cpu().numpy()
+    _, _, ref = am.alternating_minimisation(bits_to_f64(W), r, iters)
+    np.testing.assert_allclose(obj, ref, rtol=2e-3)
+    assert all(b <= a * (1 + 1e-5) for a, b in zip(obj, obj[1:])), obj
+    _check_structure(vals, meta, d_out, d_in)
+    S = _dense_S(vals, meta, d_in)
+    L = bits_to_f64(from_dev(U)) @ bits_to_f64(from_dev(V))
+    recon = np.linalg.norm(bits_to_f64(W) - S - L)
+    assert abs(recon - obj[-1]) <= 1e-2 * obj[-1], (recon, obj[-1])
+
+
+def test_decompose_start_is_eckart_young():
+    """iters = 0: U V is C_r(W) (the truncation error equals the sum of the
+    trailing squared singular values) and S the hard threshold of W - U V."""
+    d_out, d_in, r = 300, 160, 24
+    W = synth.gaussian_bf16((d_out, d_in), 1.0, 7)
+    Wf = bits_to_f64(W)
+    vals, meta, U, V, obj = slr.decompose_datafree(to_dev(W), r, 0, power_first=200, Q0=_q0(d_in, r, 8))
+    L = bits_to_f64(from_dev(U)) @ bits_to_f64(from_dev(V))
+    sv = np.linalg.svd(Wf, compute_uv=False)
+    ey = np.sqrt(np.sum(sv[r:] ** 2))
+    assert abs(np.linalg.norm(Wf - L) - ey) <= 2e-3 * ey
+    _, _, ref = am.alternating_minimisation(Wf, r, 0)
+    np.testing.assert_allclose(obj.cpu().numpy(), ref, rtol=1e-3)
+
+
+def test_decompose_recovers_planted_structure():
+    """W = S0 + L0 (2:4 with large entries plus rank 4): the objective falls
+    far below the start, as the oracle's does."""
+    rng = np.random.Generator(np.random.PCG64(11))
+    d_out, d_in, r = 384, 256, 8
+    S0 = am.hard_threshold_2to4(rng.normal(size=(d_out, d_in)) * 3.0)
+    L0 = rng.normal(size=(d_out, 4)) @ rng.normal(size=(4, d_in)) * 0.3
+    W = synth.f32_to_bf16_bits((S0 + L0).astype(np.float32))
+    _, _, _, _, obj = slr.decompose_datafree(to_dev(W), r, 12, power_first=60, power=6, Q0=_q0(d_in, r, 12))
+    obj = obj.cpu().numpy()
+    _, _, ref = am.alternating_minimisation(bits_to_f64(W), r, 12)
+    assert obj[-1] < 0.5 * obj[0]
+    assert obj[-1] <= ref[-1] * 1.05 + 1e-3 * np.linalg.norm(bits_to_f64(W)), (obj[-1], ref[-1])
+
+
+def test_decompose_deterministic():
+    W = to_dev(synth.gaussian_bf16((128, 96), 0.02, 13))
+    a = slr.decompose_datafree(W, 8, 2, Q0=_q0(96, 8, 1))
+    b = slr.decompose_datafree(W, 8, 2, Q0=_q0(96, 8, 1))
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.uint8) if x.dtype != torch.float64 else x,
+                           y.view(torch.uint8) if y.dtype != torch.float64 else y)
+
+
+def test_decompose_config_layer():
+    """The Llama-3-8B gate/up shape (14336 x 4096, r = 64), three iterations of
+    two warm-started power steps: monotone objective, valid 2:4 metadata,
+    finite factors."""
+    layer = next(l for l in synth.CONFIGS[3].layers if l.name == "gate_up")
+    W = layer.weight()
+    vals, meta, U, V, obj = slr.decompose_datafree(to_dev(W), 64, 3, power_first=8, power=2,
+                                                    Q0=_q0(layer.d_in, 64, 3))
+    torch.cuda.synchronize()
+    obj = obj.cpu().numpy()
+    assert np.all(np.isfinite(obj)) and obj[0] < np.linalg.norm(bits_to_f64(W))
+    assert all(b <= a * (1 + 1e-4) for a, b in zip(obj, obj[1:])), obj
+    _check_structure(vals, meta, layer.d_out, layer.d_in)
+    assert torch.isfinite(U.float()).all() and torch.isfinite(V.float()).all()
