@@ -295,6 +295,8 @@ def run_ours(args, rank, world, dist):
     pack = run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier) if "pack" in legs else None
     sparse28 = run_2to8_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier) \
         if "2to8" in legs else None
+    decomp = run_decompose_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier) \
+        if "decompose" in legs else None
     calibrate = run_calibrate_leg(args, slr, torch, dev, W, to_dev, peaks, max_over_ranks, barrier) \
         if "calibrate" in legs else None
     del W
@@ -323,6 +325,7 @@ def run_ours(args, rank, world, dist):
         "pack": pack,
         "calibrate": calibrate,
         "sparse_2to8": sparse28,
+        "decompose_datafree": decomp,
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": 2 * K,
@@ -636,6 +639,49 @@ def run_2to8_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier):
     return res
 
 
+def run_decompose_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier):
+    """Data-free alternating minimisation (HASSLE-free section 4, identity
+    Hessian) of the gate/up weight into 2:4 S + rank-64 U V: the start
+    (8 power steps from a random subspace) alone, then with 4 iterations of
+    2 warm-started power steps; the difference is the per-iteration time.
+    FLOPs per iteration: (4 p + 4) d_out d_in r (p power steps of Z Q and
+    Z^T P, then U = Z Q and the residual W - U V), fp32 on CUDA cores."""
+    L = layer_of(PREFILL["cfg"], PREFILL["name"])
+    d_out, d_in, r, p, iters = L.d_out, L.d_in, 64, 2, 4
+    W = to_dev(L.weight())
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    Q0 = torch.randn((d_in, r), generator=g, device=dev, dtype=torch.float32)
+
+    def run(n):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        out = slr.decompose_datafree(W, r, n, power_first=8, power=p, Q0=Q0)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1), out
+
+    run(0)
+    run(1)  # warm-up
+    barrier()
+    t0 = min(run(0)[0] for _ in range(3))
+    runs = [run(iters) for _ in range(3)]
+    t1 = min(x[0] for x in runs)
+    obj = runs[0][1][4].cpu().numpy()
+    ms_iter = max_over_ranks((t1 - t0) / iters)
+    flops = (4 * p + 4) * d_out * d_in * r
+    # fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
+    peak_fp32 = 148 * 128 * 2 * 1.965e9 / 1e12
+    tf = flops / (ms_iter * 1e-3) / 1e12
+    return {"workload": f"data-free alternating minimisation of the {d_out}x{d_in} gate/up weight, 2:4 + rank {r}, "
+                        f"{p} warm-started power steps per iteration",
+            "ms_start": round(t0, 3), "ms_per_iteration": round(ms_iter, 3), "iterations_timed": iters,
+            "tflops_fp32": round(tf, 2), "peak_fp32_tflops_derived": round(peak_fp32, 1),
+            "frac_of_fp32_peak": round(tf / peak_fp32, 4),
+            "objective": [round(float(x), 5) for x in obj]}
+
+
 def run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier):
     d_out, d_in = W.shape
     nbytes = d_out * d_in * 2 + d_out * d_in + d_out * d_in // 8   # read W, write vals + meta
@@ -778,7 +824,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024, help="token rows in the oracle CPU baseline sample")
     ap.add_argument("--ref-rows", type=int, default=64, help="token rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="prefill,e2e,decode,pack,calibrate,2to8,cpu,cfg2,cfg4,cfg5",
+    ap.add_argument("--only", default="prefill,e2e,decode,pack,calibrate,2to8,decompose,cpu,cfg2,cfg4,cfg5",
                     help="comma list of legs to run (profiling runs use one leg)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -214,8 +214,9 @@ SLR_API slr_status slr_forward_2to8(const void *X, int64_t M, const void *vals8,
  *   vals, meta device: S in the slr_pack_2to4 format (values = W - U V at the
  *              kept positions, rounded to bf16).
  *   U          device, bf16 [d_out, r];  V  device, bf16 [r, d_in].
- *   objective  device, fp64 [iters + 1], or NULL: ||W - S - U V||_F (fp32 U V,
- *              unrounded S) after the start and after every iteration.
+ *   objective  device, fp64 [iters + 1], or NULL: ||W - S - U V||_F (S as
+ *              stored in bf16, U V in fp32) after the start and after every
+ *              iteration.
  *   workspace  device scratch of slr_decompose_workspace_size() bytes.
  *
  * Requirements: d_out >= 1, d_in >= 8 with d_in % 8 == 0, 8 <= r <= 128 with

@@ -40,15 +40,26 @@ def _check_structure(vals, meta, d_out, d_in):
     assert np.all(lo < hi), "metadata nibbles must name two ascending positions"
 
 
-@pytest.mark.parametrize("d_out,d_in,r,iters", [(256, 128, 8, 4), (192, 320, 16, 3)])
-def test_decompose_matches_oracle_objectives(d_out, d_in, r, iters):
-    W = synth.gaussian_bf16((d_out, d_in), 0.02, d_out + d_in)
-    vals, meta, U, V, obj = slr.decompose_datafree(to_dev(W), r, iters, power_first=80, power=30,
-                                                    Q0=_q0(d_in, r, 5))
+def _gapped(d_out, d_in, r, seed, top=40.0):
+    """A rank-r part with singular values top .. top/2 plus a 2:4 part and noise,
+    so the spectrum has a clear gap after the r-th value (the subspace iteration
+    converges in a few dozen steps and the trajectories are comparable)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    Uo, _ = np.linalg.qr(rng.normal(size=(d_out, r)))
+    Vo, _ = np.linalg.qr(rng.normal(size=(d_in, r)))
+    L = (Uo * np.linspace(top, top / 2, r)) @ Vo.T
+    S0 = am.hard_threshold_2to4(rng.normal(size=(d_out, d_in))) * 0.5
+    return synth.f32_to_bf16_bits((L + S0 + 0.05 * rng.normal(size=(d_out, d_in))).astype(np.float32))
+
+
+def _run_and_compare(W, r, iters, power_first, power, rtol, seed):
+    d_out, d_in = W.shape
+    vals, meta, U, V, obj = slr.decompose_datafree(to_dev(W), r, iters, power_first=power_first, power=power,
+                                                    Q0=_q0(d_in, r, seed))
     torch.cuda.synchronize()
     obj = obj.cpu().numpy()
     _, _, ref = am.alternating_minimisation(bits_to_f64(W), r, iters)
-    np.testing.assert_allclose(obj, ref, rtol=2e-3)
+    np.testing.assert_allclose(obj, ref, rtol=rtol)
     assert all(b <= a * (1 + 1e-5) for a, b in zip(obj, obj[1:])), obj
     _check_structure(vals, meta, d_out, d_in)
     S = _dense_S(vals, meta, d_in)
@@ -57,13 +68,27 @@ def test_decompose_matches_oracle_objectives(d_out, d_in, r, iters):
     assert abs(recon - obj[-1]) <= 1e-2 * obj[-1], (recon, obj[-1])
 
 
+@pytest.mark.parametrize("d_out,d_in,r,iters", [(256, 128, 8, 4), (192, 320, 16, 3), (520, 264, 32, 3)])
+def test_decompose_matches_oracle_gapped(d_out, d_in, r, iters):
+    """Spectral gap after r: every objective within 1e-3 of the exact oracle's."""
+    _run_and_compare(_gapped(d_out, d_in, r, d_out + r), r, iters, 40, 10, 1e-3, 5)
+
+
+def test_decompose_matches_oracle_gaussian():
+    """A Gaussian W has almost no gap after r, so the fp32 subspace iteration and
+    the exact SVD may settle on slightly different (equally good) subspaces and
+    the trajectories drift apart: objectives within 1e-2."""
+    W = synth.gaussian_bf16((256, 128), 0.02, 384)
+    _run_and_compare(W, 8, 4, 80, 30, 1e-2, 5)
+
+
 def test_decompose_start_is_eckart_young():
     """iters = 0: U V is C_r(W) (the truncation error equals the sum of the
     trailing squared singular values) and S the hard threshold of W - U V."""
     d_out, d_in, r = 300, 160, 24
-    W = synth.gaussian_bf16((d_out, d_in), 1.0, 7)
+    W = _gapped(d_out, d_in, r, 7)
     Wf = bits_to_f64(W)
-    vals, meta, U, V, obj = slr.decompose_datafree(to_dev(W), r, 0, power_first=200, Q0=_q0(d_in, r, 8))
+    vals, meta, U, V, obj = slr.decompose_datafree(to_dev(W), r, 0, power_first=60, Q0=_q0(d_in, r, 8))
     L = bits_to_f64(from_dev(U)) @ bits_to_f64(from_dev(V))
     sv = np.linalg.svd(Wf, compute_uv=False)
     ey = np.sqrt(np.sum(sv[r:] ** 2))
@@ -73,18 +98,20 @@ def test_decompose_start_is_eckart_young():
 
 
 def test_decompose_recovers_planted_structure():
-    """W = S0 + L0 (2:4 with large entries plus rank 4): the objective falls
-    far below the start, as the oracle's does."""
+    """W = S0 + L0 (2:4 with large entries plus rank 8), r = 8: the alternation
+    all but recovers the planted pair, on the GPU as in the oracle."""
     rng = np.random.Generator(np.random.PCG64(11))
     d_out, d_in, r = 384, 256, 8
     S0 = am.hard_threshold_2to4(rng.normal(size=(d_out, d_in)) * 3.0)
-    L0 = rng.normal(size=(d_out, 4)) @ rng.normal(size=(4, d_in)) * 0.3
+    L0 = rng.normal(size=(d_out, r)) @ rng.normal(size=(r, d_in)) * 0.3
     W = synth.f32_to_bf16_bits((S0 + L0).astype(np.float32))
-    _, _, _, _, obj = slr.decompose_datafree(to_dev(W), r, 12, power_first=60, power=6, Q0=_q0(d_in, r, 12))
+    Wn = np.linalg.norm(bits_to_f64(W))
+    _, _, _, _, obj = slr.decompose_datafree(to_dev(W), r, 16, power_first=60, power=6, Q0=_q0(d_in, r, 12))
     obj = obj.cpu().numpy()
-    _, _, ref = am.alternating_minimisation(bits_to_f64(W), r, 12)
-    assert obj[-1] < 0.5 * obj[0]
-    assert obj[-1] <= ref[-1] * 1.05 + 1e-3 * np.linalg.norm(bits_to_f64(W)), (obj[-1], ref[-1])
+    _, _, ref = am.alternating_minimisation(bits_to_f64(W), r, 16)
+    assert ref[-1] < 0.01 * ref[0], ref           # the oracle recovers it ...
+    assert obj[-1] < 0.01 * obj[0], obj           # ... and so does the GPU
+    assert obj[-1] <= 1.1 * ref[-1] + 2e-3 * Wn, (obj[-1], ref[-1])
 
 
 def test_decompose_deterministic():
