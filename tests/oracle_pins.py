@@ -634,3 +634,72 @@ def pin_am_degenerate_cases(am):
 
 AM_PINS = [pin_am_truncation_exact_cases, pin_am_truncation_beats_random, pin_am_hard_threshold,
            pin_am_monotone_objective, pin_am_degenerate_cases]
+
+
+# --------------------------------------------------------------------------- LoRA backward pins
+#
+# These take the module oracle.lora_backward (or a planted-mistake copy).  The
+# gradient is pinned by its definition: the loss <dY, Y> with Y from the C
+# forward oracle is linear in U (and in V), so a central difference with
+# small integer data is exact; plus independence from S and the bound.
+
+def _lora_problem(seed, M=5, d_out=8, d_in=12, r=3):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    X = _bf16(rng.integers(-3, 4, size=(M, d_in)))
+    dY = _bf16(rng.integers(-3, 4, size=(M, d_out)))
+    W = _bf16(rng.integers(-4, 5, size=(d_out, d_in)))
+    U = _bf16(rng.integers(-2, 3, size=(d_out, r)))
+    V = _bf16(rng.integers(-2, 3, size=(r, d_in)))
+    return X, dY, W, U, V
+
+
+def _loss(o, X, dY, vals, meta, U, V):
+    Y, _ = o.forward(X, vals, meta, U, V)
+    return float(np.sum(_f64(dY) * Y))
+
+
+def pin_lora_finite_difference(lb):
+    import oracle
+    o = oracle.default()
+    for seed, shape in [(101, (5, 8, 12, 3)), (102, (3, 16, 8, 2)), (103, (7, 4, 16, 5))]:
+        X, dY, W, U, V = _lora_problem(seed, *shape)
+        vals, meta = o.pack_2to4(W)
+        dU, dV, _, _ = lb.lora_backward(X, dY, U, V)
+        for (i, k) in [(0, 0), (shape[1] - 1, shape[3] - 1), (shape[1] // 2, 1 % shape[3])]:
+            Up, Um = U.copy(), U.copy()
+            Up[i, k] = _bf16([_f64(U[i:i + 1, k:k + 1])[0, 0] + 1.0])[0]
+            Um[i, k] = _bf16([_f64(U[i:i + 1, k:k + 1])[0, 0] - 1.0])[0]
+            fd = (_loss(o, X, dY, vals, meta, Up, V) - _loss(o, X, dY, vals, meta, Um, V)) / 2.0
+            assert dU[i, k] == fd, (seed, i, k, dU[i, k], fd)
+        for (k, j) in [(0, 0), (shape[3] - 1, shape[2] - 1), (1 % shape[3], shape[2] // 2)]:
+            Vp, Vm = V.copy(), V.copy()
+            Vp[k, j] = _bf16([_f64(V[k:k + 1, j:j + 1])[0, 0] + 1.0])[0]
+            Vm[k, j] = _bf16([_f64(V[k:k + 1, j:j + 1])[0, 0] - 1.0])[0]
+            fd = (_loss(o, X, dY, vals, meta, U, Vp) - _loss(o, X, dY, vals, meta, U, Vm)) / 2.0
+            assert dV[k, j] == fd, (seed, k, j, dV[k, j], fd)
+
+
+def pin_lora_shapes_bounds_and_s_independence(lb):
+    import oracle
+    o = oracle.default()
+    X, dY, W, U, V = _lora_problem(104, 6, 8, 16, 4)
+    dU, dV, BU, BV = lb.lora_backward(X, dY, U, V)
+    assert dU.shape == (8, 4) and dV.shape == (4, 16)
+    assert np.all(np.abs(dU) <= BU) and np.all(np.abs(dV) <= BV)
+    # The gradient does not depend on S: the loss difference between two S is
+    # constant in U, so finite differences through either S agree.
+    v1, m1 = o.pack_2to4(W)
+    v2, m2 = o.pack_2to4(_bf16(np.zeros((8, 16))))
+    Up = U.copy()
+    Up[3, 2] = _bf16([_f64(U[3:4, 2:3])[0, 0] + 1.0])[0]
+    d1 = _loss(o, X, dY, v1, m1, Up, V) - _loss(o, X, dY, v1, m1, U, V)
+    d2 = _loss(o, X, dY, v2, m2, Up, V) - _loss(o, X, dY, v2, m2, U, V)
+    assert d1 == d2 == dU[3, 2]
+    # Non-negative inputs: the bound is the gradient itself.
+    Xa, dYa, Ua, Va = (_bf16(np.abs(_f64(a))) for a in (X, dY, U, V))
+    dU2, dV2, BU2, BV2 = lb.lora_backward(Xa, dYa, Ua, Va)
+    np.testing.assert_array_equal(dU2, BU2)
+    np.testing.assert_array_equal(dV2, BV2)
+
+
+LORA_PINS = [pin_lora_finite_difference, pin_lora_shapes_bounds_and_s_independence]

@@ -16,3 +16,12 @@ from oracle_pins import AM_PINS  # noqa: E402
 def test_oracle_am_pin(pin):
     import oracle.datafree_am as am
     pin(am)
+
+
+from oracle_pins import LORA_PINS  # noqa: E402
+
+
+@pytest.mark.parametrize("pin", LORA_PINS, ids=[p.__name__ for p in LORA_PINS])
+def test_oracle_lora_pin(pin):
+    import oracle.lora_backward as lb
+    pin(lb)

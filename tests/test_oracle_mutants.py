@@ -111,3 +111,34 @@ def test_am_mutant_is_caught(name, old, new, count, tmp_path):
         except (AssertionError, ValueError, IndexError, np.linalg.LinAlgError):
             caught.append(pin.__name__)
     assert caught, f"no pin caught mutant {name}"
+
+
+LORA_SRC = os.path.join(os.path.dirname(oracle.__file__), "lora_backward.py")
+LORA_MUTANTS = [
+    ("lora_v_rows_reversed", "T = Xf @ Vf.T", "T = Xf @ Vf[::-1].T", 1),
+    ("lora_dv_sign", "dV = G.T @ Xf", "dV = -(G.T @ Xf)", 1),
+    ("lora_du_uses_u", "dU = dYf.T @ T", "dU = dYf.T @ (T + 0.5 * (dYf @ Uf))", 1),
+    ("lora_bound_signed", "B_dU = np.abs(dYf).T @ (np.abs(Xf) @ np.abs(Vf).T)", "B_dU = np.abs(dYf).T @ (np.abs(Xf) @ Vf.T)", 1),
+]
+
+
+@pytest.mark.parametrize("name,old,new,count", LORA_MUTANTS, ids=[m[0] for m in LORA_MUTANTS])
+def test_lora_mutant_is_caught(name, old, new, count, tmp_path):
+    import importlib.util
+    import sys as _sys
+    _sys.path.insert(0, TESTS)
+    from oracle_pins import LORA_PINS
+    text = open(LORA_SRC).read()
+    assert text.count(old) == count, f"mutation site for {name} not found"
+    path = tmp_path / f"{name}.py"
+    path.write_text(text.replace(old, new))
+    spec = importlib.util.spec_from_file_location(f"lora_{name}", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    caught = []
+    for pin in LORA_PINS:
+        try:
+            pin(mod)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught mutant {name}"
