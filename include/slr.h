@@ -197,6 +197,40 @@ SLR_API slr_status slr_forward_2to8(const void *X, int64_t M, const void *vals8,
                             void *Y, void *workspace, size_t workspace_bytes, slr_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * Backward with respect to the low-rank factors (S frozen), for LoRA-style
+ * fine-tuning of U and V (3BASiL summary page: the low-rank components
+ * initialise LoRA; LoSparse section 3.2 for the layer).
+ *
+ * For Y = X S^T + T U^T with T = X V^T and an upstream gradient dY:
+ *     dU = dY^T T          dV = (dY U)^T X
+ * on the tensor cores (bf16 operands, fp32 accumulation; T and G = dY U are
+ * held in bf16 between the products).  The operands are read in place from the
+ * row-major X and dY (no transposes).
+ *
+ *   X       device, bf16 [M, d_in]      (the forward's input).
+ *   dY      device, bf16 [M, d_out].
+ *   U       device, bf16 [d_out, r];  V  device, bf16 [r, d_in].
+ *   T       device, bf16 [M, r], or NULL: the forward's X V^T if the caller
+ *           kept it; otherwise it is recomputed.
+ *   dU      device, fp32 [d_out, r], out;  dV  device, fp32 [r, d_in], out.
+ *   workspace  slr_lora_backward_workspace_size(M, r) bytes, 256-byte aligned.
+ *
+ * Accuracy contract (tested): relative Frobenius error <= 5e-3 and
+ * |err| <= 1e-2 * B + 1e-6 * max(B) per element against the exact gradients of
+ * the same bf16 inputs, B = |dY|^T |X| |V|^T for dU and (|dY| |U|)^T |X| for dV.
+ *
+ * Requirements: M >= 0 (M == 0 writes zero gradients), d_out >= 8 with
+ * d_out % 8 == 0, d_in >= 64 with d_in % 64 == 0, 8 <= r <= 256 with r % 8 == 0,
+ * M, d_out, d_in < 2^31; all pointers 16-byte aligned.
+ * ------------------------------------------------------------------------ */
+SLR_API slr_status slr_lora_backward(const void *X, int64_t M, const void *dY, int64_t d_out, int64_t d_in,
+                             const void *U, const void *V, int64_t r, const void *T, float *dU, float *dV,
+                             void *workspace, size_t workspace_bytes, slr_stream_t stream);
+
+/* Scratch bytes of slr_lora_backward (4 * M * r, rounded up). */
+SLR_API size_t slr_lora_backward_workspace_size(int64_t M, int64_t r);
+
+/* --------------------------------------------------------------------------
  * Data-free decomposition W ~ S + U V by alternating minimisation.
  *
  * HASSLE-free, section 4 (data-free variant: identity Hessian), started as in

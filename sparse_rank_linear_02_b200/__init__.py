@@ -12,6 +12,7 @@ Functions mirror the C ABI in ``include/slr.h``:
 * ``column_norms(X, sumsq=None) -> (norms, sumsq)``  -- ``slr_column_norms``
 * ``pack_2to8(W, dense=True, as_2to4=True)``  -- ``slr_pack_2to8``
 * ``forward_2to8(X, vals8, meta8, U, V) -> Y``  -- ``slr_forward_2to8``
+* ``lora_backward(X, dY, U, V, T=None) -> (dU, dV)``  -- ``slr_lora_backward``
 * ``decompose_datafree(W, r, iters, ...) -> (vals, meta, U, V, objective)``  --
   ``slr_decompose_datafree``
 * ``forward(X, vals, meta, U, V) -> Y``  -- ``slr_forward`` /
@@ -70,6 +71,10 @@ def _load() -> ctypes.CDLL:
                                            p, p, p, sz, p]
     lib.slr_decompose_workspace_size.restype = sz
     lib.slr_decompose_workspace_size.argtypes = [i64, i64, i64]
+    lib.slr_lora_backward.restype = st
+    lib.slr_lora_backward.argtypes = [p, i64, p, i64, i64, p, p, i64, p, p, p, p, sz, p]
+    lib.slr_lora_backward_workspace_size.restype = sz
+    lib.slr_lora_backward_workspace_size.argtypes = [i64, i64]
     lib.slr_column_norms.restype = st
     lib.slr_column_norms.argtypes = [p, i64, i64, i64, p, p, p, sz, p]
     lib.slr_column_norms_workspace_size.restype = sz
@@ -207,6 +212,23 @@ def forward_2to8(X: torch.Tensor, vals8: torch.Tensor, meta8: torch.Tensor, U: t
     _check(_lib.slr_forward_2to8(_ptr(X), M, _ptr(vals8), _ptr(meta8), d_out, d_in, _ptr(U), _ptr(V), r,
                                  _ptr(out), _ptr(workspace), ws_bytes, _stream()), "slr_forward_2to8")
     return out
+
+
+def lora_backward(X: torch.Tensor, dY: torch.Tensor, U: torch.Tensor, V: torch.Tensor,
+                  T: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Gradients of the layer w.r.t. U and V for upstream ``dY`` [M, d_out]:
+    ``dU = dY^T (X V^T)`` (fp32 [d_out, r]), ``dV = (dY U)^T X`` (fp32 [r, d_in]).
+    ``T`` is the forward's ``X V^T`` (bf16 [M, r]) if kept."""
+    M, d_in = X.shape
+    d_out = dY.shape[1]
+    r = U.shape[1]
+    dU = torch.empty((d_out, r), dtype=torch.float32, device=X.device)
+    dV = torch.empty((r, d_in), dtype=torch.float32, device=X.device)
+    need = int(_lib.slr_lora_backward_workspace_size(M, r))
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _check(_lib.slr_lora_backward(_ptr(X), M, _ptr(dY), d_out, d_in, _ptr(U), _ptr(V), r, _ptr(T), _ptr(dU),
+                                  _ptr(dV), _ptr(ws), ws.numel(), _stream()), "slr_lora_backward")
+    return dU, dV
 
 
 def decompose_datafree(W: torch.Tensor, r: int, iters: int, *, power_first: int = 8, power: int = 2,

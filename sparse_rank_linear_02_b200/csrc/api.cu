@@ -225,6 +225,41 @@ slr_status slr_forward_2to8(const void *X, int64_t M, const void *vals8, const v
     return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
 }
 
+size_t slr_lora_backward_workspace_size(int64_t M, int64_t r) {
+    if (M <= 0 || r <= 0) return 0;
+    return slr::round_up((size_t)4 * M * r, slr::kAlign);
+}
+
+slr_status slr_lora_backward(const void *X, int64_t M, const void *dY, int64_t d_out, int64_t d_in, const void *U,
+                             const void *V, int64_t r, const void *T, float *dU, float *dV, void *workspace,
+                             size_t workspace_bytes, slr_stream_t stream) {
+    if (M < 0 || d_out < 8 || d_out % 8 != 0 || d_in < 64 || d_in % 64 != 0 || r < 8 || r > 256 || r % 8 != 0 ||
+        M > INT32_MAX || d_out > INT32_MAX || d_in > INT32_MAX)
+        return SLR_ERR_SHAPE;
+    if (dU == nullptr || dV == nullptr) return SLR_ERR_NULL;
+    if (M > 0 && (X == nullptr || dY == nullptr || U == nullptr || V == nullptr || workspace == nullptr))
+        return SLR_ERR_NULL;
+    if (!slr::aligned16(dU) || !slr::aligned16(dV)) return SLR_ERR_ALIGN;
+    if (M > 0 && (!slr::aligned16(X) || !slr::aligned16(dY) || !slr::aligned16(U) || !slr::aligned16(V) ||
+                  !slr::aligned16(T) || (reinterpret_cast<uintptr_t>(workspace) % slr::kAlign) != 0))
+        return SLR_ERR_ALIGN;
+    if (workspace_bytes < slr_lora_backward_workspace_size(M, r)) return SLR_ERR_WORKSPACE;
+    const slr_status dev = slr::check_device();
+    if (dev != SLR_OK) return dev;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    if (M == 0) {
+        err = cudaMemsetAsync(dU, 0, (size_t)d_out * r * sizeof(float), st);
+        if (err == cudaSuccess) err = cudaMemsetAsync(dV, 0, (size_t)r * d_in * sizeof(float), st);
+    } else {
+        err = slr::launch_lora_backward(static_cast<const uint16_t *>(X), M, static_cast<const uint16_t *>(dY), d_out,
+                                        d_in, static_cast<const uint16_t *>(U), static_cast<const uint16_t *>(V), r,
+                                        static_cast<const uint16_t *>(T), dU, dV, static_cast<uint16_t *>(workspace),
+                                        st);
+    }
+    return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
+}
+
 size_t slr_decompose_workspace_size(int64_t d_out, int64_t d_in, int64_t r) {
     if (d_out < 1 || d_in < 8 || r < 8 || r > 128) return 0;
     return (size_t)slr::am_plan(d_out, d_in, r).bytes;
@@ -298,10 +333,11 @@ slr_path slr_forward_select_path(int64_t M, int64_t d_out, int64_t d_in, int64_t
 slr_status slr_check_kernel_error(void) {
     if (slr::check_device() != SLR_OK) return SLR_ERR_DEVICE;
     if (cudaDeviceSynchronize() != cudaSuccess) return SLR_ERR_CUDA;
-    unsigned code = 0, code28 = 0;
+    unsigned code = 0, code28 = 0, code_bwd = 0;
     if (slr::read_and_clear_kernel_error(&code) != cudaSuccess) return SLR_ERR_CUDA;
     if (slr::read_and_clear_decode28_error(&code28) != cudaSuccess) return SLR_ERR_CUDA;
-    return (code | code28) ? SLR_ERR_TIMEOUT : SLR_OK;
+    if (slr::read_and_clear_backward_error(&code_bwd) != cudaSuccess) return SLR_ERR_CUDA;
+    return (code | code28 | code_bwd) ? SLR_ERR_TIMEOUT : SLR_OK;
 }
 
 slr_status slr_selftest_wait_timeout(int64_t limit_cycles, slr_stream_t stream) {

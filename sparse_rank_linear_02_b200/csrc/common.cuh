@@ -72,6 +72,15 @@ cudaError_t launch_am_datafree(const uint16_t *W, int64_t d_out, int64_t d_in, i
                                int power, const float *Q0, uint16_t *vals, uint8_t *meta, uint16_t *U, uint16_t *V,
                                double *objective, uint8_t *ws, cudaStream_t st);
 
+// Gradients of the layer with respect to U and V (S frozen): G = dY U (bf16,
+// in ws), dU = dY^T T (fp32 [d_out, r]), dV = G^T X (fp32 [r, d_in]).  T16_in
+// is the forward's T = X V^T (bf16 [M, r]) or null (then computed into ws).
+// ws: 2 * M * r bf16.  d_in % 64 == 0, d_out % 8 == 0, 8 <= r <= 256, r % 8 == 0.
+cudaError_t launch_lora_backward(const uint16_t *X, int64_t M, const uint16_t *dY, int64_t d_out, int64_t d_in,
+                                 const uint16_t *U, const uint16_t *V, int64_t r, const uint16_t *T16_in, float *dU,
+                                 float *dV, uint16_t *ws, cudaStream_t st);
+cudaError_t read_and_clear_backward_error(unsigned *code);
+
 // Row split of the column-norm reduction: `splits` row ranges of
 // `rows_per_split` rows, each leaving d_in fp32 partial sums in the workspace.
 struct NormPlan {

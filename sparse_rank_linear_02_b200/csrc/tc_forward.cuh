@@ -1,10 +1,19 @@
 // tc_forward.cuh -- launcher of the 2:4 tcgen05 tensor-core forward (internal).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace slr {
+
+namespace tc {
+// 2-D tiled tensor map of a row-major matrix (inner x outer elements, row
+// pitch row_bytes) with the given box and swizzle; false when the driver's
+// encoder is unavailable or rejects the arguments.
+bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
+}  // namespace tc
 
 // Y = X S^T + T U^T on the tensor cores.  T16 is bf16 [M, r] (may be null when
 // r == 0).  Requires d_in % 128 == 0, d_out % 8 == 0, r % 8 == 0.

@@ -210,3 +210,20 @@ def test_decompose_argument_errors():
     assert need >= 14336 * 4096 * 4
     if not torch.cuda.is_available():
         assert f(w, 64, 64, 8, 1, 1, 1, q, v, m, u, vv, None, ws, big, None) == DEVICE
+
+
+def test_lora_backward_argument_errors():
+    f = slr.lib().slr_lora_backward
+    x, dy, u, v, du, dv, ws = (P(0x10000 * k) for k in range(1, 8))
+    big = 1 << 30
+    assert f(x, 8, dy, 12, 64, u, v, 8, None, du, dv, ws, big, None) == SHAPE     # d_out % 8
+    assert f(x, 8, dy, 16, 96, u, v, 8, None, du, dv, ws, big, None) == SHAPE     # d_in % 64
+    assert f(x, 8, dy, 16, 64, u, v, 264, None, du, dv, ws, big, None) == SHAPE   # r > 256
+    assert f(x, 8, dy, 16, 64, u, v, 8, None, P(0), dv, ws, big, None) == NULL
+    assert f(x, 8, P(0), 16, 64, u, v, 8, None, du, dv, ws, big, None) == NULL
+    assert f(x, 8, dy, 16, 64, u, v, 8, P(0x80008), du, dv, ws, big, None) == ALIGN   # T
+    assert f(x, 8, dy, 16, 64, u, v, 8, None, du, dv, ws, 16, None) == WORKSPACE
+    assert slr.lib().slr_lora_backward_workspace_size(2048, 64) == 4 * 2048 * 64
+    if not torch.cuda.is_available():
+        assert f(x, 8, dy, 16, 64, u, v, 8, None, du, dv, ws, big, None) == DEVICE
+        assert f(None, 0, None, 16, 64, None, None, 8, None, du, dv, None, 0, None) == DEVICE   # M == 0 zero-fills
