@@ -295,6 +295,8 @@ def run_ours(args, rank, world, dist):
     pack = run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier) if "pack" in legs else None
     sparse28 = run_2to8_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier) \
         if "2to8" in legs else None
+    backward = run_backward_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier) \
+        if "backward" in legs else None
     decomp = run_decompose_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier) \
         if "decompose" in legs else None
     calibrate = run_calibrate_leg(args, slr, torch, dev, W, to_dev, peaks, max_over_ranks, barrier) \
@@ -326,6 +328,7 @@ def run_ours(args, rank, world, dist):
         "calibrate": calibrate,
         "sparse_2to8": sparse28,
         "decompose_datafree": decomp,
+        "lora_backward": backward,
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": 2 * K,
@@ -682,6 +685,52 @@ def run_decompose_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barr
             "objective": [round(float(x), 5) for x in obj]}
 
 
+def run_backward_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier):
+    """Backward w.r.t. U and V (LoRA fine-tuning of the low-rank factors, S
+    frozen) on the gate/up prefill shape, with the forward's T kept:
+    G = dY U, dU = dY^T T, dV = G^T X on the tensor cores.  GB/s counts the
+    algorithmic bytes (dY, X, U, T read once; dU, dV written in fp32)."""
+    L = layer_of(PREFILL["cfg"], PREFILL["name"])
+    M, d_out, d_in, r = PREFILL["M"], L.d_out, L.d_in, L.r
+    Uh, Vh = L.factors()
+    U, V = to_dev(Uh), to_dev(Vh)
+    nbytes = 2 * M * d_out + 2 * M * d_in + 2 * d_out * r + 2 * M * r + 4 * d_out * r + 4 * r * d_in
+    n_sets = max(2, math.ceil(2.0 * L2_BYTES / nbytes))
+    sets = []
+    for i in range(n_sets):
+        X = to_dev(L.activations(M)) if i == 0 else sets[0]["X"].clone()
+        dY = torch.randn((M, d_out), device=dev, dtype=torch.float32).to(torch.bfloat16)
+        sets.append(dict(X=X, dY=dY))
+    T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(slr.workspace_size(M, d_out, d_in, r), 256), dtype=torch.uint8, device=dev)
+    slr.forward_project(sets[0]["X"], V, d_out, ws, path="tensor")
+    T.copy_(ws[: M * r * 2].view(torch.bfloat16).view(M, r))
+    lib = slr.lib()
+    dU = torch.empty((d_out, r), dtype=torch.float32, device=dev)
+    dV = torch.empty((r, d_in), dtype=torch.float32, device=dev)
+    bws = torch.empty(max(lib.slr_lora_backward_workspace_size(M, r), 256), dtype=torch.uint8, device=dev)
+
+    def bwd(k):
+        s = sets[k % n_sets]
+        st = lib.slr_lora_backward(slr._ptr(s["X"]), M, slr._ptr(s["dY"]), d_out, d_in, slr._ptr(U), slr._ptr(V), r,
+                                   slr._ptr(T), slr._ptr(dU), slr._ptr(dV), slr._ptr(bws), bws.numel(),
+                                   slr._stream())
+        assert st == 0, st
+
+    for i in range(max(args.warmup, 3)):
+        bwd(i)
+    slr.check_kernel_error()
+    K = max(10, args.steps)
+    barrier()
+    ms = max_over_ranks(graph_time_ms(torch, [lambda k=k: bwd(k) for k in range(K)])) / K
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    flops = 2.0 * M * r * (2 * d_out + d_in)
+    return {"workload": f"backward w.r.t. U, V of the {d_out}x{d_in} gate/up layer, r={r}, M={M} tokens, T kept",
+            "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 5), "algorithmic_bytes": nbytes,
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+            "launches_per_step": 3, "l2": f"rotating {n_sets} (X, dY) sets"}
+
+
 def run_pack_leg(args, slr, torch, dev, W, peaks, max_over_ranks, barrier):
     d_out, d_in = W.shape
     nbytes = d_out * d_in * 2 + d_out * d_in + d_out * d_in // 8   # read W, write vals + meta
@@ -824,7 +873,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024, help="token rows in the oracle CPU baseline sample")
     ap.add_argument("--ref-rows", type=int, default=64, help="token rows per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="prefill,e2e,decode,pack,calibrate,2to8,decompose,cpu,cfg2,cfg4,cfg5",
+    ap.add_argument("--only", default="prefill,e2e,decode,pack,calibrate,2to8,decompose,backward,cpu,cfg2,cfg4,cfg5",
                     help="comma list of legs to run (profiling runs use one leg)")
     args = ap.parse_args()
     if args.warmup < 3:
