@@ -173,6 +173,34 @@ def bus_id_of(torch, dev):
 
 # ----------------------------------------------------------------------------- our arm
 
+def rank_helpers(torch, dist, dev):
+    """barrier(): all ranks meet (process group barrier, then the device drains);
+    max_over_ranks(x): the largest of every rank's x (an all-reduce MAX on a
+    tensor of `dev`, so it works with NCCL on GPUs and with gloo on the CPU).
+    With dist None both act on the one process."""
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        if dev.type == "cuda":
+            torch.cuda.synchronize()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return barrier, max_over_ranks
+
+
+def weak_scaling_value(world, work_per_rank_step, max_total_ms, steps, unit_scale=1e12):
+    """Whole-job throughput: every rank processes its own batch of the same size
+    each step, so the job processes world x the per-rank work in the slowest
+    rank's time."""
+    return world * work_per_rank_step / (max_total_ms / steps * 1e-3) / unit_scale
+
+
 def run_ours(args, rank, world, dist):
     import torch
     import sparse_rank_linear_02_b200 as slr
@@ -184,17 +212,7 @@ def run_ours(args, rank, world, dist):
     def to_dev(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = rank_helpers(torch, dist, dev)
 
     # ------------------------------------------------ prefill workload (the metric)
     L = layer_of(PREFILL["cfg"], PREFILL["name"])
@@ -240,7 +258,7 @@ def run_ours(args, rank, world, dist):
     flops_dense = 2.0 * M * d_out * d_in                 # dense-equivalent work per step
     flops_lr = 2.0 * M * r * (d_in + d_out)
     flops_exec = M * d_out * d_in + flops_lr              # MACs on kept weights x2 / 2 + rank-r GEMMs
-    value = world * flops_dense / (total_ms / K * 1e-3) / 1e12
+    value = weak_scaling_value(world, flops_dense, total_ms, K)
 
     p_dense = peaks["bf16_tflops"]
     p_sparse = SPARSE_RATIO * p_dense

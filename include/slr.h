@@ -215,6 +215,10 @@ SLR_API slr_status slr_forward_2to8(const void *X, int64_t M, const void *vals8,
  *   dU      device, fp32 [d_out, r], out;  dV  device, fp32 [r, d_in], out.
  *   workspace  slr_lora_backward_workspace_size(M, r) bytes, 256-byte aligned.
  *
+ * The product dU runs on a library-owned second stream, forked from and joined
+ * back into `stream` with events, so the call composes with stream capture
+ * like any other work on `stream`.
+ *
  * Accuracy contract (tested): relative Frobenius error <= 5e-3 and
  * |err| <= 1e-2 * B + 1e-6 * max(B) per element against the exact gradients of
  * the same bf16 inputs, B = |dY|^T |X| |V|^T for dU and (|dY| |U|)^T |X| for dV.

@@ -165,18 +165,22 @@ __global__ void reduce_splits_kernel(const float *__restrict__ part, int splits,
 // rank-deficient block stays finite), then M = L^-T (fp32, r x r row-major).
 // Shared memory: one r x r fp64 array; L fills the lower triangle and
 // X = L^-1 (also lower triangular) is kept transposed in the strict upper
-// triangle (X[i][c] at [c][i]); its diagonal is 1 / L[i][i].
+// triangle (X[i][c] at [c][i]); its diagonal is 1 / L[i][i].  Both phases are
+// right-looking, so every step is a parallel update of the trailing block:
+//   Cholesky, column j: pivot, scale column j below it, A[i][k] -= L[i][j] L[k][j]
+//   for j < k <= i;  inverse, row i: finalise row i of X (divide by L[i][i]),
+//   then X[i'][c] -= L[i'][i] X[i][c] for i' > i, c <= i.
 __global__ void __launch_bounds__(256) chol_inv_kernel(const float *__restrict__ gpart, int splits, int r,
                                                        float *__restrict__ Mout) {
     extern __shared__ double A[];
-    const int tid = threadIdx.x;
-    for (int i = tid; i < r * r; i += blockDim.x) {
+    __shared__ double floor_pivot;
+    const int tid = threadIdx.x, nth = blockDim.x;
+    for (int i = tid; i < r * r; i += nth) {
         double s = 0.0;
         for (int k = 0; k < splits; ++k) s += (double)gpart[(int64_t)k * r * r + i];
         A[i] = s;
     }
     __syncthreads();
-    __shared__ double floor_pivot;
     if (tid == 0) {
         double tr = 0.0;
         for (int i = 0; i < r; ++i) tr += A[i * r + i];
@@ -185,30 +189,39 @@ __global__ void __launch_bounds__(256) chol_inv_kernel(const float *__restrict__
     __syncthreads();
     for (int j = 0; j < r; ++j) {
         if (tid == 0) {
-            double d = A[j * r + j];
-            for (int k = 0; k < j; ++k) d -= A[j * r + k] * A[j * r + k];
+            const double d = A[j * r + j];
             A[j * r + j] = sqrt(d > floor_pivot ? d : floor_pivot);
         }
         __syncthreads();
         const double piv = A[j * r + j];
-        for (int i = j + 1 + tid; i < r; i += blockDim.x) {
-            double s = A[i * r + j];
-            for (int k = 0; k < j; ++k) s -= A[i * r + k] * A[j * r + k];
-            A[i * r + j] = s / piv;
+        for (int i = j + 1 + tid; i < r; i += nth) A[i * r + j] /= piv;
+        __syncthreads();
+        const int n = r - j - 1;
+        for (int q = tid; q < n * n; q += nth) {
+            const int ii = q / n, kk = q % n;
+            if (kk <= ii) {
+                const int i = j + 1 + ii, k = j + 1 + kk;
+                A[i * r + k] -= A[i * r + j] * A[k * r + j];
+            }
         }
         __syncthreads();
     }
-    // Column c of X = L^-1 by forward substitution, one thread per column;
-    // X[i][c] (i > c) is stored at A[c][i], a row only this thread touches.
-    for (int c = tid; c < r; c += blockDim.x) {
-        for (int i = c + 1; i < r; ++i) {
-            double s = -A[i * r + c] / A[c * r + c];       // k = c term, X[c][c] = 1 / L[c][c]
-            for (int k = c + 1; k < i; ++k) s -= A[i * r + k] * A[c * r + k];
-            A[c * r + i] = s / A[i * r + i];
-        }
-    }
+    for (int q = tid; q < r * r; q += nth)
+        if (q % r > q / r) A[q] = 0.0;  // strict upper triangle: X starts as the identity
     __syncthreads();
-    for (int i = tid; i < r * r; i += blockDim.x) {
+    for (int i = 0; i < r; ++i) {
+        const double dinv = 1.0 / A[i * r + i];
+        for (int c = tid; c < i; c += nth) A[c * r + i] *= dinv;
+        __syncthreads();
+        const int n = r - i - 1, m = i + 1;
+        for (int q = tid; q < n * m; q += nth) {
+            const int ii = i + 1 + q / m, c = q % m;
+            const double xic = (c == i) ? dinv : A[c * r + i];
+            A[c * r + ii] -= A[ii * r + i] * xic;
+        }
+        __syncthreads();
+    }
+    for (int i = tid; i < r * r; i += nth) {
         const int k = i / r, c = i % r;  // M[k][c] = X[c][k]
         float v = 0.f;
         if (c == k) v = (float)(1.0 / A[k * r + k]);
@@ -265,27 +278,31 @@ __global__ void __launch_bounds__(256) residual_project_kernel(const uint16_t *_
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
     for (int k0 = 0; k0 < r; k0 += kRBK) {
-        // Ps[k][row]: 64 rows x 16 k = 1024 floats, 4 per thread.
+        // Ps[k][row]: 64 rows x 16 k = 1024 floats, one 16-byte load per
+        // thread.  r % 8 == 0, so a 4-wide piece starting below r lies wholly
+        // inside the row (and is 16-byte aligned); pieces at or past r are zero.
         {
             const int row = tid / 4, kq = (tid % 4) * 4;
             const int64_t gr = r0 + row;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int gk = k0 + kq + q;
-                Ps[kq + q][row] = (gr < d_out && gk < r) ? P[gr * r + gk] : 0.f;
-            }
+            const float4 v = (gr < d_out && k0 + kq < r) ? *reinterpret_cast<const float4 *>(P + gr * r + k0 + kq)
+                                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+            Ps[kq + 0][row] = v.x;
+            Ps[kq + 1][row] = v.y;
+            Ps[kq + 2][row] = v.z;
+            Ps[kq + 3][row] = v.w;
         }
-        // Qs[k][col]: 128 cols x 16 k = 2048 floats, 8 per thread.
+        // Qs[k][col]: 128 cols x 16 k = 2048 floats, two 16-byte loads per thread.
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int idx = tid + h * 256;
             const int col = idx / 4, kq = (idx % 4) * 4;
             const int64_t gc = c0 + col;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int gk = k0 + kq + q;
-                Qs[kq + q][col] = (gc < d_in && gk < r) ? Q[gc * r + gk] : 0.f;
-            }
+            const float4 v = (gc < d_in && k0 + kq < r) ? *reinterpret_cast<const float4 *>(Q + gc * r + k0 + kq)
+                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+            Qs[kq + 0][col] = v.x;
+            Qs[kq + 1][col] = v.y;
+            Qs[kq + 2][col] = v.z;
+            Qs[kq + 3][col] = v.w;
         }
         __syncthreads();
 #pragma unroll

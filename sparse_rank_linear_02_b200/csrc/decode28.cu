@@ -51,13 +51,31 @@ __device__ __forceinline__ float group28_fma(uint32_t vv, uint32_t b, uint4 xg, 
     return acc;
 }
 
-// 32 logical columns: v holds the 8 kept values, m32 the 4 index bytes, x the
-// 32 X values of one token.
-__device__ __forceinline__ float chunk28_fma(uint4 v, uint32_t m32, const uint4 (&x)[4], float acc) {
-    acc = group28_fma(v.x, m32 & 0xFFu, x[0], acc);
-    acc = group28_fma(v.y, (m32 >> 8) & 0xFFu, x[1], acc);
-    acc = group28_fma(v.z, (m32 >> 16) & 0xFFu, x[2], acc);
-    acc = group28_fma(v.w, m32 >> 24, x[3], acc);
+// The three selectors of group28_fma for every index byte b = idx0 | idx1 << 3
+// (only 64 values): low half = the in-half selector, high half = the final
+// selector (byte permutes read the low 16 bits of their selector).
+__device__ __forceinline__ uint32_t selector_entry(uint32_t b) {
+    const uint32_t sel = ((b & 3u) | ((b & 0x18u) << 5)) * 0x22u + 0x1010u;
+    const uint32_t fsel = (b & 4u) * 0x11u + (b & 0x20u) * 0x220u + 0x3210u;
+    return (sel & 0xFFFFu) | (fsel << 16);
+}
+
+// group28_fma with the selectors looked up in the shared table `lut`.
+__device__ __forceinline__ float group28_fma_lut(uint32_t vv, uint32_t e, uint4 xg, float acc) {
+    const uint32_t lo = __byte_perm(xg.x, xg.y, e), hi = __byte_perm(xg.z, xg.w, e);
+    const uint32_t xs = __byte_perm(lo, hi, e >> 16);
+    acc = fmaf(bf16lo_to_f32(vv), bf16lo_to_f32(xs), acc);
+    acc = fmaf(bf16hi_to_f32(vv), bf16hi_to_f32(xs), acc);
+    return acc;
+}
+
+// 32 logical columns: v holds the 8 kept values, e the selector entries of the
+// 4 groups, x the 32 X values of one token.
+__device__ __forceinline__ float chunk28_fma(uint4 v, const uint32_t (&e)[4], const uint4 (&x)[4], float acc) {
+    acc = group28_fma_lut(v.x, e[0], x[0], acc);
+    acc = group28_fma_lut(v.y, e[1], x[1], acc);
+    acc = group28_fma_lut(v.z, e[2], x[2], acc);
+    acc = group28_fma_lut(v.w, e[3], x[3], acc);
     return acc;
 }
 
@@ -66,6 +84,9 @@ __global__ void __launch_bounds__(kWarps28 * 32) decode28_forward_kernel(
     const uint16_t *__restrict__ X, int64_t M, const uint16_t *__restrict__ vals8,
     const uint8_t *__restrict__ meta8, int64_t d_out, int64_t d_in, const uint16_t *__restrict__ U,
     const float *__restrict__ T32, int64_t r, uint16_t *__restrict__ Y) {
+    __shared__ uint32_t lut[64];
+    if (threadIdx.x < 64) lut[threadIdx.x] = selector_entry(threadIdx.x);
+    __syncthreads();
     const int lane = threadIdx.x & 31;
     const int64_t m0 = (int64_t)blockIdx.y * MT;
     const int nt = (int)((M - m0) < MT ? (M - m0) : MT);
@@ -124,14 +145,21 @@ __global__ void __launch_bounds__(kWarps28 * 32) decode28_forward_kernel(
             for (int u = 0; u < kUnrollChunks; ++u) {
                 const int64_t c = c0 + 32 * u;
                 if (c < chunks) {
+                    uint4 x[MT][4];
 #pragma unroll
                     for (int t = 0; t < MT; ++t) {
-                        if (t < nt) {
-                            const uint4 *xr = reinterpret_cast<const uint4 *>(xbase + t * d_in + c * 32);
-                            const uint4 x[4] = {__ldg(xr), __ldg(xr + 1), __ldg(xr + 2), __ldg(xr + 3)};
+                        const uint4 *xr = reinterpret_cast<const uint4 *>(xbase + t * d_in + c * 32);
 #pragma unroll
-                            for (int q = 0; q < RW; ++q) acc[q][t] = chunk28_fma(v[u][q], mm[u][q], x, acc[q][t]);
-                        }
+                        for (int h = 0; h < 4; ++h) x[t][h] = t < nt ? __ldg(xr + h) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int q = 0; q < RW; ++q) {
+                        uint32_t e[4];
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) e[g] = lut[(mm[u][q] >> (8 * g)) & 0x3Fu];
+#pragma unroll
+                        for (int t = 0; t < MT; ++t)
+                            if (t < nt) acc[q][t] = chunk28_fma(v[u][q], e, x[t], acc[q][t]);
                     }
                 }
             }

@@ -22,7 +22,11 @@
 // shared memory and are summed over distributed shared memory (as in the
 // rank projection of the forward), then written once: fp32 row-major,
 // fp32 transposed (dV), or bf16 row-major (G).  Every wait is bounded.
+// dU runs on a second stream beside G and dV (forked and joined with events
+// on the caller's stream).
 #include <cuda.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "tc_forward.cuh"
@@ -283,16 +287,51 @@ cudaError_t gemm_tc(const uint16_t *A, int64_t lda, const uint16_t *B, int64_t l
                               (int32_t)nk);
 }
 
+// A second stream per device, so that dU (which needs only dY and T) runs
+// beside G and dV; created once, never destroyed (it lives as long as the
+// process, like the library's other per-device state).
+cudaStream_t side_stream() {
+    static std::mutex mu;
+    static cudaStream_t streams[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (streams[dev] == nullptr && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+        streams[dev] = nullptr;
+    return streams[dev];
+}
+
 template <int RN>
 cudaError_t backward_rn(const uint16_t *X, int64_t M, const uint16_t *dY, int64_t d_out, int64_t d_in,
                         const uint16_t *U, const uint16_t *T16, uint16_t *G16, int64_t r, float *dU, float *dV,
                         cudaStream_t st) {
-    // G = dY U: A = dY [M][d_out] K-major (K = d_out), B = U [d_out][r] MN-major.
-    cudaError_t e = gemm_tc<false, true, RN, kOutBF16>(dY, d_out, U, r, M, r, d_out, G16, st);
-    // dU = dY^T T: A = dY [M][d_out] MN-major (K = M), B = T [M][r] MN-major.
-    if (e == cudaSuccess) e = gemm_tc<true, true, RN, kOutF32>(dY, d_out, T16, r, d_out, r, M, dU, st);
-    // dV^T = X^T G: A = X [M][d_in] MN-major, B = G [M][r] MN-major; stored transposed as dV [r][d_in].
+    // dU = dY^T T (A = dY [M][d_out] MN-major, K = M; B = T [M][r] MN-major) on
+    // the side stream, forked from and joined back into `st` with events, while
+    // `st` runs G = dY U (A = dY K-major, K = d_out; B = U [d_out][r] MN-major)
+    // and then dV^T = X^T G (A = X [M][d_in] MN-major, B = G [M][r] MN-major,
+    // stored transposed as dV [r][d_in]).  Without a side stream, all on `st`.
+    cudaStream_t side = side_stream();
+    cudaEvent_t fork = nullptr, join = nullptr;
+    if (side != nullptr && (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
+                            cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess)) {
+        if (fork != nullptr) cudaEventDestroy(fork);
+        fork = join = nullptr;
+        side = nullptr;
+    }
+    cudaError_t e = cudaSuccess;
+    cudaStream_t su = st;
+    if (side != nullptr) {
+        e = cudaEventRecord(fork, st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
+        if (e == cudaSuccess) su = side;
+    }
+    if (e == cudaSuccess) e = gemm_tc<true, true, RN, kOutF32>(dY, d_out, T16, r, d_out, r, M, dU, su);
+    if (e == cudaSuccess && side != nullptr) e = cudaEventRecord(join, side);
+    if (e == cudaSuccess) e = gemm_tc<false, true, RN, kOutBF16>(dY, d_out, U, r, M, r, d_out, G16, st);
     if (e == cudaSuccess) e = gemm_tc<true, true, RN, kOutF32T>(X, d_in, G16, r, d_in, r, M, dV, st);
+    if (e == cudaSuccess && side != nullptr) e = cudaStreamWaitEvent(st, join, 0);
+    if (fork != nullptr) cudaEventDestroy(fork);  // released once the recorded work completes
+    if (join != nullptr) cudaEventDestroy(join);
     return e;
 }
 
