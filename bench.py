@@ -665,8 +665,10 @@ def run_decompose_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barr
     Hessian) of the gate/up weight into 2:4 S + rank-64 U V: the start
     (8 power steps from a random subspace) alone, then with 4 iterations of
     2 warm-started power steps; the difference is the per-iteration time.
-    FLOPs per iteration: (4 p + 4) d_out d_in r (p power steps of Z Q and
-    Z^T P, then U = Z Q and the residual W - U V), fp32 on CUDA cores."""
+    Per iteration with p power steps the GPU streams Z = W - S (two bf16
+    planes, 4 B per weight) 2p + 1 times through the tensor-core products,
+    and the residual pass reads W (2 B) and writes Z (4 B) and S (1.125 B):
+    (4 (2p + 1) + 7.125) B per weight, the HBM bound of the iteration."""
     L = layer_of(PREFILL["cfg"], PREFILL["name"])
     d_out, d_in, r, p, iters = L.d_out, L.d_in, 64, 2, 4
     W = to_dev(L.weight())
@@ -685,21 +687,22 @@ def run_decompose_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barr
 
     run(0)
     run(1)  # warm-up
+    slr.check_kernel_error()
     barrier()
     t0 = min(run(0)[0] for _ in range(3))
     runs = [run(iters) for _ in range(3)]
     t1 = min(x[0] for x in runs)
     obj = runs[0][1][4].cpu().numpy()
     ms_iter = max_over_ranks((t1 - t0) / iters)
+    nbytes = (4 * (2 * p + 1) + 7.125) * d_out * d_in
+    gbs = nbytes / (ms_iter * 1e-3) / 1e9
     flops = (4 * p + 4) * d_out * d_in * r
-    # fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
-    peak_fp32 = 148 * 128 * 2 * 1.965e9 / 1e12
-    tf = flops / (ms_iter * 1e-3) / 1e12
     return {"workload": f"data-free alternating minimisation of the {d_out}x{d_in} gate/up weight, 2:4 + rank {r}, "
                         f"{p} warm-started power steps per iteration",
             "ms_start": round(t0, 3), "ms_per_iteration": round(ms_iter, 3), "iterations_timed": iters,
-            "tflops_fp32": round(tf, 2), "peak_fp32_tflops_derived": round(peak_fp32, 1),
-            "frac_of_fp32_peak": round(tf / peak_fp32, 4),
+            "bound": "hbm", "algorithmic_bytes_per_iteration": int(nbytes), "gbs": round(gbs, 1),
+            "frac": round(gbs / peaks["hbm_gbs"], 4),
+            "tflops_effective": round(flops / (ms_iter * 1e-3) / 1e12, 2),
             "objective": [round(float(x), 5) for x in obj]}
 
 

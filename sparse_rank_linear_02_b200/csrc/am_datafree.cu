@@ -14,25 +14,37 @@
 //   span(Q), which converges to C_r(Z) as Q converges to the top-r right
 //   singular subspace.  The random start Q0 is an input.
 //
-// Kernels (fp32 on CUDA cores; the products are tall and skinny, r <= 128):
-//  * gemm_f32_kernel<TRANS_A>: C = A B (A d x k) or C = A^T B, 128 x 64 output
-//    tiles, 16-deep k steps through shared memory, 8 x 4 outputs per thread,
-//    split over k with the partial products summed in a fixed order by
+// Kernels:
+//  * the products P = Z Q, Z^T P and U = Z Q run on the tensor cores
+//    (tc_gemm_kernel, tc_gemm.cuh) with every operand split into two bf16
+//    planes, hi = bf16(x) and lo = bf16(x - hi), and hi*hi + hi*lo + lo*hi
+//    accumulated in fp32: about 16 significant bits per operand, so the
+//    subspace iteration behaves as in fp32.  Z = W - S is kept as its two
+//    planes (written by the residual kernel); Q and P are split before use.
+//  * gemm_f32_kernel<TRANS_A>: C = A B or A^T B in fp32 on CUDA cores, for the
+//    small Gram and basis products of the orthonormalisation (d_in x r x r).
+//    128 x 64 output tiles, 16-deep k steps through shared memory, split over
+//    k with the partial products summed in a fixed order by
 //    reduce_splits_kernel (deterministic).
-//  * chol_inv_kernel: one CTA; G = Q^T Q (from the split partials, in fp64)
-//    -> Cholesky factor L -> M = L^-T, so Q M has orthonormal columns.
+//  * chol_inv_kernel: one CTA; G = Q^T Q (fp64) -> Cholesky factor L ->
+//    M = L^-T, so Q M has orthonormal columns (one barrier per step).
 //  * residual_project_kernel: for a 64 x 128 tile, R = W - P Q^T (K = r
 //    through shared memory), then per group of four the two largest |R| are
 //    kept (ties to the lower index) and written packed (bf16 values, nibble
-//    metadata), Z = W - S is written for the next subspace iteration, and the
-//    tile's sum of (R - S)^2 goes to a per-tile partial of the objective.
+//    metadata), Z = W - S is written (as its two bf16 planes) for the next
+//    subspace iteration, and the tile's sum of (R - S)^2 goes to a per-tile
+//    partial of the objective.
 #include <math.h>
 
 #include <algorithm>
 
-#include "common.cuh"
+#include "tc_gemm.cuh"
 
 namespace slr {
+
+// Error word of the tensor-core products' bounded waits (slr_check_kernel_error).
+__device__ unsigned int g_am_error = 0;
+
 namespace {
 
 constexpr int kGT = 256;   // threads of the GEMM kernels
@@ -163,70 +175,71 @@ __global__ void reduce_splits_kernel(const float *__restrict__ part, int splits,
 // One CTA: G = sum of `splits` partial r x r Gram matrices (fp64), Cholesky
 // G = L L^T (a pivot below 1e-12 of the mean diagonal is raised to it, so a
 // rank-deficient block stays finite), then M = L^-T (fp32, r x r row-major).
-// Shared memory: one r x r fp64 array; L fills the lower triangle and
-// X = L^-1 (also lower triangular) is kept transposed in the strict upper
-// triangle (X[i][c] at [c][i]); its diagonal is 1 / L[i][i].  Both phases are
-// right-looking, so every step is a parallel update of the trailing block:
-//   Cholesky, column j: pivot, scale column j below it, A[i][k] -= L[i][j] L[k][j]
-//   for j < k <= i;  inverse, row i: finalise row i of X (divide by L[i][i]),
-//   then X[i'][c] -= L[i'][i] X[i][c] for i' > i, c <= i.
-__global__ void __launch_bounds__(256) chol_inv_kernel(const float *__restrict__ gpart, int splits, int r,
+// Shared memory: one r x r fp64 array with rows padded to r + 1 (an odd
+// stride, so column accesses do not collide in one bank) and r square roots;
+// L fills the lower triangle and X = L^-1 (also lower triangular) is kept
+// transposed in the strict upper triangle (X[i][c] at [c][i]).
+// The factorisation is a chain of r steps, so the kernel is bound by the
+// barrier between steps; both phases defer their scaling to keep one barrier
+// per step:
+//   Cholesky, column j (d_j = the current A[j][j], floored): for j < k <= i,
+//     A[i][k] -= A[i][j] A[k][j] / d_j; column j is left unscaled, and at the
+//     end L[j][j] = sqrt(d_j), L[i][j] = A[i][j] / sqrt(d_j).
+//   Inverse, row i: with R = the unscaled rows of X (R[i][i] = 1),
+//     R[i'][c] -= (L[i'][i] / L[i][i]) R[i][c] for i' > i, c <= i; at the end
+//     X[i][c] = R[i][c] / L[i][i].
+__global__ void __launch_bounds__(1024) chol_inv_kernel(const float *__restrict__ gpart, int splits, int r,
                                                        float *__restrict__ Mout) {
-    extern __shared__ double A[];
+    extern __shared__ double A[];  // r rows of ld = r + 1, then r square roots
     __shared__ double floor_pivot;
-    const int tid = threadIdx.x, nth = blockDim.x;
+    const int tid = threadIdx.x, nth = blockDim.x, ld = r + 1;
+    const int tx = tid & 31, ty = tid >> 5, ny = nth >> 5;
+    double *sq = A + r * ld;
     for (int i = tid; i < r * r; i += nth) {
         double s = 0.0;
         for (int k = 0; k < splits; ++k) s += (double)gpart[(int64_t)k * r * r + i];
-        A[i] = s;
+        A[(i / r) * ld + i % r] = s;
     }
     __syncthreads();
     if (tid == 0) {
         double tr = 0.0;
-        for (int i = 0; i < r; ++i) tr += A[i * r + i];
+        for (int i = 0; i < r; ++i) tr += A[i * ld + i];
         floor_pivot = 1e-12 * (tr > 0.0 ? tr / r : 1.0);
     }
     __syncthreads();
+    const double fl = floor_pivot;
     for (int j = 0; j < r; ++j) {
-        if (tid == 0) {
-            const double d = A[j * r + j];
-            A[j * r + j] = sqrt(d > floor_pivot ? d : floor_pivot);
-        }
-        __syncthreads();
-        const double piv = A[j * r + j];
-        for (int i = j + 1 + tid; i < r; i += nth) A[i * r + j] /= piv;
-        __syncthreads();
-        const int n = r - j - 1;
-        for (int q = tid; q < n * n; q += nth) {
-            const int ii = q / n, kk = q % n;
-            if (kk <= ii) {
-                const int i = j + 1 + ii, k = j + 1 + kk;
-                A[i * r + k] -= A[i * r + j] * A[k * r + j];
-            }
+        const double d = A[j * ld + j];
+        const double inv2 = 1.0 / (d > fl ? d : fl);
+        for (int i = j + 1 + ty; i < r; i += ny) {
+            const double f = A[i * ld + j] * inv2;
+            for (int k = j + 1 + tx; k <= i; k += 32) A[i * ld + k] -= f * A[k * ld + j];
         }
         __syncthreads();
     }
-    for (int q = tid; q < r * r; q += nth)
-        if (q % r > q / r) A[q] = 0.0;  // strict upper triangle: X starts as the identity
+    for (int j = tid; j < r; j += nth) {
+        const double d = A[j * ld + j];
+        sq[j] = sqrt(d > fl ? d : fl);
+    }
+    __syncthreads();
+    for (int i = ty; i < r; i += ny)
+        for (int c = tx; c < r; c += 32)
+            A[i * ld + c] = c < i ? A[i * ld + c] / sq[c] : (c == i ? sq[i] : 0.0);  // L, and R = I above
     __syncthreads();
     for (int i = 0; i < r; ++i) {
-        const double dinv = 1.0 / A[i * r + i];
-        for (int c = tid; c < i; c += nth) A[c * r + i] *= dinv;
-        __syncthreads();
-        const int n = r - i - 1, m = i + 1;
-        for (int q = tid; q < n * m; q += nth) {
-            const int ii = i + 1 + q / m, c = q % m;
-            const double xic = (c == i) ? dinv : A[c * r + i];
-            A[c * r + ii] -= A[ii * r + i] * xic;
+        const double inv_lii = 1.0 / sq[i];
+        for (int ii = i + 1 + ty; ii < r; ii += ny) {
+            const double f = A[ii * ld + i] * inv_lii;
+            for (int c = tx; c <= i; c += 32) A[c * ld + ii] -= f * ((c == i) ? 1.0 : A[c * ld + i]);
         }
         __syncthreads();
     }
-    for (int i = tid; i < r * r; i += nth) {
-        const int k = i / r, c = i % r;  // M[k][c] = X[c][k]
+    for (int q = tid; q < r * r; q += nth) {
+        const int k = q / r, c = q % r;  // M[k][c] = X[c][k] = R[c][k] / L[c][c]
         float v = 0.f;
-        if (c == k) v = (float)(1.0 / A[k * r + k]);
-        else if (c > k) v = (float)A[k * r + c];
-        Mout[i] = v;
+        if (c == k) v = (float)(1.0 / sq[k]);
+        else if (c > k) v = (float)(A[k * ld + c] / sq[c]);
+        Mout[q] = v;
     }
 }
 
@@ -265,7 +278,8 @@ __global__ void __launch_bounds__(256) residual_project_kernel(const uint16_t *_
                                                                const float *__restrict__ P,
                                                                const float *__restrict__ Q, int64_t d_out,
                                                                int64_t d_in, int r, uint16_t *__restrict__ vals,
-                                                               uint8_t *__restrict__ meta, float *__restrict__ Z,
+                                                               uint8_t *__restrict__ meta,
+                                                               uint16_t *__restrict__ Zhi, uint16_t *__restrict__ Zlo,
                                                                float *__restrict__ obj_part) {
     __shared__ __align__(16) float Ps[kRBK][kRBM];
     __shared__ __align__(16) float Qs[kRBK][kRBN];
@@ -360,9 +374,17 @@ __global__ void __launch_bounds__(256) residual_project_kernel(const uint16_t *_
             const float e = R[p] - S[p];
             obj = fmaf(e, e, obj);
         }
-        float4 *zp = reinterpret_cast<float4 *>(Z + gr * d_in + gc);
-        zp[0] = make_float4(zr[0], zr[1], zr[2], zr[3]);
-        zp[1] = make_float4(zr[4], zr[5], zr[6], zr[7]);
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const uint32_t h0 = f32_to_bf16_bits(zr[2 * h]), h1 = f32_to_bf16_bits(zr[2 * h + 1]);
+            const uint32_t l0 = f32_to_bf16_bits(zr[2 * h] - __uint_as_float(h0 << 16));
+            const uint32_t l1 = f32_to_bf16_bits(zr[2 * h + 1] - __uint_as_float(h1 << 16));
+            hw[h] = h0 | (h1 << 16);
+            lw[h] = l0 | (l1 << 16);
+        }
+        *reinterpret_cast<uint4 *>(Zhi + gr * d_in + gc) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4 *>(Zlo + gr * d_in + gc) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) obj += __shfl_xor_sync(0xFFFFFFFFu, obj, o);
@@ -389,9 +411,15 @@ __global__ void objective_finish_kernel(const float *__restrict__ part, int64_t 
     }
 }
 
-__global__ void bf16_to_f32_kernel(const uint16_t *__restrict__ in, int64_t n, float *__restrict__ out) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        out[i] = __uint_as_float((uint32_t)in[i] << 16);
+// hi = bf16(x), lo = bf16(x - hi), elementwise.
+__global__ void split_bf16_kernel(const float *__restrict__ in, int64_t n, uint16_t *__restrict__ hi,
+                                  uint16_t *__restrict__ lo) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float x = in[i];
+        const uint16_t h = f32_to_bf16_bits(x);
+        hi[i] = h;
+        lo[i] = f32_to_bf16_bits(x - __uint_as_float((uint32_t)h << 16));
+    }
 }
 
 // U = bf16(P) [d_out, r]; V[k][j] = bf16(Q[j][k]) [r, d_in].
@@ -420,31 +448,22 @@ int grid_cap(int64_t n, int threads) {
 
 AmPlan am_plan(int64_t d_out, int64_t d_in, int64_t r) {
     AmPlan p{};
-    auto splits_for = [](int64_t tiles, int64_t kdim) {
-        // about two CTAs per SM, each split at least 256 deep
-        int64_t s = (2 * 148 + tiles - 1) / tiles;
-        const int64_t kmax = (kdim + 255) / 256;
-        if (s > kmax) s = kmax;
-        if (s > 32) s = 32;
-        return s < 1 ? int64_t(1) : s;
-    };
-    const int64_t ctiles = (r + kGBN - 1) / kGBN;
-    p.split_nn = splits_for(((d_out + kGBM - 1) / kGBM) * ctiles, d_in);    // P = Z Q
-    p.split_tn = splits_for(((d_in + kGBM - 1) / kGBM) * ctiles, d_out);    // Z^T P
-    p.split_gram = splits_for(ctiles, d_in);                                  // Q^T Q
-    p.split_mul = 1;                                                          // Q M (k = r)
-    const int64_t part = std::max({p.split_nn * d_out * r, p.split_tn * d_in * r, p.split_gram * r * r,
-                                   d_in * r});
+    // The Gram matrix Q^T Q (r x r, k = d_in) is split over k, 64 rows of Q
+    // per CTA (at most 128 CTAs); its partials live in `part`.
+    int64_t sg = (d_in + 63) / 64;
+    p.split_gram = sg > 128 ? 128 : (sg < 1 ? 1 : sg);
+    const int64_t part = p.split_gram * r * r;
     p.tiles_res = ((d_in + kRBN - 1) / kRBN) * ((d_out + kRBM - 1) / kRBM);
     auto al = [](int64_t b) { return (b + 255) / 256 * 256; };
-    p.off_Z = 0;
-    p.off_Q = p.off_Z + al(d_out * d_in * 4);
+    p.off_Z = 0;                                   // Zhi then Zlo, bf16 d_out x d_in each
+    p.off_Q = p.off_Z + 2 * al(d_out * d_in * 2);
     p.off_Q2 = p.off_Q + al(d_in * r * 4);
     p.off_P = p.off_Q2 + al(d_in * r * 4);
     p.off_M = p.off_P + al(d_out * r * 4);
     p.off_part = p.off_M + al(r * r * 4);
     p.off_obj = p.off_part + al(part * 4);
-    p.bytes = p.off_obj + al(p.tiles_res * 4);
+    p.off_split = p.off_obj + al(p.tiles_res * 4);  // hi and lo planes of Q or P (bf16, max(d_in, d_out) x r)
+    p.bytes = p.off_split + 2 * al(std::max(d_in, d_out) * r * 2);
     return p;
 }
 
@@ -469,13 +488,14 @@ cudaError_t gemm(bool trans_a, const float *A, int64_t lda, const float *B, int6
 cudaError_t orthonormalise(float *Q, float *tmp, float *M, float *part, int64_t d_in, int r, int64_t split_gram,
                            cudaStream_t st) {
     for (int pass = 0; pass < 2; ++pass) {  // CholeskyQR2
-        int64_t kps = (d_in + split_gram - 1) / split_gram;
-        kps = (kps + kGBK - 1) / kGBK * kGBK;
-        const int64_t used = (d_in + kps - 1) / kps;
-        dim3 grid(1, (unsigned)((r + kGBN - 1) / kGBN), (unsigned)used);
-        gemm_f32_kernel<true><<<grid, kGT, 0, st>>>(Q, r, Q, r, part, r, r, d_in, kps);
-        chol_inv_kernel<<<1, 256, (size_t)r * r * sizeof(double), st>>>(part, (int)used, r, M);
-        cudaError_t e = gemm(false, Q, r, M, r, tmp, part, d_in, r, r, 1, st);
+        // G = Q^T Q into the first r x r floats of tmp (split over d_in, the
+        // splits summed in a fixed order), then L^-T, then tmp = Q L^-T.
+        cudaError_t e = gemm(true, Q, r, Q, r, tmp, part, r, r, d_in, split_gram, st);
+        if (e != cudaSuccess) return e;
+        // 32 warps: each step's trailing update gives a warp one or two rows,
+        // which keeps the per-step chain short (the kernel is latency-bound).
+        chol_inv_kernel<<<1, 1024, (size_t)r * (r + 2) * sizeof(double), st>>>(tmp, 1, r, M);
+        e = gemm(false, Q, r, M, r, tmp, part, d_in, r, r, 1, st);
         if (e != cudaSuccess) return e;
         e = cudaMemcpyAsync(Q, tmp, (size_t)d_in * r * sizeof(float), cudaMemcpyDeviceToDevice, st);
         if (e != cudaSuccess) return e;
@@ -483,43 +503,86 @@ cudaError_t orthonormalise(float *Q, float *tmp, float *M, float *part, int64_t 
     return cudaGetLastError();
 }
 
+
+// Device address of g_am_error on the current device.
+unsigned int *am_err() {
+    static unsigned int *addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (addr[dev] == nullptr) {
+        void *q = nullptr;
+        if (cudaGetSymbolAddress(&q, g_am_error) == cudaSuccess) addr[dev] = static_cast<unsigned int *>(q);
+    }
+    return addr[dev];
+}
+
+// C (rows x r, fp32) = Z B (B: d_in x r) or Z^T B (B: d_out x r) on the tensor
+// cores, with Z and B in hi/lo bf16 planes; B (fp32) is split into bh/bl first.
+cudaError_t split_product(bool transpose_z, const uint16_t *Zhi, const uint16_t *Zlo, int64_t d_out, int64_t d_in,
+                          const float *B, uint16_t *bh, uint16_t *bl, int r, float *C, cudaStream_t st) {
+    const int64_t kdim = transpose_z ? d_out : d_in, rows = transpose_z ? d_in : d_out;
+    split_bf16_kernel<<<grid_cap(kdim * r, 256), 256, 0, st>>>(B, kdim * r, bh, bl);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (r <= 64)
+        return transpose_z ? gemm_tc<true, true, 64, kOutF32, true>(Zhi, Zlo, d_in, bh, bl, r, rows, r, kdim, C, am_err(), st)
+                           : gemm_tc<false, true, 64, kOutF32, true>(Zhi, Zlo, d_in, bh, bl, r, rows, r, kdim, C, am_err(), st);
+    return transpose_z ? gemm_tc<true, true, 128, kOutF32, true>(Zhi, Zlo, d_in, bh, bl, r, rows, r, kdim, C, am_err(), st)
+                       : gemm_tc<false, true, 128, kOutF32, true>(Zhi, Zlo, d_in, bh, bl, r, rows, r, kdim, C, am_err(), st);
+}
+
 }  // namespace
+
+cudaError_t read_and_clear_am_error(unsigned *code) {
+    unsigned v = 0;
+    cudaError_t err = cudaMemcpyFromSymbol(&v, g_am_error, sizeof v);
+    if (err != cudaSuccess) return err;
+    if (v != 0) {
+        const unsigned zero = 0;
+        err = cudaMemcpyToSymbol(g_am_error, &zero, sizeof zero);
+    }
+    *code = v;
+    return err;
+}
 
 cudaError_t launch_am_datafree(const uint16_t *W, int64_t d_out, int64_t d_in, int r, int iters, int power0,
                                int power, const float *Q0, uint16_t *vals, uint8_t *meta, uint16_t *U, uint16_t *V,
                                double *objective, uint8_t *ws, cudaStream_t st) {
     const AmPlan p = am_plan(d_out, d_in, r);
-    float *Z = reinterpret_cast<float *>(ws + p.off_Z);
+    uint16_t *Zhi = reinterpret_cast<uint16_t *>(ws + p.off_Z);
+    uint16_t *Zlo = Zhi + (p.off_Q - p.off_Z) / 4;  // second half of the Z region
     float *Q = reinterpret_cast<float *>(ws + p.off_Q);
     float *Q2 = reinterpret_cast<float *>(ws + p.off_Q2);
     float *P = reinterpret_cast<float *>(ws + p.off_P);
     float *M = reinterpret_cast<float *>(ws + p.off_M);
     float *part = reinterpret_cast<float *>(ws + p.off_part);
     float *objp = reinterpret_cast<float *>(ws + p.off_obj);
+    uint16_t *bh = reinterpret_cast<uint16_t *>(ws + p.off_split);
+    uint16_t *bl = bh + (p.bytes - p.off_split) / 4;
     static bool smem_set = false;
     if (!smem_set) {
-        cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 128 * 8);
+        cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 130 * 8);
         smem_set = true;
     }
     cudaError_t e = cudaSuccess;
-    // Start: S = 0, so Z = W; Q = orth(Q0).
-    bf16_to_f32_kernel<<<grid_cap(d_out * d_in, 256), 256, 0, st>>>(W, d_out * d_in, Z);
-    e = cudaMemcpyAsync(Q, Q0, (size_t)d_in * r * sizeof(float), cudaMemcpyDeviceToDevice, st);
-    if (e != cudaSuccess) return e;
-    e = orthonormalise(Q, Q2, M, part, d_in, r, p.split_gram, st);
+    // Start: S = 0, so Z = W (hi = W, lo = 0); Q = orth(Q0).
+    e = cudaMemcpyAsync(Zhi, W, (size_t)d_out * d_in * 2, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(Zlo, 0, (size_t)d_out * d_in * 2, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(Q, Q0, (size_t)d_in * r * sizeof(float), cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = orthonormalise(Q, Q2, M, part, d_in, r, p.split_gram, st);
     const dim3 rgrid((unsigned)((d_in + kRBN - 1) / kRBN), (unsigned)((d_out + kRBM - 1) / kRBM));
     for (int t = 0; t <= iters && e == cudaSuccess; ++t) {
         // P2: subspace iteration on Z, then U = Z Q.
         const int steps = t == 0 ? power0 : power;
         for (int s = 0; s < steps && e == cudaSuccess; ++s) {
-            e = gemm(false, Z, d_in, Q, r, P, part, d_out, r, d_in, p.split_nn, st);            // P = Z Q
-            if (e == cudaSuccess) e = gemm(true, Z, d_in, P, r, Q, part, d_in, r, d_out, p.split_tn, st);  // Q = Z^T P
+            e = split_product(false, Zhi, Zlo, d_out, d_in, Q, bh, bl, r, P, st);                // P = Z Q
+            if (e == cudaSuccess) e = split_product(true, Zhi, Zlo, d_out, d_in, P, bh, bl, r, Q, st);  // Q = Z^T P
             if (e == cudaSuccess) e = orthonormalise(Q, Q2, M, part, d_in, r, p.split_gram, st);
         }
-        if (e == cudaSuccess) e = gemm(false, Z, d_in, Q, r, P, part, d_out, r, d_in, p.split_nn, st);  // U = Z Q
+        if (e == cudaSuccess) e = split_product(false, Zhi, Zlo, d_out, d_in, Q, bh, bl, r, P, st);  // U = Z Q
         if (e != cudaSuccess) break;
         // P1: S = 2:4 threshold of W - U V, Z = W - S, objective.
-        residual_project_kernel<<<rgrid, 256, 0, st>>>(W, P, Q, d_out, d_in, r, vals, meta, Z, objp);
+        residual_project_kernel<<<rgrid, 256, 0, st>>>(W, P, Q, d_out, d_in, r, vals, meta, Zhi, Zlo, objp);
         if (objective != nullptr) objective_finish_kernel<<<1, 256, 0, st>>>(objp, p.tiles_res, objective + t);
         e = cudaGetLastError();
     }

@@ -333,11 +333,12 @@ slr_path slr_forward_select_path(int64_t M, int64_t d_out, int64_t d_in, int64_t
 slr_status slr_check_kernel_error(void) {
     if (slr::check_device() != SLR_OK) return SLR_ERR_DEVICE;
     if (cudaDeviceSynchronize() != cudaSuccess) return SLR_ERR_CUDA;
-    unsigned code = 0, code28 = 0, code_bwd = 0;
+    unsigned code = 0, code28 = 0, code_bwd = 0, code_am = 0;
     if (slr::read_and_clear_kernel_error(&code) != cudaSuccess) return SLR_ERR_CUDA;
     if (slr::read_and_clear_decode28_error(&code28) != cudaSuccess) return SLR_ERR_CUDA;
     if (slr::read_and_clear_backward_error(&code_bwd) != cudaSuccess) return SLR_ERR_CUDA;
-    return (code | code28 | code_bwd) ? SLR_ERR_TIMEOUT : SLR_OK;
+    if (slr::read_and_clear_am_error(&code_am) != cudaSuccess) return SLR_ERR_CUDA;
+    return (code | code28 | code_bwd | code_am) ? SLR_ERR_TIMEOUT : SLR_OK;
 }
 
 slr_status slr_selftest_wait_timeout(int64_t limit_cycles, slr_stream_t stream) {

@@ -53,15 +53,18 @@ cudaError_t launch_decode28_forward(const uint16_t *X, int64_t M, const uint16_t
                                     int64_t d_out, int64_t d_in, const uint16_t *U, const float *T32, int64_t r,
                                     uint16_t *Y, bool after_projection, cudaStream_t stream);
 
+// Reads and clears the error word of the decomposition's tensor-core products.
+cudaError_t read_and_clear_am_error(unsigned *code);
+
 // Reads and clears the error word of the 2:8 ring kernel's bounded waits.
 cudaError_t read_and_clear_decode28_error(unsigned *code);
 
 // Data-free alternating minimisation: workspace layout (byte offsets) and the
 // split counts of its products.
 struct AmPlan {
-    int64_t split_nn, split_tn, split_gram, split_mul;
+    int64_t split_gram;
     int64_t tiles_res;
-    int64_t off_Z, off_Q, off_Q2, off_P, off_M, off_part, off_obj, bytes;
+    int64_t off_Z, off_Q, off_Q2, off_P, off_M, off_part, off_obj, off_split, bytes;
 };
 AmPlan am_plan(int64_t d_out, int64_t d_in, int64_t r);
 
