@@ -559,12 +559,10 @@ cudaError_t launch_am_datafree(const uint16_t *W, int64_t d_out, int64_t d_in, i
     float *objp = reinterpret_cast<float *>(ws + p.off_obj);
     uint16_t *bh = reinterpret_cast<uint16_t *>(ws + p.off_split);
     uint16_t *bl = bh + (p.bytes - p.off_split) / 4;
-    static bool smem_set = false;
-    if (!smem_set) {
-        cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 130 * 8);
-        smem_set = true;
-    }
-    cudaError_t e = cudaSuccess;
+    // Set on every call: the attribute belongs to the current device's copy of the kernel.
+    cudaError_t e = cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)((size_t)r * (r + 2) * sizeof(double)));
+    if (e != cudaSuccess) return e;
     // Start: S = 0, so Z = W (hi = W, lo = 0); Q = orth(Q0).
     e = cudaMemcpyAsync(Zhi, W, (size_t)d_out * d_in * 2, cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(Zlo, 0, (size_t)d_out * d_in * 2, st);

@@ -406,7 +406,9 @@ cudaError_t launch28(const uint16_t *X, int64_t M, const uint16_t *vals8, const 
                      bool after_projection, cudaStream_t stream) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    static int per_sm = 0;  // resident CTAs per SM, asked once per instantiation
+    // Resident CTAs per SM, asked once per instantiation (a property of the
+    // compiled kernel and the sm_100 architecture, the same on every B200).
+    static int per_sm = 0;
     if (per_sm == 0) {
         int n = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode28_forward_kernel<MT, RW>, kWarps28 * 32, 0) !=
@@ -497,13 +499,10 @@ cudaError_t launch_ring28(const uint16_t *X, int64_t M, const uint16_t *vals8, c
     p.nst = (int32_t)nst;
     const size_t smem = (size_t)p.nst * p.slot + 2 * (size_t)p.nst * sizeof(uint64_t) +
                         (size_t)kCWarps * RW * MT * sizeof(float) + 16;
-    static size_t smem_set = 0;  // largest dynamic shared memory enabled so far for this instantiation
-    if (smem > smem_set) {
-        const cudaError_t e = cudaFuncSetAttribute(decode28_ring_kernel<MT, RW>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        smem_set = smem;
-    }
+    // Set on every call: the attribute belongs to the current device's copy of the kernel.
+    const cudaError_t e = cudaFuncSetAttribute(decode28_ring_kernel<MT, RW>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     int64_t grid = (int64_t)sms * kRingCtasPerSm;
     if (grid > p.n_rb) grid = p.n_rb;
     cudaLaunchConfig_t cfg = {};
