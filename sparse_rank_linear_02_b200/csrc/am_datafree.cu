@@ -486,8 +486,8 @@ cudaError_t gemm(bool trans_a, const float *A, int64_t lda, const float *B, int6
 
 // Q (d_in x r) <- Q L^-T with L the Cholesky factor of Q^T Q; tmp is d_in x r.
 cudaError_t orthonormalise(float *Q, float *tmp, float *M, float *part, int64_t d_in, int r, int64_t split_gram,
-                           cudaStream_t st) {
-    for (int pass = 0; pass < 2; ++pass) {  // CholeskyQR2
+                           int passes, cudaStream_t st) {
+    for (int pass = 0; pass < passes; ++pass) {  // 2: CholeskyQR2
         // G = Q^T Q into the first r x r floats of tmp (split over d_in, the
         // splits summed in a fixed order), then L^-T, then tmp = Q L^-T.
         cudaError_t e = gemm(true, Q, r, Q, r, tmp, part, r, r, d_in, split_gram, st);
@@ -567,7 +567,7 @@ cudaError_t launch_am_datafree(const uint16_t *W, int64_t d_out, int64_t d_in, i
     e = cudaMemcpyAsync(Zhi, W, (size_t)d_out * d_in * 2, cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(Zlo, 0, (size_t)d_out * d_in * 2, st);
     if (e == cudaSuccess) e = cudaMemcpyAsync(Q, Q0, (size_t)d_in * r * sizeof(float), cudaMemcpyDeviceToDevice, st);
-    if (e == cudaSuccess) e = orthonormalise(Q, Q2, M, part, d_in, r, p.split_gram, st);
+    if (e == cudaSuccess) e = orthonormalise(Q, Q2, M, part, d_in, r, p.split_gram, 2, st);
     const dim3 rgrid((unsigned)((d_in + kRBN - 1) / kRBN), (unsigned)((d_out + kRBM - 1) / kRBM));
     for (int t = 0; t <= iters && e == cudaSuccess; ++t) {
         // P2: subspace iteration on Z, then U = Z Q.
@@ -575,7 +575,11 @@ cudaError_t launch_am_datafree(const uint16_t *W, int64_t d_out, int64_t d_in, i
         for (int s = 0; s < steps && e == cudaSuccess; ++s) {
             e = split_product(false, Zhi, Zlo, d_out, d_in, Q, bh, bl, r, P, st);                // P = Z Q
             if (e == cudaSuccess) e = split_product(true, Zhi, Zlo, d_out, d_in, P, bh, bl, r, Q, st);  // Q = Z^T P
-            if (e == cudaSuccess) e = orthonormalise(Q, Q2, M, part, d_in, r, p.split_gram, st);
+            // Between power steps one Cholesky-QR pass keeps the basis well
+            // conditioned; the last step's basis, which defines U V = Z Q Q^T,
+            // gets the second pass (CholeskyQR2) so that it is orthonormal to
+            // working precision.
+            if (e == cudaSuccess) e = orthonormalise(Q, Q2, M, part, d_in, r, p.split_gram, s + 1 < steps ? 1 : 2, st);
         }
         if (e == cudaSuccess) e = split_product(false, Zhi, Zlo, d_out, d_in, Q, bh, bl, r, P, st);  // U = Z Q
         if (e != cudaSuccess) break;
