@@ -28,12 +28,12 @@
 //    reduce_splits_kernel (deterministic).
 //  * chol_inv_kernel: one CTA; G = Q^T Q (fp64) -> Cholesky factor L ->
 //    M = L^-T, so Q M has orthonormal columns (one barrier per step).
-//  * residual_project_kernel: for a 64 x 128 tile, R = W - P Q^T (K = r
-//    through shared memory), then per group of four the two largest |R| are
-//    kept (ties to the lower index) and written packed (bf16 values, nibble
-//    metadata), Z = W - S is written (as its two bf16 planes) for the next
-//    subspace iteration, and the tile's sum of (R - S)^2 goes to a per-tile
-//    partial of the objective.
+//  * P1 is the same tensor-core product P Q^T (split planes, K = r) with the
+//    threshold in its epilogue (tc_gemm_kernel's residual mode): per group of
+//    four columns R = W - P Q^T, the two largest |R| kept (ties to the lower
+//    index) and written packed (bf16 values, nibble metadata), Z = W - S
+//    written as its two bf16 planes for the next subspace iteration, and the
+//    CTA's sum of (R - S)^2 as a partial of the objective.
 #include <math.h>
 
 #include <algorithm>
@@ -243,160 +243,6 @@ __global__ void __launch_bounds__(1024) chol_inv_kernel(const float *__restrict_
     }
 }
 
-// The two positions of a group of four kept by |value| (ties to the lower
-// index), from the fp32 magnitudes' bit patterns: the tournament of (0,1) and
-// (2,3), the better winner first, then the better of the winning pair's loser
-// and the losing pair's winner.  Returns idx0 | idx1 << 2.
-__device__ __forceinline__ uint32_t keep_two(float v0, float v1, float v2, float v3) {
-    const uint32_t k0 = __float_as_uint(fabsf(v0)), k1 = __float_as_uint(fabsf(v1));
-    const uint32_t k2 = __float_as_uint(fabsf(v2)), k3 = __float_as_uint(fabsf(v3));
-    const bool b01 = k0 >= k1, b23 = k2 >= k3;
-    const uint32_t hi01 = max(k0, k1), lo01 = min(k0, k1), hi23 = max(k2, k3), lo23 = min(k2, k3);
-    const uint32_t win01 = b01 ? 0u : 1u, los01 = b01 ? 1u : 0u;
-    const uint32_t win23 = b23 ? 2u : 3u, los23 = b23 ? 3u : 2u;
-    uint32_t first, second;
-    if (hi01 >= hi23) {
-        first = win01;
-        second = lo01 >= hi23 ? los01 : win23;
-    } else {
-        first = win23;
-        second = hi01 >= lo23 ? win01 : los23;
-    }
-    return min(first, second) | (max(first, second) << 2);
-}
-
-constexpr int kRBM = 64;   // residual tile rows
-constexpr int kRBN = 128;  // residual tile columns
-constexpr int kRBK = 16;
-
-// R = W - P Q^T on a 64 x 128 tile (P: d_out x r, Q: d_in x r, fp32), then the
-// 2:4 projection of R, the packed S, Z = W - S and the tile's sum of (R - S)^2.
-// Thread layout: 16 x 16; a thread owns 4 rows x 8 consecutive columns (two
-// groups of four per row).  d_in % 128 == 0 is not required (columns are
-// guarded); d_in % 8 == 0 is.
-__global__ void __launch_bounds__(256) residual_project_kernel(const uint16_t *__restrict__ W,
-                                                               const float *__restrict__ P,
-                                                               const float *__restrict__ Q, int64_t d_out,
-                                                               int64_t d_in, int r, uint16_t *__restrict__ vals,
-                                                               uint8_t *__restrict__ meta,
-                                                               uint16_t *__restrict__ Zhi, uint16_t *__restrict__ Zlo,
-                                                               float *__restrict__ obj_part) {
-    __shared__ __align__(16) float Ps[kRBK][kRBM];
-    __shared__ __align__(16) float Qs[kRBK][kRBN];
-    __shared__ float red[8];
-    const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
-    const int64_t r0 = (int64_t)blockIdx.y * kRBM, c0 = (int64_t)blockIdx.x * kRBN;
-    float acc[4][8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-    for (int k0 = 0; k0 < r; k0 += kRBK) {
-        // Ps[k][row]: 64 rows x 16 k = 1024 floats, one 16-byte load per
-        // thread.  r % 8 == 0, so a 4-wide piece starting below r lies wholly
-        // inside the row (and is 16-byte aligned); pieces at or past r are zero.
-        {
-            const int row = tid / 4, kq = (tid % 4) * 4;
-            const int64_t gr = r0 + row;
-            const float4 v = (gr < d_out && k0 + kq < r) ? *reinterpret_cast<const float4 *>(P + gr * r + k0 + kq)
-                                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-            Ps[kq + 0][row] = v.x;
-            Ps[kq + 1][row] = v.y;
-            Ps[kq + 2][row] = v.z;
-            Ps[kq + 3][row] = v.w;
-        }
-        // Qs[k][col]: 128 cols x 16 k = 2048 floats, two 16-byte loads per thread.
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int idx = tid + h * 256;
-            const int col = idx / 4, kq = (idx % 4) * 4;
-            const int64_t gc = c0 + col;
-            const float4 v = (gc < d_in && k0 + kq < r) ? *reinterpret_cast<const float4 *>(Q + gc * r + k0 + kq)
-                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-            Qs[kq + 0][col] = v.x;
-            Qs[kq + 1][col] = v.y;
-            Qs[kq + 2][col] = v.z;
-            Qs[kq + 3][col] = v.w;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int kk = 0; kk < kRBK; ++kk) {
-            const float4 p = *reinterpret_cast<const float4 *>(&Ps[kk][ty * 4]);
-            const float4 q0 = *reinterpret_cast<const float4 *>(&Qs[kk][tx * 8]);
-            const float4 q1 = *reinterpret_cast<const float4 *>(&Qs[kk][tx * 8 + 4]);
-            const float pa[4] = {p.x, p.y, p.z, p.w};
-            const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(pa[i], qa[j], acc[i][j]);
-        }
-        __syncthreads();
-    }
-    float obj = 0.f;
-    const int64_t gc = c0 + tx * 8;
-    const int64_t meta_row = (d_in / 4 + 1) / 2;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t gr = r0 + ty * 4 + i;
-        if (gr >= d_out || gc >= d_in) continue;
-        const uint4 w = *reinterpret_cast<const uint4 *>(W + gr * d_in + gc);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-        float R[8], S[8];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            R[2 * h] = bf16lo_to_f32(ww[h]) - acc[i][2 * h];
-            R[2 * h + 1] = bf16hi_to_f32(ww[h]) - acc[i][2 * h + 1];
-        }
-        uint32_t byte = 0, kept[2];
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-            const uint32_t nib = keep_two(R[4 * g], R[4 * g + 1], R[4 * g + 2], R[4 * g + 3]);
-            const uint32_t a = nib & 3u, b = nib >> 2;  // a in 0..2, b in 1..3
-            uint32_t sv[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                sv[p] = f32_to_bf16_bits(R[4 * g + p]);
-                S[4 * g + p] = (p == (int)a || p == (int)b) ? __uint_as_float(sv[p] << 16) : 0.f;
-            }
-            const uint32_t sa = a == 0u ? sv[0] : (a == 1u ? sv[1] : sv[2]);
-            const uint32_t sb = b == 1u ? sv[1] : (b == 2u ? sv[2] : sv[3]);
-            kept[g] = sa | (sb << 16);
-            byte |= nib << (4 * g);
-        }
-        *reinterpret_cast<uint2 *>(vals + gr * (d_in / 2) + gc / 2) = make_uint2(kept[0], kept[1]);
-        meta[gr * meta_row + gc / 8] = (uint8_t)byte;
-        float zr[8];
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            const float wv = (p & 1) ? bf16hi_to_f32(ww[p / 2]) : bf16lo_to_f32(ww[p / 2]);
-            zr[p] = wv - S[p];
-            const float e = R[p] - S[p];
-            obj = fmaf(e, e, obj);
-        }
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const uint32_t h0 = f32_to_bf16_bits(zr[2 * h]), h1 = f32_to_bf16_bits(zr[2 * h + 1]);
-            const uint32_t l0 = f32_to_bf16_bits(zr[2 * h] - __uint_as_float(h0 << 16));
-            const uint32_t l1 = f32_to_bf16_bits(zr[2 * h + 1] - __uint_as_float(h1 << 16));
-            hw[h] = h0 | (h1 << 16);
-            lw[h] = l0 | (l1 << 16);
-        }
-        *reinterpret_cast<uint4 *>(Zhi + gr * d_in + gc) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4 *>(Zlo + gr * d_in + gc) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) obj += __shfl_xor_sync(0xFFFFFFFFu, obj, o);
-    if ((tid & 31) == 0) red[tid >> 5] = obj;
-    __syncthreads();
-    if (tid == 0) {
-        float s = 0.f;
-        for (int k = 0; k < 8; ++k) s += red[k];
-        obj_part[(int64_t)blockIdx.y * gridDim.x + blockIdx.x] = s;
-    }
-}
-
 // objective[t] = sqrt(sum of the tile partials), summed in fp64 in tile order.
 __global__ void objective_finish_kernel(const float *__restrict__ part, int64_t n, double *__restrict__ out) {
     __shared__ double red[256];
@@ -453,7 +299,7 @@ AmPlan am_plan(int64_t d_out, int64_t d_in, int64_t r) {
     int64_t sg = (d_in + 63) / 64;
     p.split_gram = sg > 128 ? 128 : (sg < 1 ? 1 : sg);
     const int64_t part = p.split_gram * r * r;
-    p.tiles_res = ((d_in + kRBN - 1) / kRBN) * ((d_out + kRBM - 1) / kRBM);
+    p.tiles_res = ((d_in + 127) / 128) * ((d_out + 127) / 128);  // CTAs of the fused residual product
     auto al = [](int64_t b) { return (b + 255) / 256 * 256; };
     p.off_Z = 0;                                   // Zhi then Zlo, bf16 d_out x d_in each
     p.off_Q = p.off_Z + 2 * al(d_out * d_in * 2);
@@ -463,7 +309,8 @@ AmPlan am_plan(int64_t d_out, int64_t d_in, int64_t r) {
     p.off_part = p.off_M + al(r * r * 4);
     p.off_obj = p.off_part + al(part * 4);
     p.off_split = p.off_obj + al(p.tiles_res * 4);  // hi and lo planes of Q or P (bf16, max(d_in, d_out) x r)
-    p.bytes = p.off_split + 2 * al(std::max(d_in, d_out) * r * 2);
+    p.off_split2 = p.off_split + 2 * al(std::max(d_in, d_out) * r * 2);  // hi and lo planes of Q (d_in x r)
+    p.bytes = p.off_split2 + 2 * al(d_in * r * 2);
     return p;
 }
 
@@ -558,7 +405,9 @@ cudaError_t launch_am_datafree(const uint16_t *W, int64_t d_out, int64_t d_in, i
     float *part = reinterpret_cast<float *>(ws + p.off_part);
     float *objp = reinterpret_cast<float *>(ws + p.off_obj);
     uint16_t *bh = reinterpret_cast<uint16_t *>(ws + p.off_split);
-    uint16_t *bl = bh + (p.bytes - p.off_split) / 4;
+    uint16_t *bl = bh + (p.off_split2 - p.off_split) / 4;
+    uint16_t *qh = reinterpret_cast<uint16_t *>(ws + p.off_split2);
+    uint16_t *ql = qh + (p.bytes - p.off_split2) / 4;
     // Set on every call: the attribute belongs to the current device's copy of the kernel.
     cudaError_t e = cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)((size_t)r * (r + 2) * sizeof(double)));
@@ -568,7 +417,6 @@ cudaError_t launch_am_datafree(const uint16_t *W, int64_t d_out, int64_t d_in, i
     if (e == cudaSuccess) e = cudaMemsetAsync(Zlo, 0, (size_t)d_out * d_in * 2, st);
     if (e == cudaSuccess) e = cudaMemcpyAsync(Q, Q0, (size_t)d_in * r * sizeof(float), cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess) e = orthonormalise(Q, Q2, M, part, d_in, r, p.split_gram, 2, st);
-    const dim3 rgrid((unsigned)((d_in + kRBN - 1) / kRBN), (unsigned)((d_out + kRBM - 1) / kRBM));
     for (int t = 0; t <= iters && e == cudaSuccess; ++t) {
         // P2: subspace iteration on Z, then U = Z Q.
         const int steps = t == 0 ? power0 : power;
@@ -583,10 +431,18 @@ cudaError_t launch_am_datafree(const uint16_t *W, int64_t d_out, int64_t d_in, i
         }
         if (e == cudaSuccess) e = split_product(false, Zhi, Zlo, d_out, d_in, Q, bh, bl, r, P, st);  // U = Z Q
         if (e != cudaSuccess) break;
-        // P1: S = 2:4 threshold of W - U V, Z = W - S, objective.
-        residual_project_kernel<<<rgrid, 256, 0, st>>>(W, P, Q, d_out, d_in, r, vals, meta, Zhi, Zlo, objp);
-        if (objective != nullptr) objective_finish_kernel<<<1, 256, 0, st>>>(objp, p.tiles_res, objective + t);
+        // P1: S = 2:4 threshold of W - U V, Z = W - S, objective: the product
+        // P Q^T (both split into bf16 planes) on the tensor cores with the
+        // threshold in its epilogue.
+        split_bf16_kernel<<<grid_cap(d_out * r, 256), 256, 0, st>>>(P, d_out * r, bh, bl);
+        split_bf16_kernel<<<grid_cap(d_in * r, 256), 256, 0, st>>>(Q, d_in * r, qh, ql);
         e = cudaGetLastError();
+        if (e == cudaSuccess)
+            e = gemm_tc<false, false, 128, kOutResid, true>(bh, bl, r, qh, ql, r, d_out, d_in, r, nullptr, am_err(), st,
+                                                             ResidOut{W, vals, meta, Zhi, Zlo, objp});
+        if (e == cudaSuccess && objective != nullptr)
+            objective_finish_kernel<<<1, 256, 0, st>>>(objp, p.tiles_res, objective + t);
+        if (e == cudaSuccess) e = cudaGetLastError();
     }
     if (e == cudaSuccess) {
         factors_out_kernel<<<grid_cap((d_out + d_in) * r, 256), 256, 0, st>>>(P, Q, d_out, d_in, r, U, V);

@@ -64,7 +64,7 @@ cudaError_t read_and_clear_decode28_error(unsigned *code);
 struct AmPlan {
     int64_t split_gram;
     int64_t tiles_res;
-    int64_t off_Z, off_Q, off_Q2, off_P, off_M, off_part, off_obj, off_split, bytes;
+    int64_t off_Z, off_Q, off_Q2, off_P, off_M, off_part, off_obj, off_split, off_split2, bytes;
 };
 AmPlan am_plan(int64_t d_out, int64_t d_in, int64_t r);
 

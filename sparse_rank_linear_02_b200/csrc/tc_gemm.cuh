@@ -37,9 +37,45 @@ using namespace tc;
 constexpr int kBM = 128;       // output rows per tile (MMA M)
 constexpr int kBThreads = 192;  // producer, MMA, four epilogue warps
 
-enum OutMode { kOutF32 = 0, kOutF32T = 1, kOutBF16 = 2 };
+// Outputs: fp32 row-major, fp32 transposed, bf16 row-major, or the fused
+// residual / 2:4 threshold of the data-free decomposition (ResidOut).
+enum OutMode { kOutF32 = 0, kOutF32T = 1, kOutBF16 = 2, kOutResid = 3 };
 
-template <int RN, bool SPLIT>
+// kOutResid: C = P Q^T is the rank-r part of W; the epilogue forms R = W - C
+// per group of four columns, keeps the two largest |R| (ties to the lower
+// index), writes them packed (vals, meta) and Z = W - S as two bf16 planes,
+// and leaves the CTA's sum of (R - S)^2 in obj_part[tile].
+struct ResidOut {
+    const uint16_t *W;  // bf16 [Mc][N]
+    uint16_t *vals;     // bf16 [Mc][N / 2]
+    uint8_t *meta;      // uint8 [Mc][N / 8]
+    uint16_t *Zhi, *Zlo;  // bf16 [Mc][N] each
+    float *obj_part;    // one float per CTA
+};
+
+// The two positions of a group of four kept by |value| (ties to the lower
+// index), from the fp32 magnitudes' bit patterns: the tournament of (0,1) and
+// (2,3), the better winner first, then the better of the winning pair's loser
+// and the losing pair's winner.  Returns idx0 | idx1 << 2.
+__device__ __forceinline__ uint32_t gemm_keep_two(float v0, float v1, float v2, float v3) {
+    const uint32_t k0 = __float_as_uint(fabsf(v0)), k1 = __float_as_uint(fabsf(v1));
+    const uint32_t k2 = __float_as_uint(fabsf(v2)), k3 = __float_as_uint(fabsf(v3));
+    const bool b01 = k0 >= k1, b23 = k2 >= k3;
+    const uint32_t hi01 = max(k0, k1), lo01 = min(k0, k1), hi23 = max(k2, k3), lo23 = min(k2, k3);
+    const uint32_t win01 = b01 ? 0u : 1u, los01 = b01 ? 1u : 0u;
+    const uint32_t win23 = b23 ? 2u : 3u, los23 = b23 ? 3u : 2u;
+    uint32_t first, second;
+    if (hi01 >= hi23) {
+        first = win01;
+        second = lo01 >= hi23 ? los01 : win23;
+    } else {
+        first = win23;
+        second = hi01 >= lo23 ? win01 : los23;
+    }
+    return min(first, second) | (max(first, second) << 2);
+}
+
+template <int RN, bool SPLIT, int NSMAX = 8>
 struct CfgB {
     static constexpr int A_BYTES = kBM * 64 * 2;   // 16 KB per plane
     static constexpr int B_BYTES = RN * 64 * 2;
@@ -48,7 +84,8 @@ struct CfgB {
     static constexpr int PROW = RN + 4;
     static constexpr int P_BYTES = kBM * PROW * 4;
     static constexpr int NS_FIT = (SPLIT ? 200704 : 112640) / STAGE;
-    static constexpr int NS = NS_FIT > 8 ? 8 : (NS_FIT < 2 ? 2 : NS_FIT);
+    static constexpr int NS0 = NS_FIT > 8 ? 8 : (NS_FIT < 2 ? 2 : NS_FIT);
+    static constexpr int NS = NS0 < NSMAX ? NS0 : NSMAX;
     static constexpr int RING = NS * STAGE;
     static constexpr int BAR_OFF = RING > P_BYTES ? RING : P_BYTES;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;
@@ -66,8 +103,9 @@ template <bool A_MN, bool B_MN, int RN, int OUT, bool SPLIT>
 __global__ void __launch_bounds__(kBThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a2,
                    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b2,
-                   void *__restrict__ out, int32_t Mc, int32_t N, int32_t nk_total, unsigned int *err) {
-    using C = CfgB<RN, SPLIT>;
+                   void *__restrict__ out, int32_t Mc, int32_t N, int32_t nk_total, unsigned int *err,
+                   ResidOut ro) {
+    using C = CfgB<RN, SPLIT, OUT == kOutResid ? 1 : 8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
@@ -83,6 +121,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const uint32_t ks_q = cluster_ctarank();
     const int tile = blockIdx.x / (int)ks_n;
     const int m0 = tile * kBM;
+    const int n0 = blockIdx.y * RN;  // N tiles (the residual mode only; otherwise one)
     const int k_begin = (int)(((int64_t)nk_total * ks_q) / ks_n);
     const int k_end = (int)(((int64_t)nk_total * (ks_q + 1)) / ks_n);
 
@@ -105,6 +144,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+
+    // Residual mode: each epilogue thread's W values, loaded before the wait for
+    // the accumulator so that the loads overlap the tensor-core work (the item
+    // loop below has a fixed trip count there, so the indices are static).
+    constexpr int kResidItems = RN / 4;  // items per epilogue thread (one CTA per tile)
+    uint2 wpre[OUT == kOutResid ? kResidItems : 1];
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -131,9 +176,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
                     }
                     if (B_MN) {  // map (inner = N, outer = K), box 64 x 64
 #pragma unroll
-                        for (int p = 0; p < RN / 64; ++p) tma_load_2d(mb, b + 8192 * p, &full[s], 64 * p, ks * 64);
+                        for (int p = 0; p < RN / 64; ++p) tma_load_2d(mb, b + 8192 * p, &full[s], n0 + 64 * p, ks * 64);
                     } else {     // map (inner = K, outer = N), box 64 x RN
-                        tma_load_2d(mb, b, &full[s], ks * 64, 0);
+                        tma_load_2d(mb, b, &full[s], ks * 64, n0);
                     }
                 }
                 if (++s == (uint32_t)C::NS) {
@@ -189,6 +234,15 @@ __global__ void __launch_bounds__(kBThreads, 1)
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const bool have = k_end > k_begin;
+        if (OUT == kOutResid) {
+#pragma unroll
+            for (int k = 0; k < kResidItems; ++k) {
+                const int it = threadIdx.x - 64 + 128 * k;
+                const int m = m0 + it / (RN / 4), n = n0 + (it % (RN / 4)) * 4;
+                wpre[k] = (m < Mc && n < N) ? __ldg(reinterpret_cast<const uint2 *>(ro.W + (int64_t)m * N + n))
+                                            : make_uint2(0, 0);
+            }
+        }
         if (mbar_wait(acc_full, 0)) {
             tc_fence_after();
 #pragma unroll 1
@@ -211,7 +265,50 @@ __global__ void __launch_bounds__(kBThreads, 1)
     cluster_sync_all();  // every CTA's partial is in its shared memory
 
     // Reduction over the cluster: CTA q owns rows [q*TPC, (q+1)*TPC) of the tile.
-    if (warp >= 2) {
+    float obj = 0.f;  // the residual mode's sum of (R - S)^2
+    if (OUT == kOutResid && warp >= 2) {
+        // One CTA per tile (no K split): item it = row t, columns c..c+3, one
+        // group of four; the partner item (the next lane) holds the other
+        // group of the same metadata byte.
+        const uint32_t part_addr = smem_u32(part);
+#pragma unroll
+        for (int k = 0; k < kResidItems; ++k) {
+            const int it = threadIdx.x - 64 + 128 * k;
+            const int t = it / (RN / 4), c = (it % (RN / 4)) * 4;
+            const float4 acc = ld_shared_cluster_v4(mapa_shared(part_addr + (uint32_t)((t * C::PROW + c) * 4), 0));
+            const int m = m0 + t, n = n0 + c;
+            const bool in = m < Mc && n < N;
+            uint32_t nib = 0;
+            if (in) {
+                const uint2 w = wpre[k];
+                const float w0 = bf16lo_to_f32(w.x), w1 = bf16hi_to_f32(w.x);
+                const float w2 = bf16lo_to_f32(w.y), w3 = bf16hi_to_f32(w.y);
+                const float R[4] = {w0 - acc.x, w1 - acc.y, w2 - acc.z, w3 - acc.w};
+                const float Wv[4] = {w0, w1, w2, w3};
+                nib = gemm_keep_two(R[0], R[1], R[2], R[3]);
+                const uint32_t a = nib & 3u, b = nib >> 2;  // a in 0..2, b in 1..3
+                uint32_t sv[4], zh[4], zl[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    sv[q] = f32_to_bf16_bits(R[q]);
+                    const float sq = (q == (int)a || q == (int)b) ? __uint_as_float(sv[q] << 16) : 0.f;
+                    const float z = Wv[q] - sq, e = R[q] - sq;
+                    obj = fmaf(e, e, obj);
+                    zh[q] = f32_to_bf16_bits(z);
+                    zl[q] = f32_to_bf16_bits(z - __uint_as_float(zh[q] << 16));
+                }
+                const uint32_t sa = a == 0u ? sv[0] : (a == 1u ? sv[1] : sv[2]);
+                const uint32_t sb = b == 1u ? sv[1] : (b == 2u ? sv[2] : sv[3]);
+                *reinterpret_cast<uint32_t *>(ro.vals + (int64_t)m * (N / 2) + n / 2) = sa | (sb << 16);
+                *reinterpret_cast<uint2 *>(ro.Zhi + (int64_t)m * N + n) =
+                    make_uint2(zh[0] | (zh[1] << 16), zh[2] | (zh[3] << 16));
+                *reinterpret_cast<uint2 *>(ro.Zlo + (int64_t)m * N + n) =
+                    make_uint2(zl[0] | (zl[1] << 16), zl[2] | (zl[3] << 16));
+            }
+            const uint32_t partner = __shfl_down_sync(0xFFFFFFFFu, nib, 1);
+            if (in && (c & 4) == 0) ro.meta[(int64_t)m * (N / 8) + n / 8] = (uint8_t)(nib | (partner << 4));
+        }
+    } else if (warp >= 2) {
         const int tpc = kBM / (int)ks_n;
         const int items = tpc * (RN / 4);
         const uint32_t part_addr = smem_u32(part);
@@ -250,6 +347,15 @@ __global__ void __launch_bounds__(kBThreads, 1)
             }
         }
     }
+    if (OUT == kOutResid && warp >= 2) {
+        // The four epilogue warps' sums, added in warp order (deterministic).
+        float *red = reinterpret_cast<float *>(tmem_slot + 2);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) obj += __shfl_xor_sync(0xFFFFFFFFu, obj, o);
+        if (lane == 0) red[warp - 2] = obj;
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 64) ro.obj_part[blockIdx.y * gridDim.x + blockIdx.x] = ((red[0] + red[1]) + red[2]) + red[3];
+    }
     cluster_sync_all();  // no CTA leaves while its partial may still be read
     if (warp == 1) {
         tc_fence_after();
@@ -266,8 +372,8 @@ constexpr auto kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 template <bool A_MN, bool B_MN, int RN, int OUT, bool SPLIT = false>
 cudaError_t gemm_tc(const uint16_t *A, const uint16_t *A2, int64_t lda, const uint16_t *B, const uint16_t *B2,
                     int64_t ldb, int64_t Mc, int64_t N, int64_t K, void *out, unsigned int *err,
-                    cudaStream_t stream) {
-    using C = CfgB<RN, SPLIT>;
+                    cudaStream_t stream, ResidOut ro = ResidOut{}) {
+    using C = CfgB<RN, SPLIT, OUT == kOutResid ? 1 : 8>;
     if (err == nullptr) return cudaErrorInvalidValue;
     CUtensorMap ma, ma2, mb, mb2;
     auto map_a = [&](CUtensorMap *m, const uint16_t *p) {
@@ -290,12 +396,12 @@ cudaError_t gemm_tc(const uint16_t *A, const uint16_t *A2, int64_t lda, const ui
     const int tiles = (int)((Mc + kBM - 1) / kBM);
     const int nk = (int)((K + 63) / 64);
     int ks = 1;
-    while (ks < 8 && ks * 2 <= nk && tiles * ks * 2 <= (ks >= 4 ? sms : 2 * sms)) ks *= 2;
+    while (OUT != kOutResid && ks < 8 && ks * 2 <= nk && tiles * ks * 2 <= (ks >= 4 ? sms : 2 * sms)) ks *= 2;
     cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<A_MN, B_MN, RN, OUT, SPLIT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(tiles * ks));
+    cfg.gridDim = dim3((unsigned)(tiles * ks), OUT == kOutResid ? (unsigned)((N + RN - 1) / RN) : 1u);
     cfg.blockDim = dim3(kBThreads);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = stream;
@@ -307,7 +413,7 @@ cudaError_t gemm_tc(const uint16_t *A, const uint16_t *A2, int64_t lda, const ui
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<A_MN, B_MN, RN, OUT, SPLIT>, ma, ma2, mb, mb2, out, (int32_t)Mc,
-                              (int32_t)N, (int32_t)nk, err);
+                              (int32_t)N, (int32_t)nk, err, ro);
 }
 
 
