@@ -9,7 +9,8 @@
 //
 // C_r is computed by subspace iteration on Z = W - S, warm-started from the
 // previous iteration's right subspace Q (d_in x r, orthonormal columns):
-//   repeat p times:  P = Z Q;  Q = orth(Z^T P)      (CholeskyQR2)
+//   repeat p times:  P = Z Q;  Q = orth(Z^T P)      (Cholesky QR: one pass
+//   between power steps, two (CholeskyQR2) on the last)
 //   then U = Z Q, V = Q^T, so U V = Z Q Q^T, the best rank-r fit of Z within
 //   span(Q), which converges to C_r(Z) as Q converges to the top-r right
 //   singular subspace.  The random start Q0 is an input.
@@ -20,7 +21,7 @@
 //    planes, hi = bf16(x) and lo = bf16(x - hi), and hi*hi + hi*lo + lo*hi
 //    accumulated in fp32: about 16 significant bits per operand, so the
 //    subspace iteration behaves as in fp32.  Z = W - S is kept as its two
-//    planes (written by the residual kernel); Q and P are split before use.
+//    planes (written by the P1 product below); Q and P are split before use.
 //  * gemm_f32_kernel<TRANS_A>: C = A B or A^T B in fp32 on CUDA cores, for the
 //    small Gram and basis products of the orthonormalisation (d_in x r x r).
 //    128 x 64 output tiles, 16-deep k steps through shared memory, split over
