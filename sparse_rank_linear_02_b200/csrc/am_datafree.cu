@@ -22,13 +22,14 @@
 //    accumulated in fp32: about 16 significant bits per operand, so the
 //    subspace iteration behaves as in fp32.  Z = W - S is kept as its two
 //    planes (written by the P1 product below); Q and P are split before use.
-//  * gemm_f32_kernel<TRANS_A>: C = A B or A^T B in fp32 on CUDA cores, for the
-//    small Gram and basis products of the orthonormalisation (d_in x r x r).
+//  * gemm_f32_kernel<TRANS_A>: C = A^T A in fp32 on CUDA cores, the small Gram
+//    product of the orthonormalisation (r x r over d_in).
 //    128 x 64 output tiles, 16-deep k steps through shared memory, split over
 //    k with the partial products summed in a fixed order by
 //    reduce_splits_kernel (deterministic).
-//  * chol_inv_kernel: one CTA; G = Q^T Q (fp64) -> Cholesky factor L ->
-//    M = L^-T, so Q M has orthonormal columns (one barrier per step).
+//  * chol_kernel: one CTA; G = Q^T Q (fp64) -> Cholesky factor L (one
+//    barrier per step); solve_rows_kernel: Q <- Q L^-T, one warp per row of
+//    Q, so Q has orthonormal columns.
 //  * P1 is the same tensor-core product P Q^T (split planes, K = r) with the
 //    threshold in its epilogue (tc_gemm_kernel's residual mode): per group of
 //    four columns R = W - P Q^T, the two largest |R| kept (ties to the lower
@@ -175,22 +176,16 @@ __global__ void reduce_splits_kernel(const float *__restrict__ part, int splits,
 
 // One CTA: G = sum of `splits` partial r x r Gram matrices (fp64), Cholesky
 // G = L L^T (a pivot below 1e-12 of the mean diagonal is raised to it, so a
-// rank-deficient block stays finite), then M = L^-T (fp32, r x r row-major).
-// Shared memory: one r x r fp64 array with rows padded to r + 1 (an odd
-// stride, so column accesses do not collide in one bank) and r square roots;
-// L fills the lower triangle and X = L^-1 (also lower triangular) is kept
-// transposed in the strict upper triangle (X[i][c] at [c][i]).
-// The factorisation is a chain of r steps, so the kernel is bound by the
-// barrier between steps; both phases defer their scaling to keep one barrier
-// per step:
-//   Cholesky, column j (d_j = the current A[j][j], floored): for j < k <= i,
-//     A[i][k] -= A[i][j] A[k][j] / d_j; column j is left unscaled, and at the
-//     end L[j][j] = sqrt(d_j), L[i][j] = A[i][j] / sqrt(d_j).
-//   Inverse, row i: with R = the unscaled rows of X (R[i][i] = 1),
-//     R[i'][c] -= (L[i'][i] / L[i][i]) R[i][c] for i' > i, c <= i; at the end
-//     X[i][c] = R[i][c] / L[i][i].
-__global__ void __launch_bounds__(1024) chol_inv_kernel(const float *__restrict__ gpart, int splits, int r,
-                                                       float *__restrict__ Mout) {
+// rank-deficient block stays finite), written as fp32 L (r x r row-major,
+// zero above the diagonal).  Shared memory: the r x r fp64 array with rows
+// padded to r + 1 (an odd stride, so column accesses do not collide in one
+// bank) and r square roots.  The factorisation is a chain of r steps, so the
+// kernel is bound by the barrier between steps; the scaling of each column
+// is deferred to keep one barrier per step: for column j (d_j = the current
+// A[j][j], floored), A[i][k] -= A[i][j] A[k][j] / d_j for j < k <= i, and at
+// the end L[j][j] = sqrt(d_j), L[i][j] = A[i][j] / sqrt(d_j).
+__global__ void __launch_bounds__(1024) chol_kernel(const float *__restrict__ gpart, int splits, int r,
+                                                   float *__restrict__ Lout) {
     extern __shared__ double A[];  // r rows of ld = r + 1, then r square roots
     __shared__ double floor_pivot;
     const int tid = threadIdx.x, nth = blockDim.x, ld = r + 1;
@@ -223,24 +218,57 @@ __global__ void __launch_bounds__(1024) chol_inv_kernel(const float *__restrict_
         sq[j] = sqrt(d > fl ? d : fl);
     }
     __syncthreads();
-    for (int i = ty; i < r; i += ny)
-        for (int c = tx; c < r; c += 32)
-            A[i * ld + c] = c < i ? A[i * ld + c] / sq[c] : (c == i ? sq[i] : 0.0);  // L, and R = I above
-    __syncthreads();
-    for (int i = 0; i < r; ++i) {
-        const double inv_lii = 1.0 / sq[i];
-        for (int ii = i + 1 + ty; ii < r; ii += ny) {
-            const double f = A[ii * ld + i] * inv_lii;
-            for (int c = tx; c <= i; c += 32) A[c * ld + ii] -= f * ((c == i) ? 1.0 : A[c * ld + i]);
-        }
-        __syncthreads();
-    }
     for (int q = tid; q < r * r; q += nth) {
-        const int k = q / r, c = q % r;  // M[k][c] = X[c][k] = R[c][k] / L[c][c]
-        float v = 0.f;
-        if (c == k) v = (float)(1.0 / sq[k]);
-        else if (c > k) v = (float)(A[k * ld + c] / sq[c]);
-        Mout[q] = v;
+        const int i = q / r, c = q % r;  // L (fp32, row-major, zero above the diagonal)
+        Lout[q] = c < i ? (float)(A[i * ld + c] / sq[c]) : (c == i ? (float)sq[i] : 0.f);
+    }
+}
+
+// Q <- Q L^-T in place: every row of Q solves x L^T = q by forward
+// substitution, x[c] = (q[c] - sum_{k<c} x[k] L[c][k]) / L[c][c].  One warp
+// per row: lane l holds x[l], x[l + 32], x[l + 64], x[l + 96] (r <= 128); each
+// step's sum is split over the lanes and reduced with shuffles.  L (fp32) is
+// read from shared memory (consecutive k across lanes: no bank conflicts).
+constexpr int kSolveWarps = 8;
+__global__ void __launch_bounds__(kSolveWarps * 32) solve_rows_kernel(float *__restrict__ Q, int64_t n_rows, int r,
+                                                                      const float *__restrict__ L) {
+    extern __shared__ float Ls[];  // r x r
+    for (int i = threadIdx.x; i < r * r; i += kSolveWarps * 32) Ls[i] = L[i];
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * kSolveWarps + (threadIdx.x >> 5);
+    if (row >= n_rows) return;  // warp-uniform; no barrier follows
+    float q[4], x[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const int k = lane + 32 * h;
+        q[h] = k < r ? Q[row * r + k] : 0.f;
+        x[h] = 0.f;
+    }
+    for (int c = 0; c < r; ++c) {
+        const float *lc = Ls + c * r;
+        float part = 0.f;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const int k = lane + 32 * h;
+            if (k < c) part = fmaf(x[h], lc[k], part);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xFFFFFFFFu, part, o);
+        const int h = c >> 5;
+        if (lane == (c & 31)) {
+            const float qc = h == 0 ? q[0] : (h == 1 ? q[1] : (h == 2 ? q[2] : q[3]));
+            const float xc = (qc - part) / lc[c];
+            if (h == 0) x[0] = xc;
+            else if (h == 1) x[1] = xc;
+            else if (h == 2) x[2] = xc;
+            else x[3] = xc;
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const int k = lane + 32 * h;
+        if (k < r) Q[row * r + k] = x[h];
     }
 }
 
@@ -337,15 +365,16 @@ cudaError_t orthonormalise(float *Q, float *tmp, float *M, float *part, int64_t 
                            int passes, cudaStream_t st) {
     for (int pass = 0; pass < passes; ++pass) {  // 2: CholeskyQR2
         // G = Q^T Q into the first r x r floats of tmp (split over d_in, the
-        // splits summed in a fixed order), then L^-T, then tmp = Q L^-T.
+        // splits summed in a fixed order), its Cholesky factor L into M, then
+        // Q <- Q L^-T by forward substitution on every row.
         cudaError_t e = gemm(true, Q, r, Q, r, tmp, part, r, r, d_in, split_gram, st);
         if (e != cudaSuccess) return e;
         // 32 warps: each step's trailing update gives a warp one or two rows,
         // which keeps the per-step chain short (the kernel is latency-bound).
-        chol_inv_kernel<<<1, 1024, (size_t)r * (r + 2) * sizeof(double), st>>>(tmp, 1, r, M);
-        e = gemm(false, Q, r, M, r, tmp, part, d_in, r, r, 1, st);
-        if (e != cudaSuccess) return e;
-        e = cudaMemcpyAsync(Q, tmp, (size_t)d_in * r * sizeof(float), cudaMemcpyDeviceToDevice, st);
+        chol_kernel<<<1, 1024, (size_t)r * (r + 2) * sizeof(double), st>>>(tmp, 1, r, M);
+        solve_rows_kernel<<<(unsigned)((d_in + kSolveWarps - 1) / kSolveWarps), kSolveWarps * 32,
+                            (size_t)r * r * sizeof(float), st>>>(Q, d_in, r, M);
+        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
@@ -410,8 +439,11 @@ cudaError_t launch_am_datafree(const uint16_t *W, int64_t d_out, int64_t d_in, i
     uint16_t *qh = reinterpret_cast<uint16_t *>(ws + p.off_split2);
     uint16_t *ql = qh + (p.bytes - p.off_split2) / 4;
     // Set on every call: the attribute belongs to the current device's copy of the kernel.
-    cudaError_t e = cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)((size_t)r * (r + 2) * sizeof(double)));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(solve_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)((size_t)r * r * sizeof(float)));
     if (e != cudaSuccess) return e;
     // Start: S = 0, so Z = W (hi = W, lo = 0); Q = orth(Q0).
     e = cudaMemcpyAsync(Zhi, W, (size_t)d_out * d_in * 2, cudaMemcpyDeviceToDevice, st);
