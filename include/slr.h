@@ -308,10 +308,10 @@ SLR_API size_t slr_forward_workspace_size(int64_t M, int64_t d_out, int64_t d_in
 /* Execution paths of the forward pass. */
 typedef enum slr_path {
     SLR_PATH_AUTO = 0,   /* choose by M and layer size (slr_forward_select_path):
-                            DECODE for M <= 2 on layers of <= 2^26 weights,
+                            DECODE for M == 1 on layers of <= 2^26 weights,
                             TENSOR otherwise (and DECODE when d_out % 8 != 0)      */
     SLR_PATH_DECODE = 1, /* CUDA-core streaming kernel over S rows (any M, best
-                            for one or two tokens)                                  */
+                            for a single token)                                     */
     SLR_PATH_TENSOR = 2  /* 2:4 tcgen05 tensor-core kernels with the rank-r term
                             fused: split-K streaming kernel for M <= 64, 2-SM
                             pairs on 256-row tiles above, on 512-row tiles once

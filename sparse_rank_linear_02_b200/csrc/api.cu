@@ -37,10 +37,12 @@ slr_status check_device() {
     return verdict[dev] == 1 ? SLR_OK : SLR_ERR_DEVICE;
 }
 
-// The CUDA-core streaming path wins only for one or two tokens on layers of
-// up to 2^26 weights (measured on B200: 8.4 us vs 12.4 us for 4096 x 4096 at
-// M = 1); larger layers stream faster through the split-K tensor-core kernel.
-constexpr int64_t kDecodeMaxM = 2;
+// The CUDA-core streaming path wins only for a single token on layers of up
+// to 2^26 weights (measured on B200 with rotating weight copies: 4096 x 4096,
+// M = 1: 7.6 us against 11.8 us; M = 2: 12.5 against 11.8 us; 14336 x 4096,
+// M = 1: 18.4 against 19.3 us, M = 2: 28.1 against 19.0 us); larger layers
+// and two or more tokens stream faster through the split-K tensor-core kernel.
+constexpr int64_t kDecodeMaxM = 1;
 constexpr int64_t kDecodeMaxWeights = int64_t(1) << 26;
 
 size_t workspace_bytes_for(int64_t M, int64_t r, slr_path path) {

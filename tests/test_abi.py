@@ -54,7 +54,7 @@ def test_meta_row_bytes_and_workspace():
 
 def test_path_selection():
     assert slr.select_path(1, 4096, 4096, 64) == "decode"
-    assert slr.select_path(2, 4096, 4096, 64) == "decode"
+    assert slr.select_path(2, 4096, 4096, 64) == "tensor"     # two tokens: the split-K tensor kernel
     assert slr.select_path(4, 4096, 4096, 64) == "tensor"
     assert slr.select_path(16, 4096, 4096, 64) == "tensor"
     assert slr.select_path(1, 28672, 8192, 64) == "tensor"     # large layer: tensor-core streaming
