@@ -1478,7 +1478,7 @@ PlanChoice choose_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int sm
     PlanChoice best{-1, 0, true};
     double best_cost = 0;
     for (int kind = 0; kind < 4; ++kind) {
-        if ((kind == 0) != (M < 192)) continue;
+        if (kind == 0 && M >= 192) continue;   // 128-token chunks: below 192 tokens only
         const int cap = kind == 0 ? Cfg2<128>::CHU : kind == 3 ? Cfg2<256>::CHU : Cfg2<240>::CHU;
         const int half_n = cap * 8;
         for (int chu = cap; chu >= cap - 5 && chu >= 1; --chu) {
@@ -1820,15 +1820,42 @@ cudaError_t launch_project_splitk(const uint16_t *X, int64_t M, const uint16_t *
 
 
 // =====================================================================================
-// Small-M forward (M <= 64 tokens): Y = X S^T + T U^T when the layer is bound by
-// the bytes of S.  One cluster of KS CTAs (KS <= 4) owns a 128-row x BN-token
-// tile and splits its K stages (the 2:4 stages, then the rank stages) across
-// its CTAs, so that all SMs stream S at once even when d_out / 128 is small.
+// Split-K forward for few tokens (BN = 16 .. 128 per tile): Y = X S^T + T U^T
+// when the layer is bound by the bytes of S, or has too few row tiles to keep
+// the 2-SM pairs busy.  One cluster of KS CTAs (KS <= 4) owns a 128-row x
+// BN-token tile and splits its K stages (the 2:4 stages, then the rank stages)
+// across its CTAs, so that all SMs stream S at once even when d_out / 128 is
+// small; the token tiles of one row tile are neighbouring clusters, which
+// stream the same S tile at about the same time (one read from HBM).
 // Each CTA accumulates its partial Y^T tile in TMEM (2:4 tcgen05.mma.sp with
 // the same metadata permute as the large-M kernels, N = BN), writes it to
 // shared memory in fp32, and after a cluster barrier CTA q sums rows
 // [q*128/KS, (q+1)*128/KS) over the KS partials through distributed shared
 // memory and stores them to Y in bf16 (RNE).
+// CTAs per cluster of the split-K kernel: split K two or four ways while the
+// grid stays within two CTAs per SM.
+inline int small_cluster(int64_t work, int64_t stages, int sms) {
+    int ks = 1;
+    while (ks < 4 && ks * 2 <= stages && work * ks * 2 <= 2 * (int64_t)sms) ks *= 2;
+    return ks;
+}
+
+// Whether the split-K kernel on 128-token tiles is the faster choice for
+// M > 64.  It is when the layer has few tiles of 128 rows x 128 tokens (at
+// most a quarter of the SM count: the pair kernels then leave pairs idle or
+// stream each S tile for short token chunks), or, with a long K (d_in >=
+// 8192), when its tiles still fit one CTA per SM.  Measured on B200 with
+// r = 64 against the best pair-kernel plan: 4096 x 4096 at M = 65..128 21 vs
+// 25 us (64 tiles from M = 160: 28.6 vs 26.7 us, pairs ahead); 1024 x 4096 up
+// to M = 512 (32 tiles) 19-22 vs 19-26 us; 4096 x 14336 at M = 65..512 37-64
+// vs 60-67 us (160 tiles at M = 640: 106 vs 73 us, pairs ahead); 8192 x 28672
+// at M = 65..256 72-115 vs 111-131 us; 14336 x 4096 (112 tiles, short K) and
+// 28672 x 8192 (224 tiles) stay on the pair kernels.
+inline bool small_wins(int64_t M, int64_t d_out, int64_t d_in, int sms) {
+    const int64_t work = ((d_out + BM - 1) / BM) * ((M + 127) / 128);
+    return work * 4 <= (int64_t)sms || (d_in >= 8192 && work <= (int64_t)sms);
+}
+
 template <int BN>
 struct CfgS {
     static constexpr int A_BYTES = BM * 64 * 2;          // 16 KB of packed values (128 logical K)
@@ -1838,15 +1865,15 @@ struct CfgS {
     static constexpr int STAGE = ((A_BYTES + B_BYTES + E_BYTES + 1023) / 1024) * 1024;
     static constexpr int PROW = BN + 4;                  // padded fp32 row of the partial tile
     static constexpr int P_BYTES = BM * PROW * 4;
-    static constexpr int NS_FIT = 102400 / STAGE;        // about 100 KB: two CTAs per SM
+    static constexpr int NS_FIT = 114432 / STAGE;        // two CTAs per SM (114432 + 1280 <= 115712)
     static constexpr int NS = NS_FIT > 8 ? 8 : (NS_FIT < 2 ? 2 : NS_FIT);
     static constexpr int RING = NS * STAGE;
     static constexpr int BAR_OFF = (RING > P_BYTES ? RING : P_BYTES);
     static constexpr int SMEM = BAR_OFF + 256 + 1024;
     static constexpr uint32_t ECOL = BN;
     static constexpr uint32_t TMEM_COLS = pow2_at_least(BN + 4);
-    static_assert(SMEM <= 116736, "two CTAs per SM");
-    static_assert(BN % 16 == 0 && BN <= 64, "MMA N");
+    static_assert(SMEM <= 115712, "two CTAs per SM (228 KB less 1 KB reserved per CTA)");
+    static_assert(BN % 16 == 0 && BN <= 128, "MMA N");
 };
 
 template <int BN>
@@ -2065,8 +2092,7 @@ cudaError_t launch_sparse_small(const uint16_t *X, int64_t M, const uint16_t *va
     const int n_ttiles = (int)((M + BN - 1) / BN);
     const int work = (int)((d_out + BM - 1) / BM) * n_ttiles;
     const int nk = (int)(d_in / BK), nlr = (int)((r + 63) / 64);
-    int ks = 1;
-    while (ks < 4 && ks * 2 <= nk + nlr && work * ks * 2 <= 2 * sms) ks *= 2;
+    const int ks = small_cluster(work, nk + nlr, sms);
     cudaError_t err = cudaFuncSetAttribute(tc_small_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -2109,23 +2135,28 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
             return tc::launch_sparse_pair<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, !whole, stream);
         if (strncmp(force, "2smtall", 7) == 0)
             return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, !whole, stream);
-        if (strcmp(force, "small") == 0 && M <= 64) {
+        if (strcmp(force, "small") == 0) {
             if (M <= 16) return tc::launch_sparse_small<16>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
             if (M <= 32) return tc::launch_sparse_small<32>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
-            return tc::launch_sparse_small<64>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+            if (M <= 64) return tc::launch_sparse_small<64>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
+            return tc::launch_sparse_small<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
         }
     }
-    // Up to 64 tokens the layer streams S: the split-K small-M kernel.  Above,
-    // 2-SM pairs: on 256-row tiles with chunks of up to 128 tokens (M < 192) or
-    // 240 tokens, or on 512-row tiles, which move X into shared memory half as
-    // often but drain their accumulators between chunks; each with the last
-    // round split among all pairs or dealt as whole tiles.  The plan with the
-    // smallest estimated time of its slowest pair is launched.
+    // Up to 64 tokens the layer streams S: the split-K kernel.  Above, the
+    // split-K kernel on 128-token tiles where it wins (few row tiles, one wave,
+    // long K per CTA), else 2-SM pairs: on 256-row tiles with chunks of up to
+    // 128 tokens (M < 192) or 240 tokens, or on 512-row tiles, which move X
+    // into shared memory half as often but drain their accumulators between
+    // chunks; each with the last round split among all pairs or dealt as whole
+    // tiles.  The pair plan with the smallest estimated time of its slowest
+    // pair is launched.
     if (M <= 16) return tc::launch_sparse_small<16>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     if (M <= 32) return tc::launch_sparse_small<32>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     if (M <= 64) return tc::launch_sparse_small<64>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (tc::small_wins(M, d_out, d_in, sms))
+        return tc::launch_sparse_small<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, stream);
     const tc::PlanChoice c = tc::choose_plan(M, d_out, d_in, r, sms);
     if (c.kind == 0)
         return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream, c.chu);

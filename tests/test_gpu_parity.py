@@ -173,6 +173,10 @@ def test_forward_edges(d_out, d_in, r, M, path):
     (1024, 4096, 64, 4096),   # few row tiles, many tokens
     (2048, 8192, 64, 1000),   # 512-row tiles, ragged token count
     (3072, 4096, 128, 700),   # d_out not a multiple of 512
+    (4096, 14336, 64, 160),   # split-K kernel on two 128-token tiles, K split two ways (56 stages each)
+    (1024, 8192, 128, 200),   # split-K kernel, four-way K split, two rank stages
+    (8192, 4096, 64, 160),    # below 192 tokens: every pair-kernel kind is a candidate
+    (4096, 4096, 64, 96),     # 65..128 tokens on 32 row tiles: split-K kernel, four-way split
 ])
 def test_forward_plan_shapes(d_out, d_in, r, M):
     """Default dispatch on shapes where the pair-kernel plan choice matters
@@ -219,6 +223,7 @@ VARIANTS = ["1sm", "2sm128", "2sm240", "2sm256", "2smtall", "2smtallw", "small"]
     (1024, 2048, 128, 16),   # small M, 16-token tile, two rank stages
     (256, 4096, 64, 33),     # small M, 64-token tile
     (4096, 4096, 64, 1),     # one token, 32 row tiles x 4-CTA clusters
+    (296, 1024, 64, 100),    # 65..128 tokens: one 128-token tile (split-K kernel), ragged rows
 ])
 def test_forward_tensor_variants(variant, d_out, d_in, r, M, monkeypatch):
     """Every tensor-core kernel variant (1-SM; 2-SM pairs on 256-row tiles with
