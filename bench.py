@@ -49,7 +49,7 @@ SPARSE_RATIO = 2.0   # nominal 2:4 sparse / dense tensor throughput ratio
 
 # DRAM bytes per launch of the dominant kernel from the committed ncu capture
 # (profiles/); valid only for the kernel source it was taken on.
-NCU_TRAFFIC = {"tc_forward": {"source_sha": "f7ee71cbb743eccc", "bytes_per_launch": 119456256}}
+NCU_TRAFFIC = {"tc_forward": {"source_sha": "217ad0ba78be39d8", "bytes_per_launch": 121122560}}
 
 
 def layer_of(cfg, name):
