@@ -315,9 +315,10 @@ typedef enum slr_path {
     SLR_PATH_DECODE = 1, /* CUDA-core streaming kernel over S rows (any M, best
                             for a single token)                                     */
     SLR_PATH_TENSOR = 2  /* 2:4 tcgen05 tensor-core kernels with the rank-r term
-                            fused: split-K streaming kernel for M <= 64, 2-SM
-                            pairs on 256-row tiles above, on 512-row tiles once
-                            those fill a round of pairs                             */
+                            fused: split-K streaming kernel for M <= 64 and for
+                            layers of few 128-row tiles up to a few hundred
+                            tokens, 2-SM pairs on 256- or 512-row tiles
+                            otherwise (the plan of least estimated time)          */
 } slr_path;
 
 /* The path SLR_PATH_AUTO takes for this problem. */
