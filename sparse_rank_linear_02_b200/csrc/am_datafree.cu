@@ -22,8 +22,8 @@
 //    accumulated in fp32: about 16 significant bits per operand, so the
 //    subspace iteration behaves as in fp32.  Z = W - S is kept as its two
 //    planes (written by the P1 product below); Q and P are split before use.
-//  * gemm_f32_kernel<TRANS_A>: C = A^T A in fp32 on CUDA cores, the small Gram
-//    product of the orthonormalisation (r x r over d_in).
+//  * gemm_tn_f32_kernel: C = A^T B in fp32 on CUDA cores, for the small Gram
+//    product of the orthonormalisation (Q^T Q, r x r over d_in).
 //    128 x 64 output tiles, 16-deep k steps through shared memory, split over
 //    k with the partial products summed in a fixed order by
 //    reduce_splits_kernel (deterministic).
@@ -54,14 +54,12 @@ constexpr int kGBM = 128;  // output rows per tile
 constexpr int kGBN = 64;   // output columns per tile
 constexpr int kGBK = 16;   // k per shared-memory step
 
-// C_part[split] (rows x cols, row-major, ldc = cols) = op(A) B over the k range
-// of this split.  TRANS_A == false: A is rows x kdim (lda), C = A B.
-// TRANS_A == true: A is kdim x rows (lda), C = A^T B.  B is kdim x cols (ldb).
-template <bool TRANS_A>
-__global__ void __launch_bounds__(kGT) gemm_f32_kernel(const float *__restrict__ A, int64_t lda,
-                                                       const float *__restrict__ B, int64_t ldb,
-                                                       float *__restrict__ Cpart, int64_t rows, int64_t cols,
-                                                       int64_t kdim, int64_t k_per_split) {
+// C_part[split] (rows x cols, row-major, ldc = cols) = A^T B over the k range
+// of this split: A is kdim x rows (lda), B is kdim x cols (ldb).
+__global__ void __launch_bounds__(kGT) gemm_tn_f32_kernel(const float *__restrict__ A, int64_t lda,
+                                                          const float *__restrict__ B, int64_t ldb,
+                                                          float *__restrict__ Cpart, int64_t rows, int64_t cols,
+                                                          int64_t kdim, int64_t k_per_split) {
     __shared__ __align__(16) float As[kGBK][kGBM];
     __shared__ __align__(16) float Bs[kGBK][kGBN];
     const int tid = threadIdx.x;
@@ -77,31 +75,9 @@ __global__ void __launch_bounds__(kGT) gemm_f32_kernel(const float *__restrict__
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
     for (int64_t k0 = k_begin; k0 < k_end; k0 += kGBK) {
-        // A tile -> As[k][row]
-        if (!TRANS_A) {
-            // 128 rows x 16 k: each thread two 4-wide pieces of a row.
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int idx = tid + h * kGT;       // 0..511
-                const int row = idx / 4, kq = (idx % 4) * 4;
-                const int64_t gr = r0 + row, gk = k0 + kq;
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (gr < rows) {
-                    if (gk + 3 < k_end) {
-                        v = *reinterpret_cast<const float4 *>(A + gr * lda + gk);
-                    } else {
-                        if (gk + 0 < k_end) v.x = A[gr * lda + gk + 0];
-                        if (gk + 1 < k_end) v.y = A[gr * lda + gk + 1];
-                        if (gk + 2 < k_end) v.z = A[gr * lda + gk + 2];
-                    }
-                }
-                As[kq + 0][row] = v.x;
-                As[kq + 1][row] = v.y;
-                As[kq + 2][row] = v.z;
-                As[kq + 3][row] = v.w;
-            }
-        } else {
-            // 16 k (rows of A) x 128 output rows (columns of A): coalesced rows.
+        // A tile -> As[k][row]: 16 k (rows of A) x 128 output rows (columns of
+        // A), coalesced rows; each thread two 4-wide pieces.
+        {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int idx = tid + h * kGT;       // 0..511
@@ -345,17 +321,16 @@ AmPlan am_plan(int64_t d_out, int64_t d_in, int64_t r) {
 
 namespace {
 
-cudaError_t gemm(bool trans_a, const float *A, int64_t lda, const float *B, int64_t ldb, float *out, float *part,
-                 int64_t rows, int64_t cols, int64_t kdim, int64_t splits, cudaStream_t st) {
+// out (rows x cols) = A^T B with A kdim x rows and B kdim x cols, k split over
+// `splits` CTAs whose partials are summed in a fixed order.
+cudaError_t gemm_tn(const float *A, int64_t lda, const float *B, int64_t ldb, float *out, float *part,
+                    int64_t rows, int64_t cols, int64_t kdim, int64_t splits, cudaStream_t st) {
     int64_t kps = (kdim + splits - 1) / splits;
     kps = (kps + kGBK - 1) / kGBK * kGBK;
     const int64_t used = (kdim + kps - 1) / kps;
     dim3 grid((unsigned)((rows + kGBM - 1) / kGBM), (unsigned)((cols + kGBN - 1) / kGBN), (unsigned)used);
     float *dst = used == 1 ? out : part;
-    if (trans_a)
-        gemm_f32_kernel<true><<<grid, kGT, 0, st>>>(A, lda, B, ldb, dst, rows, cols, kdim, kps);
-    else
-        gemm_f32_kernel<false><<<grid, kGT, 0, st>>>(A, lda, B, ldb, dst, rows, cols, kdim, kps);
+    gemm_tn_f32_kernel<<<grid, kGT, 0, st>>>(A, lda, B, ldb, dst, rows, cols, kdim, kps);
     if (used > 1) reduce_splits_kernel<<<grid_cap(rows * cols, 256), 256, 0, st>>>(part, (int)used, rows * cols, out);
     return cudaGetLastError();
 }
@@ -367,7 +342,7 @@ cudaError_t orthonormalise(float *Q, float *tmp, float *M, float *part, int64_t 
         // G = Q^T Q into the first r x r floats of tmp (split over d_in, the
         // splits summed in a fixed order), its Cholesky factor L into M, then
         // Q <- Q L^-T by forward substitution on every row.
-        cudaError_t e = gemm(true, Q, r, Q, r, tmp, part, r, r, d_in, split_gram, st);
+        cudaError_t e = gemm_tn(Q, r, Q, r, tmp, part, r, r, d_in, split_gram, st);
         if (e != cudaSuccess) return e;
         // 32 warps: each step's trailing update gives a warp one or two rows,
         // which keeps the per-step chain short (the kernel is latency-bound).
