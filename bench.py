@@ -295,7 +295,8 @@ def run_ours(args, rank, world, dist):
                "frac_of_roofline_sustained_peak": round(t_roof_step_s / (ms_per_step * 1e-3), 4),
                "peak_note": "frac_of_roofline uses the burst bf16 peak; the step runs after a 0.5 s preheat "
                             "at sustained clocks, for which the sustained measured peak is the denominator",
-               "project_ms": round(project_ms, 4), "combine_ms": round(combine_ms, 4)}
+               "project_ms": round(project_ms, 4), "combine_ms": round(combine_ms, 4), "path": path,
+               "l2": f"rotating {n_copies} buffer sets of {set_bytes / 1e6:.1f} MB (> L2 126 MB)"}
     clocks = clk.summary()
 
     legs = set(args.only.split(","))
@@ -334,11 +335,7 @@ def run_ours(args, rank, world, dist):
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, Llama-3-8B gate/up shape)",
-        "config": {"workload": "Llama-3-8B gate/up prefill: d_out=14336, d_in=4096, r=64, M=2048 tokens/GPU, "
-                               "2:4 S + rank-64 U,V, bf16 in, fp32 accumulate",
-                   "tokens_per_gpu": M, "d_out": d_out, "d_in": d_in, "rank": r, "path": path,
-                   "l2": f"rotating {n_copies} buffer sets of {set_bytes / 1e6:.1f} MB (> L2 126 MB)",
-                   "parallelism": f"dp{world} (independent token batches, no collective)"},
+        "config": prefill_config(world),
         "prefill": prefill,
         "decode_m1": decode,
         **sweep,
@@ -832,6 +829,15 @@ def run_calibrate_leg(args, slr, torch, dev, W, to_dev, peaks, max_over_ranks, b
                             "bytes_per_launch": p_bytes, "frac": round(gbs_p / hbm, 4)}}
 
 
+def prefill_config(world: int) -> dict:
+    """The workload of the metric's M = 2048 point, identical in both arms."""
+    L = layer_of(PREFILL["cfg"], PREFILL["name"])
+    return {"workload": f"Llama-3-8B gate/up prefill: d_out={L.d_out}, d_in={L.d_in}, r={L.r}, "
+                        f"M={PREFILL['M']} tokens/GPU, 2:4 S + rank-{L.r} U,V, bf16 in, fp32 accumulate",
+            "tokens_per_gpu": PREFILL["M"], "d_out": L.d_out, "d_in": L.d_in, "rank": L.r,
+            "parallelism": f"dp{world} (independent token batches, no collective)"}
+
+
 def cpu_baseline_prefill(L, rows: int):
     import oracle
     W = L.weight()
@@ -877,7 +883,7 @@ def run_reference(args):
             "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "Llama-3-8B gate/up prefill: d_out=14336, d_in=4096, r=64, M=2048 tokens"},
+            "config": prefill_config(int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -22,6 +22,13 @@
  *
  * Threading: calls are safe from several host threads; calls on one stream
  * execute in order.  Outputs must not alias inputs.
+ *
+ * Per-device state: on its first use on a device the library looks up, and
+ * keeps for the life of the process, the device addresses of its own
+ * file-scope device arrays (the kernels' error words, the scratch of
+ * slr_forward_decode_noalloc).  cudaDeviceReset() unloads the module those
+ * addresses belong to, so after a reset of a device this library must not be
+ * used on that device again in the same process.
  */
 #ifndef SLR_H
 #define SLR_H
@@ -268,6 +275,17 @@ SLR_API slr_status slr_decompose_datafree(const void *W, int64_t d_out, int64_t 
                                   int power_first, int power, const float *Q0, void *vals, void *meta,
                                   void *U, void *V, double *objective, void *workspace,
                                   size_t workspace_bytes, slr_stream_t stream);
+
+/* The factors of the last slr_decompose_datafree call that used `workspace`
+ * (same d_out, d_in, r; queued on the same stream before this call), before
+ * their rounding to bf16: U32 = fp32 [d_out, r], V32 = fp32 [r, d_in], with
+ * U V = U32 V32 up to that rounding (the subspace iteration's Z Q and Q^T,
+ * HASSLE-free section 4.2.1).  Either output may be NULL (not both).  The
+ * workspace is read only.  Same shape rules as slr_decompose_datafree;
+ * SLR_ERR_NULL, SLR_ERR_ALIGN (16 bytes), SLR_ERR_WORKSPACE, SLR_ERR_DEVICE,
+ * SLR_ERR_CUDA as there. */
+SLR_API slr_status slr_decompose_factors_f32(const void *workspace, size_t workspace_bytes, int64_t d_out,
+                                             int64_t d_in, int64_t r, float *U32, float *V32, slr_stream_t stream);
 
 /* Scratch bytes of slr_decompose_datafree (about 4 * d_out * d_in + O((d_out + d_in) * r)). */
 SLR_API size_t slr_decompose_workspace_size(int64_t d_out, int64_t d_in, int64_t r);

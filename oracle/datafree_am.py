@@ -42,6 +42,14 @@ def hard_threshold_2to4(R: np.ndarray) -> np.ndarray:
     """P1 for an identity Hessian: keep the two largest |R| of each aligned
     group of four along the last axis (ties to the lower index), zero the rest."""
     R = np.asarray(R, dtype=np.float64)
+    return np.where(keep_mask_2to4(R), R, 0.0)
+
+
+def keep_mask_2to4(R: np.ndarray) -> np.ndarray:
+    """The positions P1 keeps (boolean, the shape of R): in every aligned group
+    of four along the last axis, the two of largest |R|, ties to the lower
+    index."""
+    R = np.asarray(R, dtype=np.float64)
     d_out, d_in = R.shape
     if d_in % 4:
         raise ValueError("d_in must be a multiple of 4")
@@ -56,8 +64,7 @@ def hard_threshold_2to4(R: np.ndarray) -> np.ndarray:
             if q < p:
                 beats |= g[..., q] == g[..., p]
             beaten[..., p] += beats
-    keep = (beaten < 2).reshape(d_out, d_in)
-    return np.where(keep, R, 0.0)
+    return (beaten < 2).reshape(d_out, d_in)
 
 
 def objective(W: np.ndarray, S: np.ndarray, L: np.ndarray) -> float:

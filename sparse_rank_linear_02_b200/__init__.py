@@ -69,6 +69,8 @@ def _load() -> ctypes.CDLL:
     lib.slr_decompose_datafree.restype = st
     lib.slr_decompose_datafree.argtypes = [p, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, p, p, p, p,
                                            p, p, p, sz, p]
+    lib.slr_decompose_factors_f32.restype = st
+    lib.slr_decompose_factors_f32.argtypes = [p, sz, i64, i64, i64, p, p, p]
     lib.slr_decompose_workspace_size.restype = sz
     lib.slr_decompose_workspace_size.argtypes = [i64, i64, i64]
     lib.slr_lora_backward.restype = st
@@ -232,11 +234,13 @@ def lora_backward(X: torch.Tensor, dY: torch.Tensor, U: torch.Tensor, V: torch.T
 
 
 def decompose_datafree(W: torch.Tensor, r: int, iters: int, *, power_first: int = 8, power: int = 2,
-                       Q0: torch.Tensor | None = None, seed: int = 0):
+                       Q0: torch.Tensor | None = None, seed: int = 0, factors_f32: bool = False):
     """Data-free alternating minimisation W ~ S + U V (S 2:4, rank r): returns
     ``(vals, meta, U, V, objective)`` with ``objective`` an fp64 CUDA tensor of
     ``iters + 1`` values.  ``Q0`` (fp32 [d_in, r]) is the random start of the
-    subspace iteration; by default a standard normal one from ``seed``."""
+    subspace iteration; by default a standard normal one from ``seed``.  With
+    ``factors_f32`` the fp32 factors before their rounding to bf16
+    (``slr_decompose_factors_f32``) are appended: ``(..., U32, V32)``."""
     if W.dtype != torch.bfloat16 or W.dim() != 2 or not W.is_cuda or not W.is_contiguous():
         raise ValueError("W must be a contiguous 2-D CUDA bf16 tensor")
     d_out, d_in = W.shape
@@ -255,7 +259,13 @@ def decompose_datafree(W: torch.Tensor, r: int, iters: int, *, power_first: int 
     _check(_lib.slr_decompose_datafree(_ptr(W), d_out, d_in, r, iters, power_first, power, _ptr(Q0), _ptr(vals),
                                        _ptr(meta), _ptr(U), _ptr(V), _ptr(obj), _ptr(ws), ws.numel(), _stream()),
            "slr_decompose_datafree")
-    return vals, meta, U, V, obj
+    if not factors_f32:
+        return vals, meta, U, V, obj
+    U32 = torch.empty((d_out, r), dtype=torch.float32, device=dev)
+    V32 = torch.empty((r, d_in), dtype=torch.float32, device=dev)
+    _check(_lib.slr_decompose_factors_f32(_ptr(ws), ws.numel(), d_out, d_in, r, _ptr(U32), _ptr(V32), _stream()),
+           "slr_decompose_factors_f32")
+    return vals, meta, U, V, obj, U32, V32
 
 
 def workspace_size(M: int, d_out: int, d_in: int, r: int) -> int:

@@ -288,6 +288,22 @@ __global__ void factors_out_kernel(const float *__restrict__ P, const float *__r
     }
 }
 
+// U32 = P [d_out, r] and V32[k][j] = Q[j][k] [r, d_in], both fp32 (the
+// factors before their rounding to bf16).
+__global__ void factors_f32_kernel(const float *__restrict__ P, const float *__restrict__ Q, int64_t d_out,
+                                   int64_t d_in, int r, float *__restrict__ U32, float *__restrict__ V32) {
+    const int64_t nu = d_out * r, nv = (int64_t)r * d_in;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nu + nv;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        if (i < nu) {
+            if (U32 != nullptr) U32[i] = P[i];
+        } else if (V32 != nullptr) {
+            const int64_t v = i - nu, k = v / d_in, j = v - k * d_in;
+            V32[v] = Q[j * r + k];
+        }
+    }
+}
+
 int grid_cap(int64_t n, int threads) {
     const int64_t b = (n + threads - 1) / threads;
     return (int)(b < 148 * 16 ? (b > 0 ? b : 1) : 148 * 16);
@@ -384,6 +400,15 @@ cudaError_t split_product(bool transpose_z, const uint16_t *Zhi, const uint16_t 
 }
 
 }  // namespace
+
+cudaError_t launch_am_factors_f32(const uint8_t *ws, int64_t d_out, int64_t d_in, int r, float *U32, float *V32,
+                                  cudaStream_t st) {
+    const AmPlan p = am_plan(d_out, d_in, r);
+    const float *Q = reinterpret_cast<const float *>(ws + p.off_Q);
+    const float *P = reinterpret_cast<const float *>(ws + p.off_P);
+    factors_f32_kernel<<<grid_cap((d_out + d_in) * r, 256), 256, 0, st>>>(P, Q, d_out, d_in, r, U32, V32);
+    return cudaGetLastError();
+}
 
 cudaError_t read_and_clear_am_error(unsigned *code) {
     unsigned v = 0;

@@ -294,6 +294,21 @@ slr_status slr_decompose_datafree(const void *W, int64_t d_out, int64_t d_in, in
     return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
 }
 
+slr_status slr_decompose_factors_f32(const void *workspace, size_t workspace_bytes, int64_t d_out, int64_t d_in,
+                                     int64_t r, float *U32, float *V32, slr_stream_t stream) {
+    if (d_out < 1 || d_in < 8 || d_in % 8 != 0 || r < 8 || r > 128 || r % 8 != 0 || r > d_out || r > d_in ||
+        d_out > INT32_MAX || d_in > INT32_MAX)
+        return SLR_ERR_SHAPE;
+    if (workspace == nullptr || (U32 == nullptr && V32 == nullptr)) return SLR_ERR_NULL;
+    if (!slr::aligned16(workspace) || !slr::aligned16(U32) || !slr::aligned16(V32)) return SLR_ERR_ALIGN;
+    if (workspace_bytes < slr_decompose_workspace_size(d_out, d_in, r)) return SLR_ERR_WORKSPACE;
+    const slr_status dev = slr::check_device();
+    if (dev != SLR_OK) return dev;
+    const cudaError_t err = slr::launch_am_factors_f32(static_cast<const uint8_t *>(workspace), d_out, d_in, (int)r,
+                                                       U32, V32, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
+}
+
 size_t slr_column_norms_workspace_size(int64_t M, int64_t d_in) {
     if (M <= 0 || d_in <= 0 || d_in % 8 != 0) return 0;
     const slr::NormPlan p = slr::column_norms_plan(M, d_in);

@@ -75,6 +75,11 @@ cudaError_t launch_am_datafree(const uint16_t *W, int64_t d_out, int64_t d_in, i
                                int power, const float *Q0, uint16_t *vals, uint8_t *meta, uint16_t *U, uint16_t *V,
                                double *objective, uint8_t *ws, cudaStream_t st);
 
+// The fp32 factors that the last launch_am_datafree on `ws` (same shape) left
+// in its workspace: U32 = P [d_out, r], V32 = Q^T [r, d_in]; either may be null.
+cudaError_t launch_am_factors_f32(const uint8_t *ws, int64_t d_out, int64_t d_in, int r, float *U32, float *V32,
+                                  cudaStream_t st);
+
 // Gradients of the layer with respect to U and V (S frozen): G = dY U (bf16,
 // in ws), dU = dY^T T (fp32 [d_out, r]), dV = G^T X (fp32 [r, d_in]).  T16_in
 // is the forward's T = X V^T (bf16 [M, r]) or null (then computed into ws).

@@ -36,20 +36,36 @@ def bits_to_f64(b: np.ndarray) -> np.ndarray:
 
 
 def sample_indices(n: int, k: int, seed: int, tile: int = 128) -> np.ndarray:
-    """All of range(n) when n <= k; otherwise k seeded indices that always
-    include both ends and the first/last rows of the final (ragged) tile."""
+    """All of range(n) when n <= k; otherwise the sorted union of fixed indices
+    (both ends, the first and last rows of the first and of the final, ragged
+    tile) and k seeded draws spread over the whole range, so the sample holds
+    at least k indices and always reaches the top of the range."""
     if n <= k:
         return np.arange(n, dtype=np.int64)
     rng = np.random.Generator(np.random.PCG64(seed))
-    fixed = {0, 1, n - 1, n - 2, (n - 1) // tile * tile, min(n - 1, tile), tile - 1 if tile < n else 0}
+    last_tile = (n - 1) // tile * tile
+    fixed = {0, 1, n - 2, n - 1, last_tile, max(0, last_tile - 1), min(n - 1, tile - 1), min(n - 1, tile)}
     rest = rng.choice(n, size=k, replace=False)
-    out = sorted(fixed | set(int(x) for x in rest))
-    return np.array(out[:max(k, len(fixed))], dtype=np.int64)
+    return np.array(sorted(fixed | set(int(x) for x in rest)), dtype=np.int64)
 
 
-def check_forward(Y_bits: np.ndarray, Y_ref: np.ndarray, B_ref: np.ndarray, what: str):
+def stratified_indices(n: int, block: int, seed: int) -> np.ndarray:
+    """One seeded index inside every aligned block of ``block`` indices (the
+    last, ragged block included), plus n - 1: a sample that meets every
+    16-token unit or 128-row tile a kernel's work partition can produce."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    starts = np.arange(0, n, block, dtype=np.int64)
+    widths = np.minimum(block, n - starts)
+    picks = starts + (rng.random(starts.shape[0]) * widths).astype(np.int64)
+    return np.unique(np.concatenate([picks, [n - 1]]))
+
+
+def check_forward(Y_bits: np.ndarray, Y_ref: np.ndarray, B_ref: np.ndarray, what: str,
+                  rows=None, outs=None):
     """The acceptance test on the sampled block: relative Frobenius error and
-    the per-element bound, both in fp64 on the bf16 GPU output."""
+    the per-element bound, both in fp64 on the bf16 GPU output.  ``rows`` and
+    ``outs`` (the token and output indices of the block) name the failing
+    cell in the message."""
     Y = bits_to_f64(Y_bits)
     assert np.all(np.isfinite(Y)), f"{what}: non-finite output"
     diff = Y - Y_ref
@@ -60,7 +76,9 @@ def check_forward(Y_bits: np.ndarray, Y_ref: np.ndarray, B_ref: np.ndarray, what
     bad = np.abs(diff) > bound
     if bad.any():
         i, j = np.argwhere(bad)[0]
-        raise AssertionError(f"{what}: {bad.sum()} elements out of bound; first at {i},{j}: "
+        tok = int(rows[i]) if rows is not None else int(i)
+        out = int(outs[j]) if outs is not None else int(j)
+        raise AssertionError(f"{what}: {bad.sum()} elements out of bound; first at token {tok}, output {out}: "
                              f"gpu {Y[i, j]:.6g} ref {Y_ref[i, j]:.6g} bound {bound[i, j]:.3g}")
     return rel
 

@@ -212,6 +212,20 @@ def test_decompose_argument_errors():
         assert f(w, 64, 64, 8, 1, 1, 1, q, v, m, u, vv, None, ws, big, None) == DEVICE
 
 
+def test_decompose_factors_f32_argument_errors():
+    f = slr.lib().slr_decompose_factors_f32
+    ws, u, v = P(0x10000), P(0x20000), P(0x30000)
+    big = 1 << 30
+    assert f(ws, big, 64, 64, 12, u, v, None) == SHAPE       # r % 8
+    assert f(ws, big, 64, 64, 136, u, v, None) == SHAPE      # r > 128
+    assert f(None, big, 64, 64, 8, u, v, None) == NULL
+    assert f(ws, big, 64, 64, 8, None, None, None) == NULL   # no output
+    assert f(ws, big, 64, 64, 8, P(0x20004), v, None) == ALIGN
+    assert f(ws, 16, 64, 64, 8, u, v, None) == WORKSPACE
+    if not torch.cuda.is_available():
+        assert f(ws, big, 64, 64, 8, u, None, None) == DEVICE
+
+
 def test_lora_backward_argument_errors():
     f = slr.lib().slr_lora_backward
     x, dy, u, v, du, dv, ws = (P(0x10000 * k) for k in range(1, 8))

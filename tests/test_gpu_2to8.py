@@ -98,7 +98,7 @@ def _forward_case(layer, M, seed, k_rows=16, k_outs=384):
     np.testing.assert_array_equal(from_dev(v8)[outs], rv)
     np.testing.assert_array_equal(m8.cpu().numpy()[outs], rm)
     Yref, Bref = oracle.forward_2to8(X, rv, rm, np.ascontiguousarray(U[outs]), V, rows=rows)
-    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, f"{layer.name} 2:8 M={M}")
+    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, f"{layer.name} 2:8 M={M}", rows, outs)
     return W, U, V, v4, m4
 
 
@@ -129,7 +129,7 @@ def test_forward_2to8_rows_per_warp_variants(kernel, rw, monkeypatch):
         Y = slr.forward_2to8(to_dev(X), to_dev(rv8), to_dev_u8(rm8), to_dev(U), to_dev(V))
         outs = sample_indices(d_out, 512, 75)
         Yref, Bref = oracle.forward_2to8(X, rv8, rm8, U, V, outs=outs)
-        check_forward(from_dev(Y)[:, outs], Yref, Bref, f"rw={rw} M={M}")
+        check_forward(from_dev(Y)[:, outs], Yref, Bref, f"rw={rw} M={M}", None, outs)
 
 
 def test_forward_2to8_rank_variants_and_edges():
@@ -176,4 +176,4 @@ def test_2to8_matrix_on_tensor_path():
     outs = sample_indices(layer.d_out, 256, 7)
     rv, rm = oracle.pack_2to8(np.ascontiguousarray(W[outs]))
     Yref, Bref = oracle.forward_2to8(Xp, rv, rm, np.ascontiguousarray(U[outs]), V, rows=rows)
-    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, "2:8 gate_up on the tensor path")
+    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, "2:8 gate_up on the tensor path", rows, outs)

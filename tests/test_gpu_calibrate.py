@@ -222,4 +222,4 @@ def test_calibrated_layer_forward():
     rows = sample_indices(64, 64, 3)
     outs = sample_indices(layer.d_out, 512, 4)
     Yref, Bref = oracle.forward(X, vref, mref, U, V, rows=rows, outs=outs)
-    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, "calibrated q_proj")
+    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, "calibrated q_proj", rows, outs)

@@ -137,3 +137,113 @@ def test_decompose_config_layer():
     assert all(b <= a * (1 + 1e-4) for a, b in zip(obj, obj[1:])), obj
     _check_structure(vals, meta, layer.d_out, layer.d_in)
     assert torch.isfinite(U.float()).all() and torch.isfinite(V.float()).all()
+
+
+# ----------------------------------------------------------------------------- element-wise P1 / P2
+
+def _gpu_mask(meta, d_out, d_in):
+    """Kept positions named by the packed metadata (boolean [d_out, d_in])."""
+    m = meta.cpu().numpy().astype(np.int64)
+    nib = np.stack([m & 0xF, m >> 4], axis=-1).reshape(d_out, -1)[:, : d_in // 4]
+    mask = np.zeros((d_out, d_in // 4, 4), dtype=bool)
+    rows, groups = np.indices(nib.shape)
+    mask[rows, groups, nib & 3] = True
+    mask[rows, groups, nib >> 2] = True
+    return mask.reshape(d_out, d_in)
+
+
+def _check_p1(W, vals, meta, U32, V32, what, max_ambiguous=1e-2):
+    """S must be the 2:4 hard threshold (HASSLE-free section 4.1.1) of W - L with
+    L = U32 V32, the GPU's own unrounded low-rank part: identical kept positions
+    in every group except those where the second and third largest |W - L|
+    lie within the GPU's rounding of each other, and kept values equal to
+    W - L rounded to bf16.  The GPU forms L from bf16 hi/lo planes of the two
+    factors (|error| <= 2^-16 (|U32||V32|)_ij per product, three products) and
+    W - L in fp32; the tolerance per entry is four times that estimate."""
+    d_out, d_in = W.shape
+    Wf = bits_to_f64(W)
+    Uf = U32.double().cpu().numpy()
+    Vf = V32.double().cpu().numpy()
+    L = Uf @ Vf
+    R = Wf - L
+    tol = 4.0 * (3 * 2.0 ** -16 * (np.abs(Uf) @ np.abs(Vf)) + 2.0 ** -23 * (np.abs(Wf) + np.abs(L)))
+    keep_ref = am.keep_mask_2to4(R)
+    keep_gpu = _gpu_mask(meta, d_out, d_in)
+    # ambiguous groups: the two entries either side of the cut are within tolerance
+    a = np.abs(R).reshape(d_out, -1, 4)
+    t = tol.reshape(d_out, -1, 4)
+    order = np.argsort(-a, axis=-1, kind="stable")
+    a2 = np.take_along_axis(a, order[..., 1:2], -1)[..., 0]
+    a3 = np.take_along_axis(a, order[..., 2:3], -1)[..., 0]
+    t2 = np.take_along_axis(t, order[..., 1:2], -1)[..., 0]
+    t3 = np.take_along_axis(t, order[..., 2:3], -1)[..., 0]
+    ambiguous = (a2 - a3) <= (t2 + t3)
+    differs = np.any(keep_ref.reshape(d_out, -1, 4) != keep_gpu.reshape(d_out, -1, 4), axis=-1)
+    n_groups = differs.size
+    assert not np.any(differs & ~ambiguous), \
+        f"{what}: {int(np.sum(differs & ~ambiguous))} groups keep other positions than the hard threshold " \
+        f"of W - U32 V32 outside rounding ties (first at row, group {np.argwhere(differs & ~ambiguous)[0]})"
+    assert ambiguous.sum() <= max_ambiguous * n_groups, (what, int(ambiguous.sum()), n_groups)
+    # kept values: bf16 of W - L (half an ulp of bf16, plus the tolerance)
+    S = bits_to_f64(oracle_unpack(vals, meta, d_in))
+    ok = np.repeat(~ambiguous, 4, axis=-1).reshape(d_out, d_in) & keep_gpu
+    err = np.abs(S - R)
+    bound = 2.0 ** -8 * np.abs(R) + tol + 1e-30
+    assert np.all(err[ok] <= bound[ok]), f"{what}: kept value off W - L by {float(np.max(err[ok] - bound[ok])):.3g}"
+    assert np.all(S[~keep_gpu] == 0.0)
+    return int(differs.sum()), int(ambiguous.sum()), n_groups
+
+
+def oracle_unpack(vals, meta, d_in):
+    import oracle
+    return oracle.unpack_2to4(from_dev(vals), meta.cpu().numpy(), d_in)
+
+
+@pytest.mark.parametrize("d_out,d_in,r,iters", [(256, 128, 8, 3), (192, 320, 16, 2), (520, 264, 32, 2)])
+def test_decompose_p1_and_p2_element_wise_gapped(d_out, d_in, r, iters):
+    """After `iters` iterations:
+    P1 -- S is the hard threshold of W - U32 V32 (see _check_p1);
+    P2 -- U32 V32 is C_r(W - S_prev) (HASSLE-free section 4.2.1) element by
+    element, S_prev being the GPU's S after iters - 1 iterations (the run is
+    deterministic and warm-started, so the shorter run is a prefix of the
+    longer one): |L_gpu - C_r|_ij <= 2e-4 max|C_r| (fp32 subspace iteration
+    on hi/lo planes of W - S_prev, converged on a matrix with a spectral gap),
+    and the bf16 factors U V within their rounding, 2^-7 (|U||V|)_ij, of it."""
+    W = _gapped(d_out, d_in, r, d_out + r)
+    q0 = _q0(d_in, r, 5)
+    vp, mp, _, _, _ = slr.decompose_datafree(to_dev(W), r, iters - 1, power_first=40, power=10, Q0=q0)
+    vals, meta, U, V, obj, U32, V32 = slr.decompose_datafree(to_dev(W), r, iters, power_first=40, power=10, Q0=q0,
+                                                             factors_f32=True)
+    torch.cuda.synchronize()
+    _check_p1(W, vals, meta, U32, V32, f"P1 {d_out}x{d_in} r={r}")
+    Wf = bits_to_f64(W)
+    S_prev = bits_to_f64(oracle_unpack(vp, mp, d_in))
+    L_ref = am.truncated_svd(Wf - S_prev, r)
+    L_gpu = U32.double().cpu().numpy() @ V32.double().cpu().numpy()
+    scale = np.max(np.abs(L_ref))
+    err = np.abs(L_gpu - L_ref)
+    assert np.max(err) <= 2e-4 * scale, f"P2: max |U32 V32 - C_r(W - S_prev)| = {np.max(err) / scale:.3g} of max|C_r|"
+    Ub, Vb = bits_to_f64(from_dev(U)), bits_to_f64(from_dev(V))
+    errb = np.abs(Ub @ Vb - L_ref)
+    assert np.all(errb <= 2.0 ** -7 * (np.abs(Ub) @ np.abs(Vb)) + 2e-4 * scale), "P2: bf16 factors"
+
+
+def test_decompose_config_layer_start_and_threshold():
+    """The gate/up layer (14336 x 4096, r = 64), iters = 0: the start's U32 V32
+    captures the top-r energy of W up to the subspace iteration's convergence
+    (||W - U32 V32||_F between the Eckart-Young error, from the eigenvalues of
+    W^T W, and 1.002 times it), and S is the hard threshold of W - U32 V32
+    element by element (P1 check above)."""
+    layer = next(l for l in synth.CONFIGS[3].layers if l.name == "gate_up")
+    W = layer.weight()
+    vals, meta, U, V, obj, U32, V32 = slr.decompose_datafree(to_dev(W), 64, 0, power_first=8, power=2,
+                                                             Q0=_q0(layer.d_in, 64, 3), factors_f32=True)
+    torch.cuda.synchronize()
+    Wf = bits_to_f64(W)
+    ev = np.linalg.eigvalsh(Wf.T @ Wf)
+    ey = np.sqrt(max(np.sum(Wf * Wf) - np.sum(ev[-64:]), 0.0))
+    L = U32.double().cpu().numpy() @ V32.double().cpu().numpy()
+    fit = np.linalg.norm(Wf - L)
+    assert ey * (1 - 1e-6) <= fit <= ey * 1.002, (fit, ey)
+    del L
+    _check_p1(W, vals, meta, U32, V32, "P1 gate/up start")

@@ -84,7 +84,7 @@ def _forward_case(cfg, name, M, path, k_rows=48, k_outs=384):
     outs = sample_indices(layer.d_out, k_outs, seed=cfg * 11 + layer.d_out)
     Yref, Bref = oracle.forward(X, vals, meta, U, V, rows=rows, outs=outs)
     Yg = from_dev(Y)[np.ix_(rows, outs)]
-    return check_forward(Yg, Yref, Bref, f"cfg{cfg} {name} M={M} path={path}")
+    return check_forward(Yg, Yref, Bref, f"cfg{cfg} {name} M={M} path={path}", rows, outs)
 
 
 def _cases():
@@ -119,7 +119,8 @@ def _lowrank_only(d_out, d_in, r, M, path, seed):
     rows = sample_indices(M, 40, seed)
     outs = sample_indices(d_out, 300, seed + 5)
     Yref, Bref = oracle.forward(X, vals, meta, U, V, rows=rows, outs=outs)
-    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, f"lowrank-only {d_out}x{d_in} r={r} M={M} {path}")
+    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, f"lowrank-only {d_out}x{d_in} r={r} M={M} {path}",
+                  rows, outs)
 
 
 @pytest.mark.parametrize("path", ["decode", "tensor"])
@@ -193,7 +194,7 @@ def test_forward_plan_shapes(d_out, d_in, r, M):
     rows = sample_indices(M, 48, seed)
     outs = sample_indices(d_out, 512, seed + 1)
     Yref, Bref = oracle.forward(X, vals, meta, U, V, rows=rows, outs=outs)
-    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, f"plan {d_out}x{d_in} r={r} M={M}")
+    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, f"plan {d_out}x{d_in} r={r} M={M}", rows, outs)
 
 
 def test_forward_matches_between_paths():
@@ -241,7 +242,7 @@ def test_forward_tensor_variants(variant, d_out, d_in, r, M, monkeypatch):
     slr.check_kernel_error()
     rows = sample_indices(M, 64, seed)
     Yref, Bref = oracle.forward(X, vals, meta, U, V, rows=rows)
-    check_forward(from_dev(Y)[rows], Yref, Bref, f"{variant} {d_out}x{d_in} r={r} M={M}")
+    check_forward(from_dev(Y)[rows], Yref, Bref, f"{variant} {d_out}x{d_in} r={r} M={M}", rows)
 
 
 @pytest.mark.parametrize("variant", VARIANTS)

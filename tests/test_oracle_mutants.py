@@ -82,7 +82,7 @@ def test_mutant_is_caught(name, old, new, count, tmp_path):
 AM_SRC = os.path.join(os.path.dirname(oracle.__file__), "datafree_am.py")
 AM_MUTANTS = [
     ("am_tie_to_higher", "            if q < p:\n", "            if q > p:\n", 1),
-    ("am_keep_three", "keep = (beaten < 2)", "keep = (beaten < 3)", 1),
+    ("am_keep_three", "return (beaten < 2).reshape", "return (beaten < 3).reshape", 1),
     ("am_truncation_one_more", "return (Uz[:, :r] * sz[:r]) @ Vz[:r, :]", "return (Uz[:, :r + 1] * sz[:r + 1]) @ Vz[:r + 1, :]", 1),
     ("am_smallest_singular", "return (Uz[:, :r] * sz[:r]) @ Vz[:r, :]", "return (Uz[:, -r:] * sz[-r:]) @ Vz[-r:, :]", 1),
     ("am_threshold_signed", "g = np.abs(R).reshape", "g = R.reshape", 1),
