@@ -40,6 +40,7 @@ import synth  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
 PREFILL = dict(cfg=3, name="gate_up", M=2048)
+CHAIN_MAX_M = 64   # the small-M kernels honour SLR_FWD_OVERLAP_PRECEDING up to this M
 DECODE = dict(cfg=2, name="q_proj", M=1)
 
 # Fallback peaks (the profiling recipe's earlier measurement on this machine),
@@ -388,7 +389,18 @@ def roofline_time(M, d_out, d_in, r, peaks):
 
 def measure_point(slr, torch, dev, cache, L, M, K, peaks, max_over_ranks, barrier):
     """One (layer, M) point: K forward steps in a CUDA graph over rotating
-    buffer sets (sized past L2); returns the metrics of the point."""
+    buffer sets (sized past L2); returns the metrics of the point.  Up to
+    CHAIN_MAX_M tokens the same K steps are also timed as chained calls
+    (SLR_FWD_OVERLAP_PRECEDING: each step may stream its weights while the
+    previous step finishes, as consecutive layers of a decode loop do)."""
+    point = _measure_point(slr, torch, dev, cache, L, M, K, peaks, max_over_ranks, barrier, False)
+    if M <= CHAIN_MAX_M:
+        ch = _measure_point(slr, torch, dev, cache, L, M, K, peaks, max_over_ranks, barrier, True)
+        point["chained"] = {k: ch[k] for k in ("ms", "tflops_dense_equiv", "gbs", "frac_of_roofline")}
+    return point
+
+
+def _measure_point(slr, torch, dev, cache, L, M, K, peaks, max_over_ranks, barrier, chained):
     vals, meta, U, V = cache.weights(L)
     d_out, d_in, r = L.d_out, L.d_in, L.r
     path = slr.select_path(M, d_out, d_in, r)
@@ -403,7 +415,8 @@ def measure_point(slr, torch, dev, cache, L, M, K, peaks, max_over_ranks, barrie
                          ws=torch.empty(ws_bytes, dtype=torch.uint8, device=dev)))
 
     def fwd(s):
-        slr.forward(s["X"], s["vals"], s["meta"], s["U"], s["V"], out=s["Y"], workspace=s["ws"], path=path)
+        slr.forward(s["X"], s["vals"], s["meta"], s["U"], s["V"], out=s["Y"], workspace=s["ws"], path=path,
+                    overlap_preceding=chained)
 
     for i in range(3):
         fwd(sets[i % n_copies])
@@ -587,12 +600,18 @@ def run_decode_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier
     for i in range(max(args.warmup, 10)):
         project(sets[i % n_copies])
         combine(sets[i % n_copies])
-    def fwd(s):
-        slr.forward(s["X"], s["vals"], s["meta"], s["U"], s["V"], out=s["Y"], workspace=s["ws"], path=path)
+    def fwd(s, chained=False):
+        slr.forward(s["X"], s["vals"], s["meta"], s["U"], s["V"], out=s["Y"], workspace=s["ws"], path=path,
+                    overlap_preceding=chained)
 
     step_fns = [lambda s=sets[k % n_copies]: fwd(s) for k in range(K)]
     barrier()
     total_ms = max_over_ranks(graph_time_ms(torch, step_fns))
+    barrier()
+    # the same K steps as chained calls (SLR_FWD_OVERLAP_PRECEDING), as
+    # back-to-back layers of a decode loop issue them
+    chain_ms = max_over_ranks(graph_time_ms(torch, [lambda s=sets[k % n_copies]: fwd(s, True)
+                                                    for k in range(K)])) / K
     barrier()
     combine_ms = graph_time_ms(torch, [lambda s=sets[k % n_copies]: combine(s) for k in range(K)]) / K
     ms = total_ms / K
@@ -604,6 +623,10 @@ def run_decode_leg(args, slr, torch, dev, to_dev, peaks, max_over_ranks, barrier
     return {"workload": "Llama-3-8B q_proj decode: 4096x4096, r=64, M=1", "path": path,
             "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 5), "steps": K,
             "frac": round(gbs / peaks["hbm_gbs"], 4), "algorithmic_bytes": nbytes,
+            "chained": {"ms_per_step": round(chain_ms, 5), "value": round(nbytes / (chain_ms * 1e-3) / 1e9, 1),
+                        "frac": round(nbytes / (chain_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                        "how": "slr_forward_ex with SLR_FWD_OVERLAP_PRECEDING: each step may stream its "
+                               "weights while the previous step finishes"},
             "kernel": {"name": "decode_forward_kernel", "ms": round(combine_ms, 5), "bytes": k_bytes,
                        "gbs": round(k_gbs, 1), "frac": round(k_gbs / peaks["hbm_gbs"], 4)},
             "l2": f"rotating {n_copies} buffer sets of {nbytes / 1e6:.1f} MB"}

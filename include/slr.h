@@ -349,6 +349,29 @@ SLR_API slr_status slr_forward_with_path(const void *X, int64_t M, const void *v
                                  int64_t r, void *Y, void *workspace, size_t workspace_bytes,
                                  slr_path path, slr_stream_t stream);
 
+/* Option bits of slr_forward_ex.
+ *
+ * SLR_FWD_OVERLAP_PRECEDING: the call's kernels may start while the kernel
+ * queued just before them on `stream` is still running (programmatic
+ * dependent launch).  Before that kernel has completed they only read the
+ * layer's weights (vals, meta, U, V); they wait for it before they read X,
+ * read or write the workspace, or write Y.  Back-to-back layers of a decode
+ * loop then stream the next layer's weights while the previous layer
+ * finishes, which hides the launch and ramp-up time of layers of a few tens
+ * of MB.  The caller guarantees that the kernel queued immediately before
+ * the call does not write vals, meta, U or V (weights written earlier, with
+ * at least one other kernel or any copy or event in between, are fine).
+ * Honoured for the small-M kernels (the streaming path, and the tensor-core
+ * path up to 64 tokens with r <= 256); other calls run as without the flag.
+ * The result is the same bits as without the flag. */
+#define SLR_FWD_OVERLAP_PRECEDING 1u
+
+/* slr_forward_with_path with option bits (SLR_FWD_*); unknown bits return
+ * SLR_ERR_ARG.  flags == 0 is slr_forward_with_path. */
+SLR_API slr_status slr_forward_ex(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out,
+                                  int64_t d_in, const void *U, const void *V, int64_t r, void *Y, void *workspace,
+                                  size_t workspace_bytes, slr_path path, uint32_t flags, slr_stream_t stream);
+
 /* The two stages of slr_forward, for callers that schedule or time them
  * separately.  slr_forward(...) == slr_forward_project(...) followed on the same
  * stream by slr_forward_combine(...) with the same path and workspace.

@@ -16,7 +16,7 @@ Functions mirror the C ABI in ``include/slr.h``:
 * ``decompose_datafree(W, r, iters, ...) -> (vals, meta, U, V, objective)``  --
   ``slr_decompose_datafree``
 * ``forward(X, vals, meta, U, V) -> Y``  -- ``slr_forward`` /
-  ``slr_forward_with_path``
+  ``slr_forward_with_path`` / ``slr_forward_ex``
 * ``workspace_size``, ``select_path``, ``check_kernel_error``
 
 Tensors are torch CUDA tensors (torch only provides memory and the current
@@ -85,6 +85,8 @@ def _load() -> ctypes.CDLL:
     lib.slr_forward.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, p, sz, p]
     lib.slr_forward_with_path.restype = st
     lib.slr_forward_with_path.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, p, sz, st, p]
+    lib.slr_forward_ex.restype = st
+    lib.slr_forward_ex.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, p, sz, st, ctypes.c_uint32, p]
     lib.slr_forward_workspace_size.restype = sz
     lib.slr_forward_workspace_size.argtypes = [i64, i64, i64, i64]
     lib.slr_forward_select_path.restype = st
@@ -276,10 +278,17 @@ def select_path(M: int, d_out: int, d_in: int, r: int) -> str:
     return PATH_NAMES[int(_lib.slr_forward_select_path(M, d_out, d_in, r))]
 
 
+FWD_OVERLAP_PRECEDING = 1
+
+
 def forward(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, U: torch.Tensor | None,
             V: torch.Tensor | None, *, path: str = "auto", out: torch.Tensor | None = None,
-            workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """``Y = X @ S.T + (X @ V.T) @ U.T`` with S given packed by ``pack_2to4``."""
+            workspace: torch.Tensor | None = None, overlap_preceding: bool = False) -> torch.Tensor:
+    """``Y = X @ S.T + (X @ V.T) @ U.T`` with S given packed by ``pack_2to4``.
+
+    ``overlap_preceding`` sets ``SLR_FWD_OVERLAP_PRECEDING`` (``slr_forward_ex``):
+    the call may start reading its weights while the kernel queued just before
+    it is still running, which that kernel must not write."""
     M, d_in = X.shape
     d_out = vals.shape[0]
     r = 0 if U is None else U.shape[1]
@@ -289,8 +298,9 @@ def forward(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, U: torch.Te
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(_lib.slr_forward_with_path(_ptr(X), M, _ptr(vals), _ptr(meta), d_out, d_in, _ptr(U), _ptr(V), r,
-                                      _ptr(out), _ptr(workspace), ws_bytes, PATHS[path], _stream()),
+    flags = FWD_OVERLAP_PRECEDING if overlap_preceding else 0
+    _check(_lib.slr_forward_ex(_ptr(X), M, _ptr(vals), _ptr(meta), d_out, d_in, _ptr(U), _ptr(V), r,
+                               _ptr(out), _ptr(workspace), ws_bytes, PATHS[path], flags, _stream()),
            "slr_forward")
     return out
 

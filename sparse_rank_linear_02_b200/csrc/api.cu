@@ -9,6 +9,8 @@ namespace slr {
 namespace {
 
 constexpr size_t kAlign = 256;
+// Largest M whose tensor-core path takes T from the CUDA-core projection.
+constexpr int64_t kSmallProjectM = 16;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -89,19 +91,26 @@ slr_status validate(const void *X, int64_t M, const void *vals, const void *meta
 }
 
 // Stage 1: T = X V^T into the workspace, fp32 for the streaming path and bf16
-// for the tensor-core path.
+// for the tensor-core path.  chained: see forward_impl.
 cudaError_t run_project(const void *X, int64_t M, const void *V, int64_t d_in, int64_t r, void *workspace,
-                        slr_path p, cudaStream_t stream) {
+                        slr_path p, bool chained, cudaStream_t stream) {
     if (r == 0) return cudaSuccess;
     const uint16_t *x = static_cast<const uint16_t *>(X);
     const uint16_t *vv = static_cast<const uint16_t *>(V);
-    if (p == SLR_PATH_DECODE) return launch_lowrank_project(x, M, vv, d_in, r, static_cast<float *>(workspace), nullptr, stream);
-    return launch_tc_project(x, M, vv, d_in, r, static_cast<uint16_t *>(workspace), stream);
+    if (p == SLR_PATH_DECODE)
+        return launch_lowrank_project(x, M, vv, d_in, r, static_cast<float *>(workspace), nullptr, chained, stream);
+    // Up to 16 tokens the CUDA-core projection (r x 1..2 CTAs, fp32 sums
+    // rounded to bf16) finishes well before the streaming combine needs T;
+    // the tensor-core projection runs on a handful of CTAs there.
+    if (M <= kSmallProjectM)
+        return launch_lowrank_project(x, M, vv, d_in, r, nullptr, static_cast<uint16_t *>(workspace), chained, stream);
+    return launch_tc_project(x, M, vv, d_in, r, static_cast<uint16_t *>(workspace), chained, stream);
 }
 
-// Stage 2: Y = X S^T + T U^T with T read from the workspace.
+// Stage 2: Y = X S^T + T U^T with T read from the workspace.  pdl: 0 ordinary
+// launch, 1 right after the projection, 2 chained.
 cudaError_t run_combine(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out, int64_t d_in,
-                        const void *U, int64_t r, void *Y, const void *workspace, slr_path p, bool after_projection,
+                        const void *U, int64_t r, void *Y, const void *workspace, slr_path p, int pdl,
                         cudaStream_t stream) {
     const uint16_t *x = static_cast<const uint16_t *>(X);
     const uint16_t *v = static_cast<const uint16_t *>(vals);
@@ -110,20 +119,40 @@ cudaError_t run_combine(const void *X, int64_t M, const void *vals, const void *
     uint16_t *y = static_cast<uint16_t *>(Y);
     if (p == SLR_PATH_DECODE)
         return launch_decode_forward(x, M, v, m, d_out, d_in, u, r > 0 ? static_cast<const float *>(workspace) : nullptr,
-                                     r, y, after_projection, stream);
+                                     r, y, pdl, stream);
     return launch_tc_forward(x, M, v, m, d_out, d_in, u, r > 0 ? static_cast<const uint16_t *>(workspace) : nullptr,
-                             r, y, after_projection, stream);
+                             r, y, pdl, stream);
 }
 
+// Whether a call with SLR_FWD_OVERLAP_PRECEDING runs chained: the small-M
+// kernels (the streaming path where it stages X in shared memory, and the
+// split-K tensor kernel with its projection up to kChainMaxM tokens and rank
+// 256) support it; other calls launch as without the flag, which is also
+// correct.
+bool chain_supported(slr_path p, int64_t M, int64_t d_in, int64_t r) {
+    if (p == SLR_PATH_DECODE) return decode_chain_ok(M, d_in);
+    return M <= kChainMaxM && r <= 256;
+}
+
+// Chained (flags & SLR_FWD_OVERLAP_PRECEDING, where supported): the
+// projection is a programmatic dependent of the work before the call, the
+// combine a programmatic dependent of the projection; both request only
+// weights (V; S and U) before they wait for the preceding grid, and read X,
+// read or write T, and write Y after.  Otherwise the projection is an
+// ordinary launch and the combine a programmatic dependent of it that waits
+// only before reading T.
 slr_status forward_impl(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out,
                         int64_t d_in, const void *U, const void *V, int64_t r, void *Y, void *workspace,
-                        size_t workspace_bytes, slr_path path, cudaStream_t stream) {
+                        size_t workspace_bytes, slr_path path, uint32_t flags, cudaStream_t stream) {
     slr_path p;
+    if ((flags & ~(uint32_t)SLR_FWD_OVERLAP_PRECEDING) != 0) return SLR_ERR_ARG;
     const slr_status st = validate(X, M, vals, meta, d_out, d_in, U, V, r, Y, workspace, workspace_bytes, path,
                                    true, true, true, &p);
     if (st != SLR_OK || M == 0) return st;
-    cudaError_t err = run_project(X, M, V, d_in, r, workspace, p, stream);
-    if (err == cudaSuccess) err = run_combine(X, M, vals, meta, d_out, d_in, U, r, Y, workspace, p, true, stream);
+    const bool chained = (flags & SLR_FWD_OVERLAP_PRECEDING) != 0 && chain_supported(p, M, d_in, r);
+    cudaError_t err = run_project(X, M, V, d_in, r, workspace, p, chained, stream);
+    if (err == cudaSuccess)
+        err = run_combine(X, M, vals, meta, d_out, d_in, U, r, Y, workspace, p, chained ? 2 : 1, stream);
     return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
 }
 
@@ -218,7 +247,7 @@ slr_status slr_forward_2to8(const void *X, int64_t M, const void *vals8, const v
     const uint16_t *x = static_cast<const uint16_t *>(X);
     float *T32 = r > 0 ? static_cast<float *>(workspace) : nullptr;
     cudaError_t err = cudaSuccess;
-    if (r > 0) err = slr::launch_lowrank_project(x, M, static_cast<const uint16_t *>(V), d_in, r, T32, nullptr, st);
+    if (r > 0) err = slr::launch_lowrank_project(x, M, static_cast<const uint16_t *>(V), d_in, r, T32, nullptr, false, st);
     if (err == cudaSuccess)
         err = slr::launch_decode28_forward(x, M, static_cast<const uint16_t *>(vals8),
                                            static_cast<const uint8_t *>(meta8), d_out, d_in,
@@ -371,7 +400,7 @@ slr_status slr_forward(const void *X, int64_t M, const void *vals, const void *m
                        const void *U, const void *V, int64_t r, void *Y, void *workspace, size_t workspace_bytes,
                        slr_stream_t stream) {
     return slr::forward_impl(X, M, vals, meta, d_out, d_in, U, V, r, Y, workspace, workspace_bytes, SLR_PATH_AUTO,
-                             reinterpret_cast<cudaStream_t>(stream));
+                             0u, reinterpret_cast<cudaStream_t>(stream));
 }
 
 slr_status slr_forward_project(const void *X, int64_t M, const void *V, int64_t d_out, int64_t d_in, int64_t r,
@@ -381,7 +410,8 @@ slr_status slr_forward_project(const void *X, int64_t M, const void *V, int64_t 
     const slr_status st = slr::validate(X, M, dummy, dummy, d_out, d_in, nullptr, V, r, dummy, workspace,
                                         workspace_bytes, path, false, false, true, &p);
     if (st != SLR_OK || M == 0) return st;
-    return slr::run_project(X, M, V, d_in, r, workspace, p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+    return slr::run_project(X, M, V, d_in, r, workspace, p, false, reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
                ? SLR_OK
                : SLR_ERR_CUDA;
 }
@@ -393,7 +423,7 @@ slr_status slr_forward_combine(const void *X, int64_t M, const void *vals, const
     const slr_status st = slr::validate(X, M, vals, meta, d_out, d_in, U, nullptr, r, Y, workspace, workspace_bytes,
                                         path, true, true, false, &p);
     if (st != SLR_OK || M == 0) return st;
-    return slr::run_combine(X, M, vals, meta, d_out, d_in, U, r, Y, workspace, p, false,
+    return slr::run_combine(X, M, vals, meta, d_out, d_in, U, r, Y, workspace, p, 0,
                             reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SLR_OK
                : SLR_ERR_CUDA;
@@ -402,7 +432,14 @@ slr_status slr_forward_combine(const void *X, int64_t M, const void *vals, const
 slr_status slr_forward_with_path(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out,
                                  int64_t d_in, const void *U, const void *V, int64_t r, void *Y, void *workspace,
                                  size_t workspace_bytes, slr_path path, slr_stream_t stream) {
-    return slr::forward_impl(X, M, vals, meta, d_out, d_in, U, V, r, Y, workspace, workspace_bytes, path,
+    return slr::forward_impl(X, M, vals, meta, d_out, d_in, U, V, r, Y, workspace, workspace_bytes, path, 0u,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+slr_status slr_forward_ex(const void *X, int64_t M, const void *vals, const void *meta, int64_t d_out, int64_t d_in,
+                          const void *U, const void *V, int64_t r, void *Y, void *workspace, size_t workspace_bytes,
+                          slr_path path, uint32_t flags, slr_stream_t stream) {
+    return slr::forward_impl(X, M, vals, meta, d_out, d_in, U, V, r, Y, workspace, workspace_bytes, path, flags,
                              reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -29,6 +29,31 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
     return v;
 }
 
+// Loads of data that another grid writes while this one may already run (T
+// from the projection kernel, X in a chained launch): ordinary coherent loads
+// that bypass L1 (.cg), issued from volatile asm so that the compiler keeps
+// them after the griddepcontrol.wait that precedes them.  Read-only loads
+// (__ldg, ld.global.nc) must not be used for such data: the compiler treats
+// them as invariant and may move them above the wait.
+__device__ __forceinline__ float ld_dep_f32(const float *p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ float2 ld_dep_f2(const float *p) {
+    float2 v;
+    asm volatile("ld.global.cg.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint4 ld_dep_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error; arguments were validated by
 // the API layer.
@@ -104,17 +129,23 @@ cudaError_t launch_column_norms(const uint16_t *X, int64_t M, int64_t d_in, int6
                                 float *norms, float *partial, cudaStream_t stream);
 
 // T = X * V^T for M tokens, written as fp32 [M, r] (T32, may be null) and/or
-// bf16 [M, r] (T16, may be null).
+// bf16 [M, r] (T16, may be null).  chained: launched as a programmatic
+// dependent of whatever precedes it on `stream`; V is prefetched into L2 at
+// once, X read and T written only after the wait for the preceding grid.
 cudaError_t launch_lowrank_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in,
-                                   int64_t r, float *T32, uint16_t *T16, cudaStream_t stream);
+                                   int64_t r, float *T32, uint16_t *T16, bool chained, cudaStream_t stream);
 
 // Small-M streaming forward: Y = X S^T + T U^T with T (fp32 [M, r]) precomputed.
-// after_projection: the projection kernel that writes T32 is the kernel
-// launched immediately before on `stream` (enables programmatic dependent
-// launch; must be false otherwise).
+// pdl_mode: 0 = ordinary launch; 1 = the projection kernel that writes T32 is
+// the kernel launched immediately before on `stream` (programmatic dependent
+// launch, waits before reading T32).  Chained launches (2) are not supported
+// by this kernel (decode_chain_ok).
+// Whether the streaming forward supports chained launches for this M and d_in.
+bool decode_chain_ok(int64_t M, int64_t d_in);
+
 cudaError_t launch_decode_forward(const uint16_t *X, int64_t M, const uint16_t *vals,
                                   const uint8_t *meta, int64_t d_out, int64_t d_in,
                                   const uint16_t *U, const float *T32, int64_t r, uint16_t *Y,
-                                  bool after_projection, cudaStream_t stream);
+                                  int pdl_mode, cudaStream_t stream);
 
 }  // namespace slr

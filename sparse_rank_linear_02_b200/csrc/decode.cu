@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kWarps * 32, kBlocksPerSm) decode_forward_kern
             if (r > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
             for (int t = 0; t < MT; ++t)
-                tr[t] = (rk && t < nt) ? __ldg(reinterpret_cast<const float2 *>(T32 + (m0 + t) * r) + lane) : make_float2(0.f, 0.f);
+                tr[t] = (rk && t < nt) ? ld_dep_f2(T32 + (m0 + t) * r + 2 * lane) : make_float2(0.f, 0.f);
         };
 
         for (int64_t c0 = lane; c0 < chunks; c0 += 32 * kUnroll) {
@@ -125,15 +125,17 @@ __global__ void __launch_bounds__(kWarps * 32, kBlocksPerSm) decode_forward_kern
         if (!t_loaded) load_t();   // lanes that had no weight chunk
         // Rank-r term: lanes split k, products land in the same partial sums.
         // T comes from the projection kernel, which may still be running when
-        // this kernel starts (programmatic dependent launch); it was loaded
-        // after griddepcontrol.wait above.  Ranks past 64 continue here.
+        // this kernel starts (programmatic dependent launch); it is read after
+        // griddepcontrol.wait, with ordered L2 loads (a read-only __ldg load
+        // counts as invariant and may be moved above the wait).  Ranks past
+        // 64 continue here.
 #pragma unroll
         for (int t = 0; t < MT; ++t) acc[t] = fmaf(ur1, tr[t].y, fmaf(ur0, tr[t].x, acc[t]));
         for (int64_t k = lane + 64; k < r; k += 32) {
             const float u = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(U) + row * r + k) << 16);
 #pragma unroll
             for (int t = 0; t < MT; ++t)
-                if (t < nt) acc[t] = fmaf(u, __ldg(T32 + (m0 + t) * r + k), acc[t]);
+                if (t < nt) acc[t] = fmaf(u, ld_dep_f32(T32 + (m0 + t) * r + k), acc[t]);
         }
 
 #pragma unroll
@@ -184,10 +186,16 @@ cudaError_t launch_mt(const uint16_t *X, int64_t M, const uint16_t *vals, const 
 
 }  // namespace
 
+bool decode_chain_ok(int64_t, int64_t) {
+    // Seven CTAs of this kernel fill an SM's registers, so a following launch
+    // could not start early anyway: chained calls run as ordinary ones here.
+    return false;
+}
+
 cudaError_t launch_decode_forward(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                   int64_t d_out, int64_t d_in, const uint16_t *U, const float *T32, int64_t r,
-                                  uint16_t *Y, bool after_projection, cudaStream_t stream) {
-    const bool pdl = after_projection && r > 0;
+                                  uint16_t *Y, int pdl_mode, cudaStream_t stream) {
+    const bool pdl = pdl_mode != 0 && r > 0;
     if (M <= 1) return launch_mt<1>(X, M, vals, meta, d_out, d_in, U, T32, r, Y, pdl, stream);
     if (M <= 2) return launch_mt<2>(X, M, vals, meta, d_out, d_in, U, T32, r, Y, pdl, stream);
     if (M <= 4) return launch_mt<4>(X, M, vals, meta, d_out, d_in, U, T32, r, Y, pdl, stream);

@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kWarps28 * 32) decode28_forward_kernel(
             if (r > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
             for (int t = 0; t < MT; ++t)
-                tr[t] = (rk && t < nt) ? __ldg(reinterpret_cast<const float2 *>(T32 + (m0 + t) * r) + lane)
+                tr[t] = (rk && t < nt) ? ld_dep_f2(T32 + (m0 + t) * r + 2 * lane)
                                        : make_float2(0.f, 0.f);
         };
 
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kWarps28 * 32) decode28_forward_kernel(
                     (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(U) + (row0 + q) * r + k) << 16);
 #pragma unroll
                 for (int t = 0; t < MT; ++t)
-                    if (t < nt) acc[q][t] = fmaf(u, __ldg(T32 + (m0 + t) * r + k), acc[q][t]);
+                    if (t < nt) acc[q][t] = fmaf(u, ld_dep_f32(T32 + (m0 + t) * r + k), acc[q][t]);
             }
         }
 
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtasPerSm) decode28_ring_ke
             if (p.r > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
             for (int t = 0; t < MT; ++t)
-                tr[t] = (rk && t < nt) ? __ldg(reinterpret_cast<const float2 *>(T32 + (m0 + t) * p.r) + gi)
+                tr[t] = (rk && t < nt) ? ld_dep_f2(T32 + (m0 + t) * p.r + 2 * gi)
                                        : make_float2(0.f, 0.f);
         }
 #pragma unroll
@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtasPerSm) decode28_ring_ke
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
                     if (t >= nt) continue;
-                    const float2 tk = __ldg(reinterpret_cast<const float2 *>(T32 + (m0 + t) * p.r + k));
+                    const float2 tk = ld_dep_f2(T32 + (m0 + t) * p.r + k);
                     acc[j][t] = fmaf(bf16hi_to_f32(u2), tk.y, fmaf(bf16lo_to_f32(u2), tk.x, acc[j][t]));
                 }
             }

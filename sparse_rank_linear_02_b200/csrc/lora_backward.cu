@@ -98,7 +98,7 @@ cudaError_t launch_lora_backward(const uint16_t *X, int64_t M, const uint16_t *d
     uint16_t *G16 = ws + M * r;         // M x r
     cudaError_t e = cudaSuccess;
     if (T16_in == nullptr) {
-        e = launch_tc_project(X, M, V, d_in, r, T16, st);
+        e = launch_tc_project(X, M, V, d_in, r, T16, false, st);
         T16_in = T16;
     }
     if (e != cudaSuccess) return e;

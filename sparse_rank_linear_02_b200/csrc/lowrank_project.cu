@@ -35,11 +35,23 @@ __global__ void __launch_bounds__(kThreads) lowrank_project_kernel(const uint16_
                                                                    const uint16_t *__restrict__ V,
                                                                    int64_t d_in, int64_t r,
                                                                    float *__restrict__ T32,
-                                                                   uint16_t *__restrict__ T16) {
+                                                                   uint16_t *__restrict__ T16, int chained) {
     // Let the dependent streaming kernel launch now; it only reads T after
     // its own griddepcontrol.wait, which waits for this grid to complete.
     asm volatile("griddepcontrol.launch_dependents;");
     const int64_t k = blockIdx.x;
+    if (chained) {
+        // Launched while the preceding grid may still run: V (a weight) is
+        // pulled into L2 now; X is read, and T written, only after the wait.
+        if (threadIdx.x == 0 && blockIdx.y == 0) {
+            const uint8_t *row = reinterpret_cast<const uint8_t *>(V + k * d_in);
+            for (int64_t off = 0; off < d_in * 2; off += 32768) {
+                const int64_t n = d_in * 2 - off < 32768 ? d_in * 2 - off : 32768;
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(row + off), "r"((uint32_t)n) : "memory");
+            }
+        }
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+    }
     const int64_t m0 = (int64_t)blockIdx.y * kTokens;
     const int nt = (int)((M - m0) < kTokens ? (M - m0) : kTokens);
     float acc[kTokens];
@@ -53,7 +65,7 @@ __global__ void __launch_bounds__(kThreads) lowrank_project_kernel(const uint16_
 #pragma unroll
         for (int t = 0; t < kTokens; ++t) {
             if (t < nt) {
-                const uint4 x = __ldg(reinterpret_cast<const uint4 *>(X + (m0 + t) * d_in) + c);
+                const uint4 x = ld_dep_v4(reinterpret_cast<const uint4 *>(X + (m0 + t) * d_in) + c);
                 acc[t] = dot8(v, x, acc[t]);
             }
         }
@@ -82,13 +94,21 @@ __global__ void __launch_bounds__(kThreads) lowrank_project_kernel(const uint16_
 }  // namespace
 
 cudaError_t launch_lowrank_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in,
-                                   int64_t r, float *T32, uint16_t *T16, cudaStream_t stream) {
+                                   int64_t r, float *T32, uint16_t *T16, bool chained, cudaStream_t stream) {
     if (M == 0 || r == 0) return cudaSuccess;
     const int64_t tblocks = (M + kTokens - 1) / kTokens;
     if (tblocks > 65535) return cudaErrorInvalidConfiguration;
-    dim3 grid((unsigned)r, (unsigned)tblocks);
-    lowrank_project_kernel<<<grid, kThreads, 0, stream>>>(X, M, V, d_in, r, T32, T16);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)r, (unsigned)tblocks);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = chained ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, lowrank_project_kernel, X, M, V, d_in, r, T32, T16, (int)(chained ? 1 : 0));
 }
 
 }  // namespace slr

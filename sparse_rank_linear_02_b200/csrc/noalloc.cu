@@ -94,10 +94,10 @@ extern "C" slr_status slr_forward_decode_noalloc(const void *X, int64_t M, const
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const uint16_t *x = static_cast<const uint16_t *>(X);
     cudaError_t err = cudaSuccess;
-    if (r > 0) err = slr::launch_lowrank_project(x, M, static_cast<const uint16_t *>(V), d_in, r, T, nullptr, s);
+    if (r > 0) err = slr::launch_lowrank_project(x, M, static_cast<const uint16_t *>(V), d_in, r, T, nullptr, false, s);
     if (err == cudaSuccess)
         err = slr::launch_decode_forward(x, M, static_cast<const uint16_t *>(vals), static_cast<const uint8_t *>(meta),
                                          d_out, d_in, static_cast<const uint16_t *>(U), r > 0 ? T : nullptr, r,
-                                         static_cast<uint16_t *>(Y), true, s);
+                                         static_cast<uint16_t *>(Y), 1, s);
     return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
 }

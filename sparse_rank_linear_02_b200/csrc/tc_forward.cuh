@@ -15,19 +15,28 @@ bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64
               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
 }  // namespace tc
 
+// Largest M whose tensor-core forward (the split-K kernel) and projection
+// support chained launches.
+constexpr int64_t kChainMaxM = 64;
+
 // Y = X S^T + T U^T on the tensor cores.  T16 is bf16 [M, r] (may be null when
 // r == 0).  Requires d_in % 128 == 0, d_out % 8 == 0, r % 8 == 0.
-// after_projection: the kernel launched immediately before on `stream` is the
-// projection that writes T16 (enables programmatic dependent launch; must be
-// false otherwise).
+// pdl: 0 = ordinary launch; 1 = the kernel launched immediately before on
+// `stream` is the projection that writes T16 (programmatic dependent launch,
+// waits before reading T16); 2 = chained (M <= kChainMaxM): also the work
+// before the projection may still be running, so the kernel requests only
+// the weights (S, U) before it waits, and reads X and T16 after.
 cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                               int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
-                              uint16_t *Y, bool after_projection, cudaStream_t stream);
+                              uint16_t *Y, int pdl, cudaStream_t stream);
 
 // T = X V^T on the tensor cores, written as bf16 [M, r] (dense tcgen05 mode of
-// the same kernel).  Requires d_in % 64 == 0, r % 8 == 0.
+// the same kernel).  Requires d_in % 64 == 0, r % 8 == 0.  chained: launched
+// as a programmatic dependent of whatever precedes it on `stream` (M <=
+// kChainMaxM); it requests V first and waits for the preceding grid before it
+// reads X or writes T16.
 cudaError_t launch_tc_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in, int64_t r,
-                              uint16_t *T16, cudaStream_t stream);
+                              uint16_t *T16, bool chained, cudaStream_t stream);
 
 // Launches the failure-detection self-test kernel (a bounded wait that is
 // made to expire after limit_cycles SM clock cycles).

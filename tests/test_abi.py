@@ -212,6 +212,16 @@ def test_decompose_argument_errors():
         assert f(w, 64, 64, 8, 1, 1, 1, q, v, m, u, vv, None, ws, big, None) == DEVICE
 
 
+def test_forward_ex_flags():
+    f = slr.lib().slr_forward_ex
+    x, v, m, u, vv, y, ws = (P(0x10000 * k) for k in range(1, 8))
+    assert f(x, 1, v, m, 8, 128, u, vv, 8, y, ws, 1 << 20, 0, 2, None) == ARG      # unknown option bit
+    assert f(x, 1, v, m, 8, 128, u, vv, 8, y, ws, 1 << 20, 7, 1, None) == ARG      # unknown path
+    assert f(x, 1, v, m, 8, 100, u, vv, 8, y, ws, 1 << 20, 0, 1, None) == SHAPE    # d_in % 128
+    if not torch.cuda.is_available():
+        assert f(x, 1, v, m, 8, 128, u, vv, 8, y, ws, 1 << 20, 0, 1, None) == DEVICE
+
+
 def test_decompose_factors_f32_argument_errors():
     f = slr.lib().slr_decompose_factors_f32
     ws, u, v = P(0x10000), P(0x20000), P(0x30000)

@@ -266,3 +266,78 @@ def test_forward_tensor_variants_one_hot(variant, monkeypatch):
     V = synth.gaussian_bf16((8, d_in), 1.0, 6162)
     Y = slr.forward(to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U), to_dev(V), path="tensor")
     np.testing.assert_array_equal(bits_to_f64(from_dev(Y)), bits_to_f64(np.ascontiguousarray(S.T)))
+
+
+# ----------------------------------------------------------------------------- chained launches
+
+def _layer_case(d_out, d_in, r, M, seed, outliers=True):
+    X = synth.activations_bf16(M, d_in, seed, seed + 9 if outliers else None)
+    W = synth.gaussian_bf16((d_out, d_in), 0.02, seed + 1)
+    vals, meta = oracle.pack_2to4(W)
+    U = synth.gaussian_bf16((d_out, r), 0.5, seed + 2)
+    V = synth.gaussian_bf16((r, d_in), 0.5 / np.sqrt(max(r, 1)), seed + 3)
+    return X, vals, meta, U, V
+
+
+@pytest.mark.parametrize("path", ["decode", "tensor"])
+@pytest.mark.parametrize("d_out,d_in,r,M", [
+    (4096, 4096, 64, 1), (4096, 4096, 64, 4), (4096, 4096, 64, 16),   # q_proj decode: 37 slabs of 111 rows
+    (1024, 4096, 64, 16),     # 37 slabs of 28 rows
+    (3000, 2048, 128, 33),    # BN = 64, ragged last slab
+    (2048, 1024, 256, 64),    # four rank stages
+    (1024, 2048, 0, 7),       # no projection: the combine itself is chained
+    (28672, 8192, 64, 2),     # two CTAs per SM, 296 slabs of 97 rows
+])
+def test_forward_chained_matches_unchained(path, d_out, d_in, r, M):
+    """SLR_FWD_OVERLAP_PRECEDING changes when the kernels may start, not what
+    they compute: bit-identical Y, and within the oracle's bounds."""
+    seed = d_out + 7 * d_in + 11 * r + M
+    X, vals, meta, U, V = _layer_case(d_out, d_in, r, M, seed)
+    args = (to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U) if r else None, to_dev(V) if r else None)
+    Y0 = slr.forward(*args, path=path)
+    Y1 = slr.forward(*args, path=path, overlap_preceding=True)
+    torch.cuda.synchronize()
+    slr.check_kernel_error()
+    assert torch.equal(Y0.view(torch.int16), Y1.view(torch.int16))
+    rows = sample_indices(M, 16, seed)
+    outs = sample_indices(d_out, 512, seed + 1)
+    Yref, Bref = oracle.forward(X, vals, meta, U if r else None, V if r else None, rows=rows, outs=outs)
+    check_forward(from_dev(Y1)[np.ix_(rows, outs)], Yref, Bref, f"chained {d_out}x{d_in} r={r} M={M} {path}",
+                  rows, outs)
+
+
+@pytest.mark.parametrize("path", ["decode", "tensor"])
+@pytest.mark.parametrize("M", [1, 16])
+def test_forward_chained_dependent_layers(path, M):
+    """Eight square layers back to back, each reading the previous layer's Y as
+    its X and sharing one workspace, all queued as chained calls: identical
+    bits to the same sequence without the flag (a kernel that read X or the
+    workspace before the previous layer finished would differ)."""
+    d = 4096
+    layers = []
+    for l in range(8):
+        W = synth.gaussian_bf16((d, d), 0.05, 900 + l)
+        vals, meta = oracle.pack_2to4(W)
+        U = synth.gaussian_bf16((d, 64), 0.05, 950 + l)
+        V = synth.gaussian_bf16((64, d), 0.05, 970 + l)
+        layers.append((to_dev(vals), to_dev_u8(meta), to_dev(U), to_dev(V)))
+    X0 = to_dev(synth.activations_bf16(M, d, 990, None))
+    ws = torch.empty(max(slr.workspace_size(M, d, d, 64), 256), dtype=torch.uint8, device="cuda")
+
+    def run(chained):
+        x = X0
+        outs = []
+        for vals, meta, U, V in layers:
+            y = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
+            slr.forward(x, vals, meta, U, V, path=path, out=y, workspace=ws, overlap_preceding=chained)
+            outs.append(y)
+            x = y
+        torch.cuda.synchronize()
+        return outs
+
+    ref = run(False)
+    for rep in range(3):
+        got = run(True)
+        for l, (a, b) in enumerate(zip(ref, got)):
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"layer {l} differs (repeat {rep})"
+    slr.check_kernel_error()
