@@ -128,7 +128,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(load) if load else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(self.samples),
-                "window": "nvidia-smi every 20 ms over an untimed 0.5 s replay of the timed graph and the timed replay"}
+                "window": "nvidia-smi every 20 ms over an untimed replay of the timed graph and the timed replay"}
 
 
 # ----------------------------------------------------------------------------- timing
@@ -249,7 +249,15 @@ def run_ours(args, rank, world, dist):
     step_fns = [lambda s=sets[k % n_copies]: fwd(s) for k in range(K)]
     clk = ClockSampler(bus_id_of(torch, dev) if rank == 0 else None)
     barrier()
-    total_ms = max_over_ranks(graph_time_ms(torch, step_fns, clock=clk))
+    # The K timed steps follow the warm-up directly (a 40 ms untimed replay of
+    # the same graph lets the clock sampler see the GPU under this load): the
+    # clocks of a run of milliseconds, which the burst peak describes.
+    total_ms = max_over_ranks(graph_time_ms(torch, step_fns, clock=clk, preheat_s=0.04))
+    barrier()
+    # The same K steps after a 0.5 s preheat, at the clocks a long run settles
+    # to under the power cap (reported against the sustained peak).
+    clk_s = ClockSampler(bus_id_of(torch, dev) if rank == 0 else None)
+    sustained_ms = max_over_ranks(graph_time_ms(torch, step_fns, clock=clk_s, preheat_s=0.5))
     barrier()
     # the dominant kernel alone, K launches over the same rotating buffers
     combine_ms = graph_time_ms(torch, [lambda s=sets[k % n_copies]: combine(s) for k in range(K)]) / K
@@ -293,9 +301,14 @@ def run_ours(args, rank, world, dist):
     prefill = {"tflops_dense_equiv": round(value / world, 1), "tflops_executed": round(flops_exec / (ms_per_step * 1e-3) / 1e12, 1),
                "gbs": round(step_bytes / (ms_per_step * 1e-3) / 1e9, 1),
                "frac_of_roofline": round(t_roof_step / (ms_per_step * 1e-3), 4),
-               "frac_of_roofline_sustained_peak": round(t_roof_step_s / (ms_per_step * 1e-3), 4),
-               "peak_note": "frac_of_roofline uses the burst bf16 peak; the step runs after a 0.5 s preheat "
-                            "at sustained clocks, for which the sustained measured peak is the denominator",
+               "sustained": {"ms_per_step": round(sustained_ms / K, 5),
+                             "tflops_dense_equiv": round(flops_dense / (sustained_ms / K * 1e-3) / 1e12, 1),
+                             "frac_of_roofline_sustained_peak": round(t_roof_step_s / (sustained_ms / K * 1e-3), 4),
+                             "clocks": clk_s.summary(),
+                             "how": "the same K steps after a 0.5 s untimed replay, against the sustained "
+                                    "measured peak"},
+               "peak_note": "frac_of_roofline: the K timed steps right after the warm-up, against the burst "
+                            "measured peak; 'sustained': after a 0.5 s preheat, against the sustained peak",
                "project_ms": round(project_ms, 4), "combine_ms": round(combine_ms, 4), "path": path,
                "l2": f"rotating {n_copies} buffer sets of {set_bytes / 1e6:.1f} MB (> L2 126 MB)"}
     clocks = clk.summary()

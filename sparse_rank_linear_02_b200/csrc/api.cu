@@ -9,8 +9,10 @@ namespace slr {
 namespace {
 
 constexpr size_t kAlign = 256;
-// Largest M whose tensor-core path takes T from the CUDA-core projection.
+// Largest M whose tensor-core path may take T from the CUDA-core projection,
+// and the most bytes of X that projection may re-read.
 constexpr int64_t kSmallProjectM = 16;
+constexpr double kSmallProjectXBytes = 12.0 * 1024 * 1024;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -100,9 +102,11 @@ cudaError_t run_project(const void *X, int64_t M, const void *V, int64_t d_in, i
     if (p == SLR_PATH_DECODE)
         return launch_lowrank_project(x, M, vv, d_in, r, static_cast<float *>(workspace), nullptr, chained, stream);
     // Up to 16 tokens the CUDA-core projection (r x 1..2 CTAs, fp32 sums
-    // rounded to bf16) finishes well before the streaming combine needs T;
-    // the tensor-core projection runs on a handful of CTAs there.
-    if (M <= kSmallProjectM)
+    // rounded to bf16; 2.3-3.6 us on 4096 x 4096 against 6.7 us for the
+    // tensor-core projection, which runs on a handful of CTAs there), as long
+    // as its CTAs' re-reads of X (each rank index reads the token block's X,
+    // r * M * d_in * 2 bytes in all) stay small.
+    if (M <= kSmallProjectM && (double)r * (double)M * (double)d_in * 2.0 <= kSmallProjectXBytes)
         return launch_lowrank_project(x, M, vv, d_in, r, nullptr, static_cast<uint16_t *>(workspace), chained, stream);
     return launch_tc_project(x, M, vv, d_in, r, static_cast<uint16_t *>(workspace), chained, stream);
 }

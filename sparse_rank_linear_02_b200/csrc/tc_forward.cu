@@ -36,7 +36,6 @@
 #include <cudaTypedefs.h>
 
 #include <cstdlib>
-#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -1838,27 +1837,24 @@ cudaError_t launch_project_splitk(const uint16_t *X, int64_t M, const uint16_t *
 // =====================================================================================
 // Split-K forward for few tokens (BN = 16 .. 128 per tile): Y = X S^T + T U^T
 // when the layer is bound by the bytes of S, or has too few row tiles to keep
-// the 2-SM pairs busy.  One cluster of KS CTAs (KS <= 4) owns a slab of H <= 128
-// output rows x BN tokens and splits its K stages (the 2:4 stages, then the
-// rank stages) across its CTAs.  With one token tile (M <= BN <= 64) the slab
-// height H and KS are chosen so that the clusters fill every SM with equal
-// shares of S (e.g. 37 slabs of 111 rows x 4 CTAs on a 4096-row layer), and the
-// ring holds all of a CTA's stages; with several token tiles the slabs are
-// 128-row tiles and the token tiles of one slab are neighbouring clusters,
-// which stream the same S tile at about the same time (one read from HBM).
-// The A operand is always read as 128 rows: rows H..127 of a stage hold
-// whatever the ring held before (their metadata nibbles are forced valid by
-// the permute), and the matching rows of the accumulator are never stored.
-// Each CTA accumulates its partial Y^T slab in TMEM (2:4 tcgen05.mma.sp with
+// the 2-SM pairs busy.  One cluster of KS CTAs (KS <= 4) owns a 128-row x
+// BN-token tile and splits its K stages (the 2:4 stages, then the rank stages)
+// across its CTAs, so that all SMs stream S at once even when d_out / 128 is
+// small; the token tiles of one row tile are neighbouring clusters, which
+// stream the same S tile at about the same time (one read from HBM).
+// Each CTA accumulates its partial Y^T tile in TMEM (2:4 tcgen05.mma.sp with
 // the same metadata permute as the large-M kernels, N = BN), writes it to
-// shared memory in fp32, and after a cluster barrier CTA q sums its share of
-// the H rows over the KS partials through distributed shared memory and
-// stores them to Y in bf16 (RNE).
+// shared memory in fp32, and after a cluster barrier CTA q sums rows
+// [q*128/KS, (q+1)*128/KS) over the KS partials through distributed shared
+// memory and stores them to Y in bf16 (RNE).
 //
 // Launch modes (pdl): 0 plain; 1 programmatic dependent of the projection
 // kernel that writes T (wait before the first load of T); 2 chained: also
 // the preceding work may still run, so S and U are requested first and the
 // kernel waits before its first load of X.
+//
+// CTAs per cluster of the split-K kernel: split K two or four ways while the
+// grid stays within two CTAs per SM.
 inline int small_cluster(int64_t work, int64_t stages, int sms) {
     int ks = 1;
     while (ks < 4 && ks * 2 <= stages && work * ks * 2 <= 2 * (int64_t)sms) ks *= 2;
@@ -1881,49 +1877,40 @@ inline bool small_wins(int64_t M, int64_t d_out, int64_t d_in, int sms) {
     return work * 4 <= (int64_t)sms || (d_in >= 8192 && work <= (int64_t)sms);
 }
 
-template <int BN, int PER_SM>
+template <int BN>
 struct CfgS {
     static constexpr int A_BYTES = BM * 64 * 2;          // 16 KB of packed values (128 logical K)
     static constexpr int B_HALF = BN * 64 * 2;           // BN tokens x one 128-byte panel
     static constexpr int B_BYTES = 2 * B_HALF;
     static constexpr int E_BYTES = BM * BK / 8;          // 2 KB of metadata
     static constexpr int STAGE = ((A_BYTES + B_BYTES + E_BYTES + 1023) / 1024) * 1024;
-    static constexpr int P_BYTES = BM * BN * 4;          // one fp32 partial tile (row-major, BN per row)
-    // one CTA per SM: up to 227 KB; two: 113 KB each (228 KB less 1 KB reserved per CTA)
-    static constexpr int BUDGET = PER_SM == 1 ? 232448 : 115712;
-    static constexpr int RING_OFF = 1024;                // barriers in the first 1 KB
-    static constexpr int NS_MAX = 12;
+    static constexpr int PROW = BN + 4;                  // padded fp32 row of the partial tile
+    static constexpr int P_BYTES = BM * PROW * 4;
+    static constexpr int NS_FIT = 114432 / STAGE;        // two CTAs per SM (114432 + 1280 <= 115712)
+    static constexpr int NS = NS_FIT > 8 ? 8 : (NS_FIT < 2 ? 2 : NS_FIT);
+    static constexpr int RING = NS * STAGE;
+    static constexpr int BAR_OFF = (RING > P_BYTES ? RING : P_BYTES);
+    static constexpr int SMEM = BAR_OFF + 256 + 1024;
     static constexpr uint32_t ECOL = BN;
     static constexpr uint32_t TMEM_COLS = pow2_at_least(BN + 4);
+    static_assert(SMEM <= 115712, "two CTAs per SM (228 KB less 1 KB reserved per CTA)");
     static_assert(BN % 16 == 0 && BN <= 128, "MMA N");
-    static_assert(PER_SM == 1 || PER_SM == 2, "CTAs per SM");
-    static_assert((2 * NS_MAX + 2) * 8 + 8 <= RING_OFF, "barrier area");
-    // Ring slots that fit beside the receive area of ks - 1 partial tiles
-    // (the cluster leader collects the other CTAs' partials there).
-    static constexpr int slots(int ks) {
-        const int fit = (BUDGET - 1024 - RING_OFF - (ks - 1) * P_BYTES) / STAGE;
-        return fit > NS_MAX ? NS_MAX : fit;
-    }
-    static constexpr int smem(int ns, int ks) { return RING_OFF + ns * STAGE + (ks - 1) * P_BYTES + 1024; }
 };
 
-template <int BN, int PER_SM>
-__global__ void __launch_bounds__(kThreads, PER_SM)
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 2)
     tc_small_kernel(const __grid_constant__ CUtensorMap tm_vals, const __grid_constant__ CUtensorMap tm_meta,
                     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_u,
                     const __grid_constant__ CUtensorMap tm_t, uint16_t *__restrict__ Y, int32_t M, int32_t d_out,
-                    int32_t n_ttiles, int32_t nk, int32_t nlr, int32_t H, int32_t pdl, int32_t NS, int32_t push) {
-    using C = CfgS<BN, PER_SM>;
+                    int32_t n_ttiles, int32_t nk, int32_t nlr, int32_t pdl) {
+    using C = CfgS<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-    uint64_t *empty = full + C::NS_MAX;
-    uint64_t *acc_full = empty + C::NS_MAX;
-    uint64_t *red_full = acc_full + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(red_full + 1);
-    uint8_t *ring = smem + C::RING_OFF;
-    float *part = reinterpret_cast<float *>(ring);      // own partial: reuses the ring after the K loop
-    float *recv = reinterpret_cast<float *>(ring + NS * C::STAGE);   // leader: the other CTAs' partials
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *empty = full + C::NS;
+    uint64_t *acc_full = empty + C::NS;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    float *part = reinterpret_cast<float *>(smem);      // reuses the ring after the K loop
 
     // The next kernel on the stream may be scheduled now (a chained forward
     // waits for this grid before it reads anything this grid writes).
@@ -1934,29 +1921,21 @@ __global__ void __launch_bounds__(kThreads, PER_SM)
     asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(ks_n));
     const uint32_t ks_q = cluster_ctarank();
     const int work = blockIdx.x / (int)ks_n;
-    const int d0 = (work / n_ttiles) * H;
+    const int d0 = (work / n_ttiles) * BM;
     const int tok0 = (work % n_ttiles) * BN;
     const int total = nk + nlr;
     const int k_begin = (int)(((int64_t)total * ks_q) / ks_n);
     const int k_end = (int)(((int64_t)total * (ks_q + 1)) / ks_n);
-    const uint32_t part_bytes = (uint32_t)H * BN * 4u;   // rows 0..H-1 of a partial tile
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < C::NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
-        mbar_init(red_full, 1);
-        // The leader expects one partial tile from each other CTA of the cluster.
-        if (push && ks_q == 0 && ks_n > 1) mbar_expect_tx(red_full, (ks_n - 1) * part_bytes);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async_smem();
     }
-    __syncthreads();
-    // Every CTA of the cluster has initialised its barriers once all have
-    // arrived here; the wait for that comes before the partials are pushed.
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     // The producer needs no TMEM: warp 0 arrives on the start barrier and
     // streams at once; the other warps wait there for the TMEM allocation.
     uint32_t tmem_base = 0;
@@ -1976,31 +1955,26 @@ __global__ void __launch_bounds__(kThreads, PER_SM)
 
     if (warp == 0) {
         if (lane == 0) {
-            // Bytes a stage's copies deliver: boxes of H rows of values or U
-            // (128 B each) and of metadata (16 B), BN rows of X or T (two
-            // 128-byte panels of X, one of T).
-            const uint32_t sparse_tx = (uint32_t)H * 144u + (uint32_t)C::B_BYTES;
-            const uint32_t rank_tx = (uint32_t)H * 128u + (uint32_t)C::B_HALF;
-            // Weight operands (S tile and metadata, or a U tile) first: they do
-            // not depend on earlier work on the stream.  In chained mode the
-            // first ring's X / T loads follow the wait for the preceding grid.
-            const int prologue = pdl == 2 ? min(k_end - k_begin, NS) : 0;
+            // Chained launch (pdl == 2): the preceding grid may still run.  The
+            // first ring's weight operands (S tile and metadata, or a U tile)
+            // are requested now; its X / T loads follow the wait.
+            const int prologue = pdl == 2 ? min(k_end - k_begin, C::NS) : 0;
             for (int i = 0; i < prologue; ++i) {
                 const int ks = k_begin + i;
-                uint8_t *st = ring + i * C::STAGE;
+                uint8_t *st = smem + i * C::STAGE;
                 if (ks < nk) {
-                    mbar_expect_tx(&full[i], sparse_tx);
+                    mbar_expect_tx(&full[i], C::A_BYTES + C::B_BYTES + C::E_BYTES);
                     tma_load_2d(&tm_vals, smem_u32(st), &full[i], ks * 64, d0);
                     tma_load_2d(&tm_meta, smem_u32(st + C::A_BYTES + C::B_BYTES), &full[i], ks * (BK / 8), d0);
                 } else {
-                    mbar_expect_tx(&full[i], rank_tx);
+                    mbar_expect_tx(&full[i], C::A_BYTES + C::B_HALF);
                     tma_load_2d(&tm_u, smem_u32(st), &full[i], (ks - nk) * 64, d0);
                 }
             }
             if (pdl == 2) asm volatile("griddepcontrol.wait;" ::: "memory");
             for (int i = 0; i < prologue; ++i) {
                 const int ks = k_begin + i;
-                const uint32_t b = smem_u32(ring + i * C::STAGE + C::A_BYTES);
+                const uint32_t b = smem_u32(smem + i * C::STAGE + C::A_BYTES);
                 if (ks < nk) {
                     tma_load_2d(&tm_x, b, &full[i], ks * BK, tok0);
                     tma_load_2d(&tm_x, b + C::B_HALF, &full[i], ks * BK + 64, tok0);
@@ -2008,18 +1982,18 @@ __global__ void __launch_bounds__(kThreads, PER_SM)
                     tma_load_2d(&tm_t, b, &full[i], (ks - nk) * 64, tok0);
                 }
             }
-            uint32_t s = (uint32_t)(prologue % NS), ph = prologue == NS ? 1u : 0u;
+            uint32_t s = (uint32_t)(prologue % C::NS), ph = prologue == C::NS ? 1u : 0u;
             bool t_ready = pdl != 1;
             for (int ks = k_begin + prologue; ks < k_end; ++ks) {
                 if (!mbar_wait(&empty[s], ph ^ 1)) {
                     atomicOr(&g_tc_error, 4096u);
                     break;
                 }
-                uint8_t *st = ring + s * C::STAGE;
+                uint8_t *st = smem + s * C::STAGE;
                 const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES),
                                e = smem_u32(st + C::A_BYTES + C::B_BYTES);
                 if (ks < nk) {
-                    mbar_expect_tx(&full[s], sparse_tx);
+                    mbar_expect_tx(&full[s], C::A_BYTES + C::B_BYTES + C::E_BYTES);
                     tma_load_2d(&tm_vals, a, &full[s], ks * 64, d0);
                     tma_load_2d(&tm_x, b, &full[s], ks * BK, tok0);
                     tma_load_2d(&tm_x, b + C::B_HALF, &full[s], ks * BK + 64, tok0);
@@ -2031,11 +2005,11 @@ __global__ void __launch_bounds__(kThreads, PER_SM)
                         t_ready = true;
                     }
                     const int j = ks - nk;
-                    mbar_expect_tx(&full[s], rank_tx);
+                    mbar_expect_tx(&full[s], C::A_BYTES + C::B_HALF);
                     tma_load_2d(&tm_u, a, &full[s], j * 64, d0);
                     tma_load_2d(&tm_t, b, &full[s], j * 64, tok0);
                 }
-                if (++s == (uint32_t)NS) {
+                if (++s == (uint32_t)C::NS) {
                     s = 0;
                     ph ^= 1;
                 }
@@ -2045,18 +2019,6 @@ __global__ void __launch_bounds__(kThreads, PER_SM)
         constexpr uint32_t kIdescSp = idesc_bf16(BM, BN, true);
         constexpr uint32_t kIdescDense = idesc_bf16(BM, BN, false);
         const uint32_t e_tmem = tmem_base + C::ECOL;
-        // Metadata rows H..127 are never loaded (TMA writes rows 0..H-1 only):
-        // give them the valid pattern (0, 1) once.  The permute below moves
-        // whole 16-bit words between rows, so they stay valid in every later
-        // use of the slot.
-        if (H < BM) {
-            for (int s2 = 0; s2 < NS; ++s2) {
-                uint8_t *e = ring + s2 * C::STAGE + C::A_BYTES + C::B_BYTES;
-                for (int row = H + lane; row < BM; row += 32)
-                    *reinterpret_cast<uint4 *>(e + row * 16) = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
-            }
-            __syncwarp();
-        }
         uint32_t s = 0, ph = 0;
         bool ok = true;
         for (int ks = k_begin; ks < k_end; ++ks) {
@@ -2064,12 +2026,10 @@ __global__ void __launch_bounds__(kThreads, PER_SM)
                 ok = false;
                 break;
             }
-            uint8_t *st = ring + s * C::STAGE;
+            uint8_t *st = smem + s * C::STAGE;
             const uint32_t a = smem_u32(st), b = smem_u32(st + C::A_BYTES);
             const uint32_t first = (ks == k_begin) ? 1u : 0u;
             if (ks < nk) {
-                // Rows H..127 of the values were not loaded (stale shared
-                // memory); the accumulator rows they produce are never stored.
                 permute_meta_tile(st + C::A_BYTES + C::B_BYTES, lane);
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -2094,7 +2054,7 @@ __global__ void __launch_bounds__(kThreads, PER_SM)
                 mma_commit(&empty[s]);
             }
             __syncwarp();
-            if (++s == (uint32_t)NS) {
+            if (++s == (uint32_t)C::NS) {
                 s = 0;
                 ph ^= 1;
             }
@@ -2103,8 +2063,7 @@ __global__ void __launch_bounds__(kThreads, PER_SM)
         if (lane == 0) mma_commit(acc_full);  // fires at once when this CTA had no stages
         __syncwarp();
     } else {
-        // TMEM partial (lane = output row, column = token) -> shared memory,
-        // rows 0..H-1 (fp32, BN per row)
+        // TMEM partial (lane = output row, column = token) -> shared memory
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const bool have = k_end > k_begin;
@@ -2114,100 +2073,37 @@ __global__ void __launch_bounds__(kThreads, PER_SM)
             for (int q = 0; q < BN / 16; ++q) {
                 uint32_t v[16];
                 tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(q * 16), v);
-                if (row < H) {
-                    float4 *dst = reinterpret_cast<float4 *>(part + row * BN + q * 16);
+                float4 *dst = reinterpret_cast<float4 *>(part + row * C::PROW + q * 16);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        dst[j] = have ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                                    __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
+                for (int j = 0; j < 4; ++j)
+                    dst[j] = have ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         } else {
             atomicOr(&g_tc_error, 16384u);
         }
     }
     tc_fence_before();
-    __syncthreads();   // the partial is in shared memory; TMEM is no longer read
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-    if (warp == 1) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
-    }
+    cluster_sync_all();  // every CTA's partial is in its shared memory
 
-    if (!push) {
-        // No room for a receive area: every CTA keeps its partial, and after a
-        // cluster barrier CTA q sums rows [q*RPC, (q+1)*RPC) over the cluster
-        // through distributed shared memory.
-        cluster_sync_all();
-        if (warp >= 2) {
-            const int rpc = (H + (int)ks_n - 1) / (int)ks_n;
-            const int items = rpc * (BN / 4);
-            const uint32_t part_addr = smem_u32(part);
-            for (int it = threadIdx.x - 64; it < items; it += 128) {
-                const int row = (int)ks_q * rpc + it % rpc;
-                const int tg = it / rpc;
-                if (row >= H) continue;
-                const uint32_t off = (uint32_t)((row * BN + 4 * tg) * 4);
-                float4 p[4];
-#pragma unroll
-                for (uint32_t q = 0; q < 4; ++q)
-                    p[q] = q < ks_n ? ld_shared_cluster_v4(mapa_shared(part_addr + off, q)) : make_float4(0.f, 0.f, 0.f, 0.f);
-                const float sum[4] = {p[0].x + p[1].x + p[2].x + p[3].x, p[0].y + p[1].y + p[2].y + p[3].y,
-                                      p[0].z + p[1].z + p[2].z + p[3].z, p[0].w + p[1].w + p[2].w + p[3].w};
-                const int out_row = d0 + row;
-                if (out_row < d_out) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int tok = tok0 + 4 * tg + j;
-                        if (tok < M) Y[(int64_t)tok * d_out + out_row] = f32_to_bf16_bits(sum[j]);
-                    }
-                }
-            }
-        }
-        cluster_sync_all();  // no CTA leaves while its partial may still be read
-        return;
-    }
-
-    if (ks_q != 0) {
-        // Push the partial into the leader's receive slot q - 1; the copy
-        // completes on the leader's red_full barrier.  The CTA stays until
-        // the copy has read its shared memory.
-        if (threadIdx.x == 64) {
-            fence_proxy_async_smem();
-            const uint32_t dst = mapa_shared(smem_u32(recv) + (ks_q - 1) * (uint32_t)C::P_BYTES, 0);
-            asm volatile(
-                "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                "r"(smem_u32(part)), "r"(part_bytes), "r"(mapa_shared(smem_u32(red_full), 0))
-                : "memory");
-            bulk_commit();
-            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-        }
-        return;
-    }
-
-    // Leader: rows [0, H) of the slab, all BN tokens, summed over its own
-    // partial and the KS - 1 received ones in rank order; thread -> (row,
-    // group of 4 tokens), rows fastest so that the bf16 stores of one token
-    // are contiguous in Y.
+    // CTA q: rows [q*RPC, (q+1)*RPC) of the tile, all BN tokens, summed over
+    // the cluster; thread -> (row, group of 4 tokens), rows fastest so that
+    // the bf16 stores of one token are contiguous in Y.
     if (warp >= 2) {
-        if (ks_n > 1 && !mbar_wait(red_full, 0)) {
-            atomicOr(&g_tc_error, 32768u);
-            return;
-        }
-        const int items = H * (BN / 4);
+        const int rpc = BM / (int)ks_n;
+        const int items = rpc * (BN / 4);
+        const uint32_t part_addr = smem_u32(part);
         for (int it = threadIdx.x - 64; it < items; it += 128) {
-            const int row = it % H;
-            const int tg = it / H;
-            float4 acc = *reinterpret_cast<const float4 *>(part + row * BN + 4 * tg);
-            for (uint32_t q = 1; q < ks_n; ++q) {
-                const float4 p = *reinterpret_cast<const float4 *>(recv + (q - 1) * (C::P_BYTES / 4) + row * BN + 4 * tg);
-                acc.x += p.x;
-                acc.y += p.y;
-                acc.z += p.z;
-                acc.w += p.w;
-            }
-            const float sum[4] = {acc.x, acc.y, acc.z, acc.w};
+            const int row = (int)ks_q * rpc + it % rpc;
+            const int tg = it / rpc;
+            const uint32_t off = (uint32_t)((row * C::PROW + 4 * tg) * 4);
+            float4 p[4];
+#pragma unroll
+            for (uint32_t q = 0; q < 4; ++q)
+                p[q] = q < ks_n ? ld_shared_cluster_v4(mapa_shared(part_addr + off, q)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float sum[4] = {p[0].x + p[1].x + p[2].x + p[3].x, p[0].y + p[1].y + p[2].y + p[3].y,
+                                  p[0].z + p[1].z + p[2].z + p[3].z, p[0].w + p[1].w + p[2].w + p[3].w};
             const int out_row = d0 + row;
             if (out_row < d_out) {
 #pragma unroll
@@ -2218,96 +2114,44 @@ __global__ void __launch_bounds__(kThreads, PER_SM)
             }
         }
     }
-}
-
-// Plan of the split-K kernel for one token tile: slab height H <= 128, KS
-// CTAs per slab (a cluster), one or two CTAs per SM.  The number of slabs is
-// the number of clusters the device holds at once (cudaOccupancyMaxActive-
-// Clusters: clusters are placed within GPCs, so 4-CTA clusters of a full SM
-// each do not reach every SM), so the grid is a single wave.  Among the
-// plans whose slabs are at most 128 rows, the one with the fewest bytes per
-// CTA (S once, plus X once per slab, split over its KS CTAs) is taken, with a
-// penalty when the ring cannot hold all of a CTA's stages; ties keep the
-// smaller cluster.
-struct SlabPlan {
-    int H, ks, per_sm, slabs, ns;
-};
-
-template <int BN, int PER_SM>
-int small_max_clusters(int ks, int ns) {
-    using C = CfgS<BN, PER_SM>;
-    static std::mutex mu;
-    static int cache[64][5] = {};   // per device, per ks
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    std::lock_guard<std::mutex> lock(mu);
-    if (cache[dev][ks] == 0) {
-        const int smem = C::smem(ns, ks);
-        if (cudaFuncSetAttribute(tc_small_kernel<BN, PER_SM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess)
-            return 0;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)ks * 8u);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = (size_t)smem;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)ks;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, tc_small_kernel<BN, PER_SM>, &cfg) != cudaSuccess || n <= 0) {
-            cudaGetLastError();
-            return 0;
-        }
-        cache[dev][ks] = n;
+    cluster_sync_all();  // no CTA leaves while its partial may still be read
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
     }
-    return cache[dev][ks];
 }
 
+// pdl: 0 plain launch, 1 after the projection kernel (waits before T), 2
+// chained (waits before X and T).
 template <int BN>
-SlabPlan slab_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r) {
-    SlabPlan best{0, 0, 0, 0, 0};
-    double best_cost = -1.0;
-    const int64_t stages = d_in / BK + (r + 63) / 64;
-    const double row_bytes = (double)d_in + d_in / 8.0;   // packed values + metadata per row
-    for (int per_sm = 1; per_sm <= 2; ++per_sm) {
-        for (int ks = 1; ks <= 4; ks *= 2) {
-            if (ks > stages) continue;
-            const int ns = per_sm == 1 ? CfgS<BN, 1>::slots(ks) : CfgS<BN, 2>::slots(ks);
-            if (ns < 2) continue;
-            const int clusters = per_sm == 1 ? small_max_clusters<BN, 1>(ks, ns) : small_max_clusters<BN, 2>(ks, ns);
-            if (clusters < 1) continue;
-            const int64_t H = (d_out + clusters - 1) / clusters;
-            if (H > BM || H < 8) continue;
-            const int used = (int)((d_out + H - 1) / H);
-            const int64_t per_cta = (stages + ks - 1) / ks;
-            const double cta = (H * row_bytes + (double)M * d_in * 2.0) / ks;
-            const double cost = cta * (per_cta <= ns ? 1.0 : 1.25) + (ks > 1 ? 1024.0 : 0.0);
-            if (best_cost < 0.0 || cost < best_cost * 0.999) {
-                best_cost = cost;
-                best = SlabPlan{(int)H, ks, per_sm, used, ns};
-            }
-        }
-    }
-    return best;
-}
-
-template <int BN, int PER_SM>
-cudaError_t launch_small_cfg(const CUtensorMap &m_vals, const CUtensorMap &m_meta, const CUtensorMap &m_x,
-                             const CUtensorMap &m_u, const CUtensorMap &m_t, uint16_t *Y, int64_t M, int64_t d_out,
-                             int n_ttiles, int work, int ks, int nk, int nlr, int H, int pdl, int ns, bool push,
-                             cudaStream_t stream) {
-    using C = CfgS<BN, PER_SM>;
-    const int smem = C::smem(ns, push ? ks : 1);
-    cudaError_t err = cudaFuncSetAttribute(tc_small_kernel<BN, PER_SM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+cudaError_t launch_sparse_small(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
+                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
+                                uint16_t *Y, int pdl, cudaStream_t stream) {
+    using C = CfgS<BN>;
+    CUtensorMap m_vals, m_meta, m_x, m_u, m_t;
+    memset(&m_u, 0, sizeof m_u);
+    memset(&m_t, 0, sizeof m_t);
+    bool ok = make_map(&m_vals, kBF16, vals, d_in / 2, d_out, d_in, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&m_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, d_in / 8, d_out, d_in / 8, 16, BM,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map(&m_x, kBF16, X, d_in, M, d_in * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (ok && r > 0)
+        ok = make_map(&m_u, kBF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+             make_map(&m_t, kBF16, T16, r, M, r * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int n_ttiles = (int)((M + BN - 1) / BN);
+    const int work = (int)((d_out + BM - 1) / BM) * n_ttiles;
+    const int nk = (int)(d_in / BK), nlr = (int)((r + 63) / 64);
+    const int ks = small_cluster(work, nk + nlr, sms);
+    cudaError_t err = cudaFuncSetAttribute(tc_small_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(work * ks));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -2317,65 +2161,10 @@ cudaError_t launch_small_cfg(const CUtensorMap &m_vals, const CUtensorMap &m_met
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl != 0 ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, tc_small_kernel<BN, PER_SM>, m_vals, m_meta, m_x, m_u, m_t, Y, (int32_t)M,
-                              (int32_t)d_out, (int32_t)n_ttiles, (int32_t)nk, (int32_t)nlr, (int32_t)H, (int32_t)pdl,
-                              (int32_t)ns, (int32_t)(push ? 1 : 0));
-}
-
-// pdl: 0 plain launch, 1 after the projection kernel (waits before T), 2
-// chained (waits before X and T).  A plan of a single token tile uses row
-// slabs sized to fill the SMs; otherwise 128-row tiles.
-template <int BN>
-cudaError_t launch_sparse_small(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
-                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
-                                uint16_t *Y, int pdl, cudaStream_t stream) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int n_ttiles = (int)((M + BN - 1) / BN);
-    const int nk = (int)(d_in / BK), nlr = (int)((r + 63) / 64);
-    SlabPlan plan{0, 0, 0, 0, 0};
-    // SLR_SMALL_PLAN=H:ks:per_sm forces a slab plan (A/B measurements).
-    const char *force = getenv("SLR_SMALL_PLAN");
-    int fh = 0, fks = 0, fps = 0;
-    if (force != nullptr && sscanf(force, "%d:%d:%d", &fh, &fks, &fps) == 3 && fh >= 8 && fh <= BM &&
-        (fks == 1 || fks == 2 || fks == 4) && (fps == 1 || fps == 2) && n_ttiles == 1) {
-        const int ns = fps == 1 ? CfgS<BN, 1>::slots(fks) : CfgS<BN, 2>::slots(fks);
-        plan = SlabPlan{fh, fks, fps, (int)((d_out + fh - 1) / fh), ns};
-    } else if (n_ttiles == 1 && BN <= 64) {
-        plan = slab_plan<BN>(M, d_out, d_in, r);
-    }
-    if (plan.H == 0) {   // several token tiles, or no slab plan in one wave: 128-row tiles
-        const int tiles = (int)((d_out + BM - 1) / BM);
-        const int ks = small_cluster((int64_t)tiles * n_ttiles, nk + nlr, sms);
-        plan = SlabPlan{BM, ks, 2, tiles, CfgS<BN, 2>::slots(ks)};
-    }
-    if (plan.ks > nk + nlr) plan.ks = 1;
-    // Push reduction when the leader's receive area leaves a ring of two or
-    // more slots; otherwise the cluster reduces through remote reads.
-    bool push = plan.ns >= 2;
-    if (!push) plan.ns = plan.per_sm == 1 ? CfgS<BN, 1>::slots(1) : CfgS<BN, 2>::slots(1);
-    if (plan.ns < 2) return cudaErrorInvalidConfiguration;
-    CUtensorMap m_vals, m_meta, m_x, m_u, m_t;
-    memset(&m_u, 0, sizeof m_u);
-    memset(&m_t, 0, sizeof m_t);
-    const uint32_t h = (uint32_t)plan.H;
-    bool ok = make_map(&m_vals, kBF16, vals, d_in / 2, d_out, d_in, 64, h, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map(&m_meta, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, d_in / 8, d_out, d_in / 8, 16, h,
-                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
-              make_map(&m_x, kBF16, X, d_in, M, d_in * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (ok && r > 0)
-        ok = make_map(&m_u, kBF16, U, r, d_out, r * 2, 64, h, CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_map(&m_t, kBF16, T16, r, M, r * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (!ok) return cudaErrorInvalidValue;
-    const int work = plan.slabs * n_ttiles;
     const int mode = (pdl == 1 && r == 0) ? 0 : pdl;
-    if (plan.per_sm == 1)
-        return launch_small_cfg<BN, 1>(m_vals, m_meta, m_x, m_u, m_t, Y, M, d_out, n_ttiles, work, plan.ks, nk, nlr,
-                                       plan.H, mode, plan.ns, push, stream);
-    return launch_small_cfg<BN, 2>(m_vals, m_meta, m_x, m_u, m_t, Y, M, d_out, n_ttiles, work, plan.ks, nk, nlr,
-                                   plan.H, mode, plan.ns, push, stream);
+    cfg.numAttrs = mode != 0 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, tc_small_kernel<BN>, m_vals, m_meta, m_x, m_u, m_t, Y, (int32_t)M,
+                              (int32_t)d_out, (int32_t)n_ttiles, (int32_t)nk, (int32_t)nlr, (int32_t)mode);
 }
 
 }  // namespace tc

@@ -281,12 +281,12 @@ def _layer_case(d_out, d_in, r, M, seed, outliers=True):
 
 @pytest.mark.parametrize("path", ["decode", "tensor"])
 @pytest.mark.parametrize("d_out,d_in,r,M", [
-    (4096, 4096, 64, 1), (4096, 4096, 64, 4), (4096, 4096, 64, 16),   # q_proj decode: 37 slabs of 111 rows
-    (1024, 4096, 64, 16),     # 37 slabs of 28 rows
-    (3000, 2048, 128, 33),    # BN = 64, ragged last slab
+    (4096, 4096, 64, 1), (4096, 4096, 64, 4), (4096, 4096, 64, 16),   # q_proj decode
+    (1024, 4096, 64, 16),     # 8 row tiles, K split four ways
+    (3000, 2048, 128, 33),    # BN = 64, ragged last row tile
     (2048, 1024, 256, 64),    # four rank stages
     (1024, 2048, 0, 7),       # no projection: the combine itself is chained
-    (28672, 8192, 64, 2),     # two CTAs per SM, 296 slabs of 97 rows
+    (28672, 8192, 64, 2),     # 224 row tiles, two CTAs per SM
 ])
 def test_forward_chained_matches_unchained(path, d_out, d_in, r, M):
     """SLR_FWD_OVERLAP_PRECEDING changes when the kernels may start, not what
