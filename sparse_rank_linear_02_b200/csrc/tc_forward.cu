@@ -429,6 +429,8 @@ struct Params2 {
     int32_t cyc;        // rounds of the cyclic phase
     int32_t chu;        // most 16-token units per chunk (<= the kernel's BN / 16)
     int64_t n_tiles;    // tiles dealt in the cyclic phase (a last round may be partial)
+    const uint8_t *meta;  // packed metadata [d_out, meta_ld] (copied with cp.async by the 512-row kernel)
+    int64_t meta_ld;      // bytes per metadata row (d_in / 8)
     int64_t tail[kMaxPairs + 1];  // pair p's tail units are [tail[p], tail[p+1])
 };
 
@@ -943,7 +945,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
             mbar_init(&empty[s], 1);
         }
         for (int m = 0; m < C::MS; ++m) {
-            mbar_init(&mfull[m], 1);
+            mbar_init(&mfull[m], 32);   // one cp.async arrival per lane of the metadata warp
             mbar_init(&mready[m], 1);
             mbar_init(&mempty[m], 1);
         }
@@ -1034,15 +1036,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
             ld.advance(prm.chu);
             use.advance(prm.chu);
         }
+        // A stage's metadata is 16 bytes per row: as TMA boxes it would cost
+        // one copy request per row, as many as the 128-byte rows of the
+        // values, on the SM's TMA engine.  The warp's lanes copy the 256 rows
+        // (both halves) with 16-byte cp.async instead, eight per lane, and each
+        // lane arrives on the slot's barrier when its copies have landed.
+        // Rows past d_out are zero-filled, as TMA would.
         auto issue = [&](int slot) {
-            if (elect_one()) {
-                uint8_t *e = meta_ring + slot * 2 * C::E_BYTES;
-                mbar_expect_tx(&mfull[slot], 2 * C::E_BYTES);
-                const int r0 = ld.ch.d0 + (int)rank * BM;
-                tma_load_2d(&maps.meta, smem_u32(e), &mfull[slot], ld.ks * (BK / 8), r0);
-                tma_load_2d(&maps.meta, smem_u32(e + C::E_BYTES), &mfull[slot], ld.ks * (BK / 8), r0 + 2 * BM);
+            uint8_t *e = meta_ring + slot * 2 * C::E_BYTES;
+            const int r0 = ld.ch.d0 + (int)rank * BM;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int q = lane + 32 * i;            // 0..255: half q >> 7, row q & 127
+                const int row = r0 + (q >> 7) * 2 * BM + (q & 127);
+                const bool in = row < d_out;
+                const uint8_t *src = prm.meta + (in ? (int64_t)row * prm.meta_ld + (int64_t)ld.ks * (BK / 8) : 0);
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                                 smem_u32(e + (q >> 7) * C::E_BYTES + (q & 127) * 16)),
+                             "l"(src), "r"(in ? 16 : 0)
+                             : "memory");
             }
-            __syncwarp();
+            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&mfull[slot])) : "memory");
             ld.advance(prm.chu);
             if (ld.valid) ld.advance(prm.chu);
         };
@@ -1578,6 +1592,8 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
     int pairs = 0;
     if (chu <= 0 || chu > C::CHU) chu = C::CHU;
     plan_pairs(M, d_out, d_in, r, chu, 4 * BM, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, split_tail, &prm, &pairs);
+    prm.meta = meta;
+    prm.meta_ld = d_in / 8;
     // Directly after the projection kernel on this stream: programmatic
     // dependent launch (the producer waits before it loads T).  Otherwise an
     // ordinary launch, which must not overlap an unrelated preceding kernel.
