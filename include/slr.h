@@ -309,7 +309,10 @@ SLR_API size_t slr_decompose_workspace_size(int64_t d_out, int64_t d_in, int64_t
  *
  * Arithmetic: products of bf16 inputs are accumulated in fp32.  T is kept in
  * fp32 on the small-M path and rounded to bf16 before the second product on
- * the tensor-core path.  Accuracy contract (tested): relative Frobenius error
+ * the tensor-core path.  Above 64 tokens the 512-row tensor-core kernel forms
+ * T in the same launch (a projection phase before its main loop: partial
+ * products of 256-token tiles over slices of K, summed in a fixed order), and
+ * the other kernels take it from a projection kernel launched just before.  Accuracy contract (tested): relative Frobenius error
  * <= 5e-3 and |err_ij| <= 1e-2 * (|X| |W'|^T)_ij + 1e-3 against the exact
  * result on the same bf16 inputs.
  *
@@ -322,7 +325,11 @@ SLR_API slr_status slr_forward(const void *X, int64_t M, const void *vals, const
                        int64_t d_out, int64_t d_in, const void *U, const void *V, int64_t r,
                        void *Y, void *workspace, size_t workspace_bytes, slr_stream_t stream);
 
-/* Scratch bytes slr_forward needs for this problem (0 when none). */
+/* Scratch bytes slr_forward needs for this problem (0 when none): T (fp32
+ * [M, r] on the streaming path, bf16 [M, r] on the tensor-core path) and,
+ * above 64 tokens with 0 < r <= 128, room for the partial products with which
+ * the 512-row tensor-core kernel forms T itself (a single launch after a
+ * memset of two counters; 64 B + 128 x 256 x 64 or 128 fp32 values). */
 SLR_API size_t slr_forward_workspace_size(int64_t M, int64_t d_out, int64_t d_in, int64_t r);
 
 /* Execution paths of the forward pass. */

@@ -52,6 +52,9 @@ constexpr int64_t kDecodeMaxWeights = int64_t(1) << 26;
 size_t workspace_bytes_for(int64_t M, int64_t r, slr_path path) {
     if (M <= 0 || r <= 0) return 0;
     if (path == SLR_PATH_DECODE) return round_up((size_t)M * r * sizeof(float), kAlign);
+    // Above kChainMaxM tokens (r <= 128) the single-call forward may form T
+    // inside the 512-row kernel: T, the phase counters and the partials.
+    if (M > kChainMaxM && r <= 128) return round_up(fused_layout(M, r).bytes, kAlign);
     return round_up((size_t)M * r * sizeof(uint16_t), kAlign);
 }
 
@@ -154,7 +157,17 @@ slr_status forward_impl(const void *X, int64_t M, const void *vals, const void *
                                    true, true, true, &p);
     if (st != SLR_OK || M == 0) return st;
     const bool chained = (flags & SLR_FWD_OVERLAP_PRECEDING) != 0 && chain_supported(p, M, d_in, r);
-    cudaError_t err = run_project(X, M, V, d_in, r, workspace, p, chained, stream);
+    cudaError_t err = cudaSuccess;
+    if (p == SLR_PATH_TENSOR && M > kChainMaxM) {
+        // One call: the 512-row kernel with its projection phase where it is
+        // the dispatched kernel, else projection then combine.
+        err = launch_tc_forward_fused(static_cast<const uint16_t *>(X), M, static_cast<const uint16_t *>(vals),
+                                      static_cast<const uint8_t *>(meta), d_out, d_in,
+                                      static_cast<const uint16_t *>(U), static_cast<const uint16_t *>(V), r,
+                                      static_cast<uint16_t *>(Y), static_cast<uint8_t *>(workspace), stream);
+        return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
+    }
+    err = run_project(X, M, V, d_in, r, workspace, p, chained, stream);
     if (err == cudaSuccess)
         err = run_combine(X, M, vals, meta, d_out, d_in, U, r, Y, workspace, p, chained ? 2 : 1, stream);
     return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;

@@ -411,6 +411,7 @@ struct Maps2 {
     CUtensorMap vals, meta, u, y32, y16;
     CUtensorMap xs[5];
     CUtensorMap ts[5];
+    CUtensorMap xt, vt;   // projection phase: X in 128-row boxes, V in RN/2-row boxes (two 64-wide panels)
 };
 
 __host__ __device__ constexpr int box_rows(int i, int half_n) { return i < 4 ? (8 << i) : half_n; }
@@ -431,6 +432,14 @@ struct Params2 {
     int64_t n_tiles;    // tiles dealt in the cyclic phase (a last round may be partial)
     const uint8_t *meta;  // packed metadata [d_out, meta_ld] (copied with cp.async by the 512-row kernel)
     int64_t meta_ld;      // bytes per metadata row (d_in / 8)
+    // Projection phase of the 512-row kernel (tp_on): T = X V^T for 256-token
+    // tiles, K split tp_ks ways over the first tp_tiles * tp_ks pairs, partial
+    // sums in tp_part, reduced by every CTA into T16; tp_count[0] counts the
+    // CTAs whose partials are written, tp_count[1] those whose share of T16 is.
+    int32_t tp_on, tp_tiles, tp_ks, tp_rn, r;
+    float *tp_part;       // [tp_tiles * tp_ks][256][tp_rn] fp32
+    uint16_t *tp_t16;     // T [M, r] bf16
+    unsigned int *tp_count;
     int64_t tail[kMaxPairs + 1];  // pair p's tail units are [tail[p], tail[p+1])
 };
 
@@ -905,10 +914,22 @@ struct CfgT {
     static_assert(NS >= 2, "need at least two stages");
     static_assert(MLEAD < MS && MLEAD % 2 == 0, "metadata lead");
     static_assert(SMEM <= 232448, "shared memory budget");
-    static_assert((2 * NS + 3 * MS + 4) * 8 + 8 <= 1024, "barrier area");
+    static_assert((2 * NS + 3 * MS + 6) * 8 + 8 <= 1024, "barrier area");
 };
 
 constexpr int kThreadsT = 384;  // 12 warps
+
+// Bounded spin until *p >= target (acquire, GPU scope); false on expiry.
+__device__ __forceinline__ bool spin_count_ge(const unsigned int *p, unsigned int target) {
+    const long long t0 = clock64();
+    while (true) {
+        unsigned int v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        if (v >= target) return true;
+        if (clock64() - t0 > kWaitCycles) return false;
+        __nanosleep(64);
+    }
+}
 
 template <int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
@@ -923,7 +944,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
     uint64_t *mempty = mready + C::MS;
     uint64_t *acc_full = mempty + C::MS;
     uint64_t *acc_empty = acc_full + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
+    uint64_t *tp_full = acc_empty + 1;    // projection phase: T partial complete in TMEM
+    uint64_t *tp_empty = tp_full + 1;     // projection phase: T partial drained (leader)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tp_empty + 1);
     volatile uint32_t *fail = tmem_slot + 1;
     uint8_t *meta_ring = smem + C::META_OFF;
     uint8_t *dummy = smem + C::DUMMY_OFF;   // MS signal slots + 1 source slot
@@ -938,6 +961,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
     const int nstages = nk + prm.nlr;
     const int M = prm.M;
     const int d_out = prm.d_out;
+    // Projection phase (T = X V^T inside this kernel, LoSparse section 3.2's
+    // low-rank term): pair p < tp_tiles * tp_ks computes the partial product
+    // of token tile p / tp_ks over the p % tp_ks-th slice of the K stages.
+    const bool tp_busy = prm.tp_on && pair < prm.tp_tiles * prm.tp_ks;
+    const int tp_tile = tp_busy ? pair / prm.tp_ks : 0, tp_q = tp_busy ? pair % prm.tp_ks : 0;
+    const int tp_k0 = tp_busy ? (int)(((int64_t)nk * tp_q) / prm.tp_ks) : 0;
+    const int tp_k1 = tp_busy ? (int)(((int64_t)nk * (tp_q + 1)) / prm.tp_ks) : 0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NS; ++s) {
@@ -951,6 +981,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 16);
+        mbar_init(tp_full, 1);
+        mbar_init(tp_empty, 8);
         *fail = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async_smem();
@@ -975,6 +1007,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
         const uint32_t full_leader0 = mapa_shared(smem_u32(&full[0]), 0);
         uint32_t s = 0, ph = 0;
         bool t_ready = false;
+        // Projection phase: per stage, this CTA's 128 tokens of X (two
+        // 128-byte panels, 32 KB) and its tp_rn / 2 rows of V through the
+        // same ring as the main loop.
+        for (int ks = tp_k0; ks < tp_k1; ++ks) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(&empty[s], ph ^ 1))) {
+                if (lane == 0) {
+                    *fail = 1;
+                    atomicOr(&g_tc_error, 65536u);
+                }
+                break;
+            }
+            uint8_t *st = smem + s * C::STAGE;
+            const uint32_t a = smem_u32(st), b = smem_u32(st + C::B_OFF);
+            const uint32_t bar = full_leader0 + s * (uint32_t)sizeof(uint64_t);
+            if (elect_one()) {
+                if (leader) mbar_expect_tx(&full[s], 2u * (32768u + (uint32_t)prm.tp_rn * 128u));
+                tma_load_3d_pair(&maps.xt, a, bar, 0, tp_tile * 256 + (int)rank * 128, ks * 2);
+                tma_load_3d_pair(&maps.vt, b, bar, 0, (int)rank * (prm.tp_rn / 2), ks * 2);
+            }
+            __syncwarp();
+            if (++s == (uint32_t)C::NS) {
+                s = 0;
+                ph ^= 1;
+            }
+        }
         ChunkIter iter(prm, pair, npairs);
         Chunk ch;
         while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(prm.chu, ch)) {
@@ -1006,9 +1063,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
                 } else {
                     const int j = ks - nk;
                     if (!t_ready) {
-                        // T comes from the projection kernel, which may still
-                        // be running (programmatic dependent launch).
-                        asm volatile("griddepcontrol.wait;" ::: "memory");
+                        if (prm.tp_on) {
+                            // T comes from this grid's projection phase: every
+                            // CTA has written its share of T16 (global writes,
+                            // then read here through the async proxy).
+                            if (!__all_sync(0xFFFFFFFFu, spin_count_ge(prm.tp_count + 1, gridDim.x))) {
+                                if (lane == 0) {
+                                    *fail = 1;
+                                    atomicOr(&g_tc_error, 131072u);
+                                }
+                                break;
+                            }
+                            asm volatile("fence.proxy.async.global;" ::: "memory");
+                        } else {
+                            // T comes from the projection kernel, which may
+                            // still be running (programmatic dependent launch).
+                            asm volatile("griddepcontrol.wait;" ::: "memory");
+                        }
                         t_ready = true;
                     }
                     if (elect_one()) {
@@ -1120,6 +1191,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
             uint32_t s = 0, ph = 0;
             int it = 0;
             int64_t k = 0;   // sparse stages consumed (metadata slot sequence)
+            if (tp_busy) {
+                // Projection phase: D = T partial (M = 256 tokens of the pair,
+                // N = tp_rn ranks) in TMEM columns 0..tp_rn-1, dense MMAs with
+                // A = the X tile and B = the V tile, K = 16 each.
+                const uint32_t idesc_t = idesc_bf16(2 * BM, prm.tp_rn, false);
+                const uint32_t vpanel = (uint32_t)prm.tp_rn * 64u;   // tp_rn / 2 rows of 128 bytes
+                bool ok = true;
+                for (int ks = tp_k0; ks < tp_k1; ++ks) {
+                    if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(&full[s], ph))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint8_t *st = smem + s * C::STAGE;
+                    const uint32_t a = smem_u32(st), b = smem_u32(st + C::B_OFF);
+                    if (elect_one()) {
+#pragma unroll
+                        for (int pn = 0; pn < 2; ++pn)
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)
+                                mma_dense_pair(tmem_base, desc_sw128(a + pn * 16384 + 32 * c),
+                                               desc_sw128(b + pn * vpanel + 32 * c), idesc_t,
+                                               (ks > tp_k0 || pn > 0 || c > 0) ? 1u : 0u);
+                        mma_commit_pair(&empty[s]);
+                    }
+                    __syncwarp();
+                    if (++s == (uint32_t)C::NS) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                if (elect_one()) mma_commit_pair(tp_full);
+                __syncwarp();
+                // The main loop accumulates into the same TMEM columns: wait
+                // until both CTAs have drained the partial.
+                if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait_cluster(tp_empty, 0));
+                if (!ok) {
+                    if (lane == 0) {
+                        *fail = 1;
+                        atomicOr(&g_tc_error, 262144u);
+                    }
+                }
+                tc_fence_after();
+            }
             ChunkIter iter(prm, pair, npairs);
             Chunk ch;
             while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(prm.chu, ch)) {
@@ -1207,6 +1322,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
         const bool store_thread = ((warp - 2) % 4 == 0 && lane == 0);
         uint16_t *out = reinterpret_cast<uint16_t *>(smem + C::OUT_OFF + grp * C::OUT_BYTES);
         const uint32_t empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+        if (prm.tp_on) {
+            // Projection phase, part 1 (warps 2..5, one per TMEM lane quarter,
+            // pairs with a K slice): the fp32 partial of this CTA's 128 tokens
+            // goes to tp_part, then the leader learns that TMEM is free.
+            const int etid = (int)threadIdx.x - 64;   // 0..255
+            if (tp_busy && warp <= 5) {
+                const int quarter = warp & 3;
+                const int trow = quarter * 32 + lane;
+                if (mbar_wait_cluster(tp_full, 0)) {
+                    tc_fence_after();
+                    float *dst = prm.tp_part +
+                                 ((int64_t)(tp_q * prm.tp_tiles + tp_tile) * 256 + (int)rank * 128 + trow) * prm.tp_rn;
+                    for (int q = 0; q < prm.tp_rn / 16; ++q) {
+                        uint32_t v[16];
+                        tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(q * 16), v);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            reinterpret_cast<float4 *>(dst + q * 16)[j] =
+                                make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                    }
+                } else {
+                    *fail = 1;
+                    atomicOr(&g_tc_error, 524288u);
+                }
+                __threadfence();   // the partial, before the count that publishes it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote_relaxed(mapa_shared(smem_u32(tp_empty), 0));
+                named_bar_sync(3, 128);
+                if (etid == 0) {
+                    __threadfence();
+                    atomicAdd(prm.tp_count, 1u);
+                }
+            }
+            // Part 2 (all eight warps of every CTA): once every partial is
+            // written, this CTA's share of T = the sum of the tp_ks partials in
+            // slice order, rounded to bf16 (RNE) into tp_t16; four ranks per
+            // step (r % 8 == 0).
+            if (spin_count_ge(prm.tp_count, 2u * (unsigned)(prm.tp_tiles * prm.tp_ks))) {
+                const int64_t total = (int64_t)M * prm.r;
+                const int64_t per = ((total + gridDim.x - 1) / gridDim.x + 3) / 4 * 4;
+                const int64_t e0 = (int64_t)blockIdx.x * per;
+                const int64_t e1 = e0 + per < total ? e0 + per : total;
+                for (int64_t e = e0 + 4 * etid; e < e1; e += 4 * 256) {
+                    const int64_t m = e / prm.r;
+                    const int j = (int)(e - m * prm.r);
+                    const int tile = (int)(m / 256), trow = (int)(m % 256);
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int q = 0; q < prm.tp_ks; ++q) {
+                        const uint4 p4 = ld_dep_v4(prm.tp_part +
+                                                   ((int64_t)(q * prm.tp_tiles + tile) * 256 + trow) * prm.tp_rn + j);
+                        acc.x += __uint_as_float(p4.x);
+                        acc.y += __uint_as_float(p4.y);
+                        acc.z += __uint_as_float(p4.z);
+                        acc.w += __uint_as_float(p4.w);
+                    }
+                    uint2 packed;
+                    packed.x = (uint32_t)f32_to_bf16_bits(acc.x) | ((uint32_t)f32_to_bf16_bits(acc.y) << 16);
+                    packed.y = (uint32_t)f32_to_bf16_bits(acc.z) | ((uint32_t)f32_to_bf16_bits(acc.w) << 16);
+                    *reinterpret_cast<uint2 *>(prm.tp_t16 + e) = packed;
+                }
+            } else {
+                *fail = 1;
+                atomicOr(&g_tc_error, 1048576u);
+            }
+            __threadfence();   // this thread's part of T, before the count that publishes it
+            named_bar_sync(4, 256);
+            if (etid == 0) {
+                __threadfence();
+                atomicAdd(prm.tp_count + 1, 1u);
+            }
+        }
         int it = 0;
         ChunkIter iter(prm, pair, npairs);
         Chunk ch;
@@ -1565,8 +1753,13 @@ cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *val
 template <int BN>
 cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
-                               uint16_t *Y, bool after_projection, bool split_tail, cudaStream_t stream, int chu = 0) {
+                               uint16_t *Y, bool after_projection, bool split_tail, cudaStream_t stream, int chu = 0,
+                               const uint16_t *V = nullptr, uint8_t *fused_ws = nullptr) {
     using C = CfgT<BN>;
+    // With V and a fused workspace the kernel forms T itself (projection
+    // phase); T16 is then the workspace's first region.
+    bool tp = V != nullptr && fused_ws != nullptr && r > 0 && r <= 128;
+    if (tp) T16 = reinterpret_cast<const uint16_t *>(fused_ws);
     Maps2 maps;
     memset(&maps, 0, sizeof maps);
     bool ok = make_map(&maps.vals, kBF16, vals, d_in / 2, d_out, d_in, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -1582,6 +1775,9 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
             ok = make_map(&maps.ts[i], kBF16, T16, r, M, r * 2, 64, (uint32_t)box_rows(i, C::HALF_N),
                           CU_TENSOR_MAP_SWIZZLE_128B);
     }
+    const int tp_rn = r <= 64 ? 64 : 128;
+    if (ok && tp)
+        ok = make_map_panels(&maps.xt, X, d_in, M, 128) && make_map_panels(&maps.vt, V, d_in, r, tp_rn / 2);
     if (!ok) return cudaErrorInvalidValue;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -1591,9 +1787,53 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
     Params2 prm;
     int pairs = 0;
     if (chu <= 0 || chu > C::CHU) chu = C::CHU;
-    plan_pairs(M, d_out, d_in, r, chu, 4 * BM, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, split_tail, &prm, &pairs);
+    int max_pairs = sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs;
+    if (tp) {
+        // The projection phase waits on counters that every CTA of the grid
+        // advances, so the whole grid must be resident at once: no more pairs
+        // than the device holds clusters of this kernel.
+        int ncl = 0;
+        cudaLaunchConfig_t occ = {};
+        occ.gridDim = dim3((unsigned)(2 * max_pairs));
+        occ.blockDim = dim3(kThreadsT);
+        occ.dynamicSmemBytes = C::SMEM;
+        err = cudaOccupancyMaxActiveClusters(&ncl, tc2t_forward_kernel<BN>, &occ);
+        if (err != cudaSuccess) return err;
+        if (ncl < max_pairs) max_pairs = ncl;
+    }
+    plan_pairs(M, d_out, d_in, r, chu, 4 * BM, max_pairs, split_tail, &prm, &pairs);
+    if (tp && (M + 255) / 256 > pairs) {
+        // Fewer pairs than 256-token tiles: T from the projection kernel instead.
+        err = launch_tc_project(X, M, V, d_in, r, const_cast<uint16_t *>(T16), false, stream);
+        if (err != cudaSuccess) return err;
+        tp = false;
+        after_projection = true;
+    }
     prm.meta = meta;
     prm.meta_ld = d_in / 8;
+    prm.tp_on = 0;
+    prm.r = (int32_t)r;
+    prm.tp_rn = tp_rn;
+    prm.tp_tiles = (int32_t)((M + 255) / 256);
+    prm.tp_ks = 1;
+    prm.tp_part = nullptr;
+    prm.tp_t16 = const_cast<uint16_t *>(T16);
+    prm.tp_count = nullptr;
+    if (tp) {
+        // Token tiles of 256 over the pairs, K split as far as the pairs go
+        // (every tile has a pair: M <= 256 * pairs, checked above).
+        const int nk = (int)(d_in / BK);
+        int ks = pairs / prm.tp_tiles;
+        if (ks > nk) ks = nk;
+        prm.tp_on = 1;
+        prm.tp_ks = ks < 1 ? 1 : ks;
+        const FusedLayout L = fused_layout(M, r);
+        prm.tp_count = reinterpret_cast<unsigned int *>(fused_ws + L.off_count);
+        prm.tp_part = reinterpret_cast<float *>(fused_ws + L.off_part);
+        // The two phase counters start at zero (the kernel reads, never resets them).
+        err = cudaMemsetAsync(prm.tp_count, 0, 2 * sizeof(unsigned int), stream);
+        if (err != cudaSuccess) return err;
+    }
     // Directly after the projection kernel on this stream: programmatic
     // dependent launch (the producer waits before it loads T).  Otherwise an
     // ordinary launch, which must not overlap an unrelated preceding kernel.
@@ -1606,7 +1846,7 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = (after_projection && r > 0) ? 1 : 0;
+    cfg.numAttrs = (after_projection && r > 0 && !tp) ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, tc2t_forward_kernel<BN>, maps, prm);
 }
 
@@ -2238,6 +2478,44 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
     if (c.kind == 3)
         return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream, c.chu);
     return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream, c.chu);
+}
+
+cudaError_t launch_tc_forward_fused(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
+                                    int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *V, int64_t r,
+                                    uint16_t *Y, uint8_t *ws, cudaStream_t stream) {
+    if (M <= 0) return cudaSuccess;
+    if (M > INT32_MAX || d_out > INT32_MAX || d_in > INT32_MAX) return cudaErrorInvalidValue;
+    uint16_t *T16 = reinterpret_cast<uint16_t *>(ws);
+    // The 512-row kernel forms T itself when it is the kernel the dispatch
+    // picks (or SLR_TC_KERNEL=2smtall[w] forces it), r <= 128 and every
+    // 256-token tile has a pair; otherwise the projection kernel runs first.
+    bool tall = false, split = true;
+    int chu = 0;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const char *force = getenv("SLR_TC_KERNEL");
+    if (M > kChainMaxM && r > 0 && r <= 128 && (M + 255) / 256 <= sms / 2) {
+        if (force != nullptr) {
+            if (strncmp(force, "2smtall", 7) == 0) {
+                tall = true;
+                split = force[strlen(force) - 1] != 'w';
+            }
+        } else if (!tc::small_wins(M, d_out, d_in, sms)) {
+            const tc::PlanChoice c = tc::choose_plan(M, d_out, d_in, r, sms);
+            if (c.kind == 2) {
+                tall = true;
+                split = c.split;
+                chu = c.chu;
+            }
+        }
+    }
+    if (tall)
+        return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, false, split, stream, chu, V,
+                                           ws);
+    cudaError_t err = cudaSuccess;
+    if (r > 0) err = launch_tc_project(X, M, V, d_in, r, T16, false, stream);
+    if (err == cudaSuccess) err = launch_tc_forward(X, M, vals, meta, d_out, d_in, U, r > 0 ? T16 : nullptr, r, Y, 1, stream);
+    return err;
 }
 
 cudaError_t launch_tc_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in, int64_t r,

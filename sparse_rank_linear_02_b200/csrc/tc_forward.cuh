@@ -19,6 +19,24 @@ bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64
 // support chained launches.
 constexpr int64_t kChainMaxM = 64;
 
+// Workspace of the single-call tensor-core forward above kChainMaxM tokens:
+// T (bf16 [M, r], read by the combine's rank stages), two phase counters, and
+// the fp32 partial products of the 512-row kernel's projection phase (at most
+// kFusedMaxParts slices of a 256-token tile, tile rows of up to 128 ranks).
+constexpr int64_t kFusedMaxParts = 128;
+struct FusedLayout {
+    size_t off_count, off_part, bytes;
+};
+inline FusedLayout fused_layout(int64_t M, int64_t r) {
+    const size_t t16 = ((size_t)M * (size_t)r * 2 + 255) / 256 * 256;
+    const size_t rn = r <= 64 ? 64 : 128;
+    FusedLayout L;
+    L.off_count = t16;
+    L.off_part = t16 + 256;
+    L.bytes = L.off_part + (size_t)kFusedMaxParts * 256 * rn * 4;
+    return L;
+}
+
 // Y = X S^T + T U^T on the tensor cores.  T16 is bf16 [M, r] (may be null when
 // r == 0).  Requires d_in % 128 == 0, d_out % 8 == 0, r % 8 == 0.
 // pdl: 0 = ordinary launch; 1 = the kernel launched immediately before on
@@ -29,6 +47,15 @@ constexpr int64_t kChainMaxM = 64;
 cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                               int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
                               uint16_t *Y, int pdl, cudaStream_t stream);
+
+// The single-call forward on the tensor cores (M > kChainMaxM): the 512-row
+// pair kernel with its projection phase when the dispatch picks that kernel and
+// r <= 128 (one launch after a memset of the phase counters), otherwise the
+// projection kernel followed by launch_tc_forward as its programmatic dependent.
+// ws: fused_layout(M, r).bytes when r <= 128, else M * r * 2 (rounded to 256).
+cudaError_t launch_tc_forward_fused(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
+                                    int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *V, int64_t r,
+                                    uint16_t *Y, uint8_t *ws, cudaStream_t stream);
 
 // T = X V^T on the tensor cores, written as bf16 [M, r] (dense tcgen05 mode of
 // the same kernel).  Requires d_in % 64 == 0, r % 8 == 0.  chained: launched
