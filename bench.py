@@ -50,7 +50,7 @@ SPARSE_RATIO = 2.0   # nominal 2:4 sparse / dense tensor throughput ratio
 
 # DRAM bytes per launch of the dominant kernel from the committed ncu capture
 # (profiles/); valid only for the kernel source it was taken on.
-NCU_TRAFFIC = {"tc_forward": {"source_sha": "df62f645efde6b7f", "bytes_per_launch": 118750976}}
+NCU_TRAFFIC = {"tc_forward": {"source_sha": "b0630a1d9862f229", "bytes_per_launch": 117836032}}
 
 
 def layer_of(cfg, name):
@@ -238,13 +238,15 @@ def run_ours(args, rank, world, dist):
     def combine(s):
         slr.forward_combine(s["X"], s["vals"], s["meta"], s["U"], s["Y"], s["ws"], path=path)
 
+    def fwd(s):  # one step through the single-call entry point (one launch: projection phase + main loop)
+        slr.forward(s["X"], s["vals"], s["meta"], s["U"], s["V"], out=s["Y"], workspace=s["ws"], path=path)
+
     for i in range(args.warmup):
-        project(sets[i % n_copies])
-        combine(sets[i % n_copies])
+        fwd(sets[i % n_copies])
+    project(sets[0])
+    combine(sets[0])
     slr.check_kernel_error()
     K = args.steps
-    def fwd(s):  # one step through the single-call entry point (projection + fused kernel)
-        slr.forward(s["X"], s["vals"], s["meta"], s["U"], s["V"], out=s["Y"], workspace=s["ws"], path=path)
 
     step_fns = [lambda s=sets[k % n_copies]: fwd(s) for k in range(K)]
     clk = ClockSampler(bus_id_of(torch, dev) if rank == 0 else None)
