@@ -312,7 +312,11 @@ SLR_API size_t slr_decompose_workspace_size(int64_t d_out, int64_t d_in, int64_t
  * the tensor-core path.  Above 64 tokens the 512-row tensor-core kernel forms
  * T in the same launch (a projection phase before its main loop: partial
  * products of 256-token tiles over slices of K, summed in a fixed order), and
- * the other kernels take it from a projection kernel launched just before.  Accuracy contract (tested): relative Frobenius error
+ * the other kernels take it from a projection kernel launched just before.
+ * When that kernel splits its last round of tiles along K, the slices' fp32
+ * partial tiles are summed in slice order before the rounding to bf16: the
+ * result does not depend on timing, but may differ in the last bit from an
+ * unsplit evaluation of the same tile.  Accuracy contract (tested): relative Frobenius error
  * <= 5e-3 and |err_ij| <= 1e-2 * (|X| |W'|^T)_ij + 1e-3 against the exact
  * result on the same bf16 inputs.
  *
@@ -327,9 +331,12 @@ SLR_API slr_status slr_forward(const void *X, int64_t M, const void *vals, const
 
 /* Scratch bytes slr_forward needs for this problem (0 when none): T (fp32
  * [M, r] on the streaming path, bf16 [M, r] on the tensor-core path) and,
- * above 64 tokens with 0 < r <= 128, room for the partial products with which
- * the 512-row tensor-core kernel forms T itself (a single launch after a
- * memset of two counters; 64 B + 128 x 256 x 64 or 128 fp32 values). */
+ * above 64 tokens with r > 0, 1 KB of counters, room for the partial products
+ * with which the 512-row tensor-core kernel forms T itself (r <= 128:
+ * 128 x 256 x 64 or 128 fp32 values) and for the fp32 partial tiles of its
+ * last round when that round is split along K (128 x 2 x 2 x 240 x 128 fp32
+ * values, 62.9 MB).  The counters are zeroed on the stream before each such
+ * launch. */
 SLR_API size_t slr_forward_workspace_size(int64_t M, int64_t d_out, int64_t d_in, int64_t r);
 
 /* Execution paths of the forward pass. */

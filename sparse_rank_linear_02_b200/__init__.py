@@ -202,11 +202,19 @@ def pack_2to8(W: torch.Tensor, *, dense: bool = True, as_2to4: bool = True):
 
 def forward_2to8(X: torch.Tensor, vals8: torch.Tensor, meta8: torch.Tensor, U: torch.Tensor | None,
                  V: torch.Tensor | None, *, out: torch.Tensor | None = None,
-                 workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """``Y = X @ S.T + (X @ V.T) @ U.T`` with S in the dense 2:8 packing."""
+                 workspace: torch.Tensor | None = None, vals4: torch.Tensor | None = None,
+                 meta4: torch.Tensor | None = None) -> torch.Tensor:
+    """``Y = X @ S.T + (X @ V.T) @ U.T`` with S in the dense 2:8 packing.
+
+    The 2:8 streaming kernel is issue-bound and only pays at one token; given
+    the 2:4 packing of the same matrix (``vals4``, ``meta4`` from
+    :func:`pack_2to8`), calls with more than one token run ``slr_forward`` on
+    it instead (the same product: a 2:8 pattern is a 2:4 pattern)."""
     M, d_in = X.shape
     d_out = vals8.shape[0]
     r = 0 if U is None else U.shape[1]
+    if M > 1 and vals4 is not None and meta4 is not None:
+        return forward(X, vals4, meta4, U, V, out=out, workspace=workspace)
     if out is None:
         out = torch.empty((M, d_out), dtype=torch.bfloat16, device=X.device)
     need = workspace_size(M, d_out, d_in, r)

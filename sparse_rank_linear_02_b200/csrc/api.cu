@@ -52,9 +52,10 @@ constexpr int64_t kDecodeMaxWeights = int64_t(1) << 26;
 size_t workspace_bytes_for(int64_t M, int64_t r, slr_path path) {
     if (M <= 0 || r <= 0) return 0;
     if (path == SLR_PATH_DECODE) return round_up((size_t)M * r * sizeof(float), kAlign);
-    // Above kChainMaxM tokens (r <= 128) the single-call forward may form T
-    // inside the 512-row kernel: T, the phase counters and the partials.
-    if (M > kChainMaxM && r <= 128) return round_up(fused_layout(M, r).bytes, kAlign);
+    // Above kChainMaxM tokens the single-call forward may run the 512-row
+    // kernel with its projection phase and K-split last round: T, counters,
+    // partial products and partial tiles.
+    if (M > kChainMaxM) return round_up(fused_layout(M, r).bytes, kAlign);
     return round_up((size_t)M * r * sizeof(uint16_t), kAlign);
 }
 

@@ -440,36 +440,71 @@ struct Params2 {
     float *tp_part;       // [tp_tiles * tp_ks][256][tp_rn] fp32
     uint16_t *tp_t16;     // T [M, r] bf16
     unsigned int *tp_count;
-    int64_t tail[kMaxPairs + 1];  // pair p's tail units are [tail[p], tail[p+1])
+    // K-split last round (ksplit, 512-row kernel): tail[p] = tile << 16 |
+    // q << 8 | g when pair p runs K slice q of g of that tile (-1: no tail
+    // work); each slice's fp32 partial tile goes to ks_part slot p, and
+    // ks_count[i] counts the CTAs whose partial of tail tile i is written.
+    int32_t ksplit;
+    float *ks_part;       // [kKsSlots][2 CTAs][2 halves][240 tokens][128 rows] fp32
+    unsigned int *ks_count;
+    uint16_t *y;          // Y [M, d_out]: the reduction of a K-split tile stores it directly
+    // Token-split or whole tail: pair p's tail units are [tail[p], tail[p+1]).
+    int64_t tail[kMaxPairs + 1];
 };
 
 struct Chunk {
     int32_t d0;         // first output row of the pair's 256-row tile
     int32_t tok0;       // first token
     int32_t n;          // tokens (multiple of 16)
+    int32_t k0, k1;     // sparse K stages [k0, k1) of the chunk
+    int32_t lr;         // the rank stages follow the sparse ones
+    int32_t part;       // a K slice of a tail tile: partial sums, then a share of the reduction
 };
 
 // The chunk sequence of one pair; every warp role of the pair walks the same
 // sequence.  All partition parameters are copied into registers when the
 // iterator is built, so the loops never read the kernel parameters again.
 struct ChunkIter {
-    int32_t j, cyc, ut, ttiles, wu, wr, pair, npairs, tile_rows;
+    int32_t j, cyc, ut, ttiles, wu, wr, pair, npairs, tile_rows, nk, ksplit;
     int64_t n_tiles, lo, hi;
 
     __host__ __device__ __forceinline__ ChunkIter(const Params2 &prm, int pair_, int npairs_)
         : j(0), cyc(prm.cyc), ut(prm.ut), ttiles(prm.ttiles), wu(prm.wu), wr(prm.wr), pair(pair_), npairs(npairs_),
-          tile_rows(prm.tile_rows), n_tiles(prm.n_tiles), lo(prm.tail[pair_]), hi(prm.tail[pair_ + 1]) {}
+          tile_rows(prm.tile_rows), nk(prm.nk), ksplit(prm.ksplit), n_tiles(prm.n_tiles), lo(prm.tail[pair_]),
+          hi(prm.ksplit ? 0 : prm.tail[pair_ + 1]) {}
+
+    __host__ __device__ __forceinline__ void whole_tile(int64_t tile, Chunk &c) const {
+        const int64_t rt = tile / ttiles;
+        const int32_t tt = (int32_t)(tile - rt * ttiles);
+        const int32_t u0 = tt * wu + (tt < wr ? tt : wr);
+        c.d0 = (int32_t)(rt * tile_rows);
+        c.tok0 = u0 * 16;
+        c.n = (wu + (tt < wr ? 1 : 0)) * 16;
+        c.k0 = 0;
+        c.k1 = nk;
+        c.lr = 1;
+        c.part = 0;
+    }
 
     __host__ __device__ __forceinline__ bool next(int32_t chu, Chunk &c) {
         const int64_t tile = (int64_t)j * npairs + (pair + j) % npairs;
         if (j < cyc && tile < n_tiles) {
-            const int64_t rt = tile / ttiles;
-            const int32_t tt = (int32_t)(tile - rt * ttiles);
-            const int32_t u0 = tt * wu + (tt < wr ? tt : wr);
-            c.d0 = (int32_t)(rt * tile_rows);
-            c.tok0 = u0 * 16;
-            c.n = (wu + (tt < wr ? 1 : 0)) * 16;
+            whole_tile(tile, c);
             ++j;
+            return true;
+        }
+        if (ksplit) {
+            // One K slice of one tail tile (the slices of a tile together
+            // cover its K stages once; slice 0 also runs the rank stages).
+            if (lo < 0) return false;
+            const int64_t t = lo >> 16;
+            const int32_t q = (int32_t)((lo >> 8) & 255), g = (int32_t)(lo & 255);
+            whole_tile(t, c);
+            c.k0 = (int32_t)(((int64_t)nk * q) / g);
+            c.k1 = (int32_t)(((int64_t)nk * (q + 1)) / g);
+            c.lr = q == 0;
+            c.part = g > 1;
+            lo = -1;
             return true;
         }
         if (lo >= hi) return false;
@@ -484,6 +519,10 @@ struct ChunkIter {
             c.tok0 = ui * 16;
             c.n = nu * 16;
             lo += nu;
+            c.k0 = 0;
+            c.k1 = nk;
+            c.lr = 1;
+            c.part = 0;
         } else {
             const int64_t rt = (hi - 1) / ut;
             const int64_t start = rt * ut;
@@ -495,27 +534,32 @@ struct ChunkIter {
             c.tok0 = (int32_t)(hi - nu - start) * 16;
             c.n = nu * 16;
             hi -= nu;
+            c.k0 = 0;
+            c.k1 = nk;
+            c.lr = 1;
+            c.part = 0;
         }
         return true;
     }
 };
 
-// Cursor over a pair's sparse stages (chunk by chunk, nk stages each), for the
-// metadata warp.
+// Cursor over a pair's sparse stages (chunk by chunk, stages [k0, k1) each),
+// for the metadata warp.
 struct SparseCursor {
     ChunkIter iter;
     Chunk ch;
-    int32_t ks, nk;
+    int32_t ks;
     bool valid;
 
-    __device__ __forceinline__ SparseCursor(const Params2 &prm, int pair, int npairs, int nk_, int32_t chu)
-        : iter(prm, pair, npairs), ks(0), nk(nk_) {
+    __device__ __forceinline__ SparseCursor(const Params2 &prm, int pair, int npairs, int32_t chu)
+        : iter(prm, pair, npairs), ks(0) {
         valid = iter.next(chu, ch);
+        if (valid) ks = ch.k0;
     }
     __device__ __forceinline__ void advance(int32_t chu) {
-        if (++ks == nk) {
-            ks = 0;
+        if (++ks == ch.k1) {
             valid = iter.next(chu, ch);
+            if (valid) ks = ch.k0;
         }
     }
 };
@@ -649,7 +693,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         // its tiles MLEAD stages ahead into slots of its own parity.
         const int par = warp - 6;
         const uint32_t src_slot = smem_u32(dummy + 16 * C::MS);
-        SparseCursor ld(prm, pair, npairs, nk, prm.chu), use(prm, pair, npairs, nk, prm.chu);
+        SparseCursor ld(prm, pair, npairs, prm.chu), use(prm, pair, npairs, prm.chu);
         if (par) {
             ld.advance(prm.chu);
             use.advance(prm.chu);
@@ -918,6 +962,7 @@ struct CfgT {
 };
 
 constexpr int kThreadsT = 384;  // 12 warps
+static_assert(kKsSlotFloats == 4 * 240 * BM, "K-split slot: 2 CTAs x 2 halves x 240 tokens x 128 rows");
 
 // Bounded spin until *p >= target (acquire, GPU scope); false on expiry.
 __device__ __forceinline__ bool spin_count_ge(const unsigned int *p, unsigned int target) {
@@ -958,7 +1003,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
     const int pair = blockIdx.x >> 1;
     const int npairs = gridDim.x >> 1;
     const int nk = prm.nk;
-    const int nstages = nk + prm.nlr;
     const int M = prm.M;
     const int d_out = prm.d_out;
     // Projection phase (T = X V^T inside this kernel, LoSparse section 3.2's
@@ -1042,7 +1086,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
             const uint32_t brows = (uint32_t)box_rows(bi, C::HALF_N);
             const CUtensorMap *xmap = &maps.xs[bi];
             const CUtensorMap *tmap = &maps.ts[bi];
-            for (int ks = 0; ks < nstages; ++ks) {
+            const int nsp = ch.k1 - ch.k0;
+            const int nst = nsp + (ch.lr ? prm.nlr : 0);
+            for (int i = 0; i < nst; ++i) {
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait_cluster(&empty[s], ph ^ 1))) {
                     if (lane == 0) {
                         *fail = 1;
@@ -1053,7 +1099,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
                 uint8_t *st = smem + s * C::STAGE;
                 const uint32_t a = smem_u32(st), b = smem_u32(st + C::B_OFF);
                 const uint32_t bar = full_leader0 + s * (uint32_t)sizeof(uint64_t);
-                if (ks < nk) {
+                if (i < nsp) {
+                    const int ks = ch.k0 + i;
                     if (elect_one()) {
                         if (leader) mbar_expect_tx(&full[s], 2u * (2u * C::A_BYTES + brows * 256u));
                         tma_load_2d_pair(&maps.vals, a, bar, ks * 64, d0);
@@ -1061,7 +1108,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
                         tma_load_3d_pair(xmap, b, bar, 0, tok, ks * 2);
                     }
                 } else {
-                    const int j = ks - nk;
+                    const int j = i - nsp;
                     if (!t_ready) {
                         if (prm.tp_on) {
                             // T comes from this grid's projection phase: every
@@ -1102,7 +1149,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
         // holds both halves' tiles (2 x 2 KB).
         const int par = warp - 10;
         const uint32_t src_slot = smem_u32(dummy + 16 * C::MS);
-        SparseCursor ld(prm, pair, npairs, nk, prm.chu), use(prm, pair, npairs, nk, prm.chu);
+        SparseCursor ld(prm, pair, npairs, prm.chu), use(prm, pair, npairs, prm.chu);
         if (par) {
             ld.advance(prm.chu);
             use.advance(prm.chu);
@@ -1250,8 +1297,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
                     break;
                 }
                 tc_fence_after();
-                for (int ks = 0; ks < nstages; ++ks) {
-                    const bool sparse = ks < nk;
+                const int nsp = ch.k1 - ch.k0;
+                const int nst = nsp + (ch.lr ? prm.nlr : 0);
+                for (int i = 0; i < nst; ++i) {
+                    const bool sparse = i < nsp;
                     const int m = (int)(k % C::MS);
                     bool got = mbar_wait_cluster(&full[s], ph);
                     if (got && sparse) got = mbar_wait_cluster(&mready[m], (uint32_t)((k / C::MS) & 1));
@@ -1274,7 +1323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
                                     const uint64_t adesc = desc_sw128(a + h * C::A_BYTES + 32 * c);
                                     const uint64_t bdesc = desc_sw128(b + (c >> 1) * panel + (c & 1) * 64);
                                     mma_sp_pair(tmem_base + h * BN, adesc, bdesc, e_tmem + 4 * h + (uint32_t)(c & 2),
-                                                idesc_sp | (uint32_t)(c & 1), (ks | c) != 0);
+                                                idesc_sp | (uint32_t)(c & 1), (i | c) != 0);
                                 }
                             mma_commit_pair(&mempty[m]);
                         } else {
@@ -1398,7 +1447,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
         int it = 0;
         ChunkIter iter(prm, pair, npairs);
         Chunk ch;
+        bool part = false;   // the pair's last chunk is a K slice of a tail tile
         while (!*fail && iter.next(prm.chu, ch)) {
+            if (ch.part) {
+                part = true;
+                break;
+            }
             const int d0 = ch.d0 + grp * 2 * BM + (int)rank * BM;
             if (!mbar_wait_cluster(acc_full, (uint32_t)(it & 1))) {
                 *fail = 1;
@@ -1452,6 +1506,101 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
                 }
             }
             ++it;
+        }
+        if (part && !*fail) {
+            // K slice q of g of tail tile tt (decoded from the plan).  This
+            // thread's row of the slice's fp32 partial goes to the pair's slot
+            // in blocks of four tokens ([token / 4][row][4]: a warp's 16-byte
+            // stores, and the reduction's 16-byte loads, cover 512 consecutive
+            // bytes); the accumulators are released; the CTA's count is added
+            // once all its threads have written.
+            const int64_t e = prm.tail[pair];
+            const int cq = (int)((e >> 8) & 255), cg = (int)(e & 255);
+            const int tt = (int)((e >> 16) - (int64_t)prm.cyc * npairs);
+            const int d0 = ch.d0 + grp * 2 * BM + (int)rank * BM;
+            const int64_t sub = ((int)rank * 2 + grp) * (BN * BM);
+            bool ok = mbar_wait_cluster(acc_full, (uint32_t)(it & 1));
+            if (ok) {
+                tc_fence_after();
+                const uint32_t acc = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(grp * BN);
+                float4 *own = reinterpret_cast<float4 *>(prm.ks_part + (int64_t)pair * kKsSlotFloats + sub) + row;
+#pragma unroll 1
+                for (int q = 0; q < kPieces && q * 16 < ch.n; ++q) {
+                    uint32_t h[16];
+                    tmem_ld_32x32b_x16(acc + (uint32_t)(q * 16), h);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        own[(q * 4 + u) * BM] = make_float4(__uint_as_float(h[4 * u]), __uint_as_float(h[4 * u + 1]),
+                                                            __uint_as_float(h[4 * u + 2]), __uint_as_float(h[4 * u + 3]));
+                }
+            } else {
+                *fail = 1;
+                atomicOr(&g_tc_error, 128u);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote_relaxed(empty_leader);
+            __threadfence();
+            named_bar_sync(5, 256);
+            if (threadIdx.x == 64) {
+                __threadfence();
+                atomicAdd(prm.ks_count + tt, 1u);
+            }
+            // Once the 2g CTAs of the tile's slices have written theirs, the
+            // pair sums its share of the token blocks of its rows over the g
+            // slots in slice order (a fixed order), rounds to bf16 (RNE) and
+            // stores them to Y; eight 16-byte loads per thread in flight.
+            if (lane == 0) ok = spin_count_ge(prm.ks_count + tt, 2u * (unsigned)cg) && ok;
+            ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+            __syncwarp();
+            if (!ok) {
+                *fail = 1;
+                if (lane == 0) atomicOr(&g_tc_error, 2097152u);
+            } else {
+                const float *first = prm.ks_part + (int64_t)(pair - cq) * kKsSlotFloats + sub + 4 * row;
+                const int yrow = d0 + row;
+                const int nb = ch.n / 4;
+                const int b0 = (nb * cq) / cg, b1 = (nb * (cq + 1)) / cg;
+#pragma unroll 1
+                for (int b = b0; b < b1; b += 8) {
+                    float4 sum[8];
+#pragma unroll 1
+                    for (int sl = 0; sl < cg; ++sl) {
+                        const float *src = first + (int64_t)sl * kKsSlotFloats;
+                        uint4 v[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            if (b + u < b1) v[u] = ld_dep_v4(src + (int64_t)(b + u) * (BM * 4));
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            if (b + u < b1) {
+                                const float4 f = make_float4(__uint_as_float(v[u].x), __uint_as_float(v[u].y),
+                                                             __uint_as_float(v[u].z), __uint_as_float(v[u].w));
+                                if (sl == 0) {
+                                    sum[u] = f;
+                                } else {
+                                    sum[u].x += f.x;
+                                    sum[u].y += f.y;
+                                    sum[u].z += f.z;
+                                    sum[u].w += f.w;
+                                }
+                            }
+                        }
+                    }
+                    if (yrow < d_out) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int tok = ch.tok0 + 4 * (b + u);
+                            if (b + u < b1) {
+                                const float e4[4] = {sum[u].x, sum[u].y, sum[u].z, sum[u].w};
+#pragma unroll
+                                for (int w = 0; w < 4; ++w)
+                                    if (tok + w < M) prm.y[(int64_t)(tok + w) * d_out + yrow] = f32_to_bf16_bits(e4[w]);
+                            }
+                        }
+                    }
+                }
+            }
         }
         if (store_thread) bulk_wait_all();
     }
@@ -1569,7 +1718,7 @@ cudaError_t launch_project(const uint16_t *X, int64_t M, const uint16_t *V, int6
 // tiles, the cyclic rounds and the tail ranges, sized so that every pair gets
 // the same number of units in total when the cyclic phase allows it.
 void plan_pairs(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int chu, int tile_rows, int max_pairs,
-                bool split_tail, Params2 *prm, int *pairs_out) {
+                int tail_mode, Params2 *prm, int *pairs_out) {
     memset(prm, 0, sizeof *prm);
     prm->M = (int32_t)M;
     prm->d_out = (int32_t)d_out;
@@ -1586,13 +1735,15 @@ void plan_pairs(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int chu, int 
     prm->wu = (int32_t)(ut / ttiles);
     prm->wr = (int32_t)(ut % ttiles);
     const int P = (int)(units < max_pairs ? units : max_pairs);
-    // Whole rounds of tiles first.  With split_tail the tiles of the last,
-    // partial round are then split among all pairs, each pair taking one
-    // piece of one tile (a piece never crosses a tile, so no pair gets an
-    // extra chunk); without it the last round is dealt as whole tiles too.
+    // Whole rounds of tiles first.  tail_mode 0: the last, partial round is
+    // dealt as whole tiles too.  1: its tiles are split among all pairs, each
+    // pair taking one piece (a run of tokens) of one tile (a piece never
+    // crosses a tile, so no pair gets an extra chunk).  2 (512-row kernel
+    // with a workspace): its tiles are split along K, each pair taking one
+    // slice of the K stages of one tile at the tile's full token width.
     const int64_t T = rows * ttiles;
     prm->n_tiles = T;
-    if (!split_tail) {
+    if (tail_mode == 0) {
         prm->cyc = (int32_t)((T + P - 1) / P);
         for (int p = 0; p <= P; ++p) prm->tail[p] = units;
         *pairs_out = P;
@@ -1602,6 +1753,22 @@ void plan_pairs(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int chu, int 
     prm->cyc = (int32_t)cyc;
     const int64_t c_tiles = cyc * P;
     const int64_t rem = T - c_tiles;                   // tiles left, fewer than P
+    if (tail_mode == 2) {
+        // Pairs [first(i), first(i+1)) share tile c_tiles + i, at most
+        // max(1, nk / 4) of them (a slice keeps at least four stages); the
+        // others have no tail work.
+        prm->ksplit = 1;
+        for (int p = 0; p <= kMaxPairs; ++p) prm->tail[p] = -1;
+        int gmax = prm->nk / 4;
+        gmax = gmax < 1 ? 1 : gmax > 255 ? 255 : gmax;
+        for (int64_t i = 0; i < rem; ++i) {
+            const int first = (int)(i * P / rem), last = (int)((i + 1) * P / rem);
+            const int g = last - first < gmax ? last - first : gmax;
+            for (int q = 0; q < g; ++q) prm->tail[first + q] = ((c_tiles + i) << 16) | ((int64_t)q << 8) | g;
+        }
+        *pairs_out = P;
+        return;
+    }
     auto tile_u0 = [&](int64_t tile) {                 // first unit of a tile, row-major unit order
         const int64_t rt = tile / ttiles, tt = tile % ttiles;
         return rt * ut + tt * prm->wu + (tt < prm->wr ? tt : prm->wr);
@@ -1630,8 +1797,11 @@ void plan_pairs(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int chu, int 
 // kernel is not overlapped).  Only used to rank plans.
 double plan_cycles(const Params2 &prm, int pairs, int chu, int half_n, int mode) {
     // mode 0: 256-row tiles, two accumulators; 1: 256-row, one accumulator;
-    // 2: 512-row tiles (one accumulator per half).
-    const int nstages = prm.nk + prm.nlr;
+    // 2: 512-row tiles (one accumulator per half).  A K slice of a split tail
+    // tile also writes its fp32 partial (256 rows x n tokens per CTA) and
+    // reads as many values back in the reduction, at ~32 B per cycle (fitted:
+    // on the gate/up prefill the K split and the token split of the last
+    // round measured within 1.5%).
     const bool tall = mode == 2;
     const double overhead = mode == 0 ? 800.0 : 3000.0;
     double worst = 0;
@@ -1643,7 +1813,9 @@ double plan_cycles(const Params2 &prm, int pairs, int chu, int half_n, int mode)
             const double brows = box_rows(pick_box(ch.n / 2), half_n);
             const double bytes = tall ? 2.0 * 16384 + brows * 256 + 4096 : 16384 + brows * 256 + 2048;
             const double mma = (tall ? 4.0 : 2.0) * ch.n;
-            cyc += nstages * (mma > bytes / 44.0 ? mma : bytes / 44.0) + overhead;
+            const int nst = ch.k1 - ch.k0 + (ch.lr ? prm.nlr : 0);
+            cyc += nst * (mma > bytes / 44.0 ? mma : bytes / 44.0) + overhead;
+            if (ch.part) cyc += 2.0 * 256 * 4 * ch.n / 32.0;
         }
         if (cyc > worst) worst = cyc;
     }
@@ -1658,13 +1830,14 @@ double plan_cycles(const Params2 &prm, int pairs, int chu, int half_n, int mode)
 // tiles can make the tile count fit the pairs better); cached per shape.
 struct PlanChoice {
     int kind, chu;
-    bool split;
+    int tail;   // plan_pairs' tail_mode
 };
 
-PlanChoice choose_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int sms) {
+PlanChoice choose_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int sms, bool allow_ksplit) {
     struct Key {
         int64_t M, d_out, d_in, r;
         int sms;
+        bool ks;
     };
     static std::mutex mu;
     static Key keys[64];
@@ -1673,31 +1846,34 @@ PlanChoice choose_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int sm
     {
         std::lock_guard<std::mutex> lock(mu);
         for (int i = 0; i < n_cached; ++i)
-            if (keys[i].M == M && keys[i].d_out == d_out && keys[i].d_in == d_in && keys[i].r == r && keys[i].sms == sms)
+            if (keys[i].M == M && keys[i].d_out == d_out && keys[i].d_in == d_in && keys[i].r == r &&
+                keys[i].sms == sms && keys[i].ks == allow_ksplit)
                 return vals[i];
     }
     const int maxp = sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs;
-    PlanChoice best{-1, 0, true};
+    PlanChoice best{-1, 0, 1};
     double best_cost = 0;
     for (int kind = 0; kind < 4; ++kind) {
         if (kind == 0 && M >= 192) continue;   // 128-token chunks: below 192 tokens only
         const int cap = kind == 0 ? Cfg2<128>::CHU : kind == 3 ? Cfg2<256>::CHU : Cfg2<240>::CHU;
         const int half_n = cap * 8;
+        const int n_modes = kind == 2 && allow_ksplit ? 3 : 2;
         for (int chu = cap; chu >= cap - 5 && chu >= 1; --chu) {
-            for (int sp = 0; sp < 2; ++sp) {
+            for (int t = 0; t < n_modes; ++t) {
+                const int tm = t == 0 ? 1 : t == 1 ? 0 : 2;   // token split, whole, K split
                 Params2 plan;
                 int pairs = 0;
-                plan_pairs(M, d_out, d_in, r, chu, kind == 2 ? 4 * BM : 2 * BM, maxp, sp == 0, &plan, &pairs);
+                plan_pairs(M, d_out, d_in, r, chu, kind == 2 ? 4 * BM : 2 * BM, maxp, tm, &plan, &pairs);
                 const double cost = plan_cycles(plan, pairs, chu, half_n, kind == 2 ? 2 : kind == 3 ? 1 : 0);
                 if (best.kind < 0 || cost < best_cost) {
-                    best = PlanChoice{kind, chu, sp == 0};
+                    best = PlanChoice{kind, chu, tm};
                     best_cost = cost;
                 }
             }
         }
     }
     std::lock_guard<std::mutex> lock(mu);
-    keys[next_slot] = Key{M, d_out, d_in, r, sms};
+    keys[next_slot] = Key{M, d_out, d_in, r, sms, allow_ksplit};
     vals[next_slot] = best;
     next_slot = (next_slot + 1) % 64;
     if (n_cached < 64) ++n_cached;
@@ -1707,8 +1883,9 @@ PlanChoice choose_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int sm
 template <int BN>
 cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
-                               uint16_t *Y, bool after_projection, bool split_tail, cudaStream_t stream, int chu = 0) {
+                               uint16_t *Y, bool after_projection, int tail_mode, cudaStream_t stream, int chu = 0) {
     using C = Cfg2<BN>;
+    if (tail_mode == 2) tail_mode = 1;   // the K split is the 512-row kernel's
     Maps2 maps;
     memset(&maps, 0, sizeof maps);
     bool ok = make_map(&maps.vals, kBF16, vals, d_in / 2, d_out, d_in, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -1733,7 +1910,7 @@ cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *val
     Params2 prm;
     int pairs = 0;
     if (chu <= 0 || chu > C::CHU) chu = C::CHU;
-    plan_pairs(M, d_out, d_in, r, chu, 2 * BM, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, split_tail, &prm, &pairs);
+    plan_pairs(M, d_out, d_in, r, chu, 2 * BM, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, tail_mode, &prm, &pairs);
     // Directly after the projection kernel on this stream: programmatic
     // dependent launch (the producer waits before it loads T).  Otherwise an
     // ordinary launch, which must not overlap an unrelated preceding kernel.
@@ -1753,13 +1930,17 @@ cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *val
 template <int BN>
 cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
-                               uint16_t *Y, bool after_projection, bool split_tail, cudaStream_t stream, int chu = 0,
+                               uint16_t *Y, bool after_projection, int tail_mode, cudaStream_t stream, int chu = 0,
                                const uint16_t *V = nullptr, uint8_t *fused_ws = nullptr) {
     using C = CfgT<BN>;
-    // With V and a fused workspace the kernel forms T itself (projection
-    // phase); T16 is then the workspace's first region.
-    bool tp = V != nullptr && fused_ws != nullptr && r > 0 && r <= 128;
-    if (tp) T16 = reinterpret_cast<const uint16_t *>(fused_ws);
+    // With a fused workspace (single-call forward, r > 0) T lives in its
+    // first region; the kernel forms T itself (projection phase) when r <=
+    // 128, and the last round may be split along K (partials and counters in
+    // the workspace).  Without one the K split falls back to the token split.
+    const bool fused = V != nullptr && fused_ws != nullptr && r > 0;
+    bool tp = fused && r <= 128;
+    if (fused) T16 = reinterpret_cast<const uint16_t *>(fused_ws);
+    if (tail_mode == 2 && !fused) tail_mode = 1;
     Maps2 maps;
     memset(&maps, 0, sizeof maps);
     bool ok = make_map(&maps.vals, kBF16, vals, d_in / 2, d_out, d_in, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -1788,10 +1969,11 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
     int pairs = 0;
     if (chu <= 0 || chu > C::CHU) chu = C::CHU;
     int max_pairs = sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs;
-    if (tp) {
-        // The projection phase waits on counters that every CTA of the grid
-        // advances, so the whole grid must be resident at once: no more pairs
-        // than the device holds clusters of this kernel.
+    if (tp || tail_mode == 2) {
+        // The projection phase and the K-split reduction wait on counters
+        // that other CTAs of the grid advance, so the whole grid must be
+        // resident at once: no more pairs than the device holds clusters of
+        // this kernel.
         int ncl = 0;
         cudaLaunchConfig_t occ = {};
         occ.gridDim = dim3((unsigned)(2 * max_pairs));
@@ -1800,15 +1982,11 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
         err = cudaOccupancyMaxActiveClusters(&ncl, tc2t_forward_kernel<BN>, &occ);
         if (err != cudaSuccess) return err;
         if (ncl < max_pairs) max_pairs = ncl;
+        if (max_pairs < 1) return cudaErrorInvalidConfiguration;
     }
-    plan_pairs(M, d_out, d_in, r, chu, 4 * BM, max_pairs, split_tail, &prm, &pairs);
-    if (tp && (M + 255) / 256 > pairs) {
-        // Fewer pairs than 256-token tiles: T from the projection kernel instead.
-        err = launch_tc_project(X, M, V, d_in, r, const_cast<uint16_t *>(T16), false, stream);
-        if (err != cudaSuccess) return err;
-        tp = false;
-        after_projection = true;
-    }
+    plan_pairs(M, d_out, d_in, r, chu, 4 * BM, max_pairs, tail_mode, &prm, &pairs);
+    // Fewer pairs than 256-token tiles: T from the projection kernel instead.
+    if (tp && (M + 255) / 256 > pairs) tp = false;
     prm.meta = meta;
     prm.meta_ld = d_in / 8;
     prm.tp_on = 0;
@@ -1819,20 +1997,34 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
     prm.tp_part = nullptr;
     prm.tp_t16 = const_cast<uint16_t *>(T16);
     prm.tp_count = nullptr;
+    prm.ks_part = nullptr;
+    prm.ks_count = nullptr;
+    prm.y = Y;
+    const FusedLayout L = fused_layout(M, r);
     if (tp) {
         // Token tiles of 256 over the pairs, K split as far as the pairs go
-        // (every tile has a pair: M <= 256 * pairs, checked above).
+        // (every tile has a pair: M <= 256 * pairs).
         const int nk = (int)(d_in / BK);
         int ks = pairs / prm.tp_tiles;
         if (ks > nk) ks = nk;
         prm.tp_on = 1;
         prm.tp_ks = ks < 1 ? 1 : ks;
-        const FusedLayout L = fused_layout(M, r);
         prm.tp_count = reinterpret_cast<unsigned int *>(fused_ws + L.off_count);
         prm.tp_part = reinterpret_cast<float *>(fused_ws + L.off_part);
-        // The two phase counters start at zero (the kernel reads, never resets them).
-        err = cudaMemsetAsync(prm.tp_count, 0, 2 * sizeof(unsigned int), stream);
+    }
+    if (prm.ksplit) {
+        prm.ks_count = reinterpret_cast<unsigned int *>(fused_ws + L.off_ks_count);
+        prm.ks_part = reinterpret_cast<float *>(fused_ws + L.off_ks_part);
+    }
+    if (tp || prm.ksplit) {
+        // The counters start at zero (the kernel reads, never resets them).
+        err = cudaMemsetAsync(fused_ws + L.off_count, 0, 1024, stream);
         if (err != cudaSuccess) return err;
+    }
+    if (fused && !tp) {
+        err = launch_tc_project(X, M, V, d_in, r, const_cast<uint16_t *>(T16), false, stream);
+        if (err != cudaSuccess) return err;
+        after_projection = true;
     }
     // Directly after the projection kernel on this stream: programmatic
     // dependent launch (the producer waits before it loads T).  Otherwise an
@@ -2440,14 +2632,15 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
     if (force != nullptr) {
         if (strcmp(force, "1sm") == 0) return tc::launch_sparse<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, stream);
         const bool whole = force[0] != 0 && force[strlen(force) - 1] == 'w';
+        const int tail = whole ? 0 : 1;
         if (strncmp(force, "2sm128", 6) == 0)
-            return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, !whole, stream);
+            return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, tail, stream);
         if (strncmp(force, "2sm256", 6) == 0)
-            return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, !whole, stream);
+            return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, tail, stream);
         if (strncmp(force, "2sm240", 6) == 0)
-            return tc::launch_sparse_pair<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, !whole, stream);
+            return tc::launch_sparse_pair<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, tail, stream);
         if (strncmp(force, "2smtall", 7) == 0)
-            return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, !whole, stream);
+            return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, tail, stream);
         if (strcmp(force, "small") == 0) {
             if (M <= 16) return tc::launch_sparse_small<16>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, pdl, stream);
             if (M <= 32) return tc::launch_sparse_small<32>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, pdl, stream);
@@ -2470,14 +2663,14 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (tc::small_wins(M, d_out, d_in, sms))
         return tc::launch_sparse_small<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, pdl, stream);
-    const tc::PlanChoice c = tc::choose_plan(M, d_out, d_in, r, sms);
+    const tc::PlanChoice c = tc::choose_plan(M, d_out, d_in, r, sms, false);
     if (c.kind == 0)
-        return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream, c.chu);
+        return tc::launch_sparse_pair<128>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.tail, stream, c.chu);
     if (c.kind == 1)
-        return tc::launch_sparse_pair<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream, c.chu);
+        return tc::launch_sparse_pair<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.tail, stream, c.chu);
     if (c.kind == 3)
-        return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream, c.chu);
-    return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.split, stream, c.chu);
+        return tc::launch_sparse_pair<256>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.tail, stream, c.chu);
+    return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, after_projection, c.tail, stream, c.chu);
 }
 
 cudaError_t launch_tc_forward_fused(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
@@ -2486,31 +2679,31 @@ cudaError_t launch_tc_forward_fused(const uint16_t *X, int64_t M, const uint16_t
     if (M <= 0) return cudaSuccess;
     if (M > INT32_MAX || d_out > INT32_MAX || d_in > INT32_MAX) return cudaErrorInvalidValue;
     uint16_t *T16 = reinterpret_cast<uint16_t *>(ws);
-    // The 512-row kernel forms T itself when it is the kernel the dispatch
-    // picks (or SLR_TC_KERNEL=2smtall[w] forces it), r <= 128 and every
-    // 256-token tile has a pair; otherwise the projection kernel runs first.
-    bool tall = false, split = true;
+    // Where the dispatch picks the 512-row kernel (or SLR_TC_KERNEL=
+    // 2smtall[w|k] forces it), it runs with the workspace: T formed in its
+    // projection phase (r <= 128), and its last round dealt as the plan says
+    // (k: split along K).  Otherwise the projection kernel runs first.
+    int tail = -1;   // >= 0: the 512-row kernel with this tail mode
     int chu = 0;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const char *force = getenv("SLR_TC_KERNEL");
-    if (M > kChainMaxM && r > 0 && r <= 128 && (M + 255) / 256 <= sms / 2) {
+    if (r > 0) {
         if (force != nullptr) {
             if (strncmp(force, "2smtall", 7) == 0) {
-                tall = true;
-                split = force[strlen(force) - 1] != 'w';
+                const char last = force[strlen(force) - 1];
+                tail = last == 'w' ? 0 : last == 'k' ? 2 : 1;
             }
         } else if (!tc::small_wins(M, d_out, d_in, sms)) {
-            const tc::PlanChoice c = tc::choose_plan(M, d_out, d_in, r, sms);
+            const tc::PlanChoice c = tc::choose_plan(M, d_out, d_in, r, sms, true);
             if (c.kind == 2) {
-                tall = true;
-                split = c.split;
+                tail = c.tail;
                 chu = c.chu;
             }
         }
     }
-    if (tall)
-        return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, false, split, stream, chu, V,
+    if (tail >= 0)
+        return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, false, tail, stream, chu, V,
                                            ws);
     cudaError_t err = cudaSuccess;
     if (r > 0) err = launch_tc_project(X, M, V, d_in, r, T16, false, stream);

@@ -19,21 +19,29 @@ bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64
 // support chained launches.
 constexpr int64_t kChainMaxM = 64;
 
-// Workspace of the single-call tensor-core forward above kChainMaxM tokens:
-// T (bf16 [M, r], read by the combine's rank stages), two phase counters, and
-// the fp32 partial products of the 512-row kernel's projection phase (at most
-// kFusedMaxParts slices of a 256-token tile, tile rows of up to 128 ranks).
+// Workspace of the single-call tensor-core forward above kChainMaxM tokens
+// (r > 0): T (bf16 [M, r], read by the rank stages), a 1 KB block of counters
+// (the projection phase's two at byte 0, one per K-split tail tile from byte
+// 64), the fp32 partial products of the 512-row kernel's projection phase (at
+// most kFusedMaxParts slices of a 256-token tile, tile rows of up to 128 ranks;
+// r <= 128 only), and the fp32 partial tiles of its K-split last round (one
+// slot of 2 CTAs x 2 halves x 240 tokens x 128 rows per pair).
 constexpr int64_t kFusedMaxParts = 128;
+constexpr int64_t kKsSlots = 128;                 // one per pair (at most kMaxPairs)
+constexpr int64_t kKsSlotFloats = 2 * 2 * 240 * 128;
+constexpr int64_t kKsMaxTiles = 128;              // counters: tail tiles < pairs
 struct FusedLayout {
-    size_t off_count, off_part, bytes;
+    size_t off_count, off_ks_count, off_part, off_ks_part, bytes;
 };
 inline FusedLayout fused_layout(int64_t M, int64_t r) {
     const size_t t16 = ((size_t)M * (size_t)r * 2 + 255) / 256 * 256;
     const size_t rn = r <= 64 ? 64 : 128;
     FusedLayout L;
     L.off_count = t16;
-    L.off_part = t16 + 256;
-    L.bytes = L.off_part + (size_t)kFusedMaxParts * 256 * rn * 4;
+    L.off_ks_count = t16 + 64;
+    L.off_part = t16 + 1024;
+    L.off_ks_part = L.off_part + (r <= 128 ? (size_t)kFusedMaxParts * 256 * rn * 4 : 0);
+    L.bytes = L.off_ks_part + (size_t)kKsSlots * kKsSlotFloats * 4;
     return L;
 }
 
@@ -48,11 +56,13 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
                               int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
                               uint16_t *Y, int pdl, cudaStream_t stream);
 
-// The single-call forward on the tensor cores (M > kChainMaxM): the 512-row
-// pair kernel with its projection phase when the dispatch picks that kernel and
-// r <= 128 (one launch after a memset of the phase counters), otherwise the
-// projection kernel followed by launch_tc_forward as its programmatic dependent.
-// ws: fused_layout(M, r).bytes when r <= 128, else M * r * 2 (rounded to 256).
+// The single-call forward on the tensor cores (M > kChainMaxM): where the
+// dispatch picks the 512-row pair kernel, that kernel with its projection phase
+// (r <= 128; else after the projection kernel) and its last round split along
+// K (one launch after a memset of the counters); otherwise the projection
+// kernel followed by launch_tc_forward as its programmatic dependent.
+// ws: fused_layout(M, r).bytes (null when r == 0: no projection phase, no K
+// split).
 cudaError_t launch_tc_forward_fused(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                     int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *V, int64_t r,
                                     uint16_t *Y, uint8_t *ws, cudaStream_t stream);

@@ -47,10 +47,12 @@ def test_meta_row_bytes_and_workspace():
     assert lib.slr_meta_row_bytes(12) == 2
     assert lib.slr_meta_row_bytes(4) == 1
     assert slr.workspace_size(16, 4096, 4096, 64) == 16 * 64 * 4
-    # above 64 tokens (r <= 128): bf16 T, two counters, the projection phase's partials
-    assert slr.workspace_size(2048, 14336, 4096, 64) == 2048 * 64 * 2 + 256 + 128 * 256 * 64 * 4
-    assert slr.workspace_size(2048, 14336, 4096, 128) == 2048 * 128 * 2 + 256 + 128 * 256 * 128 * 4
-    assert slr.workspace_size(2048, 14336, 4096, 256) == 2048 * 256 * 4     # fp32 T of the streaming path
+    # above 64 tokens: bf16 T, 1 KB of counters, the projection phase's partials
+    # (r <= 128) and the K-split slots (128 pairs x 2 CTAs x 2 halves x 240 x 128 fp32)
+    ks = 128 * 2 * 2 * 240 * 128 * 4
+    assert slr.workspace_size(2048, 14336, 4096, 64) == 2048 * 64 * 2 + 1024 + 128 * 256 * 64 * 4 + ks
+    assert slr.workspace_size(2048, 14336, 4096, 128) == 2048 * 128 * 2 + 1024 + 128 * 256 * 128 * 4 + ks
+    assert slr.workspace_size(2048, 14336, 4096, 256) == 2048 * 256 * 2 + 1024 + ks
     assert slr.workspace_size(8, 256, 256, 0) == 0
     assert slr.workspace_size(0, 256, 256, 8) == 0
 

@@ -177,3 +177,30 @@ def test_2to8_matrix_on_tensor_path():
     rv, rm = oracle.pack_2to8(np.ascontiguousarray(W[outs]))
     Yref, Bref = oracle.forward_2to8(Xp, rv, rm, np.ascontiguousarray(U[outs]), V, rows=rows)
     check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, "2:8 gate_up on the tensor path", rows, outs)
+
+
+@pytest.mark.parametrize("M", [1, 4, 300])
+def test_forward_2to8_routes_multi_token_calls_to_2to4(M):
+    """Given both packings, forward_2to8 keeps one token on the 2:8 streaming
+    kernel and sends more tokens to slr_forward on the 2:4 packing: the result
+    is bit-identical to the matching direct call and within the oracle's
+    bounds."""
+    layer = _layer(2, "q_proj")
+    W = layer.weight()
+    U, V = layer.factors()
+    X = layer.activations(M)
+    v8, m8, v4, m4 = slr.pack_2to8(to_dev(W))
+    args = (to_dev(X),)
+    Y = slr.forward_2to8(args[0], v8, m8, to_dev(U), to_dev(V), vals4=v4, meta4=m4)
+    if M == 1:
+        direct = slr.forward_2to8(args[0], v8, m8, to_dev(U), to_dev(V))
+    else:
+        direct = slr.forward(args[0], v4, m4, to_dev(U), to_dev(V))
+    torch.cuda.synchronize()
+    slr.check_kernel_error()
+    np.testing.assert_array_equal(from_dev(Y), from_dev(direct))
+    rows = sample_indices(M, 16, 31)
+    outs = sample_indices(layer.d_out, 256, 32)
+    rv, rm = oracle.pack_2to8(np.ascontiguousarray(W[outs]))
+    Yref, Bref = oracle.forward_2to8(X, rv, rm, np.ascontiguousarray(U[outs]), V, rows=rows)
+    check_forward(from_dev(Y)[np.ix_(rows, outs)], Yref, Bref, f"2:8 routed M={M}", rows, outs)

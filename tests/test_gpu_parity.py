@@ -211,7 +211,7 @@ def test_no_kernel_timeouts():
     slr.check_kernel_error()
 
 
-VARIANTS = ["1sm", "2sm128", "2sm240", "2sm256", "2smtall", "2smtallw", "small"]
+VARIANTS = ["1sm", "2sm128", "2sm240", "2sm256", "2smtall", "2smtallw", "2smtallk", "small"]
 
 
 @pytest.mark.parametrize("variant", VARIANTS)
@@ -266,6 +266,32 @@ def test_forward_tensor_variants_one_hot(variant, monkeypatch):
     V = synth.gaussian_bf16((8, d_in), 1.0, 6162)
     Y = slr.forward(to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U), to_dev(V), path="tensor")
     np.testing.assert_array_equal(bits_to_f64(from_dev(Y)), bits_to_f64(np.ascontiguousarray(S.T)))
+
+
+@pytest.mark.parametrize("d_out,d_in,r,M", [
+    (1000, 8192, 64, 250),    # 4 tiles on every pair: 16 K slices of 4 stages, ragged rows and tokens
+    (1024, 8192, 128, 256),   # two rank stages in slice 0, projection phase at r = 128
+    (2048, 4096, 256, 700),   # r > 128: T from the projection kernel, then the K-split kernel
+    (14336, 4096, 8, 2048),   # the gate/up shape: whole rounds, then 2-3 slices per tail tile
+])
+def test_forward_ksplit_tail(d_out, d_in, r, M, monkeypatch):
+    """The 512-row kernel with its last round split along K (SLR_TC_KERNEL=
+    2smtallk): each slice's fp32 partial tile, the fixed-order reduction and
+    the direct bf16 store, every element (or every output of sampled tokens)
+    against the oracle, and the output bit-identical on a second call."""
+    monkeypatch.setenv("SLR_TC_KERNEL", "2smtallk")
+    seed = d_out + d_in + r + M + 77
+    X, vals, meta, U, V = _layer_case(d_out, d_in, r, M, seed)
+    args = (to_dev(X), to_dev(vals), to_dev_u8(meta), to_dev(U), to_dev(V))
+    Y1 = slr.forward(*args, path="tensor")
+    Y2 = slr.forward(*args, path="tensor")
+    torch.cuda.synchronize()
+    slr.check_kernel_error()
+    b1, b2 = from_dev(Y1), from_dev(Y2)
+    np.testing.assert_array_equal(b1, b2)
+    rows = np.arange(M) if M * d_out <= 2_000_000 else sample_indices(M, 48, seed)
+    Yref, Bref = oracle.forward(X, vals, meta, U, V, rows=rows)
+    check_forward(b1[rows], Yref, Bref, f"K-split {d_out}x{d_in} r={r} M={M}", rows)
 
 
 # ----------------------------------------------------------------------------- chained launches
