@@ -334,9 +334,11 @@ SLR_API slr_status slr_forward(const void *X, int64_t M, const void *vals, const
  * above 64 tokens with r > 0, 1 KB of counters, room for the partial products
  * with which the 512-row tensor-core kernel forms T itself (r <= 128:
  * 128 x 256 x 64 or 128 fp32 values) and for the fp32 partial tiles of its
- * last round when that round is split along K (128 x 2 x 2 x 240 x 128 fp32
- * values, 62.9 MB).  The counters are zeroed on the stream before each such
- * launch. */
+ * last round when that round is split along K (one slot of 2 x 2 x 240 x 128
+ * fp32 values per SM pair of the current device: 36.4 MB on a 148-SM B200).
+ * The size is computed for the current device; a workspace sized on a device
+ * with fewer SMs is still valid (that round is then split by tokens).  The
+ * counters are zeroed on the stream before each launch that uses them. */
 SLR_API size_t slr_forward_workspace_size(int64_t M, int64_t d_out, int64_t d_in, int64_t r);
 
 /* Execution paths of the forward pass. */

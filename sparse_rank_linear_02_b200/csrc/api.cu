@@ -55,7 +55,15 @@ size_t workspace_bytes_for(int64_t M, int64_t r, slr_path path) {
     // Above kChainMaxM tokens the single-call forward may run the 512-row
     // kernel with its projection phase and K-split last round: T, counters,
     // partial products and partial tiles.
-    if (M > kChainMaxM) return round_up(fused_layout(M, r).bytes, kAlign);
+    if (M > kChainMaxM) {
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            sms = 148;   // no device: size for a B200
+        }
+        return round_up(fused_layout(M, r, fused_pairs_for(sms)).bytes, kAlign);
+    }
     return round_up((size_t)M * r * sizeof(uint16_t), kAlign);
 }
 
@@ -165,7 +173,8 @@ slr_status forward_impl(const void *X, int64_t M, const void *vals, const void *
         err = launch_tc_forward_fused(static_cast<const uint16_t *>(X), M, static_cast<const uint16_t *>(vals),
                                       static_cast<const uint8_t *>(meta), d_out, d_in,
                                       static_cast<const uint16_t *>(U), static_cast<const uint16_t *>(V), r,
-                                      static_cast<uint16_t *>(Y), static_cast<uint8_t *>(workspace), stream);
+                                      static_cast<uint16_t *>(Y), static_cast<uint8_t *>(workspace), workspace_bytes,
+                                      stream);
         return err == cudaSuccess ? SLR_OK : SLR_ERR_CUDA;
     }
     err = run_project(X, M, V, d_in, r, workspace, p, chained, stream);

@@ -445,7 +445,7 @@ struct Params2 {
     // work); each slice's fp32 partial tile goes to ks_part slot p, and
     // ks_count[i] counts the CTAs whose partial of tail tile i is written.
     int32_t ksplit;
-    float *ks_part;       // [kKsSlots][2 CTAs][2 halves][240 tokens][128 rows] fp32
+    float *ks_part;       // [pairs][2 CTAs][2 halves][240 / 4 token blocks][128 rows][4] fp32
     unsigned int *ks_count;
     uint16_t *y;          // Y [M, d_out]: the reduction of a K-split tile stores it directly
     // Token-split or whole tail: pair p's tail units are [tail[p], tail[p+1]).
@@ -963,6 +963,7 @@ struct CfgT {
 
 constexpr int kThreadsT = 384;  // 12 warps
 static_assert(kKsSlotFloats == 4 * 240 * BM, "K-split slot: 2 CTAs x 2 halves x 240 tokens x 128 rows");
+static_assert(kMaxPairs == 128, "fused_pairs_for caps the pairs at 128");
 
 // Bounded spin until *p >= target (acquire, GPU scope); false on expiry.
 __device__ __forceinline__ bool spin_count_ge(const unsigned int *p, unsigned int target) {
@@ -1931,7 +1932,7 @@ template <int BN>
 cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *T16, int64_t r,
                                uint16_t *Y, bool after_projection, int tail_mode, cudaStream_t stream, int chu = 0,
-                               const uint16_t *V = nullptr, uint8_t *fused_ws = nullptr) {
+                               const uint16_t *V = nullptr, uint8_t *fused_ws = nullptr, size_t ws_bytes = 0) {
     using C = CfgT<BN>;
     // With a fused workspace (single-call forward, r > 0) T lives in its
     // first region; the kernel forms T itself (projection phase) when r <=
@@ -1985,6 +1986,10 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
         if (max_pairs < 1) return cudaErrorInvalidConfiguration;
     }
     plan_pairs(M, d_out, d_in, r, chu, 4 * BM, max_pairs, tail_mode, &prm, &pairs);
+    const FusedLayout L = fused_layout(M, r, 0);
+    if (prm.ksplit && (ws_bytes < L.off_ks_part || (ws_bytes - L.off_ks_part) / (kKsSlotFloats * 4) < (size_t)pairs))
+        // A workspace sized for a device with fewer SMs: not enough slots.
+        plan_pairs(M, d_out, d_in, r, chu, 4 * BM, max_pairs, 1, &prm, &pairs);
     // Fewer pairs than 256-token tiles: T from the projection kernel instead.
     if (tp && (M + 255) / 256 > pairs) tp = false;
     prm.meta = meta;
@@ -2000,7 +2005,6 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
     prm.ks_part = nullptr;
     prm.ks_count = nullptr;
     prm.y = Y;
-    const FusedLayout L = fused_layout(M, r);
     if (tp) {
         // Token tiles of 256 over the pairs, K split as far as the pairs go
         // (every tile has a pair: M <= 256 * pairs).
@@ -2675,7 +2679,7 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
 
 cudaError_t launch_tc_forward_fused(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                     int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *V, int64_t r,
-                                    uint16_t *Y, uint8_t *ws, cudaStream_t stream) {
+                                    uint16_t *Y, uint8_t *ws, size_t ws_bytes, cudaStream_t stream) {
     if (M <= 0) return cudaSuccess;
     if (M > INT32_MAX || d_out > INT32_MAX || d_in > INT32_MAX) return cudaErrorInvalidValue;
     uint16_t *T16 = reinterpret_cast<uint16_t *>(ws);
@@ -2704,7 +2708,7 @@ cudaError_t launch_tc_forward_fused(const uint16_t *X, int64_t M, const uint16_t
     }
     if (tail >= 0)
         return tc::launch_sparse_tall<240>(X, M, vals, meta, d_out, d_in, U, T16, r, Y, false, tail, stream, chu, V,
-                                           ws);
+                                           ws, ws_bytes);
     cudaError_t err = cudaSuccess;
     if (r > 0) err = launch_tc_project(X, M, V, d_in, r, T16, false, stream);
     if (err == cudaSuccess) err = launch_tc_forward(X, M, vals, meta, d_out, d_in, U, r > 0 ? T16 : nullptr, r, Y, 1, stream);

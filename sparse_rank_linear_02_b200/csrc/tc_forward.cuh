@@ -25,15 +25,18 @@ constexpr int64_t kChainMaxM = 64;
 // 64), the fp32 partial products of the 512-row kernel's projection phase (at
 // most kFusedMaxParts slices of a 256-token tile, tile rows of up to 128 ranks;
 // r <= 128 only), and the fp32 partial tiles of its K-split last round (one
-// slot of 2 CTAs x 2 halves x 240 tokens x 128 rows per pair).
+// slot of 2 CTAs x 2 halves x 240 tokens x 128 rows per pair; `pairs` is the
+// most pairs a launch may use on the device, fused_pairs_for(SM count)).
 constexpr int64_t kFusedMaxParts = 128;
-constexpr int64_t kKsSlots = 128;                 // one per pair (at most kMaxPairs)
 constexpr int64_t kKsSlotFloats = 2 * 2 * 240 * 128;
-constexpr int64_t kKsMaxTiles = 128;              // counters: tail tiles < pairs
+inline int64_t fused_pairs_for(int sms) {
+    const int64_t p = sms / 2;
+    return p < 128 ? p : 128;
+}
 struct FusedLayout {
     size_t off_count, off_ks_count, off_part, off_ks_part, bytes;
 };
-inline FusedLayout fused_layout(int64_t M, int64_t r) {
+inline FusedLayout fused_layout(int64_t M, int64_t r, int64_t pairs) {
     const size_t t16 = ((size_t)M * (size_t)r * 2 + 255) / 256 * 256;
     const size_t rn = r <= 64 ? 64 : 128;
     FusedLayout L;
@@ -41,7 +44,7 @@ inline FusedLayout fused_layout(int64_t M, int64_t r) {
     L.off_ks_count = t16 + 64;
     L.off_part = t16 + 1024;
     L.off_ks_part = L.off_part + (r <= 128 ? (size_t)kFusedMaxParts * 256 * rn * 4 : 0);
-    L.bytes = L.off_ks_part + (size_t)kKsSlots * kKsSlotFloats * 4;
+    L.bytes = L.off_ks_part + (size_t)pairs * kKsSlotFloats * 4;
     return L;
 }
 
@@ -61,11 +64,12 @@ cudaError_t launch_tc_forward(const uint16_t *X, int64_t M, const uint16_t *vals
 // (r <= 128; else after the projection kernel) and its last round split along
 // K (one launch after a memset of the counters); otherwise the projection
 // kernel followed by launch_tc_forward as its programmatic dependent.
-// ws: fused_layout(M, r).bytes (null when r == 0: no projection phase, no K
-// split).
+// ws: ws_bytes >= fused_layout(M, r, pairs).bytes for the device's pairs
+// (null when r == 0: no projection phase, no K split); with fewer slots than
+// a K-split plan needs, the last round is split by tokens instead.
 cudaError_t launch_tc_forward_fused(const uint16_t *X, int64_t M, const uint16_t *vals, const uint8_t *meta,
                                     int64_t d_out, int64_t d_in, const uint16_t *U, const uint16_t *V, int64_t r,
-                                    uint16_t *Y, uint8_t *ws, cudaStream_t stream);
+                                    uint16_t *Y, uint8_t *ws, size_t ws_bytes, cudaStream_t stream);
 
 // T = X V^T on the tensor cores, written as bf16 [M, r] (dense tcgen05 mode of
 // the same kernel).  Requires d_in % 64 == 0, r % 8 == 0.  chained: launched

@@ -48,8 +48,12 @@ def test_meta_row_bytes_and_workspace():
     assert lib.slr_meta_row_bytes(4) == 1
     assert slr.workspace_size(16, 4096, 4096, 64) == 16 * 64 * 4
     # above 64 tokens: bf16 T, 1 KB of counters, the projection phase's partials
-    # (r <= 128) and the K-split slots (128 pairs x 2 CTAs x 2 halves x 240 x 128 fp32)
-    ks = 128 * 2 * 2 * 240 * 128 * 4
+    # (r <= 128) and the K-split slots (one per pair of the device, 74 pairs on
+    # 148 SMs, the size assumed without a GPU: 2 CTAs x 2 halves x 240 x 128 fp32)
+    pairs = 74
+    if torch.cuda.is_available():
+        pairs = min(128, torch.cuda.get_device_properties(0).multi_processor_count // 2)
+    ks = pairs * 2 * 2 * 240 * 128 * 4
     assert slr.workspace_size(2048, 14336, 4096, 64) == 2048 * 64 * 2 + 1024 + 128 * 256 * 64 * 4 + ks
     assert slr.workspace_size(2048, 14336, 4096, 128) == 2048 * 128 * 2 + 1024 + 128 * 256 * 128 * 4 + ks
     assert slr.workspace_size(2048, 14336, 4096, 256) == 2048 * 256 * 2 + 1024 + ks

@@ -269,10 +269,11 @@ def test_forward_tensor_variants_one_hot(variant, monkeypatch):
 
 
 @pytest.mark.parametrize("d_out,d_in,r,M", [
-    (1000, 8192, 64, 250),    # 4 tiles on every pair: 16 K slices of 4 stages, ragged rows and tokens
+    (1000, 8192, 64, 250),    # 4 tiles over 32 pairs: 8 K slices of 8 stages, ragged rows and tokens
     (1024, 8192, 128, 256),   # two rank stages in slice 0, projection phase at r = 128
     (2048, 4096, 256, 700),   # r > 128: T from the projection kernel, then the K-split kernel
     (14336, 4096, 8, 2048),   # the gate/up shape: whole rounds, then 2-3 slices per tail tile
+    (2048, 28672, 64, 512),   # long K: 12 tiles, 6-7 slices of 32-37 stages each
 ])
 def test_forward_ksplit_tail(d_out, d_in, r, M, monkeypatch):
     """The 512-row kernel with its last round split along K (SLR_TC_KERNEL=
