@@ -63,11 +63,6 @@ __global__ void __launch_bounds__(kWarps * 32, kBlocksPerSm) decode_forward_kern
     const int64_t nwarps = (int64_t)gridDim.x * kWarps;
     const uint16_t *xbase = X + m0 * d_in;
     constexpr int kUnroll = unroll_for<MT>();
-    // The weights take the registers, so the X values are loaded only once a
-    // row's weights have arrived; pull the CTA's X rows into L1 now, while the
-    // weights are in flight, so those loads hit L1.
-    for (int64_t line = threadIdx.x; line < (int64_t)nt * d_in * 2 / 128; line += kWarps * 32)
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const uint8_t *>(xbase) + line * 128));
 
     for (int64_t row = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); row < d_out; row += nwarps) {
         float acc[MT];
