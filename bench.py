@@ -86,9 +86,10 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, bus_id: str | None):
+    def __init__(self, bus_id: str | None, window: str = ""):
         self.bus_id = bus_id
         self.proc = None
+        self.window = window
 
     def __enter__(self):
         cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "20"]
@@ -128,18 +129,28 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(load) if load else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(self.samples),
-                "window": "nvidia-smi every 20 ms over an untimed replay of the timed graph and the timed replay"}
+                "window": "nvidia-smi every 20 ms over " + (self.window or "the timed replay")}
 
 
 # ----------------------------------------------------------------------------- timing
 
-def graph_time_ms(torch, fns, clock=None, preheat_s=0.5):
+def _replay_for(g, torch, seconds):
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        g.replay()
+        torch.cuda.synchronize()
+
+
+def graph_time_ms(torch, fns, clock=None, preheat_s=0.0, rest_s=0.2, postheat_s=0.0):
     """Capture the callables (one kernel sequence each) into one CUDA graph,
-    replay it once untimed, then once between CUDA events; returns the total
-    device time in ms of the timed replay.  With a clock sampler, sampling
-    starts before an untimed ~preheat_s replay loop of the same graph and
-    stops after the timed replay, so the loaded-clock samples bracket the
-    timed region even when it is only milliseconds long."""
+    replay it once untimed, let the GPU rest `rest_s` seconds (a 1 kW part
+    under a dense load reaches its power cap within tens of milliseconds and
+    recovers while idle, so every measurement starts from the same state),
+    replay it for `preheat_s` seconds untimed, then once between CUDA events;
+    returns the total device time in ms of the timed replay.  With a clock
+    sampler, sampling runs from before the rest to after `postheat_s` seconds
+    of further untimed replays, so that samples under this load bracket the
+    timed region even when it lasts only milliseconds."""
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for f in fns:
@@ -149,15 +160,14 @@ def graph_time_ms(torch, fns, clock=None, preheat_s=0.5):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if clock is not None:
         clock.__enter__()
-        t0 = time.perf_counter()
-        while time.perf_counter() - t0 < preheat_s:
-            g.replay()
-            torch.cuda.synchronize()
+    time.sleep(rest_s)
+    _replay_for(g, torch, preheat_s)
     e0.record()
     g.replay()
     e1.record()
     torch.cuda.synchronize()
     if clock is not None:
+        _replay_for(g, torch, postheat_s)
         clock.__exit__(None, None, None)
     ms = e0.elapsed_time(e1)
     del g
@@ -249,16 +259,20 @@ def run_ours(args, rank, world, dist):
     K = args.steps
 
     step_fns = [lambda s=sets[k % n_copies]: fwd(s) for k in range(K)]
-    clk = ClockSampler(bus_id_of(torch, dev) if rank == 0 else None)
+    clk = ClockSampler(bus_id_of(torch, dev) if rank == 0 else None,
+                       "0.5 s idle, 5 ms of untimed replays of the timed graph, the timed replay, then 40 ms of "
+                       "untimed replays")
     barrier()
-    # The K timed steps follow the warm-up directly (a 40 ms untimed replay of
-    # the same graph lets the clock sampler see the GPU under this load): the
-    # clocks of a run of milliseconds, which the burst peak describes.
-    total_ms = max_over_ranks(graph_time_ms(torch, step_fns, clock=clk, preheat_s=0.04))
+    # The K timed steps (milliseconds of work) start 5 ms into a load that
+    # follows 0.5 s of rest: the clocks of a short burst, which the burst peak
+    # describes.
+    total_ms = max_over_ranks(graph_time_ms(torch, step_fns, clock=clk, preheat_s=0.005, rest_s=0.5,
+                                            postheat_s=0.04))
     barrier()
     # The same K steps after a 0.5 s preheat, at the clocks a long run settles
     # to under the power cap (reported against the sustained peak).
-    clk_s = ClockSampler(bus_id_of(torch, dev) if rank == 0 else None)
+    clk_s = ClockSampler(bus_id_of(torch, dev) if rank == 0 else None,
+                         "a 0.5 s untimed replay loop of the timed graph and the timed replay")
     sustained_ms = max_over_ranks(graph_time_ms(torch, step_fns, clock=clk_s, preheat_s=0.5))
     barrier()
     # the dominant kernel, K launches over the same rotating buffers: the
@@ -317,8 +331,9 @@ def run_ours(args, rank, world, dist):
                              "clocks": clk_s.summary(),
                              "how": "the same K steps after a 0.5 s untimed replay, against the sustained "
                                     "measured peak"},
-               "peak_note": "frac_of_roofline: the K timed steps right after the warm-up, against the burst "
-                            "measured peak; 'sustained': after a 0.5 s preheat, against the sustained peak",
+               "peak_note": "frac_of_roofline: the K timed steps 5 ms into a load after 0.5 s of rest (a burst "
+                            "of milliseconds), against the burst measured peak; 'sustained': after a 0.5 s "
+                            "preheat, against the sustained peak",
                "two_launch_mode": {"project_ms": round(project_ms, 4), "combine_ms": round(combine_ms, 4),
                                    "how": "T from the projection kernel, then the combine kernel alone "
                                           "(slr_forward_project / slr_forward_combine)"},
