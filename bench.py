@@ -312,7 +312,7 @@ def run_ours(args, rank, world, dist):
                 "kernel_ms": round(kernel_ms, 4),
                 "peak_source": f"{peak_src}: 2:4 peak = {SPARSE_RATIO:g} x bf16_tflops {p_dense:g} (burst) for "
                                f"2*M*d_out*d_in, bf16_tflops for 2*M*r*(d_in+d_out)"}
-    # whole-step roofline (all kernels, the SURVEY's model)
+    # whole-step roofline (all kernels: the larger of the HBM time and the tensor time)
     step_bytes = algorithmic_bytes(M, d_out, d_in, r)
     t_roof_step = max(step_bytes / (peaks["hbm_gbs"] * 1e9),
                       flops_dense / (p_sparse * 1e12) + flops_lr / (p_dense * 1e12))

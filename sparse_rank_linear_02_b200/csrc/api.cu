@@ -26,19 +26,19 @@ slr_status check_device() {
         return SLR_ERR_DEVICE;
     }
     static std::mutex mu;
-    static int verdict[64] = {0};  // 0 unknown, 1 ok, 2 bad
+    static int device_ok[64] = {0};  // 0 unknown, 1 ok, 2 bad
     if (dev >= 64) return SLR_ERR_DEVICE;
     std::lock_guard<std::mutex> lock(mu);
-    if (verdict[dev] == 0) {
+    if (device_ok[dev] == 0) {
         int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
             cudaGetLastError();
             return SLR_ERR_DEVICE;
         }
-        verdict[dev] = (major == 10 && minor == 0) ? 1 : 2;
+        device_ok[dev] = (major == 10 && minor == 0) ? 1 : 2;
     }
-    return verdict[dev] == 1 ? SLR_OK : SLR_ERR_DEVICE;
+    return device_ok[dev] == 1 ? SLR_OK : SLR_ERR_DEVICE;
 }
 
 // The CUDA-core streaming path wins only for a single token on layers of up
