@@ -461,6 +461,30 @@ SLR_API slr_status slr_check_kernel_error(void);
  * without an sm_100 device, SLR_ERR_CUDA if the launch fails. */
 SLR_API slr_status slr_selftest_wait_timeout(int64_t limit_cycles, slr_stream_t stream);
 
+/* Host-only check of the work plan of the 2-SM pair kernels of slr_forward
+ * (no device needed, nothing launched).  The layer's product is a sum over
+ * the K stages of every output tile (LoSparse, section 3.2); the plan deals
+ * the tiles, pieces of tiles (runs of tokens) and K slices of tiles to the
+ * pairs.  This builds the plan for a problem shape as a launch would and walks
+ * every pair's chunk sequence, counting violations: every (row tile, 16-token
+ * unit, K stage) covered by exactly one chunk, the rank stages of every (row
+ * tile, unit) by exactly one, chunk rows and tokens inside the problem, a K
+ * slice only as a pair's last chunk, with its slice, slot and counter indices
+ * in range.
+ *
+ *   kernel       0: 256-row tiles, chunks of up to 128 tokens; 1: 240;
+ *                3: 256; 2: 512-row tiles, 240 tokens.
+ *   tail_mode    0: the last round dealt as whole tiles; 1: split by tokens;
+ *                2: split along K (kernel 2 only).
+ *   max_pairs    1..128 (the device's pairs, e.g. 74 on a 148-SM B200).
+ *   chunk_units  most 16-token units per chunk (0: the kernel's maximum).
+ *
+ * Returns the number of violations (0: the plan is sound), or -1 when an
+ * argument is out of range (as for slr_forward, d_in % 128 == 0, r % 8 == 0)
+ * or the problem needs more than 2^26 (tile, unit, stage) entries. */
+SLR_API int64_t slr_plan_check(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int32_t kernel, int32_t tail_mode,
+                               int32_t max_pairs, int32_t chunk_units);
+
 #ifdef __cplusplus
 }
 #endif

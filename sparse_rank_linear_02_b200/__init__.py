@@ -101,10 +101,25 @@ def _load() -> ctypes.CDLL:
     lib.slr_forward_decode_noalloc.argtypes = [p, i64, p, p, i64, i64, p, p, i64, p, p]
     lib.slr_selftest_wait_timeout.restype = st
     lib.slr_selftest_wait_timeout.argtypes = [i64, p]
+    i32 = ctypes.c_int32
+    lib.slr_plan_check.restype = i64
+    lib.slr_plan_check.argtypes = [i64, i64, i64, i64, i32, i32, i32, i32]
     return lib
 
 
 _lib = _load()
+
+
+PLAN_KERNELS = {"2sm128": 0, "2sm240": 1, "2smtall": 2, "2sm256": 3}
+PLAN_TAILS = {"whole": 0, "tokens": 1, "k": 2}
+
+
+def plan_check(M: int, d_out: int, d_in: int, r: int, kernel: str, tail: str, max_pairs: int,
+               chunk_units: int = 0) -> int:
+    """``slr_plan_check``: the number of violations in the pair kernels' work
+    plan for this shape (0 = sound; host only, no device needed)."""
+    return int(_lib.slr_plan_check(M, d_out, d_in, r, PLAN_KERNELS[kernel], PLAN_TAILS[tail], max_pairs,
+                                   chunk_units))
 
 
 def lib() -> ctypes.CDLL:

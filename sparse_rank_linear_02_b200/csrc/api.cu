@@ -414,6 +414,11 @@ slr_status slr_check_kernel_error(void) {
     return (code | code28 | code_bwd | code_am) ? SLR_ERR_TIMEOUT : SLR_OK;
 }
 
+int64_t slr_plan_check(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int32_t kernel, int32_t tail_mode,
+                       int32_t max_pairs, int32_t chunk_units) {
+    return slr::tc::plan_check(M, d_out, d_in, r, kernel, tail_mode, max_pairs, chunk_units);
+}
+
 slr_status slr_selftest_wait_timeout(int64_t limit_cycles, slr_stream_t stream) {
     if (limit_cycles < 1 || limit_cycles > INT32_MAX) return SLR_ERR_ARG;
     if (slr::check_device() != SLR_OK) return SLR_ERR_DEVICE;

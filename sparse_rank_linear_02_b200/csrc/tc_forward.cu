@@ -38,6 +38,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "tc_forward.cuh"
@@ -1879,6 +1880,76 @@ PlanChoice choose_plan(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int sm
     next_slot = (next_slot + 1) % 64;
     if (n_cached < 64) ++n_cached;
     return best;
+}
+
+// Host-only check of a pair plan (slr_plan_check): builds the plan as a
+// launch would and walks every pair's chunk sequence.  Counts violations:
+// each (row tile, 16-token unit, K stage) covered by exactly one chunk, the
+// rank stages of each (row tile, unit) by exactly one chunk, chunk rows and
+// tokens inside the problem, a K slice only as a pair's last chunk and with
+// slice, slot and counter indices in range.  -1 for arguments out of range.
+int64_t plan_check(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int kernel, int tail_mode, int max_pairs,
+                   int chu) {
+    if (M < 1 || M > INT32_MAX || d_out < 1 || d_out > INT32_MAX || d_in < BK || d_in % BK != 0 || r < 0 ||
+        r % 8 != 0 || kernel < 0 || kernel > 3 || tail_mode < 0 || tail_mode > 2 || max_pairs < 1 ||
+        max_pairs > kMaxPairs || (tail_mode == 2 && kernel != 2))
+        return -1;
+    const int cap = kernel == 0 ? Cfg2<128>::CHU : kernel == 1 ? Cfg2<240>::CHU : kernel == 3 ? Cfg2<256>::CHU
+                                                                                              : CfgT<240>::CHU;
+    if (chu <= 0 || chu > cap) chu = cap;
+    const int tile_rows = kernel == 2 ? 4 * BM : 2 * BM;
+    Params2 prm;
+    int P = 0;
+    plan_pairs(M, d_out, d_in, r, chu, tile_rows, max_pairs, tail_mode, &prm, &P);
+    const int64_t rows = (d_out + tile_rows - 1) / tile_rows, ut = prm.ut, nk = prm.nk;
+    if (rows * ut * nk > ((int64_t)1 << 26)) return -1;   // keeps the check's memory bounded
+    std::vector<uint8_t> cover((size_t)(rows * ut * nk), 0), rank((size_t)(rows * ut), 0);
+    int64_t bad = (P < 1 || P > max_pairs) ? 1 : 0;
+    for (int p = 0; p < P; ++p) {
+        ChunkIter it(prm, p, P);
+        Chunk ch;
+        bool part_seen = false;
+        int64_t guard = 0;
+        while (it.next(chu, ch)) {
+            if (++guard > rows * ut + 1) {   // more chunks than units: a loop that does not end
+                ++bad;
+                break;
+            }
+            if (part_seen) ++bad;   // a K slice is the pair's last chunk
+            if (ch.d0 < 0 || ch.d0 % tile_rows != 0 || ch.d0 / tile_rows >= rows || ch.n <= 0 || ch.n % 16 != 0 ||
+                ch.n > 16 * cap || ch.tok0 < 0 || ch.tok0 % 16 != 0 || ch.k0 < 0 || ch.k1 > nk || ch.k0 >= ch.k1) {
+                ++bad;
+                continue;
+            }
+            if (ch.part) {
+                part_seen = true;
+                const int64_t e = prm.tail[p];
+                const int q = (int)((e >> 8) & 255), g = (int)(e & 255);
+                const int64_t tt = (e >> 16) - (int64_t)prm.cyc * P;
+                if (!prm.ksplit || g < 2 || q >= g || p - q < 0 || p - q + g > P || tt < 0 || tt >= P ||
+                    64 + 4 * tt + 4 > 1024)
+                    ++bad;
+            }
+            const int64_t rt = ch.d0 / tile_rows;
+            for (int64_t u = ch.tok0 / 16; u < (ch.tok0 + ch.n) / 16; ++u) {
+                if (u >= ut) {
+                    ++bad;
+                    continue;
+                }
+                for (int64_t k = ch.k0; k < ch.k1; ++k) {
+                    uint8_t &c = cover[(size_t)((rt * ut + u) * nk + k)];
+                    if (c < 255) ++c;
+                }
+                if (ch.lr) {
+                    uint8_t &c = rank[(size_t)(rt * ut + u)];
+                    if (c < 255) ++c;
+                }
+            }
+        }
+    }
+    for (uint8_t c : cover) bad += c != 1;
+    for (uint8_t c : rank) bad += c != 1;
+    return bad;
 }
 
 template <int BN>

@@ -79,6 +79,13 @@ cudaError_t launch_tc_forward_fused(const uint16_t *X, int64_t M, const uint16_t
 cudaError_t launch_tc_project(const uint16_t *X, int64_t M, const uint16_t *V, int64_t d_in, int64_t r,
                               uint16_t *T16, bool chained, cudaStream_t stream);
 
+// Host-only check of the pair kernels' work plan (see slr_plan_check in
+// slr.h): the number of violations, 0 for a sound plan, -1 for bad arguments.
+namespace tc {
+int64_t plan_check(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int kernel, int tail_mode, int max_pairs,
+                   int chu);
+}  // namespace tc
+
 // Launches the failure-detection self-test kernel (a bounded wait that is
 // made to expire after limit_cycles SM clock cycles).
 cudaError_t launch_wait_timeout_selftest(long long limit_cycles, cudaStream_t stream);
