@@ -277,7 +277,7 @@ def run_ours(args, rank, world, dist):
     barrier()
     # the dominant kernel, K launches over the same rotating buffers: the
     # 512-row kernel with its projection phase (one forward() call: the kernel
-    # and the 8-byte memset of its two phase counters)
+    # and the 1 KB memset of its counters)
     kernel_ms = graph_time_ms(torch, step_fns) / K
     # the two-launch mode of the same step, for comparison: T from the
     # projection kernel, then the combine kernel reading it
@@ -388,7 +388,7 @@ def run_ours(args, rank, world, dist):
         "lora_backward": backward,
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": K,   # one tc2t_forward_kernel launch per timed step (and an 8-byte memset node)
+        "gpu_launches": K,   # one tc2t_forward_kernel launch per timed step (and a 1 KB memset node)
         "clocks": clocks,
         "cpu_baseline": cpu,
         "peaks": {"source": peak_src, **peaks},
