@@ -407,16 +407,23 @@ struct Cfg2 {
 // 64-element K panels of a stage in one copy (a 3-D view of X: element, row,
 // panel), landing as panel 0's rows then panel 1's rows; ts[i] loads
 // box_rows(i) rows of T (one panel).  A chunk uses the smallest box that holds
-// its rows; rows past the chunk are loaded but not read by the MMA.
+// its rows; rows past the chunk are loaded but not read by the MMA.  Boxes of
+// 8, 16, 32 and 64 rows, then `b4` and b4 + 8 rows (the rows of the plan's two
+// widths of whole token tiles, so that neither loads padding) and the
+// kernel's most (half_n).
 struct Maps2 {
     CUtensorMap vals, meta, u, y32, y16;
-    CUtensorMap xs[5];
-    CUtensorMap ts[5];
+    CUtensorMap xs[7];
+    CUtensorMap ts[7];
     CUtensorMap xt, vt;   // projection phase: X in 128-row boxes, V in RN/2-row boxes (two 64-wide panels)
 };
 
-__host__ __device__ constexpr int box_rows(int i, int half_n) { return i < 4 ? (8 << i) : half_n; }
-__host__ __device__ constexpr int pick_box(int rows) { return rows <= 8 ? 0 : rows <= 16 ? 1 : rows <= 32 ? 2 : rows <= 64 ? 3 : 4; }
+__host__ __device__ constexpr int box_rows(int i, int half_n, int b4) {
+    return i < 4 ? (8 << i) : i == 4 ? b4 : i == 5 ? (b4 + 8 < half_n ? b4 + 8 : half_n) : half_n;
+}
+__host__ __device__ constexpr int pick_box(int rows, int b4) {
+    return rows <= 8 ? 0 : rows <= 16 ? 1 : rows <= 32 ? 2 : rows <= 64 ? 3 : rows <= b4 ? 4 : rows <= b4 + 8 ? 5 : 6;
+}
 
 constexpr int kMaxPairs = 128;
 
@@ -430,6 +437,7 @@ struct Params2 {
     int32_t wu, wr;     // token tile tt has wu + (tt < wr) units
     int32_t cyc;        // rounds of the cyclic phase
     int32_t chu;        // most 16-token units per chunk (<= the kernel's BN / 16)
+    int32_t box4;       // rows of X box 4: those of the narrower whole token tiles (8 * wu, 64..8 * chu); box 5: 8 more
     int64_t n_tiles;    // tiles dealt in the cyclic phase (a last round may be partial)
     const uint8_t *meta;  // packed metadata [d_out, meta_ld] (copied with cp.async by the 512-row kernel)
     int64_t meta_ld;      // bytes per metadata row (d_in / 8)
@@ -640,8 +648,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
             const int d0 = ch.d0 + (int)rank * BM;
             const int rows = ch.n / 2;
             const int tok = ch.tok0 + (int)rank * rows;
-            const int bi = pick_box(rows);
-            const uint32_t brows = (uint32_t)box_rows(bi, C::HALF_N);
+            const int bi = pick_box(rows, prm.box4);
+            const uint32_t brows = (uint32_t)box_rows(bi, C::HALF_N, prm.box4);
             const CUtensorMap *xmap = &maps.xs[bi];
             const CUtensorMap *tmap = &maps.ts[bi];
             for (int ks = 0; ks < nstages; ++ks) {
@@ -770,7 +778,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
             while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(prm.chu, ch)) {
                 const uint32_t idesc_sp = idesc_bf16(2 * BM, ch.n, true);
                 const uint32_t idesc_dense = idesc_bf16(2 * BM, ch.n, false);
-                const uint32_t panel = (uint32_t)box_rows(pick_box(ch.n / 2), C::HALF_N) * 128u;
+                const uint32_t panel = (uint32_t)box_rows(pick_box(ch.n / 2, prm.box4), C::HALF_N, prm.box4) * 128u;
                 const int buf = C::NACC == 2 ? (it & 1) : 0;
                 const uint32_t use = (uint32_t)(C::NACC == 2 ? (it >> 1) : it);
                 bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_cluster(&acc_empty[buf], (use & 1) ^ 1));
@@ -1084,8 +1092,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
             const int d0 = ch.d0 + (int)rank * BM;        // half 0 rows of this CTA; half 1 at +256
             const int rows = ch.n / 2;
             const int tok = ch.tok0 + (int)rank * rows;
-            const int bi = pick_box(rows);
-            const uint32_t brows = (uint32_t)box_rows(bi, C::HALF_N);
+            const int bi = pick_box(rows, prm.box4);
+            const uint32_t brows = (uint32_t)box_rows(bi, C::HALF_N, prm.box4);
             const CUtensorMap *xmap = &maps.xs[bi];
             const CUtensorMap *tmap = &maps.ts[bi];
             const int nsp = ch.k1 - ch.k0;
@@ -1289,7 +1297,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT, 1)
             while (!__any_sync(0xFFFFFFFFu, *fail != 0) && iter.next(prm.chu, ch)) {
                 const uint32_t idesc_sp = idesc_bf16(2 * BM, ch.n, true);
                 const uint32_t idesc_dense = idesc_bf16(2 * BM, ch.n, false);
-                const uint32_t panel = (uint32_t)box_rows(pick_box(ch.n / 2), C::HALF_N) * 128u;
+                const uint32_t panel = (uint32_t)box_rows(pick_box(ch.n / 2, prm.box4), C::HALF_N, prm.box4) * 128u;
                 bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_cluster(acc_empty, (uint32_t)((it & 1) ^ 1)));
                 if (!ok) {
                     if (lane == 0) {
@@ -1736,6 +1744,12 @@ void plan_pairs(int64_t M, int64_t d_out, int64_t d_in, int64_t r, int chu, int 
     prm->ttiles = (int32_t)ttiles;
     prm->wu = (int32_t)(ut / ttiles);
     prm->wr = (int32_t)(ut % ttiles);
+    {
+        int b4 = 8 * prm->wu;
+        if (b4 < 64) b4 = 64;
+        if (b4 > 8 * chu) b4 = 8 * chu;
+        prm->box4 = b4;
+    }
     const int P = (int)(units < max_pairs ? units : max_pairs);
     // Whole rounds of tiles first.  tail_mode 0: the last, partial round is
     // dealt as whole tiles too.  1: its tiles are split among all pairs, each
@@ -1812,7 +1826,7 @@ double plan_cycles(const Params2 &prm, int pairs, int chu, int half_n, int mode)
         Chunk ch;
         double cyc = 0;
         while (it.next(chu, ch)) {
-            const double brows = box_rows(pick_box(ch.n / 2), half_n);
+            const double brows = box_rows(pick_box(ch.n / 2, prm.box4), half_n, prm.box4);
             const double bytes = tall ? 2.0 * 16384 + brows * 256 + 4096 : 16384 + brows * 256 + 2048;
             const double mma = (tall ? 4.0 : 2.0) * ch.n;
             const int nst = ch.k1 - ch.k0 + (ch.lr ? prm.nlr : 0);
@@ -1965,14 +1979,7 @@ cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *val
                        CU_TENSOR_MAP_SWIZZLE_NONE) &&
               make_map(&maps.y32, kBF16, Y, d_out, M, d_out * 2, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE) &&
               make_map(&maps.y16, kBF16, Y, d_out, M, d_out * 2, BM, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
-    for (int i = 0; i < 5 && ok; ++i)
-        ok = make_map_panels(&maps.xs[i], X, d_in, M, (uint32_t)box_rows(i, C::HALF_N));
-    if (ok && r > 0) {
-        ok = make_map(&maps.u, kBF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
-        for (int i = 0; i < 5 && ok; ++i)
-            ok = make_map(&maps.ts[i], kBF16, T16, r, M, r * 2, 64, (uint32_t)box_rows(i, C::HALF_N),
-                          CU_TENSOR_MAP_SWIZZLE_128B);
-    }
+    if (ok && r > 0) ok = make_map(&maps.u, kBF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -1983,6 +1990,13 @@ cudaError_t launch_sparse_pair(const uint16_t *X, int64_t M, const uint16_t *val
     int pairs = 0;
     if (chu <= 0 || chu > C::CHU) chu = C::CHU;
     plan_pairs(M, d_out, d_in, r, chu, 2 * BM, sms / 2 < kMaxPairs ? sms / 2 : kMaxPairs, tail_mode, &prm, &pairs);
+    // X and T boxes, now that the plan fixes box 4's rows.
+    for (int i = 0; i < 7; ++i) {
+        const uint32_t rows_i = (uint32_t)box_rows(i, C::HALF_N, prm.box4);
+        if (!make_map_panels(&maps.xs[i], X, d_in, M, rows_i)) return cudaErrorInvalidValue;
+        if (r > 0 && !make_map(&maps.ts[i], kBF16, T16, r, M, r * 2, 64, rows_i, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
     // Directly after the projection kernel on this stream: programmatic
     // dependent launch (the producer waits before it loads T).  Otherwise an
     // ordinary launch, which must not overlap an unrelated preceding kernel.
@@ -2020,14 +2034,7 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
                        CU_TENSOR_MAP_SWIZZLE_NONE) &&
               make_map(&maps.y32, kBF16, Y, d_out, M, d_out * 2, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE) &&
               make_map(&maps.y16, kBF16, Y, d_out, M, d_out * 2, BM, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
-    for (int i = 0; i < 5 && ok; ++i)
-        ok = make_map_panels(&maps.xs[i], X, d_in, M, (uint32_t)box_rows(i, C::HALF_N));
-    if (ok && r > 0) {
-        ok = make_map(&maps.u, kBF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
-        for (int i = 0; i < 5 && ok; ++i)
-            ok = make_map(&maps.ts[i], kBF16, T16, r, M, r * 2, 64, (uint32_t)box_rows(i, C::HALF_N),
-                          CU_TENSOR_MAP_SWIZZLE_128B);
-    }
+    if (ok && r > 0) ok = make_map(&maps.u, kBF16, U, r, d_out, r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
     const int tp_rn = r <= 64 ? 64 : 128;
     if (ok && tp)
         ok = make_map_panels(&maps.xt, X, d_in, M, 128) && make_map_panels(&maps.vt, V, d_in, r, tp_rn / 2);
@@ -2061,6 +2068,13 @@ cudaError_t launch_sparse_tall(const uint16_t *X, int64_t M, const uint16_t *val
     if (prm.ksplit && (ws_bytes < L.off_ks_part || (ws_bytes - L.off_ks_part) / (kKsSlotFloats * 4) < (size_t)pairs))
         // A workspace sized for a device with fewer SMs: not enough slots.
         plan_pairs(M, d_out, d_in, r, chu, 4 * BM, max_pairs, 1, &prm, &pairs);
+    // X and T boxes, now that the plan fixes box 4's rows.
+    for (int i = 0; i < 7; ++i) {
+        const uint32_t rows_i = (uint32_t)box_rows(i, C::HALF_N, prm.box4);
+        if (!make_map_panels(&maps.xs[i], X, d_in, M, rows_i)) return cudaErrorInvalidValue;
+        if (r > 0 && !make_map(&maps.ts[i], kBF16, T16, r, M, r * 2, 64, rows_i, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
     // Fewer pairs than 256-token tiles: T from the projection kernel instead.
     if (tp && (M + 255) / 256 > pairs) tp = false;
     prm.meta = meta;
