@@ -50,7 +50,7 @@ SPARSE_RATIO = 2.0   # nominal 2:4 sparse / dense tensor throughput ratio
 
 # DRAM bytes per launch of the dominant kernel from the committed ncu capture
 # (profiles/); valid only for the kernel source it was taken on.
-NCU_TRAFFIC = {"tc_forward": {"source_sha": "92bc7dc317066cbd", "bytes_per_launch": 118821888}}
+NCU_TRAFFIC = {"tc_forward": {"source_sha": "b30c665dc4dd5528", "bytes_per_launch": 119173632}}
 
 
 def layer_of(cfg, name):
