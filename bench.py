@@ -335,6 +335,10 @@ def run_ours(args, rank, world, dist):
                             "of milliseconds), against the burst measured peak; 'sustained': after a 0.5 s "
                             "preheat, against the sustained peak",
                "two_launch_mode": {"project_ms": round(project_ms, 4), "combine_ms": round(combine_ms, 4),
+                                   # the combine alone against its own flops (no T to form)
+                                   "combine_frac": round((flops_dense / (p_sparse * 1e12) +
+                                                          2.0 * M * r * d_out / (p_dense * 1e12)) /
+                                                         (combine_ms * 1e-3), 4),
                                    "how": "T from the projection kernel, then the combine kernel alone "
                                           "(slr_forward_project / slr_forward_combine)"},
                "path": path,
